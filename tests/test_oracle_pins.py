@@ -1,0 +1,395 @@
+"""Pins of the fp64 oracle to what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a special case that
+reduces to an older, simpler update; an independent complex-valued derivation; the
+parallel (masked matrix) form; a closed form; an exact ODE solution's convergence order;
+a hand-checkable rotation example; or an invariant. A plausible mistake in the oracle (a
+dropped beta term, beta_{t-1} instead of beta_t, a missing alpha in beta, the wrong rotation
+direction or pairing, bias before the norm, B and C swapped in MIMO, a state-passing slip)
+fails at least one of them.
+
+Page references are to "Mamba-3: Improved Sequence Modeling using State Space Principles".
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+
+
+def rnd_problem(rng, b=2, L=24, H=3, G=1, P=5, N=8, R=1, norm=True, bias=True, lam=None,
+                theta_scale=math.pi, dt_shift=-1.0):
+    x = rng.standard_normal((b, L, H, R, P))
+    B = rng.standard_normal((b, L, G, R, N))
+    C = rng.standard_normal((b, L, G, R, N))
+    th = rng.uniform(-1, 1, (b, L, H, N // 2)) * theta_scale
+    dt = np.log1p(np.exp(rng.standard_normal((b, L, H)) + dt_shift))
+    A = -np.exp(rng.uniform(-1, 1, (b, L, H)))
+    lm = (1 / (1 + np.exp(-rng.standard_normal((b, L, H))))) if lam is None else np.full(
+        (b, L, H), float(lam))
+    Bb = rng.standard_normal((H, R, N)) * 0.3 if bias else None
+    Cb = rng.standard_normal((H, R, N)) * 0.3 if bias else None
+    return dict(x=x, B=B, C=C, theta=th, dt=dt, A=A, lam=lm, B_bias=Bb, C_bias=Cb,
+                bc_norm=norm)
+
+
+def rand_state(rng, b, H, N, P, R):
+    return oracle.State(rng.standard_normal((b, H, N, P)),
+                        rng.uniform(-math.pi, math.pi, (b, H, N // 2)),
+                        rng.standard_normal((b, H, R, N)),
+                        rng.standard_normal((b, H, R, P)))
+
+
+def normed(v, bias, norm, eps=1e-6):
+    """B or C after the optional RMS norm over N and the bias (Sec. 3.4)."""
+    if norm:
+        v = v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    return v + (0 if bias is None else bias)
+
+
+# --------------------------------------------------------------------------------------
+# Independent complex-valued derivation (Appendix B.3, eq. 25 in complex form; Prop. 2).
+# The state is complex of size N/2 in the ORIGINAL (un-rotated) frame: the transition is
+# exp(dt (A + i theta)), the previous input gets rotated by the current step's angle, and
+# the real readout is Re(c^T h) with c = C_re - i C_im (Prop. 2: C = [C; -C_hat]).
+# --------------------------------------------------------------------------------------
+def complex_reference(p, state=None):
+    x, B, C, th, dt, A, lm = (p[k] for k in ("x", "B", "C", "theta", "dt", "A", "lam"))
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    half = N // 2
+    y = np.zeros((b, L, H, R, P))
+    out = oracle.State.zeros(b, H, N, P, R)
+    for bb in range(b):
+        for hh in range(H):
+            g = hh // (H // G)
+            Bb = None if p["B_bias"] is None else p["B_bias"][hh]
+            Cb = None if p["C_bias"] is None else p["C_bias"][hh]
+            if state is None:
+                phi0 = np.zeros(half)
+                hc = np.zeros((half, P), complex)
+                bprev = np.zeros((R, half), complex)
+                xprev = np.zeros((R, P))
+                praw = np.zeros((R, N))
+            else:
+                phi0 = state.phi[bb, hh].copy()
+                ht = state.h[bb, hh]
+                hc = np.exp(1j * phi0)[:, None] * (ht[:half] + 1j * ht[half:])
+                bn = normed(state.prev_B[bb, hh], Bb, p["bc_norm"])
+                bprev = bn[:, :half] + 1j * bn[:, half:]
+                xprev = state.prev_x[bb, hh].copy()
+                praw = state.prev_B[bb, hh].copy()
+            phi = phi0.copy()
+            for t in range(L):
+                d, a, l = dt[bb, t, hh], A[bb, t, hh], lm[bb, t, hh]
+                w = d * th[bb, t, hh]
+                bn = normed(B[bb, t, g], Bb, p["bc_norm"])
+                cn = normed(C[bb, t, g], Cb, p["bc_norm"])
+                bc = bn[:, :half] + 1j * bn[:, half:]
+                cc = cn[:, :half] - 1j * cn[:, half:]
+                beta = (1 - l) * d * math.exp(d * a)
+                gamma = l * d
+                hc = (np.exp(d * (a + 1j * th[bb, t, hh]))[:, None] * hc
+                      + beta * np.exp(1j * w)[:, None] * np.einsum("rn,rp->np", bprev, xprev)
+                      + gamma * np.einsum("rn,rp->np", bc, x[bb, t, hh]))
+                y[bb, t, hh] = np.real(np.einsum("rn,np->rp", cc, hc))
+                phi = phi + w
+                bprev, xprev, praw = bc, x[bb, t, hh].copy(), B[bb, t, g].copy()
+            ht = np.exp(-1j * phi)[:, None] * hc
+            out.h[bb, hh] = np.concatenate([ht.real, ht.imag], 0)
+            out.phi[bb, hh] = phi
+            out.prev_B[bb, hh] = praw
+            out.prev_x[bb, hh] = xprev
+    return y, out
+
+
+def run(p, state=None, **kw):
+    return oracle.scan(p["x"], p["B"], p["C"], p["theta"], p["dt"], p["A"], p["lam"],
+                       p["B_bias"], p["C_bias"], state=state, bc_norm=p["bc_norm"], **kw)
+
+
+def assert_state_close(s1, s2, tol=1e-11):
+    for f in ("h", "phi", "prev_B", "prev_x"):
+        a, b = getattr(s1, f), getattr(s2, f)
+        assert np.max(np.abs(a - b)) <= tol * max(1.0, np.max(np.abs(b))), f
+
+
+@pytest.mark.parametrize("R,G,H", [(1, 1, 3), (1, 3, 3), (2, 1, 2), (4, 2, 4)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_complex_valued_derivation(R, G, H, with_state):
+    """Rotated-frame real recurrence == complex recurrence in the original frame (App. B.3).
+
+    Pins the rotation direction (R^T), the (i, i+N/2) pairing, the sign convention of C,
+    the beta term's rotation by the current step, and the rotated-frame final state."""
+    rng = np.random.default_rng(10 + R + G + H + with_state)
+    p = rnd_problem(rng, H=H, G=G, R=R)
+    st = rand_state(rng, 2, H, 8, 5, R) if with_state else None
+    y, fs = run(p, st)
+    yc, fc = complex_reference(p, st)
+    np.testing.assert_allclose(y, yc, rtol=0, atol=1e-11 * np.max(np.abs(yc)))
+    assert_state_close(fs, fc, 1e-11)
+
+
+def test_lambda_one_is_exponential_euler():
+    """lam == 1 reduces to Mamba-2's exponential-Euler update h = e^{dt A} h + dt B x
+    (Sec. 3.1.1 Remark 2, eq. 4), written here in the complex form of Prop. 2."""
+    rng = np.random.default_rng(1)
+    p = rnd_problem(rng, lam=1.0, R=2)
+    y, fs = run(p)
+    x, B, C, th, dt, A = (p[k] for k in ("x", "B", "C", "theta", "dt", "A"))
+    b, L, H, R, P = x.shape
+    half = B.shape[-1] // 2
+    for bb in range(b):
+        for hh in range(H):
+            hc = np.zeros((half, P), complex)
+            for t in range(L):
+                bn = normed(B[bb, t, 0], p["B_bias"][hh], True)
+                cn = normed(C[bb, t, 0], p["C_bias"][hh], True)
+                hc = np.exp(dt[bb, t, hh] * (A[bb, t, hh] + 1j * th[bb, t, hh]))[:, None] * hc \
+                    + dt[bb, t, hh] * np.einsum("rn,rp->np", bn[:, :half] + 1j * bn[:, half:],
+                                                x[bb, t, hh])
+                ye = np.real(np.einsum("rn,np->rp", cn[:, :half] - 1j * cn[:, half:], hc))
+                np.testing.assert_allclose(y[bb, t, hh], ye, atol=1e-11)
+
+
+def test_theta_zero_is_real_ssm():
+    """theta == 0: no rotation (R_t = I), the angle stays 0 and the state equals the plain
+    real exponential-trapezoidal recurrence of Prop. 1 on the normalised, biased B, C."""
+    rng = np.random.default_rng(2)
+    p = rnd_problem(rng, theta_scale=0.0, R=1, G=1, H=2)
+    y, fs = run(p)
+    assert np.all(fs.phi == 0)
+    x, B, C, dt, A, lm = (p[k] for k in ("x", "B", "C", "dt", "A", "lam"))
+    for hh in range(2):
+        h = np.zeros((8, 5))
+        vprev = np.zeros((8, 5))
+        for t in range(x.shape[1]):
+            v = np.outer(normed(B[0, t, 0, 0], p["B_bias"][hh, 0], True), x[0, t, hh, 0])
+            al = math.exp(dt[0, t, hh] * A[0, t, hh])
+            h = al * h + (1 - lm[0, t, hh]) * dt[0, t, hh] * al * vprev + lm[0, t, hh] * dt[0, t, hh] * v
+            vprev = v
+            np.testing.assert_allclose(
+                y[0, t, hh, 0], h.T @ normed(C[0, t, 0, 0], p["C_bias"][hh, 0], True), atol=1e-11)
+
+
+@pytest.mark.parametrize("R", [1, 3])
+def test_parallel_mask_form(R):
+    """Y = (L o C B^T) X with L = L1 . L2 (Sec. 3.1.3 eq. 7): L1 the 1-semiseparable decay
+    matrix, L2 the 2-band matrix with gamma_t on the diagonal and beta_t below it. For MIMO
+    the token mask is expanded by the Kronecker product with a full R x R block of ones.
+    Rotations enter through B_bar, C_bar computed as complex products e^{-i Phi} b."""
+    rng = np.random.default_rng(3 + R)
+    T = 40
+    p = rnd_problem(rng, b=1, L=T, H=1, R=R, N=6, P=3)
+    y, _ = run(p)
+    dt, A, lm = p["dt"][0, :, 0], p["A"][0, :, 0], p["lam"][0, :, 0]
+    al = np.exp(dt * A)
+    beta = (1 - lm) * dt * al
+    gam = lm * dt
+    L1 = np.zeros((T, T))
+    for t in range(T):
+        for s in range(t + 1):
+            L1[t, s] = np.prod(al[s + 1:t + 1])
+    L2 = np.diag(gam) + np.diag(beta[1:], -1)
+    Lm = np.kron(L1 @ L2, np.ones((R, R)))
+    phi = np.cumsum(dt[:, None] * p["theta"][0, :, 0], axis=0)  # [T, N/2]
+    half = 3
+
+    def bar(v, bias):
+        vn = normed(v, bias, True)                    # [T, R, N]
+        z = (vn[..., :half] + 1j * vn[..., half:]) * np.exp(-1j * phi)[:, None, :]
+        return np.concatenate([z.real, z.imag], -1).reshape(T * R, 2 * half)
+
+    Bb = bar(p["B"][0, :, 0], p["B_bias"][0])
+    Cb = bar(p["C"][0, :, 0], p["C_bias"][0])
+    X = p["x"][0, :, 0].reshape(T * R, 3)
+    Y = (Lm * (Cb @ Bb.T)) @ X
+    np.testing.assert_allclose(y[0, :, 0].reshape(T * R, 3), Y, atol=1e-11 * np.max(np.abs(Y)))
+
+
+def test_mimo_is_sum_of_R2_siso():
+    """MIMO output i == sum over j of SISO runs with (B^(j), C^(i), x^(j)) (Sec. 3.3,
+    eq. 12-14). Catches B/C or x rank-index mix-ups."""
+    rng = np.random.default_rng(4)
+    R = 3
+    p = rnd_problem(rng, b=1, L=20, H=2, R=R)
+    y, _ = run(p)
+    acc = np.zeros_like(y)
+    for i in range(R):
+        for j in range(R):
+            q = dict(p)
+            q["x"] = p["x"][:, :, :, j:j + 1]
+            q["B"] = p["B"][:, :, :, j:j + 1]
+            q["C"] = p["C"][:, :, :, i:i + 1]
+            q["B_bias"] = p["B_bias"][:, j:j + 1]
+            q["C_bias"] = p["C_bias"][:, i:i + 1]
+            yij, _ = run(q)
+            acc[:, :, :, i] += yij[:, :, :, 0]
+    np.testing.assert_allclose(y, acc, atol=1e-11 * np.max(np.abs(acc)))
+
+
+def test_mimo_rank1_equals_siso_bitwise():
+    rng = np.random.default_rng(5)
+    p = rnd_problem(rng, R=1)
+    y1, s1 = run(p)
+    y2, s2 = run(p, nthreads=1)
+    assert np.array_equal(y1, y2) and np.array_equal(s1.h, s2.h)
+
+
+@pytest.mark.parametrize("lam", [0.5, 0.3, 1.0])
+def test_constant_alpha_closed_form(lam):
+    """Constant dt, A, lam, x, B, C and theta = 0: h_t = v [gamma + w alpha (1-alpha^t)/(1-alpha)]
+    with v = B x^T and w = gamma + (1-lam) dt, from unrolling Prop. 1 from h_0 = gamma_0 B_0 x_0."""
+    T, N, P = 50, 4, 3
+    rng = np.random.default_rng(6)
+    Bv, Cv, xv = rng.standard_normal(N), rng.standard_normal(N), rng.standard_normal(P)
+    d, a = 0.3, -0.7
+    p = dict(x=np.broadcast_to(xv, (1, T, 1, 1, P)).copy(),
+             B=np.broadcast_to(Bv, (1, T, 1, 1, N)).copy(),
+             C=np.broadcast_to(Cv, (1, T, 1, 1, N)).copy(),
+             theta=np.zeros((1, T, 1, N // 2)), dt=np.full((1, T, 1), d),
+             A=np.full((1, T, 1), a), lam=np.full((1, T, 1), lam), B_bias=None, C_bias=None,
+             bc_norm=False)
+    y, fs = run(p)
+    al, gam = math.exp(d * a), lam * d
+    w = gam + (1 - lam) * d
+    for t in range(T):
+        coef = gam + w * al * (1 - al ** t) / (1 - al)
+        np.testing.assert_allclose(y[0, t, 0, 0], coef * (Cv @ Bv) * xv, rtol=1e-12)
+    np.testing.assert_allclose(fs.h[0, 0], (gam + w * al * (1 - al ** (T - 1)) / (1 - al))
+                               * np.outer(Bv, xv), rtol=1e-12)
+
+
+def _ode_error(lam, n_steps, T_end=2.0, a=-0.8):
+    """Max error of the scheme against the exact solution of h' = a h + sin(tau), h(0) = 0,
+    sampled at tau_t = (t+1) dt, with x(tau) = sin(tau) (so x_{-1} = sin(0) = 0 and the
+    all-zero initial state is exact)."""
+    d = T_end / n_steps
+    tau = d * np.arange(1, n_steps + 1)
+    N, P = 2, 1
+    p = dict(x=np.sin(tau).reshape(1, -1, 1, 1, 1),
+             B=np.broadcast_to(np.array([1.0, 0.0]), (1, n_steps, 1, 1, N)).copy(),
+             C=np.broadcast_to(np.array([1.0, 0.0]), (1, n_steps, 1, 1, N)).copy(),
+             theta=np.zeros((1, n_steps, 1, 1)), dt=np.full((1, n_steps, 1), d),
+             A=np.full((1, n_steps, 1), a), lam=np.full((1, n_steps, 1), lam),
+             B_bias=None, C_bias=None, bc_norm=False)
+    y, _ = run(p)
+    # exact: h(t) = int_0^t e^{a(t-s)} sin s ds = (e^{at} - a sin t - cos t) / (1 + a^2)
+    exact = (np.exp(a * tau) - a * np.sin(tau) - np.cos(tau)) / (1 + a * a)
+    return np.max(np.abs(y[0, :, 0, 0, 0] - exact))
+
+
+def test_exact_solution_reference_is_right():
+    """The closed form used below solves h' = a h + sin(t), h(0) = 0 (checked by finite
+    differences), so the convergence test measures the scheme, not the reference."""
+    a = -0.8
+    t = np.linspace(0.1, 2, 50)
+    f = lambda t: (np.exp(a * t) - a * np.sin(t) - np.cos(t)) / (1 + a * a)
+    e = 1e-6
+    np.testing.assert_allclose((f(t + e) - f(t - e)) / (2 * e), a * f(t) + np.sin(t), atol=1e-8)
+    assert abs(f(0.0)) < 1e-15
+
+
+def test_convergence_order():
+    """lam = 1/2 is the classical trapezoid: global error O(dt^2); lam = 1 (Euler) is O(dt)
+    (Sec. 3.1.1 Remark 3, Appendix A.2). A beta without the e^{dt A} factor, or beta_{t-1}
+    in place of beta_t, degrades lam = 1/2 to first order and fails here."""
+    r_trap = _ode_error(0.5, 200) / _ode_error(0.5, 400)
+    r_euler = _ode_error(1.0, 200) / _ode_error(1.0, 400)
+    assert 3.6 < r_trap < 4.4, r_trap
+    assert 1.8 < r_euler < 2.2, r_euler
+    assert _ode_error(0.5, 400) < 1e-4
+
+
+def test_parity_by_rotation():
+    """State tracking by rotation (Sec. 3.2): with alpha = 1, dt = 1, lam = 1, one unit
+    impulse at t = 0 and theta_t = pi * bit_t, y_t = cos(pi * sum_{s=1..t} bit_s), i.e. the
+    parity of the bits seen after the impulse: +1 even, -1 odd."""
+    rng = np.random.default_rng(7)
+    T = 33
+    bits = rng.integers(0, 2, T)
+    x = np.zeros((1, T, 1, 1, 1))
+    x[0, 0] = 1.0
+    p = dict(x=x, B=np.broadcast_to(np.array([1.0, 0.0]), (1, T, 1, 1, 2)).copy(),
+             C=np.broadcast_to(np.array([1.0, 0.0]), (1, T, 1, 1, 2)).copy(),
+             theta=(math.pi * bits).reshape(1, T, 1, 1).astype(float),
+             dt=np.ones((1, T, 1)), A=np.zeros((1, T, 1)), lam=np.ones((1, T, 1)),
+             B_bias=None, C_bias=None, bc_norm=False)
+    y, _ = run(p)
+    par = np.cumsum(bits) - bits[0]
+    expect = np.where(par % 2 == 0, 1.0, -1.0)
+    np.testing.assert_allclose(y[0, :, 0, 0, 0], expect, atol=1e-12)
+
+
+@pytest.mark.parametrize("split", [1, 7, 23])
+def test_split_sequence_state_passing(split):
+    """scan(L1) -> state -> scan(L2) == scan(L1 + L2) (Appendix G.2 state passing)."""
+    rng = np.random.default_rng(8)
+    p = rnd_problem(rng, L=24, R=2, G=1, H=2)
+    st0 = rand_state(rng, 2, 2, 8, 5, 2)
+    y, fs = run(p, st0)
+    a = {k: (v[:, :split] if isinstance(v, np.ndarray) and v.ndim >= 3 and k not in ("B_bias", "C_bias") else v) for k, v in p.items()}
+    c = {k: (v[:, split:] if isinstance(v, np.ndarray) and v.ndim >= 3 and k not in ("B_bias", "C_bias") else v) for k, v in p.items()}
+    y1, s1 = run(a, st0)
+    y2, s2 = run(c, s1)
+    np.testing.assert_allclose(np.concatenate([y1, y2], 1), y, atol=1e-11)
+    assert_state_close(s2, fs)
+
+
+def test_decode_steps_equal_scan():
+    rng = np.random.default_rng(9)
+    p = rnd_problem(rng, L=9, R=2, H=2)
+    st0 = rand_state(rng, 2, 2, 8, 5, 2)
+    y, fs = run(p, st0)
+    st = st0
+    for t in range(9):
+        yt, st = oracle.decode_step(*(p[k][:, t] for k in ("x", "B", "C", "theta", "dt", "A", "lam")),
+                                    B_bias=p["B_bias"], C_bias=p["C_bias"], state=st,
+                                    bc_norm=True)
+        np.testing.assert_allclose(yt, y[:, t], atol=1e-12)
+    assert_state_close(st, fs)
+
+
+def test_bcnorm_scale_invariance_and_bias_after_norm():
+    """RMS norm then bias (Sec. 3.4): scaling B_raw and C_raw by any k > 0 per token leaves
+    the output unchanged (eps -> 0; 1e-30 keeps the all-zero initial prev_B finite); adding the bias before the norm would break this."""
+    rng = np.random.default_rng(11)
+    p = rnd_problem(rng, R=2)
+    y, _ = oracle.scan(p["x"], p["B"], p["C"], p["theta"], p["dt"], p["A"], p["lam"],
+                       p["B_bias"], p["C_bias"], bc_norm=True, norm_eps=1e-30)
+    k = rng.uniform(0.1, 10, p["B"].shape[:-1] + (1,))
+    y2, _ = oracle.scan(p["x"], p["B"] * k, p["C"] * k[..., ::-1, :], p["theta"], p["dt"],
+                        p["A"], p["lam"], p["B_bias"], p["C_bias"], bc_norm=True, norm_eps=1e-30)
+    np.testing.assert_allclose(y, y2, atol=1e-11 * np.max(np.abs(y)))
+    # RMS norm value itself: a constant vector c*1 normalises to 1 for any c.
+    q = dict(p)
+    q["B"] = np.full_like(p["B"], 3.7)
+    yb, _ = oracle.scan(q["x"], q["B"], p["C"], p["theta"], p["dt"], p["A"], p["lam"],
+                        None, p["C_bias"], bc_norm=True, norm_eps=1e-30)
+    q["B"] = np.full_like(p["B"], 1.0)
+    yc, _ = oracle.scan(q["x"], q["B"], normed(p["C"], None, True, 1e-30), p["theta"], p["dt"],
+                        p["A"], p["lam"], None, p["C_bias"], bc_norm=False)
+    np.testing.assert_allclose(yb, yc, atol=1e-11 * np.max(np.abs(yc)))
+
+
+def test_global_angle_offset_invariance():
+    """From a zero state, adding a constant to the initial angle leaves y unchanged: scores
+    depend only on angle differences (Appendix B.2)."""
+    rng = np.random.default_rng(12)
+    p = rnd_problem(rng, R=2)
+    st = oracle.State.zeros(2, 3, 8, 5, 2)
+    st.phi[:] = rng.uniform(-5, 5, st.phi.shape)
+    y0, f0 = run(p)
+    y1, f1 = run(p, st)
+    np.testing.assert_allclose(y0, y1, atol=1e-11 * np.max(np.abs(y0)))
+    np.testing.assert_allclose(f1.phi - f0.phi, st.phi, atol=1e-12)
+
+
+def test_empty_sequence_keeps_state():
+    rng = np.random.default_rng(13)
+    p = rnd_problem(rng, L=0)
+    st = rand_state(rng, 2, 3, 8, 5, 1)
+    y, fs = run(p, st)
+    assert y.shape[1] == 0
+    assert_state_close(fs, st, 0)
