@@ -1,0 +1,345 @@
+"""Benchmark of the Mamba-3 SSM core on B200.
+
+Headline: prefill throughput (tokens/s) of the SISO chunked scan at 1.5B-layer shapes
+(batch 4, 64 heads, head dim 64, state 128, L 2048, chunk 64, bf16 inputs, fp32 state,
+BC norm + bias), one m3_scan_fwd per step, inputs resident in HBM. Also reported: the
+decode step (batch 128, 64 heads, SISO and MIMO R=4) as us/step over 1000 consecutive steps
+captured in one CUDA graph, the end-to-end prefill through the public API with host buffers,
+the roofline of the dominant kernel, SM clocks during the timed region, and the CPU oracle.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-decode]
+For N > 1 launch under torch.distributed.run; every rank runs its own copy of the workload
+(independent sequences: weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roofline"
+WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        sm = sorted(r[0] for r in rows)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def scan_bytes(pr) -> int:
+    """Algorithmic HBM bytes of one scan: every input read once, y written once, final
+    state written once (no initial state)."""
+    t = pr.tensors()
+    n = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
+    n += t["x"].numel() * t["x"].element_size()  # y
+    d = pr.dims
+    es = t["x"].element_size()
+    units = d.batch * d.nheads
+    n += units * (d.dstate * d.headdim * 4 + d.dstate // 2 * 4 + d.rank * (d.dstate + d.headdim) * es)
+    return int(n)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from state_space_sequence_mamba_b200 import binding as m3
+    from state_space_sequence_mamba_b200.inputs import make_config, make_decode
+    m3.load_library()
+    hbm, tc, peak_kind = peaks()
+
+    # two input sets (each > L2) alternate between steps so no step reads the previous
+    # step's inputs from L2
+    sets = [make_config(1, device=dev, seed=1 + 100 * rank + i) for i in range(2)]
+    d = sets[0].dims
+    y = torch.empty_like(sets[0].x)
+    fin = m3.State.empty(d.batch, d.nheads, d.dstate, d.headdim, d.rank, d.dtype, dev)
+    ws = torch.zeros(max(256, m3.scan_workspace_bytes(m3.make_dims(sets[0].x, sets[0].B,
+                                                                   d.chunk, True, 1e-6))),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        m3.scan_fwd(**sets[i % 2].tensors(), init=None, final=fin, y=y, workspace=ws,
+                    chunk=d.chunk, bc_norm=True, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = ("GPU-" + str(props.uuid)) if getattr(props, "uuid", None) else str(local)
+    with ClockSampler(gpu_id) as clk:
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+    m3.scan_check(ws)
+    total_ms = ev[0].elapsed_time(ev[-1])
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    tokens = d.batch * d.seqlen
+    value = tokens * world * args.steps / (total_ms / 1e3)
+    byts = scan_bytes(sets[0])
+    launch_ms = sum(per_launch) / len(per_launch)
+    achieved = byts / (launch_ms / 1e3) / 1e9
+
+    # ---- end to end through the public API: pinned host inputs in, y out ----
+    host = {k: (v.cpu().pin_memory() if v is not None else None)
+            for k, v in sets[0].tensors().items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    dev_in = {k: (torch.empty_like(v, device=dev) if v is not None else None)
+              for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_host.numel() * y_host.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dev_in[k].copy_(v, non_blocking=True)
+        m3.scan_fwd(**dev_in, init=None, final=fin, y=y, workspace=ws, chunk=d.chunk,
+                    bc_norm=True, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = tokens * world * e2e_steps / (e2e_ms / 1e3)
+    del host, dev_in, y_host
+
+    # ---- decode: 1000 consecutive steps in one CUDA graph, SISO and MIMO R=4 ----
+    decode = {}
+    if not args.no_decode:
+        for R in (1, 4):
+            decode[f"R{R}"] = bench_decode(m3, dev, R, args.decode_steps, hbm, world, dist)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": d.batch, "seq_len": d.seqlen,
+                   "nheads": d.nheads, "headdim": d.headdim, "dstate": d.dstate,
+                   "chunk": d.chunk, "parallelism": f"independent sequences x{world}",
+                   "l2": "two alternating input sets of 144 MB each (> 126 MB L2), no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "bytes_per_launch": byts, "launch_ms": launch_ms,
+                     "peak_source": peak_kind},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "decode": decode,
+    }
+    if rank == 0:
+        line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def bench_decode(m3, dev, R, steps, hbm, world, dist):
+    import torch
+    from state_space_sequence_mamba_b200.inputs import make_decode
+    pr = make_decode(R, steps, device=dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in pr.state.items()})
+    yb = torch.empty(pr.dims.batch, pr.dims.nheads, R, pr.dims.headdim, dtype=torch.bfloat16,
+                     device=dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def run(n):
+        for t in range(n):
+            m3.decode_step(pr.x[t], pr.B[t], pr.C[t], pr.theta[t], pr.dt[t], pr.A[t], pr.lam[t],
+                           state_in=st, y=yb, stream=s)
+
+    with torch.cuda.stream(s):
+        run(3)  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run(steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):  # replay() launches on the current stream
+        g.replay()  # warm-up replay
+        torch.cuda.synchronize()
+        e0.record(s)
+        g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    us = ms * 1e3 / steps
+    units = pr.dims.batch * pr.dims.nheads
+    es = 2
+    N, P = pr.dims.dstate, pr.dims.headdim
+    per_unit = (2 * N * P * 4 + 2 * (N // 2) * 4 + 2 * R * N * es + 2 * R * P * es
+                + R * P * es + R * P * es + (N // 2) * es + 3 * 4)
+    byts = units * per_unit + pr.dims.batch * 2 * R * N * es
+    ach = byts / (us / 1e6) / 1e9
+    del g
+    return {"us_per_step": us, "steps": steps, "graph": True, "bytes_per_step": byts,
+            "achieved_gbs": ach, "frac_hbm": ach / hbm, "gpu_launches": steps}
+
+
+def cpu_baseline(pr):
+    """The fp64 oracle as it stands, on all host cores, on one of the workload's sequences
+    (batch 0, all heads, full length)."""
+    import oracle
+    t = {k: (v[:1].cpu() if (v is not None and k not in ("B_bias", "C_bias")) else
+             (v.cpu() if v is not None else None)) for k, v in pr.tensors().items()}
+    cores = oracle.max_threads()
+    t0 = time.perf_counter()
+    oracle.scan(**t, bc_norm=True, nthreads=cores)
+    dt = time.perf_counter() - t0
+    tokens = t["x"].shape[1]
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"1 of {pr.dims.batch} sequences (all {pr.dims.nheads} heads, "
+                      f"L={pr.dims.seqlen}), {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from state_space_sequence_mamba_b200.inputs import make_config
+    pr = make_config(1)
+    t = {k: (v[:1] if (v is not None and k not in ("B_bias", "C_bias")) else v)
+         for k, v in pr.tensors().items()}
+    cores = oracle.max_threads()
+    for _ in range(args.warmup):
+        oracle.scan(**t, bc_norm=True, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.scan(**t, bc_norm=True, nthreads=cores)
+    el = time.perf_counter() - t0
+    tokens = t["x"].shape[1]
+    v = tokens * args.steps / el
+    sample = (f"1 of {pr.dims.batch} sequences per step (all {pr.dims.nheads} heads, "
+              f"L={pr.dims.seqlen})")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

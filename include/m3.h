@@ -1,0 +1,136 @@
+/*
+ * m3.h -- C ABI of the Mamba-3 selective-SSM core on NVIDIA B200 (sm_100a).
+ *
+ * The operation is the recurrence of "Mamba-3: Improved Sequence Modeling using State Space
+ * Principles": the exponential-trapezoidal update (Sec. 3.1.1, Prop. 1)
+ *     h_t = alpha_t h_{t-1} + beta_t B_{t-1} x_{t-1}^T + gamma_t B_t x_t^T,
+ *     alpha_t = exp(dt_t A_t), beta_t = (1 - lam_t) dt_t alpha_t, gamma_t = lam_t dt_t,
+ * over a complex diagonal state realised as a cumulative data-dependent rotation of B and C
+ * (Sec. 3.2.1 Prop. 2, Sec. 3.2.2 Prop. 4 and Appendix B.3: Bbar_t = (prod_{s<=t} R_s^T) B_t,
+ * R_s = Block{R(dt_s theta_s[i])}), with B and C RMS-normalised and biased per head
+ * (Sec. 3.4), in single-input (rank R = 1) and rank-R MIMO form (Sec. 3.3, Appendix C:
+ * H_t = a_t H_{t-1} + B_t X_t^T, Y_t = H_t^T C_t), with y_t = H_t^T Cbar_t.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers to contiguous row-major buffers owned by the
+ *    caller, 16-byte aligned. The library never allocates or frees device memory, never
+ *    synchronises the device, and launches only on the given stream (a cudaStream_t passed
+ *    as void*; NULL = the legacy default stream).
+ *  - The complex state of size N/2 is stored as [Re; Im] halves: rotation pair i is
+ *    (i, i + N/2) (Prop. 2: B = [B; B_hat]).
+ *  - Head h reads B/C group h / (H / G).
+ *  - Errors: an invalid argument returns M3_ERR_INVALID_ARG, a valid but unsupported shape
+ *    M3_ERR_UNSUPPORTED, both before anything is launched; a launch failure returns
+ *    M3_ERR_CUDA. m3_last_error() describes the most recent failure of the calling thread.
+ *    No C++ exception crosses this interface.
+ *  - Inputs that hold NaN or Inf propagate into the affected (batch, head) outputs only.
+ */
+#ifndef M3_H_
+#define M3_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define M3_API __attribute__((visibility("default")))
+#else
+#define M3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    M3_OK = 0,
+    M3_ERR_INVALID_ARG = 1,
+    M3_ERR_UNSUPPORTED = 2,
+    M3_ERR_CUDA = 3,
+    M3_ERR_TIMEOUT = 4
+} m3_status;
+
+/* Storage type of x, B, C, theta, y, prev_B and prev_x. dt, A, lam, the biases and the
+ * state's h and phi are always fp32. */
+typedef enum { M3_F32 = 0, M3_BF16 = 1 } m3_dtype;
+
+typedef struct {
+    int64_t batch;    /* b >= 0                                                     */
+    int64_t seqlen;   /* L >= 0 (m3_decode_step: must be 1)                         */
+    int64_t nheads;   /* H >= 1                                                     */
+    int64_t ngroups;  /* G >= 1, H % G == 0: heads that share one B/C              */
+    int64_t headdim;  /* P in {16, 32, 64, 128}                                    */
+    int64_t dstate;   /* N, a multiple of 16, <= 256                               */
+    int64_t rank;     /* R in {1, 2, 4, 8}; 1 = SISO                                */
+    int64_t chunk;    /* tokens per chunk of the prefill scan (chunk * R <= 128)    */
+    int32_t in_dtype; /* m3_dtype                                                   */
+    int32_t bc_norm;  /* nonzero: RMS-normalise B and C over N before the bias      */
+    float norm_eps;   /* epsilon of the RMS norm (1e-6 is the usual value)          */
+} m3_dims;
+
+typedef struct {
+    const void* x;        /* [b, L, H, R, P]   in_dtype                                   */
+    const void* B;        /* [b, L, G, R, N]   in_dtype, raw (before norm and bias)       */
+    const void* C;        /* [b, L, G, R, N]   in_dtype, raw                              */
+    const void* theta;    /* [b, L, H, N/2]    in_dtype: per-step angle rate; the step's
+                             rotation angle is dt * theta (Prop. 2)                     */
+    const float* dt;      /* [b, L, H] step size, > 0 (after softplus)                     */
+    const float* A;       /* [b, L, H] decay rate, < 0                                     */
+    const float* lam;     /* [b, L, H] trapezoid weight in [0, 1] (lam = 1: Euler)         */
+    const float* B_bias;  /* [H, R, N] added after the norm, or NULL for zero              */
+    const float* C_bias;  /* [H, R, N] or NULL                                             */
+} m3_inputs;
+
+/* Recurrent state of every (batch, head) unit. Each unit owns its slice of every field. */
+typedef struct {
+    float* h;      /* [b, H, N, P] fp32, state in the rotated (RoPE) frame: prod R_s^T h  */
+    float* phi;    /* [b, H, N/2]  fp32 cumulative angle sum_s dt_s theta_s               */
+    void* prev_B;  /* [b, H, R, N] in_dtype: raw B of the last token seen (per head copy) */
+    void* prev_x;  /* [b, H, R, P] in_dtype: x of the last token seen                     */
+} m3_state;
+/* An all-zero state is the state of an empty sequence: h_{-1} = 0, x_{-1} = 0, so the first
+ * step is h_0 = gamma_0 B_0 x_0 (Sec. 3.1.3). */
+
+/* Bytes of device workspace m3_scan_fwd needs for these dims (>= 256), or 0 if the dims are
+ * invalid or unsupported. */
+M3_API size_t m3_scan_workspace_bytes(const m3_dims* dims);
+
+/* Chunked parallel prefill scan over a whole sequence (Sec. 3.1.3 parallel form, Sec. 3.3
+ * chunked algorithm).
+ *   init      state before token 0, or NULL for a fresh sequence (all zeros).
+ *   final     where to write the state after token L-1, or NULL to skip; may alias init.
+ *   y         [b, L, H, R, P] in_dtype output, y_t = H_t^T Cbar_t.
+ *   workspace device buffer of at least m3_scan_workspace_bytes(dims) bytes, 256-byte
+ *             aligned, zero-filled before its first use (e.g. one cudaMemsetAsync). Every
+ *             call leaves it zero-filled again, so it is reused without resetting. Two calls
+ *             that may run at the same time need separate workspaces.
+ * Asynchronous: returns after launching. A device-side timeout (a wait between CTAs that
+ * exceeded its bound) is reported by m3_scan_check after the stream has synchronised. */
+M3_API m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                      const m3_state* final_state, void* y, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* One-token decode step: exactly one iteration of the recurrence for every unit.
+ *   dims->seqlen must be 1; `in` points at one token: x [b,1,H,R,P], B, C [b,1,G,R,N] ...
+ *   state_in  the state before the token (required).
+ *   state_out where to write the state after it; may be the same buffers as state_in.
+ *   y         [b, H, R, P] in_dtype. */
+M3_API m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,
+                         const m3_state* state_out, void* y, void* stream);
+
+/* After the stream that ran m3_scan_fwd has synchronised: M3_OK, or M3_ERR_TIMEOUT if a
+ * bounded inter-CTA wait gave up (the outputs of that call are then incomplete). Performs
+ * one blocking 4-byte device-to-host copy; after a timeout it also re-zeroes the workspace
+ * header (blocking) so the workspace can be reused. */
+M3_API m3_status m3_scan_check(void* workspace);
+
+/* Static description of a status code. */
+M3_API const char* m3_status_str(m3_status s);
+
+/* Human-readable reason for the most recent failed call on this thread ("" if none). */
+M3_API const char* m3_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H_ */

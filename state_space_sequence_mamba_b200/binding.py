@@ -1,0 +1,202 @@
+"""ctypes binding of the C ABI in include/m3.h. Argument marshalling only.
+
+torch supplies device memory and streams; every step of the computation runs in the CUDA
+kernels of ``libm3.so``. If the library is missing this module raises: there is no fallback
+implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libm3.so")
+
+M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
+M3_F32, M3_BF16 = 0, 1
+
+
+class M3Error(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"m3 status {status}: {msg}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64),
+                ("rank", ctypes.c_int64), ("chunk", ctypes.c_int64),
+                ("in_dtype", ctypes.c_int32), ("bc_norm", ctypes.c_int32),
+                ("norm_eps", ctypes.c_float)]
+
+
+class Inputs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("x", "B", "C", "theta", "dt", "A", "lam", "B_bias", "C_bias")]
+
+
+class StateC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("h", "phi", "prev_B", "prev_x")]
+
+
+# Symbols include/m3.h declares (checked by the CPU test suite).
+EXPORTS = ("m3_scan_workspace_bytes", "m3_scan_fwd", "m3_decode_step", "m3_scan_check",
+           "m3_status_str", "m3_last_error")
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libm3.so and declares the signatures. Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m state_space_sequence_mamba_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER
+    lib.m3_scan_workspace_bytes.argtypes = [P(Dims)]
+    lib.m3_scan_workspace_bytes.restype = ctypes.c_size_t
+    lib.m3_scan_fwd.argtypes = [P(Dims), P(Inputs), P(StateC), P(StateC), ctypes.c_void_p,
+                                ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    lib.m3_scan_fwd.restype = ctypes.c_int
+    lib.m3_decode_step.argtypes = [P(Dims), P(Inputs), P(StateC), P(StateC), ctypes.c_void_p,
+                                   ctypes.c_void_p]
+    lib.m3_decode_step.restype = ctypes.c_int
+    lib.m3_scan_check.argtypes = [ctypes.c_void_p]
+    lib.m3_scan_check.restype = ctypes.c_int
+    lib.m3_status_str.argtypes = [ctypes.c_int]
+    lib.m3_status_str.restype = ctypes.c_char_p
+    lib.m3_last_error.argtypes = []
+    lib.m3_last_error.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != M3_OK:
+        lib = load_library()
+        raise M3Error(rc, lib.m3_last_error().decode() or lib.m3_status_str(rc).decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return M3_BF16
+    if dt == torch.float32:
+        return M3_F32
+    raise ValueError(f"unsupported input dtype {dt}")
+
+
+class State:
+    """Device state of every (batch, head) unit: h [b,H,N,P] fp32, phi [b,H,N/2] fp32,
+    prev_B [b,H,R,N] and prev_x [b,H,R,P] in the input dtype."""
+
+    def __init__(self, h, phi, prev_B, prev_x):
+        self.h, self.phi, self.prev_B, self.prev_x = h, phi, prev_B, prev_x
+
+    @staticmethod
+    def empty(batch, nheads, dstate, headdim, rank, dtype, device):
+        return State(torch.empty(batch, nheads, dstate, headdim, device=device),
+                     torch.empty(batch, nheads, dstate // 2, device=device),
+                     torch.empty(batch, nheads, rank, dstate, dtype=dtype, device=device),
+                     torch.empty(batch, nheads, rank, headdim, dtype=dtype, device=device))
+
+    @staticmethod
+    def from_dict(d):
+        return State(d["h"], d["phi"], d["prev_B"], d["prev_x"])
+
+    def as_dict(self):
+        return dict(h=self.h, phi=self.phi, prev_B=self.prev_B, prev_x=self.prev_x)
+
+    def c(self):
+        return StateC(*(_ptr(t) for t in (self.h, self.phi, self.prev_B, self.prev_x)))
+
+
+def make_dims(x, B, chunk, bc_norm, norm_eps):
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    return Dims(b, L, H, G, P, N, R, int(chunk), _dtype_code(x.dtype), 1 if bc_norm else 0,
+                float(norm_eps))
+
+
+def scan_workspace_bytes(dims: Dims) -> int:
+    return int(load_library().m3_scan_workspace_bytes(ctypes.byref(dims)))
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def scan_fwd(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, init: State | None = None,
+             final: State | None | bool = True, y=None, workspace=None, chunk=64,
+             bc_norm=False, norm_eps=1e-6, stream=None):
+    """m3_scan_fwd on torch CUDA tensors (shapes as in include/m3.h).
+
+    ``final=True`` allocates a new State for the result, ``False``/None skips it, or pass a
+    State (it may be ``init`` itself). Returns (y, final State or None)."""
+    lib = load_library()
+    dims = make_dims(x, B, chunk, bc_norm, norm_eps)
+    dev = x.device
+    if y is None:
+        y = torch.empty_like(x)
+    if final is True:
+        final = State.empty(dims.batch, dims.nheads, dims.dstate, dims.headdim, dims.rank,
+                            x.dtype, dev)
+    elif final is False:
+        final = None
+    need = scan_workspace_bytes(dims)
+    if need == 0:
+        # invalid or unsupported dims: let the call report why
+        need = 256
+    if workspace is None:
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias)))
+    ic = init.c() if init is not None else None
+    fc = final.c() if final is not None else None
+    rc = lib.m3_scan_fwd(ctypes.byref(dims), ctypes.byref(ins),
+                         ctypes.byref(ic) if ic is not None else None,
+                         ctypes.byref(fc) if fc is not None else None,
+                         _ptr(y), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc)
+    return y, final
+
+
+def scan_check(workspace):
+    _check(load_library().m3_scan_check(_ptr(workspace)))
+
+
+def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state_in: State = None,
+                state_out: State | None = None, y=None, bc_norm=False, norm_eps=1e-6,
+                stream=None):
+    """m3_decode_step: x [b,1,H,R,P], B, C [b,1,G,R,N], theta [b,1,H,N/2], dt/A/lam [b,1,H].
+
+    ``state_out`` defaults to ``state_in`` (in-place). Returns (y [b,H,R,P], state_out)."""
+    lib = load_library()
+    dims = make_dims(x, B, 1, bc_norm, norm_eps)
+    if state_out is None:
+        state_out = state_in
+    if y is None:
+        y = torch.empty(dims.batch, dims.nheads, dims.rank, dims.headdim, dtype=x.dtype,
+                        device=x.device)
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias)))
+    si, so = state_in.c(), state_out.c()
+    rc = lib.m3_decode_step(ctypes.byref(dims), ctypes.byref(ins), ctypes.byref(si),
+                            ctypes.byref(so), _ptr(y), _stream_handle(stream))
+    _check(rc)
+    return y, state_out

@@ -1,0 +1,223 @@
+// Host side of the C ABI declared in include/m3.h: argument validation, workspace layout and
+// dispatch to the kernels. Nothing here allocates device memory or synchronises a stream
+// (m3_scan_check excepted, which is documented to block).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "m3_internal.h"
+
+namespace m3 {
+namespace {
+
+thread_local char g_err[512] = "";
+
+m3_status fail(m3_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+m3_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(M3_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kWsHeader = 256;  // status word + padding
+
+m3_status check_dims(const m3_dims* d, bool scan) {
+    if (!d) return fail(M3_ERR_INVALID_ARG, "dims is NULL");
+    if (d->in_dtype != M3_F32 && d->in_dtype != M3_BF16)
+        return fail(M3_ERR_INVALID_ARG, "in_dtype %d is not M3_F32 or M3_BF16", d->in_dtype);
+    if (d->batch < 0 || d->seqlen < 0)
+        return fail(M3_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+    if (d->nheads < 1 || d->ngroups < 1 || d->nheads % d->ngroups != 0)
+        return fail(M3_ERR_INVALID_ARG, "nheads (%lld) must be a positive multiple of ngroups (%lld)",
+                    (long long)d->nheads, (long long)d->ngroups);
+    if (d->headdim < 1 || d->dstate < 2 || d->dstate % 2 != 0 || d->rank < 1)
+        return fail(M3_ERR_INVALID_ARG, "headdim >= 1, even dstate >= 2 and rank >= 1 required");
+    if (!(d->norm_eps >= 0.f) || !std::isfinite(d->norm_eps))
+        return fail(M3_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
+    if (d->headdim != 16 && d->headdim != 32 && d->headdim != 64 && d->headdim != 128)
+        return fail(M3_ERR_UNSUPPORTED, "headdim %lld not in {16, 32, 64, 128}",
+                    (long long)d->headdim);
+    if (d->dstate % 16 != 0 || d->dstate > 256)
+        return fail(M3_ERR_UNSUPPORTED, "dstate %lld must be a multiple of 16 and <= 256",
+                    (long long)d->dstate);
+    if (d->rank != 1 && d->rank != 2 && d->rank != 4 && d->rank != 8)
+        return fail(M3_ERR_UNSUPPORTED, "rank %lld not in {1, 2, 4, 8}", (long long)d->rank);
+    if (scan) {
+        if (d->chunk < 1) return fail(M3_ERR_INVALID_ARG, "chunk must be >= 1");
+        if (d->chunk * d->rank > 128)
+            return fail(M3_ERR_UNSUPPORTED, "chunk * rank = %lld exceeds 128",
+                        (long long)(d->chunk * d->rank));
+    }
+    if (d->batch * d->nheads > (int64_t)0x7fffffff)
+        return fail(M3_ERR_UNSUPPORTED, "batch * nheads exceeds the grid limit");
+    return M3_OK;
+}
+
+m3_status check_inputs(const m3_inputs* in, bool need) {
+    if (!in) return fail(M3_ERR_INVALID_ARG, "inputs is NULL");
+    if (!need) return M3_OK;
+    const void* req[] = {in->x, in->B, in->C, in->theta, in->dt, in->A, in->lam};
+    const char* names[] = {"x", "B", "C", "theta", "dt", "A", "lam"};
+    for (int i = 0; i < 7; ++i) {
+        if (!req[i]) return fail(M3_ERR_INVALID_ARG, "input %s is NULL", names[i]);
+        if (!aligned16(req[i]))
+            return fail(M3_ERR_INVALID_ARG, "input %s is not 16-byte aligned", names[i]);
+    }
+    if (in->B_bias && !aligned16(in->B_bias)) return fail(M3_ERR_INVALID_ARG, "B_bias misaligned");
+    if (in->C_bias && !aligned16(in->C_bias)) return fail(M3_ERR_INVALID_ARG, "C_bias misaligned");
+    return M3_OK;
+}
+
+m3_status check_state(const m3_state* s, const char* what) {
+    if (!s) return M3_OK;
+    const void* f[] = {s->h, s->phi, s->prev_B, s->prev_x};
+    const char* names[] = {"h", "phi", "prev_B", "prev_x"};
+    for (int i = 0; i < 4; ++i) {
+        if (!f[i]) return fail(M3_ERR_INVALID_ARG, "%s state field %s is NULL", what, names[i]);
+        if (!aligned16(f[i]))
+            return fail(M3_ERR_INVALID_ARG, "%s state field %s is not 16-byte aligned", what, names[i]);
+    }
+    return M3_OK;
+}
+
+ScanParams make_params(const m3_dims* d, const m3_inputs* in, const m3_state* init,
+                       const m3_state* fin, void* y) {
+    ScanParams p{};
+    p.b = d->batch; p.L = d->seqlen; p.H = d->nheads; p.G = d->ngroups; p.P = d->headdim;
+    p.N = d->dstate; p.R = d->rank; p.Q = d->chunk;
+    p.bc_norm = d->bc_norm ? 1 : 0; p.eps = d->norm_eps;
+    p.x = in->x; p.B = in->B; p.C = in->C; p.theta = in->theta;
+    p.dt = in->dt; p.A = in->A; p.lam = in->lam; p.Bbias = in->B_bias; p.Cbias = in->C_bias;
+    if (init) { p.h0 = init->h; p.phi0 = init->phi; p.prevB0 = init->prev_B; p.prevx0 = init->prev_x; }
+    if (fin) { p.h1 = fin->h; p.phi1 = fin->phi; p.prevB1 = fin->prev_B; p.prevx1 = fin->prev_x; }
+    p.y = y;
+    return p;
+}
+
+size_t elem_size(const m3_dims* d) { return d->in_dtype == M3_BF16 ? 2 : 4; }
+
+// Sequence of length 0: the final state is the initial one (or zeros).
+m3_status empty_sequence(const m3_dims* d, const m3_state* init, const m3_state* fin,
+                         cudaStream_t s) {
+    if (!fin) return M3_OK;
+    const size_t u = static_cast<size_t>(d->batch * d->nheads);
+    const size_t bytes[4] = {u * d->dstate * d->headdim * 4, u * (d->dstate / 2) * 4,
+                             u * d->rank * d->dstate * elem_size(d),
+                             u * d->rank * d->headdim * elem_size(d)};
+    void* dst[4] = {fin->h, fin->phi, fin->prev_B, fin->prev_x};
+    const void* src[4] = {init ? init->h : nullptr, init ? init->phi : nullptr,
+                          init ? init->prev_B : nullptr, init ? init->prev_x : nullptr};
+    for (int i = 0; i < 4; ++i) {
+        if (bytes[i] == 0) continue;
+        cudaError_t e = src[i] ? (src[i] == dst[i] ? cudaSuccess
+                                                   : cudaMemcpyAsync(dst[i], src[i], bytes[i],
+                                                                     cudaMemcpyDeviceToDevice, s))
+                               : cudaMemsetAsync(dst[i], 0, bytes[i], s);
+        if (e != cudaSuccess) return cuda_fail(e, "empty-sequence state copy");
+    }
+    return M3_OK;
+}
+
+}  // namespace
+}  // namespace m3
+
+using namespace m3;
+
+extern "C" {
+
+size_t m3_scan_workspace_bytes(const m3_dims* dims) {
+    if (check_dims(dims, true) != M3_OK) return 0;
+    return kWsHeader;
+}
+
+m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                      const m3_state* final_state, void* y, void* workspace, size_t ws_bytes,
+                      void* stream) {
+    g_err[0] = 0;
+    m3_status st = check_dims(dims, true);
+    if (st != M3_OK) return st;
+    const bool any = dims->batch * dims->seqlen * dims->nheads > 0;
+    if ((st = check_inputs(in, any)) != M3_OK) return st;
+    if ((st = check_state(init, "initial")) != M3_OK) return st;
+    if ((st = check_state(final_state, "final")) != M3_OK) return st;
+    if (any && !y) return fail(M3_ERR_INVALID_ARG, "y is NULL");
+    if (y && !aligned16(y)) return fail(M3_ERR_INVALID_ARG, "y is not 16-byte aligned");
+    const size_t need = m3_scan_workspace_bytes(dims);
+    if (!workspace) return fail(M3_ERR_INVALID_ARG, "workspace is NULL");
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(M3_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    if (ws_bytes < need)
+        return fail(M3_ERR_INVALID_ARG, "workspace has %zu bytes, %zu needed", ws_bytes, need);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ScanParams p = make_params(dims, in, init, final_state, y);
+    p.ws = workspace;
+    p.ws_bytes = ws_bytes;
+    p.status = static_cast<int32_t*>(workspace);
+    cudaError_t e;
+    if (dims->seqlen == 0 || dims->batch == 0) return empty_sequence(dims, init, final_state, s);
+
+    const bool bf16 = dims->in_dtype == M3_BF16;
+    const size_t smem = simt_scan_smem_bytes(p);
+    if (smem > 227 * 1024)
+        return fail(M3_ERR_UNSUPPORTED, "shape needs %zu bytes of shared memory", smem);
+    e = launch_scan_simt(p, bf16, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return M3_OK;
+}
+
+m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,
+                         const m3_state* state_out, void* y, void* stream) {
+    g_err[0] = 0;
+    m3_status st = check_dims(dims, false);
+    if (st != M3_OK) return st;
+    if (dims->seqlen != 1) return fail(M3_ERR_INVALID_ARG, "decode needs seqlen == 1");
+    if (!state_in || !state_out) return fail(M3_ERR_INVALID_ARG, "state_in and state_out are required");
+    const bool any = dims->batch > 0;
+    if ((st = check_inputs(in, any)) != M3_OK) return st;
+    if ((st = check_state(state_in, "input")) != M3_OK) return st;
+    if ((st = check_state(state_out, "output")) != M3_OK) return st;
+    if (any && (!y || !aligned16(y))) return fail(M3_ERR_INVALID_ARG, "y is NULL or misaligned");
+    if (!any) return M3_OK;
+    ScanParams p = make_params(dims, in, state_in, state_out, y);
+    const size_t smem = decode_smem_bytes(p);
+    if (smem > 227 * 1024) return fail(M3_ERR_UNSUPPORTED, "decode shape too large");
+    cudaError_t e = launch_decode(p, dims->in_dtype == M3_BF16, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return M3_OK;
+}
+
+m3_status m3_scan_check(void* workspace) {
+    if (!workspace) return fail(M3_ERR_INVALID_ARG, "workspace is NULL");
+    int32_t w = 0;
+    cudaError_t e = cudaMemcpy(&w, workspace, sizeof(w), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    if (w == 0) return M3_OK;
+    // Re-arm the workspace: zero the whole header so the next call starts clean.
+    e = cudaMemset(workspace, 0, kWsHeader);
+    if (e != cudaSuccess) return cuda_fail(e, "status reset");
+    return fail(M3_ERR_TIMEOUT, "a bounded wait between CTAs gave up (code %d)", w);
+}
+
+const char* m3_status_str(m3_status s) {
+    switch (s) {
+        case M3_OK: return "ok";
+        case M3_ERR_INVALID_ARG: return "invalid argument";
+        case M3_ERR_UNSUPPORTED: return "unsupported shape";
+        case M3_ERR_CUDA: return "CUDA error";
+        case M3_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* m3_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,49 @@
+// Internal declarations shared by the host entry points and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/m3.h"
+
+namespace m3 {
+
+// Everything a scan or decode launch needs, already validated by the host entry point.
+struct ScanParams {
+    int64_t b, L, H, G, P, N, R, Q;
+    int32_t bc_norm;
+    float eps;
+    const void* x;
+    const void* B;
+    const void* C;
+    const void* theta;
+    const float* dt;
+    const float* A;
+    const float* lam;
+    const float* Bbias;  // may be null
+    const float* Cbias;  // may be null
+    // initial state; all null = zero state
+    const float* h0;
+    const float* phi0;
+    const void* prevB0;
+    const void* prevx0;
+    // final state; all null = not written
+    float* h1;
+    float* phi1;
+    void* prevB1;
+    void* prevx1;
+    void* y;
+    int32_t* status;  // device status word (workspace), may be null for decode
+    void* ws;         // workspace base
+    size_t ws_bytes;
+};
+
+// Launchers. Each returns cudaSuccess or the launch error; none synchronises.
+cudaError_t launch_decode(const ScanParams& p, bool bf16, cudaStream_t s);
+// Shared-memory bytes the SIMT scan needs for these dims (0 = cannot run).
+size_t simt_scan_smem_bytes(const ScanParams& p);
+cudaError_t launch_scan_simt(const ScanParams& p, bool bf16, cudaStream_t s);
+// Size of the decode kernel's dynamic shared memory for these dims.
+size_t decode_smem_bytes(const ScanParams& p);
+
+}  // namespace m3

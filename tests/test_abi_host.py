@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every entry
+point include/m3.h declares, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import __graft_entry__
+from state_space_sequence_mamba_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    __graft_entry__.build()
+    return bd.load_library()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(m3_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    decl = declared_functions()
+    assert {"m3_scan_fwd", "m3_decode_step", "m3_scan_workspace_bytes", "m3_scan_check"} <= decl
+    for name in decl:
+        assert hasattr(lib, name), name
+    assert set(bd.EXPORTS) == decl
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.m3_status_str(s).decode()
+    assert lib.m3_status_str(99).decode() == "unknown status"
+
+
+def dims(**kw):
+    d = dict(batch=2, seqlen=10, nheads=4, ngroups=1, headdim=64, dstate=128, rank=1, chunk=64,
+             in_dtype=bd.M3_BF16, bc_norm=1, norm_eps=1e-6)
+    d.update(kw)
+    return bd.Dims(*(d[f] for f, _ in bd.Dims._fields_))
+
+
+def test_struct_layout_matches_header(lib):
+    assert ctypes.sizeof(bd.Dims) == 8 * 8 + 4 + 4 + 4 + 4  # trailing padding to 8
+    assert ctypes.sizeof(bd.Inputs) == 9 * 8 and ctypes.sizeof(bd.StateC) == 4 * 8
+
+
+@pytest.mark.parametrize("kw,ok", [
+    ({}, True), (dict(nheads=3, ngroups=2), False), (dict(dstate=15), False),
+    (dict(headdim=48), False), (dict(rank=3), False), (dict(chunk=0), False),
+    (dict(chunk=64, rank=4), False), (dict(chunk=16, rank=4), True), (dict(in_dtype=7), False),
+    (dict(dstate=272), False), (dict(norm_eps=-1.0), False), (dict(batch=-1), False),
+])
+def test_workspace_query_validates(lib, kw, ok):
+    n = lib.m3_scan_workspace_bytes(ctypes.byref(dims(**kw)))
+    assert (n >= 256) == ok
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any launch
+
+
+def fake_inputs(**kw):
+    f = {n: FAKE for n, _ in bd.Inputs._fields_}
+    f.update(kw)
+    return bd.Inputs(*(f[n] for n, _ in bd.Inputs._fields_))
+
+
+def test_scan_rejects_bad_arguments_without_launching(lib):
+    d = dims()
+    ins = fake_inputs()
+    ws = ctypes.c_void_p(0x100000)
+    call = lambda dd=d, ii=ins, y=FAKE, w=ws, nb=4096, init=None, fin=None: lib.m3_scan_fwd(
+        ctypes.byref(dd), ctypes.byref(ii), init, fin, y, w, nb, None)
+    assert call(ii=fake_inputs(x=None)) == bd.M3_ERR_INVALID_ARG
+    assert b"x" in lib.m3_last_error()
+    assert call(ii=fake_inputs(theta=FAKE + 2)) == bd.M3_ERR_INVALID_ARG
+    assert call(y=None) == bd.M3_ERR_INVALID_ARG
+    assert call(w=None) == bd.M3_ERR_INVALID_ARG
+    assert call(nb=16) == bd.M3_ERR_INVALID_ARG
+    assert call(w=ctypes.c_void_p(0x100010)) == bd.M3_ERR_INVALID_ARG  # not 256-aligned
+    bad = bd.StateC(FAKE, None, FAKE, FAKE)
+    assert call(init=ctypes.byref(bad)) == bd.M3_ERR_INVALID_ARG
+    assert b"phi" in lib.m3_last_error()
+    assert call(dd=dims(headdim=48)) == bd.M3_ERR_UNSUPPORTED
+    assert call(dd=dims(nheads=3, ngroups=2)) == bd.M3_ERR_INVALID_ARG
+    assert lib.m3_scan_fwd(None, ctypes.byref(ins), None, None, FAKE, ws, 4096, None) == \
+        bd.M3_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments_without_launching(lib):
+    d = dims(seqlen=1)
+    ins = fake_inputs()
+    st = bd.StateC(FAKE, FAKE, FAKE, FAKE)
+    assert lib.m3_decode_step(ctypes.byref(dims(seqlen=2)), ctypes.byref(ins), ctypes.byref(st),
+                              ctypes.byref(st), FAKE, None) == bd.M3_ERR_INVALID_ARG
+    assert lib.m3_decode_step(ctypes.byref(d), ctypes.byref(ins), None, ctypes.byref(st), FAKE,
+                              None) == bd.M3_ERR_INVALID_ARG
+    assert lib.m3_decode_step(ctypes.byref(d), ctypes.byref(fake_inputs(lam=None)),
+                              ctypes.byref(st), ctypes.byref(st), FAKE, None) == bd.M3_ERR_INVALID_ARG
+    assert lib.m3_decode_step(ctypes.byref(d), ctypes.byref(ins), ctypes.byref(st),
+                              ctypes.byref(st), None, None) == bd.M3_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(ImportError):
+        bd._lib_backup = bd._lib
+        try:
+            bd._lib = None
+            bd.load_library(str(tmp_path / "nope.so"))
+        finally:
+            bd._lib = bd._lib_backup

@@ -1,0 +1,222 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle on the same
+seeded inputs. Small cases span several chunks plus a ragged tail; the full-size workloads
+are checked on sampled heads / units that the oracle computes one by one."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_common import TOL, compare, gpu_scan, oracle_scan, oracle_state, rel
+from state_space_sequence_mamba_b200 import binding as m3
+from state_space_sequence_mamba_b200.inputs import make_config, make_decode, make_problem
+
+pytestmark = pytest.mark.gpu
+
+
+def test_config0_fp32_exact_path(cuda_dev):
+    pr = make_config(0)
+    y, fin = gpu_scan(pr, cuda_dev)
+    yo, so = oracle_scan(pr)
+    errs = compare(pr, y, fin, yo, so, tol=1e-4)
+    assert errs["y"] < 1e-4
+
+
+SMALL = [
+    # b, L, H, G, P, N, R, chunk, dtype, norm, bias, state
+    (2, 200, 4, 1, 64, 128, 1, 64, torch.bfloat16, True, 0.1, True),
+    (2, 200, 4, 1, 64, 128, 1, 64, torch.bfloat16, True, 0.1, False),
+    (1, 65, 4, 2, 64, 128, 1, 64, torch.bfloat16, False, 0.0, True),
+    (1, 63, 4, 4, 64, 128, 1, 64, torch.bfloat16, True, 0.1, True),
+    (2, 64, 3, 1, 64, 128, 1, 64, torch.bfloat16, True, 0.1, True),
+    (1, 1, 4, 1, 64, 128, 1, 64, torch.bfloat16, True, 0.1, True),
+    (2, 100, 4, 1, 64, 128, 4, 16, torch.bfloat16, True, 0.1, True),
+    (1, 17, 2, 1, 64, 128, 4, 16, torch.bfloat16, True, 0.1, False),
+    (1, 70, 2, 1, 32, 64, 2, 32, torch.bfloat16, True, 0.1, True),
+    (1, 40, 2, 2, 16, 16, 8, 8, torch.bfloat16, False, 0.0, True),
+    (1, 130, 2, 1, 64, 128, 1, 64, torch.float32, True, 0.1, True),
+    (1, 90, 2, 1, 128, 32, 1, 32, torch.float32, False, 0.0, True),
+    (1, 77, 2, 1, 16, 16, 4, 16, torch.float32, True, 0.3, True),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "b{}L{}H{}G{}P{}N{}R{}Q{}{}{}{}".format(
+    *c[:8], "f32" if c[8] == torch.float32 else "bf16", "n" if c[9] else "", "s" if c[11] else ""))
+def test_scan_small(cuda_dev, case):
+    b, L, H, G, P, N, R, Q, dt, norm, bias, st = case
+    pr = make_problem(b, L, H, G, P, N, rank=R, chunk=Q, dtype=dt, bc_norm=norm,
+                      bias_std=bias, seed=L + 13 * R + P, with_state=True)
+    y, fin = gpu_scan(pr, cuda_dev, use_state=st)
+    yo, so = oracle_scan(pr, use_state=st)
+    compare(pr, y, fin, yo, so)
+
+
+def test_final_state_may_alias_init(cuda_dev):
+    pr = make_problem(2, 150, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
+                      seed=5, with_state=True)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    y, fin = m3.scan_fwd(**g.tensors(), init=st, final=st, chunk=64, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, y, fin, yo, so)
+
+
+def test_empty_sequence(cuda_dev):
+    pr = make_problem(2, 0, 4, 1, 64, 128, seed=6, with_state=True)
+    g = pr.to(cuda_dev)
+    y, fin = m3.scan_fwd(**g.tensors(), init=m3.State.from_dict(g.state), chunk=64)
+    torch.cuda.synchronize()
+    for k in ("h", "phi", "prev_B", "prev_x"):
+        assert torch.equal(getattr(fin, k), g.state[k])
+    y, fin = m3.scan_fwd(**g.tensors(), init=None, chunk=64)
+    torch.cuda.synchronize()
+    assert float(fin.h.abs().max()) == 0.0 and float(fin.phi.abs().max()) == 0.0
+
+
+def test_split_sequence_on_gpu(cuda_dev):
+    """scan(L1) -> state -> scan(L2) matches the oracle's single scan(L1 + L2)."""
+    pr = make_problem(2, 300, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
+                      seed=21, with_state=True)
+    g = pr.to(cuda_dev)
+    t = g.tensors()
+    cut = 137
+    first = {k: (v[:, :cut].contiguous() if k not in ("B_bias", "C_bias") else v) for k, v in t.items()}
+    second = {k: (v[:, cut:].contiguous() if k not in ("B_bias", "C_bias") else v) for k, v in t.items()}
+    y1, s1 = m3.scan_fwd(**first, init=m3.State.from_dict(g.state), chunk=64, bc_norm=True)
+    y2, s2 = m3.scan_fwd(**second, init=s1, chunk=64, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.cat([y1, y2], 1), s2, yo, so)
+
+
+def test_deterministic(cuda_dev):
+    pr = make_problem(2, 200, 4, 1, 64, 128, rank=4, chunk=16, bc_norm=True, bias_std=0.1,
+                      seed=9, with_state=True)
+    y1, f1 = gpu_scan(pr, cuda_dev)
+    y2, f2 = gpu_scan(pr, cuda_dev)
+    assert torch.equal(y1, y2) and torch.equal(f1.h, f2.h)
+
+
+def test_nan_stays_in_its_unit(cuda_dev):
+    pr = make_problem(2, 100, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
+                      seed=10, with_state=True)
+    pr.x[1, 50, 2, 0, 3] = float("nan")
+    y, fin = gpu_scan(pr, cuda_dev)
+    bad = torch.isnan(y).any(dim=(1, 3, 4))  # [b, H]
+    assert bad[1, 2]
+    bad[1, 2] = False
+    assert not bad.any()
+    assert torch.isfinite(fin.h[0]).all() and torch.isfinite(fin.h[1, :2]).all()
+    assert torch.isfinite(fin.h[1, 3]).all()
+
+
+def test_unsupported_shape_reports_cleanly(cuda_dev):
+    pr = make_problem(1, 8, 2, 1, 128, 256, rank=1, chunk=64, seed=11)
+    with pytest.raises(m3.M3Error) as ei:
+        gpu_scan(pr, cuda_dev, use_state=False)
+    assert ei.value.status == m3.M3_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- decode
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_decode_steps_small(cuda_dev, R):
+    steps = 5
+    pr = make_problem(2, steps, 4, 1, 64, 128, rank=R, chunk=1, bc_norm=True, bias_std=0.1,
+                      seed=30 + R, with_state=True)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    ys = []
+    for t in range(steps):
+        tok = {k: (v[:, t:t + 1].contiguous() if k not in ("B_bias", "C_bias") else v)
+               for k, v in g.tensors().items()}
+        y, st = m3.decode_step(**tok, state_in=st, bc_norm=True)
+        ys.append(y.clone())
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.stack(ys, 1), st, yo, so)
+
+
+def test_decode_out_of_place_and_fp32(cuda_dev):
+    pr = make_problem(2, 1, 4, 2, 32, 64, rank=2, chunk=1, dtype=torch.float32, bc_norm=True,
+                      bias_std=0.2, seed=40, with_state=True)
+    g = pr.to(cuda_dev)
+    sin = m3.State.from_dict(g.state)
+    sout = m3.State.empty(2, 4, 64, 32, 2, torch.float32, cuda_dev)
+    y, sout = m3.decode_step(**g.tensors(), state_in=sin, state_out=sout, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, y[:, None], sout, yo, so, tol=1e-4)
+    for k in ("h", "phi"):
+        assert torch.equal(getattr(sin, k), g.state[k])  # input state untouched
+
+
+# ---------------------------------------------------------------- full-size workloads
+@pytest.mark.slow
+def test_config1_full_size_sampled_heads(cuda_dev):
+    pr = make_config(1)
+    y, fin = gpu_scan(pr, cuda_dev, use_state=False)
+    heads = [0, 17, 38, 63]
+    yo, so = oracle_scan(pr, use_state=False, heads=heads)
+    compare(pr, y, fin, yo, so, heads=heads)
+
+
+@pytest.mark.slow
+def test_config2_mimo_full_size_sampled_heads(cuda_dev):
+    pr = make_config(2)
+    y, fin = gpu_scan(pr, cuda_dev, use_state=False)
+    heads = [5, 44]
+    yo, so = oracle_scan(pr, use_state=False, heads=heads)
+    compare(pr, y, fin, yo, so, heads=heads)
+
+
+@pytest.mark.slow
+def test_config4_long_context_with_carry_in(cuda_dev):
+    """L = 65536 from the final state of the SISO prefill workload's sequence 0 (computed by
+    the oracle, stored as fp32 / bf16 like any state), checked on sampled heads."""
+    p1 = make_config(1)
+    for k in ("x", "B", "C", "theta", "dt", "A", "lam"):
+        setattr(p1, k, getattr(p1, k)[:1])
+    _, s1 = oracle_scan(p1, use_state=False)
+    pr = make_config(4)
+    pr.B_bias, pr.C_bias = p1.B_bias, p1.C_bias   # same layer parameters as the carried state
+    pr.state = dict(h=torch.from_numpy(s1.h).float(), phi=torch.from_numpy(s1.phi).float(),
+                    prev_B=torch.from_numpy(s1.prev_B).to(torch.bfloat16),
+                    prev_x=torch.from_numpy(s1.prev_x).to(torch.bfloat16))
+    y, fin = gpu_scan(pr, cuda_dev, use_state=True)
+    heads = [3, 60]
+    yo, so = oracle_scan(pr, use_state=True, heads=heads)
+    compare(pr, y, fin, yo, so, heads=heads)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("R", [1, 4])
+def test_config3_decode_1000_steps_sampled_units(cuda_dev, R):
+    steps = 1000
+    pr = make_decode(R, steps, device=cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in pr.state.items()})
+    bsel = [0, 77]
+    hsel = list(range(0, 64, 8)) if R == 4 else list(range(0, 64, 2))
+    ys = []
+    for t in range(steps):
+        y, st = m3.decode_step(pr.x[t], pr.B[t], pr.C[t], pr.theta[t], pr.dt[t], pr.A[t],
+                               pr.lam[t], state_in=st)
+        ys.append(y[bsel][:, hsel].float())
+    torch.cuda.synchronize()
+    ys = torch.stack(ys, 1)  # [nb, steps, nh, R, P]
+    b_i, h_i = torch.as_tensor(bsel), torch.as_tensor(hsel)
+    cpu = lambda t: t.cpu()
+    xo = cpu(pr.x[:, b_i][:, :, 0][:, :, h_i]).transpose(0, 1)
+    Bo = cpu(pr.B[:, b_i][:, :, 0]).transpose(0, 1)
+    Co = cpu(pr.C[:, b_i][:, :, 0]).transpose(0, 1)
+    tho = cpu(pr.theta[:, b_i][:, :, 0][:, :, h_i]).transpose(0, 1)
+    sc = lambda t: cpu(t[:, b_i][:, :, 0][:, :, h_i]).transpose(0, 1)
+    s0 = {k: cpu(v[b_i][:, h_i]) for k, v in pr.state.items()}
+    yo, so = oracle.scan(xo, Bo, Co, tho, sc(pr.dt), sc(pr.A), sc(pr.lam),
+                         state=oracle_state(s0))
+    e_y = rel(ys, yo)
+    e_h = rel(st.h[b_i][:, h_i], so.h)
+    e_phi = rel(st.phi[b_i][:, h_i], so.phi)
+    assert e_y <= TOL[torch.bfloat16] and e_h <= TOL[torch.bfloat16] and e_phi <= 2e-2, \
+        (e_y, e_h, e_phi)
