@@ -55,7 +55,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if pr.returncode != 0:
             raise RuntimeError("nvcc failed: " + " ".join(cmd))
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"])
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

@@ -166,6 +166,11 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
     if (dims->seqlen == 0 || dims->batch == 0) return empty_sequence(dims, init, final_state, s);
 
     const bool bf16 = dims->in_dtype == M3_BF16;
+    if (tc_scan_supported(p, bf16)) {
+        e = launch_scan_tc(p, s);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
+        return M3_OK;
+    }
     const size_t smem = simt_scan_smem_bytes(p);
     if (smem > 227 * 1024)
         return fail(M3_ERR_UNSUPPORTED, "shape needs %zu bytes of shared memory", smem);

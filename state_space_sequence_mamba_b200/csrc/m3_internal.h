@@ -43,6 +43,9 @@ cudaError_t launch_decode(const ScanParams& p, bool bf16, cudaStream_t s);
 // Shared-memory bytes the SIMT scan needs for these dims (0 = cannot run).
 size_t simt_scan_smem_bytes(const ScanParams& p);
 cudaError_t launch_scan_simt(const ScanParams& p, bool bf16, cudaStream_t s);
+// Tensor-core scan (bf16, N = 128, P = 64, chunk * R = 64).
+bool tc_scan_supported(const ScanParams& p, bool bf16);
+cudaError_t launch_scan_tc(const ScanParams& p, cudaStream_t s);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 
