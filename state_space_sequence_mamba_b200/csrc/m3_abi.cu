@@ -135,7 +135,11 @@ extern "C" {
 
 size_t m3_scan_workspace_bytes(const m3_dims* dims) {
     if (check_dims(dims, true) != M3_OK) return 0;
-    return kWsHeader;
+    const m3_inputs none{};
+    const ScanParams p = make_params(dims, &none, nullptr, nullptr, nullptr);
+    size_t body = 0;
+    if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_bytes(p);
+    return kWsHeader + (body + 255) / 256 * 256;
 }
 
 m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
@@ -167,7 +171,7 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
 
     const bool bf16 = dims->in_dtype == M3_BF16;
     if (tc_scan_supported(p, bf16)) {
-        e = launch_scan_tc(p, s);
+        e = launch_scan_tc(p, static_cast<char*>(workspace) + kWsHeader, s);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
         return M3_OK;
     }

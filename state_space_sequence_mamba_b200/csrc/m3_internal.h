@@ -45,7 +45,9 @@ size_t simt_scan_smem_bytes(const ScanParams& p);
 cudaError_t launch_scan_simt(const ScanParams& p, bool bf16, cudaStream_t s);
 // Tensor-core scan (bf16, N = 128, P = 64, chunk * R = 64).
 bool tc_scan_supported(const ScanParams& p, bool bf16);
-cudaError_t launch_scan_tc(const ScanParams& p, cudaStream_t s);
+// Workspace bytes the tensor-core scan needs beyond the status header.
+size_t tc_scan_workspace_bytes(const ScanParams& p);
+cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 

@@ -15,12 +15,15 @@
 //     y   = Yd + diag(e^{cum}) Yo ;  H1 = e^{cum_end} H0 + dH   (CUDA cores, fp32)
 // MIMO rows are (token, rank) pairs, the token mask applied to full R x R blocks.
 //
-// Data flow per CTA (one (batch, head) unit, 8 warps): X arrives by TMA in the 128-byte
-// swizzled layout the MMA reads; B, C, theta are read from global (B and C are shared by all
-// heads, so they come from L2), normalised, biased and rotated on the CUDA cores straight into
-// swizzled bf16 operand tiles; the fp32 state lives in registers (row n of the state in lane n
-// of the TMEM datapath, matching the dH accumulator) and is rounded to bf16 only as the Yo
-// operand. All waits are bounded; a timeout sets the status word and the CTA exits cleanly.
+// Data flow per CTA (one (batch, head) unit, 8 warps, two CTAs per SM): every per-chunk
+// input of the next chunk (X, theta, dt, A, lam) is fetched by TMA into the other half of a
+// double buffer while the current chunk computes; X lands in the 128-byte swizzled layout the
+// MMA reads. B and C are shared by all heads, so their rows come from L2; their RMS scales are
+// computed once per token by a small pre-pass instead of once per head. Normalisation, bias
+// and rotation run on the CUDA cores straight into swizzled bf16 operand tiles. The fp32
+// state lives in registers (row n of the state in lane n of the TMEM datapath, matching the
+// dH accumulator) and is rounded to bf16 only as the Yo operand. All waits are bounded; a
+// timeout sets the status word and the CTA exits cleanly.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -37,32 +40,42 @@ using namespace sm100;
 constexpr int kTcThreads = 256;
 constexpr int kN = 128, kP = 64, kHalf = 64;
 
+__host__ __device__ constexpr uint32_t round_up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
 template <int R>
 struct TcCfg {
     static constexpr int Q = 64 / R;                        // tokens per chunk
-    static constexpr int TPL = Q >= 32 ? Q / 32 : 1;        // tokens per lane (rotation)
+    static constexpr int TPL = Q >= 16 ? Q / 16 : 1;        // tokens per lane (rotation)
     static constexpr int PPL = (Q / 4) / TPL;               // pairs per lane (rotation)
     static constexpr int LPT = 8 / PPL;                     // lanes per token group
     static_assert(LPT * (Q / TPL) == 32, "rotation lane mapping");
+    // shared-memory byte layout after 1024-byte alignment
+    static constexpr uint32_t X0 = 0, X1 = 8192;             // X chunk (TMA, swizzled), x2
+    static constexpr uint32_t XP = 16384;                    // X' = diag(dw) X
+    static constexpr uint32_t OB = 24576;                    // Bbar, 2 slabs of 64 x 128 B
+    static constexpr uint32_t OC = 40960;                    // Cbar, 2 slabs
+    static constexpr uint32_t OP = 57344;                    // P = S o M
+    static constexpr uint32_t OH = 65536;                    // H0 bf16, 128 x 128 B
+    static constexpr uint32_t TH_BYTES = round_up(Q * 128, 1024);
+    static constexpr uint32_t TH0 = 81920, TH1 = TH0 + TH_BYTES;   // theta (TMA, swizzled)
+    static constexpr uint32_t SC_ONE = (Q + 1) * 16;                // [Q+1 tokens][4 heads] fp32
+    static constexpr uint32_t SC_SLOT = round_up(SC_ONE, 128);      // 128-byte aligned slots
+    static constexpr uint32_t SC_BYTES = 3 * SC_SLOT;
+    static constexpr uint32_t SC0 = TH1 + TH_BYTES, SC1 = SC0 + SC_BYTES;  // dt, A, lam boxes
+    static constexpr uint32_t OF = SC1 + SC_BYTES;                  // fp32 scratch
+    static constexpr uint32_t X_TX = 8192;                          // bytes of one X box
+    static constexpr uint32_t TS_TX = Q * 128 + 3 * SC_ONE;         // theta + scalar boxes
 };
-
-// smem byte layout (after 1024-byte alignment)
-constexpr uint32_t OFF_X = 0;           // X chunk, 64 rows x 128 B, swizzled (TMA)
-constexpr uint32_t OFF_XP = 8192;       // X' = diag(dw) X
-constexpr uint32_t OFF_B = 16384;       // Bbar, 2 slabs of 64 rows x 128 B
-constexpr uint32_t OFF_C = 32768;       // Cbar, 2 slabs
-constexpr uint32_t OFF_P = 49152;       // P = S o M, 64 rows x 128 B
-constexpr uint32_t OFF_H = 57344;       // H0 bf16, 128 rows x 128 B
-constexpr uint32_t OFF_F = 73728;       // fp32 scratch
-// fp32 scratch (float offsets from OFF_F)
+// fp32 scratch (float offsets)
 constexpr int F_CUM = 0, F_GAM = 64, F_W = 128, F_ECUM = 192, F_DW = 256, F_DT = 320,
-              F_RSB = 384, F_RSC = 448, F_MISC = 512, F_BIAS = 576;
-// F_BIAS: bias_B [R][128] then bias_C [R][128]; then prev-token fold scratch
+              F_MISC = 384, F_BLK = 448;   // one block of chunk scalars; two blocks (by parity)
+constexpr int F_BIAS = 2 * F_BLK;          // then bias_B [R][128], bias_C [R][128], fold scratch
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
 
-__host__ __device__ constexpr uint32_t tc_smem_bytes(int R) {
-    return OFF_F + 4u * (F_BIAS + 2 * R * 128 + R * 128 + R * 64) + 1024u;
+template <int R>
+__host__ __device__ constexpr uint32_t tc_smem_bytes() {
+    return TcCfg<R>::OF + 4u * (F_BIAS + 2 * R * kN + R * kN + R * kP) + 2u * 2 * R * kN + 1024u;
 }
 
 // Cody-Waite reduction of x by 2*pi (Cody & Waite, "Software Manual for the Elementary
@@ -78,38 +91,54 @@ __device__ __forceinline__ void sincos_2pi_reduced(float x, float* s, float* c) 
     __sincosf(r, s, c);
 }
 
+// 2^x by the hardware approximation (relative error ~2^-22), x <= 0 here.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Loads PPL consecutive bf16 as floats (PPL in {2, 4, 8}).
+// PPL consecutive bf16 held as raw words (PPL in {2, 4, 8}).
 template <int PPL>
-__device__ __forceinline__ void ld_bf16(const __nv_bfloat16* src, float (&v)[PPL]) {
+struct RawV { uint32_t w[PPL / 2]; };
+
+template <int PPL>
+__device__ __forceinline__ RawV<PPL> ldg_raw(const __nv_bfloat16* src) {
+    RawV<PPL> r;
     if constexpr (PPL == 8) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-            v[2 * i] = __low2float(h);
-            v[2 * i + 1] = __high2float(h);
-        }
+        r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
     } else if constexpr (PPL == 4) {
         const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-        const uint32_t w[2] = {u.x, u.y};
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-            v[2 * i] = __low2float(h);
-            v[2 * i + 1] = __high2float(h);
-        }
+        r.w[0] = u.x; r.w[1] = u.y;
     } else {
-        const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(src));
-        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&u);
-        v[0] = __low2float(h);
-        v[1] = __high2float(h);
+        r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(src));
     }
+    return r;
+}
+template <int PPL>
+__device__ __forceinline__ RawV<PPL> lds_raw(const uint8_t* src) {
+    RawV<PPL> r;
+    if constexpr (PPL == 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src);
+        r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
+    } else if constexpr (PPL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(src);
+        r.w[0] = u.x; r.w[1] = u.y;
+    } else {
+        r.w[0] = *reinterpret_cast<const uint32_t*>(src);
+    }
+    return r;
+}
+template <int PPL>
+__device__ __forceinline__ float raw_f(const RawV<PPL>& r, int j) {
+    const uint32_t w = r.w[j >> 1];
+    return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
 }
 
 template <int PPL>
@@ -128,52 +157,177 @@ __device__ __forceinline__ void st_bf16_smem(uint8_t* dst, const float (&v)[PPL]
     }
 }
 
-__device__ __forceinline__ void set_status(int32_t* status, int code) {
-    if (status) atomicExch(status, code);
+template <int PPL>
+__device__ __forceinline__ void sts_raw(uint8_t* dst, const RawV<PPL>& v) {
+    if constexpr (PPL == 8) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
+    } else if constexpr (PPL == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(v.w[0], v.w[1]);
+    } else {
+        *reinterpret_cast<uint32_t*>(dst) = v.w[0];
+    }
+}
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) {
+    return *reinterpret_cast<const __nv_bfloat162*>(&w);
+}
+__device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct TcMaps {
+    CUtensorMap x, theta, dt, A, lam;
+};
+
+// RMS scale of every B and C row (shared by all heads): one warp per row of N = 128.
+__global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __restrict__ B,
+                                                        const __nv_bfloat16* __restrict__ C,
+                                                        int64_t rows, float eps,
+                                                        float2* __restrict__ out) {
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const uint2 ub = __ldg(reinterpret_cast<const uint2*>(B + row * kN) + lane);
+    const uint2 uc = __ldg(reinterpret_cast<const uint2*>(C + row * kN) + lane);
+    float sb = 0.f, sc = 0.f;
+    const uint32_t wb[2] = {ub.x, ub.y}, wc[2] = {uc.x, uc.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float b0 = __uint_as_float(wb[i] << 16), b1 = __uint_as_float(wb[i] & 0xFFFF0000u);
+        const float c0 = __uint_as_float(wc[i] << 16), c1 = __uint_as_float(wc[i] & 0xFFFF0000u);
+        sb = fmaf(b0, b0, fmaf(b1, b1, sb));
+        sc = fmaf(c0, c0, fmaf(c1, c1, sc));
+    }
+    sb = warp_sum(sb);
+    sc = warp_sum(sc);
+    if (lane == 0) out[row] = make_float2(rsqrtf(sb / kN + eps), rsqrtf(sc / kN + eps));
 }
 
 template <int R>
 __global__ void __launch_bounds__(kTcThreads, 2)
-scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
+scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const float2* __restrict__ rsrow) {
     using Cfg = TcCfg<R>;
     constexpr int Q = Cfg::Q, TPL = Cfg::TPL, PPL = Cfg::PPL, LPT = Cfg::LPT;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float* sf = reinterpret_cast<float*>(sm + OFF_F);
+    float* sf = reinterpret_cast<float*>(sm + Cfg::OF);   // two blocks of chunk scalars
     float* s_biasB = sf + F_BIAS;
     float* s_biasC = s_biasB + R * kN;
     float* s_fold = s_biasC + R * kN;     // [R][128] Bbar of the stored previous token
     float* s_foldx = s_fold + R * kN;     // [R][64]  its x
-    __shared__ uint64_t bar_x, bar_m1, bar_m2;
+    __nv_bfloat16* s_biasB2 = reinterpret_cast<__nv_bfloat16*>(s_foldx + R * kP);  // [R][128] bf16
+    __nv_bfloat16* s_biasC2 = s_biasB2 + R * kN;
+    __shared__ uint64_t bar_x[2], bar_t[2], bar_m1, bar_m2;
     __shared__ uint32_t tslot;
     __shared__ int s_abort;
+    // async work thread 0 has started (for draining it if a wait gives up)
+    __shared__ int s_issued[4];  // last X / TS chunk issued, MMA groups committed (m1, m2)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3, wh = warp >> 2;  // TMEM subpartition, column half
     const int64_t u = blockIdx.x;
     const int64_t bb = u / p.H, hh = u % p.H, g = hh / (p.H / p.G);
-    const int64_t L = p.L;
-    const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
-    const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
-    const __nv_bfloat16* Cg = static_cast<const __nv_bfloat16*>(p.C);
-    const __nv_bfloat16* thg = static_cast<const __nv_bfloat16*>(p.theta);
-    __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
-    auto sidx = [&](int64_t t) { return (bb * L + t) * p.H + hh; };
+    const int hc = static_cast<int>(hh & 3);  // column of this head in the scalar boxes
+    const int L = static_cast<int>(p.L);
+    const int H = static_cast<int>(p.H), G = static_cast<int>(p.G);
+    // Per-unit base pointers; offsets below fit in 32 bits (checked on the host).
+    const __nv_bfloat16* Bu = static_cast<const __nv_bfloat16*>(p.B) + (bb * p.L * G + g) * R * kN;
+    const __nv_bfloat16* Cu = static_cast<const __nv_bfloat16*>(p.C) + (bb * p.L * G + g) * R * kN;
+    const float2* rsu = rsrow ? rsrow + (bb * p.L * G + g) * R : nullptr;
+    const __nv_bfloat16* xu = static_cast<const __nv_bfloat16*>(p.x) + (bb * p.L * H + hh) * R * kP;
+    __nv_bfloat16* yu = static_cast<__nv_bfloat16*>(p.y) + (bb * p.L * H + hh) * R * kP;
+    const int tokB = G * R * kN, tokY = H * R * kP;  // element stride of one token
+    const int nchunks = (L + Q - 1) / Q;
+
+    auto issue_x = [&](int c) {
+        const int st = c & 1;
+        mbar_arrive_expect_tx(&bar_x[st], Cfg::X_TX);
+        tma_load_5d(sm + (st ? Cfg::X1 : Cfg::X0), &maps.x, &bar_x[st], 0, 0,
+                    static_cast<int>(hh), c * Q, static_cast<int>(bb));
+    };
+    auto issue_ts = [&](int c) {  // theta and the dt, A, lam boxes of chunk c
+        const int st = c & 1;
+        uint64_t* bar = &bar_t[st];
+        mbar_arrive_expect_tx(bar, Cfg::TS_TX);
+        const int ic0 = c * Q, ih = static_cast<int>(hh), ib = static_cast<int>(bb);
+        tma_load_4d(sm + (st ? Cfg::TH1 : Cfg::TH0), &maps.theta, bar, 0, ih, ic0, ib);
+        uint8_t* sc = sm + (st ? Cfg::SC1 : Cfg::SC0);
+        const int h4 = ih & ~3;
+        tma_load_3d(sc, &maps.dt, bar, h4, ic0, ib);
+        tma_load_3d(sc + Cfg::SC_SLOT, &maps.A, bar, h4, ic0, ib);
+        tma_load_3d(sc + 2 * Cfg::SC_SLOT, &maps.lam, bar, h4, ic0, ib);
+    };
+    // Chunk scalars (one full warp): cumulative log-decay, gamma, trapezoid weight w, ...
+    auto scalars = [&](int c) {
+        const int st = c & 1;
+        if (!mbar_wait(&bar_t[st], (c >> 1) & 1)) {
+            if (lane == 0) s_abort = 1;
+        }
+        const float* sSc = reinterpret_cast<const float*>(sm + (st ? Cfg::SC1 : Cfg::SC0));
+        float* blk = sf + st * F_BLK;
+        const int T = (L - c * Q) < Q ? (L - c * Q) : Q;
+        constexpr int oA = Cfg::SC_SLOT / 4, oL = 2 * Cfg::SC_SLOT / 4;
+        float a[2], d[2], ga[2], w[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = lane + 32 * k;
+            a[k] = d[k] = ga[k] = w[k] = 0.f;
+            if (t < T) {
+                const float dd = sSc[t * 4 + hc], lm = sSc[oL + t * 4 + hc];
+                d[k] = dd;
+                a[k] = dd * sSc[oA + t * 4 + hc];
+                ga[k] = lm * dd;
+                // next token (the box holds Q + 1 tokens, zero-filled past the sequence end)
+                w[k] = ga[k] + (1.f - sSc[oL + (t + 1) * 4 + hc]) * sSc[(t + 1) * 4 + hc];
+            }
+        }
+        const float c0s = warp_inclusive_scan(a[0]);
+        const float tot0 = __shfl_sync(0xffffffffu, c0s, 31);
+        const float c1s = warp_inclusive_scan(a[1]) + tot0;
+        const float cum_end = __shfl_sync(0xffffffffu, (T - 1) < 32 ? c0s : c1s, (T - 1) & 31);
+        constexpr float kLog2e = 1.4426950408889634f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = lane + 32 * k;
+            const float cm = (t < T) ? (k ? c1s : c0s) : cum_end;
+            blk[F_CUM + t] = cm * kLog2e;   // log2-scaled: decays are exp2 of differences
+            blk[F_GAM + t] = ga[k];
+            blk[F_W + t] = w[k];
+            blk[F_ECUM + t] = __expf(cm);
+            blk[F_DW + t] = (t < T) ? __expf(cum_end - cm) * w[k] : 0.f;
+            blk[F_DT + t] = d[k];
+        }
+        if (lane == 0) blk[F_MISC] = __expf(cum_end);
+    };
 
     // ---------------- setup ----------------
     if (tid == 0) {
-        mbar_init(&bar_x, 1);
+        mbar_init(&bar_x[0], 1);
+        mbar_init(&bar_x[1], 1);
+        mbar_init(&bar_t[0], 1);
+        mbar_init(&bar_t[1], 1);
         mbar_init(&bar_m1, 1);
         mbar_init(&bar_m2, 1);
         fence_mbar_init();
         s_abort = 0;
+        if (nchunks > 0) {
+            issue_x(0);
+            issue_ts(0);
+        }
+        if (nchunks > 1) issue_ts(1);
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
+    if (tid == 0) {
+        s_issued[0] = nchunks > 0 ? 0 : -1;
+        s_issued[1] = nchunks > 1 ? 1 : (nchunks > 0 ? 0 : -1);
+        s_issued[2] = s_issued[3] = 0;
+    }
     for (int i = tid; i < R * kN; i += kTcThreads) {
         s_biasB[i] = p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f;
         s_biasC[i] = p.Cbias ? p.Cbias[hh * R * kN + i] : 0.f;
+        s_biasB2[i] = __float2bfloat16_rn(s_biasB[i]);
+        s_biasC2[i] = __float2bfloat16_rn(s_biasC[i]);
     }
     fence_before_sync();
     __syncthreads();
@@ -228,7 +382,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
             s_fold[r * kN + i + kHalf] = u1 * cs - u0 * sn;
         }
         __syncthreads();
-        const float f = (1.f - p.lam[sidx(0)]) * p.dt[sidx(0)];
+        const int64_t s0 = bb * p.L * p.H + hh;
+        const float f = (1.f - p.lam[s0]) * p.dt[s0];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             float acc = 0.f;
@@ -238,104 +393,100 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
         }
     }
 
-    const uint32_t aB = smem_u32(sm + OFF_B), aC = smem_u32(sm + OFF_C);
-    const uint32_t aX = smem_u32(sm + OFF_X), aXP = smem_u32(sm + OFF_XP);
-    const uint32_t aP = smem_u32(sm + OFF_P), aH = smem_u32(sm + OFF_H);
+    const uint32_t aB = smem_u32(sm + Cfg::OB), aC = smem_u32(sm + Cfg::OC);
+    const uint32_t aXP = smem_u32(sm + Cfg::XP);
+    const uint32_t aP = smem_u32(sm + Cfg::OP), aH = smem_u32(sm + Cfg::OH);
     const uint32_t id_s = idesc_bf16(64, 64, false, false);   // S  = C . B^T
     const uint32_t id_yo = idesc_bf16(64, 64, false, true);   // Yo = C . H
     const uint32_t id_dh = idesc_bf16(128, 64, true, true);   // dH = B^T . X'
     const uint32_t id_yd = idesc_bf16(64, 64, false, true);   // Yd = P . X
 
-    const int64_t nchunks = (L + Q - 1) / Q;
-    for (int64_t c = 0; c < nchunks; ++c) {
-        const int64_t c0 = c * Q;
-        const int T = static_cast<int>((L - c0) < Q ? (L - c0) : Q);
-        const uint32_t par = static_cast<uint32_t>(c & 1);
-
-        // ---- A. TMA of X, chunk scalars, norms ----
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_x, 64 * 128);
-            tma_load_5d(sm + OFF_X, &tmx, &bar_x, 0, 0, static_cast<int>(hh), static_cast<int>(c0),
-                        static_cast<int>(bb));
-        }
-        __syncwarp();
-        if (warp == 0) {
-            // token t = lane (+32): a = dt*A, inclusive scan -> cum; gamma, w
-            float a[2], d[2], ga[2], w[2];
+    // raw B / C rows of one chunk for this lane (issued a chunk ahead)
+    RawV<PPL> rb0[TPL][R], rb1[TPL][R], rc0[TPL][R], rc1[TPL][R];
+    float2 rsv[TPL][R];
+    auto load_raw = [&](int c) {
+        const int c0 = c * Q;
+        const int T = (L - c0) < Q ? (L - c0) : Q;
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int t = lane + 32 * k;
-                a[k] = d[k] = ga[k] = w[k] = 0.f;
+        for (int k = 0; k < TPL; ++k) {
+            const int t = tg * TPL + k;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
                 if (t < T) {
-                    const int64_t si = sidx(c0 + t);
-                    const float dd = p.dt[si], lm = p.lam[si];
-                    d[k] = dd;
-                    a[k] = dd * p.A[si];
-                    ga[k] = lm * dd;
-                    w[k] = ga[k];
-                    if (c0 + t + 1 < L) {
-                        const int64_t sn = sidx(c0 + t + 1);
-                        w[k] += (1.f - p.lam[sn]) * p.dt[sn];
-                    }
+                    const int row = (c0 + t) * G * R + r;
+                    const int off = (c0 + t) * tokB + r * kN + pp0;
+                    rb0[k][r] = ldg_raw<PPL>(Bu + off);
+                    rb1[k][r] = ldg_raw<PPL>(Bu + off + kHalf);
+                    rc0[k][r] = ldg_raw<PPL>(Cu + off);
+                    rc1[k][r] = ldg_raw<PPL>(Cu + off + kHalf);
+                    rsv[k][r] = rsu ? __ldg(rsu + row) : make_float2(1.f, 1.f);
                 }
             }
-            float c0s = warp_inclusive_scan(a[0]);
-            const float tot0 = __shfl_sync(0xffffffffu, c0s, 31);
-            float c1s = warp_inclusive_scan(a[1]) + tot0;
-            const float cum_end = __shfl_sync(0xffffffffu, (T - 1) < 32 ? c0s : c1s, (T - 1) & 31);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int t = lane + 32 * k;
-                if (t < 64) {
-                    const float cm = (t < T) ? (k ? c1s : c0s) : cum_end;
-                    sf[F_CUM + t] = cm;
-                    sf[F_GAM + t] = ga[k];
-                    sf[F_W + t] = w[k];
-                    sf[F_ECUM + t] = __expf(cm);
-                    sf[F_DW + t] = (t < T) ? __expf(cum_end - cm) * w[k] : 0.f;
-                    sf[F_DT + t] = d[k];
-                }
-            }
-            if (lane == 0) sf[F_MISC] = __expf(cum_end);
         }
-        {
-            // RMS scales: 2 threads per (row, tensor)
-            const int pr = tid >> 1, half = tid & 1;
-            const int tensor = pr >> 6, row = pr & 63;
-            const int t = row / R, r = row % R;
-            float ss = 0.f;
-            if (t < T) {
-                const __nv_bfloat16* src = (tensor ? Cg : Bg) +
-                    (((bb * L + c0 + t) * p.G + g) * R + r) * kN + half * 64;
+    };
+    // y of chunk c from the Yd / Yo accumulators (TMEM): y = Yd + e^{cum_t} Yo
+    auto epilogue = [&](int c) {
+        float yd[16], yo[16];
+        const uint32_t lanebase = (32u * q4) << 16;
+        tmem_ld_16x32bx2_x16(tmem + lanebase + T_YD + 16u * wh, yd);
+        tmem_ld_16x32bx2_x16(tmem + lanebase + T_YO + 16u * wh, yo);
+        const int trow = 16 * q4 + (lane & 15);
+        const int col0 = 16 * wh + ((lane >> 4) ? 32 : 0);
+        const int t = trow / R, r = trow % R;
+        const int c0 = c * Q;
+        const int T = (L - c0) < Q ? (L - c0) : Q;
+        const float e = sf[(c & 1) * F_BLK + F_ECUM + t];
+        tmem_wait_ld();
+        if (t < T) {
+            __nv_bfloat16* dst = yu + (c0 + t) * tokY + r * kP + col0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float v[8];
-                    ld_bf16<8>(src + 8 * j, v);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
-                }
+            for (int i = 0; i < 2; ++i) {
+                uint4 v;
+                v.x = pack_bf16(fmaf(e, yo[8 * i + 0], yd[8 * i + 0]), fmaf(e, yo[8 * i + 1], yd[8 * i + 1]));
+                v.y = pack_bf16(fmaf(e, yo[8 * i + 2], yd[8 * i + 2]), fmaf(e, yo[8 * i + 3], yd[8 * i + 3]));
+                v.z = pack_bf16(fmaf(e, yo[8 * i + 4], yd[8 * i + 4]), fmaf(e, yo[8 * i + 5], yd[8 * i + 5]));
+                v.w = pack_bf16(fmaf(e, yo[8 * i + 6], yd[8 * i + 6]), fmaf(e, yo[8 * i + 7], yd[8 * i + 7]));
+                *reinterpret_cast<uint4*>(dst + 8 * i) = v;
             }
-            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-            if (half == 0) sf[(tensor ? F_RSC : F_RSB) + row] = p.bc_norm ? rsqrtf(ss / kN + p.eps) : 1.f;
         }
-        __syncthreads();
+    };
 
-        // ---- B. cumulative angle (warp scan over tokens) and rotation into Bbar / Cbar ----
+    if (nchunks > 0) {
+        load_raw(0);
+        if (warp == 1) scalars(0);
+    }
+    __syncthreads();
+
+    for (int c = 0; c < nchunks && !s_abort; ++c) {
+        const int c0 = c * Q;
+        const int T = (L - c0) < Q ? (L - c0) : Q;
+        const int st = c & 1;
+        const uint32_t par = static_cast<uint32_t>(c & 1);
+        const uint8_t* sTh = sm + (st ? Cfg::TH1 : Cfg::TH0);
+        const float* blk = sf + st * F_BLK;
+
+        // ======== I1: rotation(c), H0 and X' operands, epilogue(c-1) ========
+        if (warp == 0) {
+            // X of chunk c+1 goes where X of chunk c-1 was: Yd(c-1) must have finished
+            if (elect_one()) {
+                if (c > 0 && !mbar_wait(&bar_m2, (c - 1) & 1)) s_abort = 1;
+                if (c + 1 < nchunks) {
+                    issue_x(c + 1);
+                    s_issued[0] = c + 1;
+                }
+            }
+            __syncwarp();
+        }
+        (void)mbar_try_wait(smem_u32(&bar_t[st]), (c >> 1) & 1);  // landed (warp 1 waited)
         {
             float inc[TPL][PPL];
 #pragma unroll
             for (int k = 0; k < TPL; ++k) {
                 const int t = tg * TPL + k;
-                float th[PPL];
-                if (t < T) {
-                    ld_bf16<PPL>(thg + sidx(c0 + t) * kHalf + pp0, th);
-                } else {
+                const RawV<PPL> th = lds_raw<PPL>(sTh + swz128(t, pp0));
+                const float dd = blk[F_DT + t];  // 0 past the end: no rotation there
 #pragma unroll
-                    for (int j = 0; j < PPL; ++j) th[j] = 0.f;
-                }
-                const float dd = sf[F_DT + t];
-#pragma unroll
-                for (int j = 0; j < PPL; ++j) inc[k][j] = dd * th[j] + (k ? inc[k - 1][j] : 0.f);
+                for (int j = 0; j < PPL; ++j) inc[k][j] = fmaf(dd, raw_f<PPL>(th, j), k ? inc[k - 1][j] : 0.f);
             }
             float incl[PPL], base[PPL];
 #pragma unroll
@@ -356,42 +507,49 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
 #pragma unroll
             for (int k = 0; k < TPL; ++k) {
                 const int t = tg * TPL + k;
-                float cs[PPL], sn[PPL];
+                uint32_t cw[PPL / 2], sw[PPL / 2];  // packed bf16 cos / sin of the lane's pairs
 #pragma unroll
-                for (int j = 0; j < PPL; ++j) sincos_2pi_reduced(base[j] + inc[k][j], &sn[j], &cs[j]);
+                for (int j = 0; j < PPL; j += 2) {
+                    float s0, c0v, s1, c1v;
+                    sincos_2pi_reduced(base[j] + inc[k][j], &s0, &c0v);
+                    sincos_2pi_reduced(base[j + 1] + inc[k][j + 1], &s1, &c1v);
+                    cw[j / 2] = pack_bf16(c0v, c1v);
+                    sw[j / 2] = pack_bf16(s0, s1);
+                }
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const int row = t * R + r;
-                    float ob0[PPL], ob1[PPL], oc0[PPL], oc1[PPL];
+                    RawV<PPL> ob0, ob1, oc0, oc1;
                     if (t < T) {
-                        const int64_t gi = (((bb * L + c0 + t) * p.G + g) * R + r) * kN + pp0;
-                        float b0[PPL], b1[PPL], cc0[PPL], cc1[PPL];
-                        ld_bf16<PPL>(Bg + gi, b0);
-                        ld_bf16<PPL>(Bg + gi + kHalf, b1);
-                        ld_bf16<PPL>(Cg + gi, cc0);
-                        ld_bf16<PPL>(Cg + gi + kHalf, cc1);
-                        const float rb = sf[F_RSB + row], rc = sf[F_RSC + row];
+                        const __nv_bfloat162 rb2 = __float2bfloat162_rn(rsv[k][r].x);
+                        const __nv_bfloat162 rc2 = __float2bfloat162_rn(rsv[k][r].y);
+                        const RawV<PPL> bB0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0));
+                        const RawV<PPL> bB1 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0 + kHalf));
+                        const RawV<PPL> bC0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasC2 + r * kN + pp0));
+                        const RawV<PPL> bC1 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasC2 + r * kN + pp0 + kHalf));
 #pragma unroll
-                        for (int j = 0; j < PPL; ++j) {
-                            const int n = pp0 + j;
-                            float u0 = fmaf(b0[j], rb, s_biasB[r * kN + n]);
-                            float u1 = fmaf(b1[j], rb, s_biasB[r * kN + n + kHalf]);
-                            ob0[j] = fmaf(u0, cs[j], u1 * sn[j]);
-                            ob1[j] = fmaf(u1, cs[j], -u0 * sn[j]);
-                            u0 = fmaf(cc0[j], rc, s_biasC[r * kN + n]);
-                            u1 = fmaf(cc1[j], rc, s_biasC[r * kN + n + kHalf]);
-                            oc0[j] = fmaf(u0, cs[j], u1 * sn[j]);
-                            oc1[j] = fmaf(u1, cs[j], -u0 * sn[j]);
+                        for (int q = 0; q < PPL / 2; ++q) {
+                            const __nv_bfloat162 c2 = as_bf2(cw[q]), s2 = as_bf2(sw[q]);
+                            // u = rs * raw + bias on both halves of each rotation pair, then
+                            // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
+                            __nv_bfloat162 u0 = __hfma2(as_bf2(rb0[k][r].w[q]), rb2, as_bf2(bB0.w[q]));
+                            __nv_bfloat162 u1 = __hfma2(as_bf2(rb1[k][r].w[q]), rb2, as_bf2(bB1.w[q]));
+                            ob0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
+                            ob1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
+                            u0 = __hfma2(as_bf2(rc0[k][r].w[q]), rc2, as_bf2(bC0.w[q]));
+                            u1 = __hfma2(as_bf2(rc1[k][r].w[q]), rc2, as_bf2(bC1.w[q]));
+                            oc0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
+                            oc1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < PPL; ++j) ob0[j] = ob1[j] = oc0[j] = oc1[j] = 0.f;
+                        for (int q = 0; q < PPL / 2; ++q) ob0.w[q] = ob1.w[q] = oc0.w[q] = oc1.w[q] = 0u;
                     }
                     const uint32_t o = swz128(row, pp0);
-                    st_bf16_smem<PPL>(sm + OFF_B + o, ob0);
-                    st_bf16_smem<PPL>(sm + OFF_B + 8192 + o, ob1);
-                    st_bf16_smem<PPL>(sm + OFF_C + o, oc0);
-                    st_bf16_smem<PPL>(sm + OFF_C + 8192 + o, oc1);
+                    sts_raw<PPL>(sm + Cfg::OB + o, ob0);
+                    sts_raw<PPL>(sm + Cfg::OB + 8192 + o, ob1);
+                    sts_raw<PPL>(sm + Cfg::OC + o, oc0);
+                    sts_raw<PPL>(sm + Cfg::OC + 8192 + o, oc1);
                 }
             }
         }
@@ -403,25 +561,30 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
             v.y = pack_bf16(hreg[8 * i + 2], hreg[8 * i + 3]);
             v.z = pack_bf16(hreg[8 * i + 4], hreg[8 * i + 5]);
             v.w = pack_bf16(hreg[8 * i + 6], hreg[8 * i + 7]);
-            *reinterpret_cast<uint4*>(sm + OFF_H + swz128(nrow, 32 * wh + 8 * i)) = v;
+            *reinterpret_cast<uint4*>(sm + Cfg::OH + swz128(nrow, 32 * wh + 8 * i)) = v;
         }
-
-        // ---- C. X' = diag(dw) X once X has landed ----
-        if (!mbar_wait(&bar_x, par)) {
-            if (lane == 0) s_abort = 1;
-        }
-        for (int e = tid; e < 64 * 8; e += kTcThreads) {
-            const int row = e >> 3, ch = e & 7;
-            const float sc = sf[F_DW + row / R];
-            const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
-            uint4 v = *reinterpret_cast<const uint4*>(sm + OFF_X + o);
-            uint32_t wds[4] = {v.x, v.y, v.z, v.w};
+        // X' = diag(dw) X
+        {
+            uint8_t* sX = sm + (st ? Cfg::X1 : Cfg::X0);
+            if (!mbar_wait(&bar_x[st], (c >> 1) & 1)) s_abort = 1;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                __nv_bfloat162 h2 = *reinterpret_cast<__nv_bfloat162*>(&wds[i]);
-                wds[i] = pack_bf16(__low2float(h2) * sc, __high2float(h2) * sc);
+            for (int i = 0; i < 2; ++i) {
+                const int e = tid + i * kTcThreads;
+                const int row = e >> 3, ch = e & 7;
+                const __nv_bfloat162 sc2 = __float2bfloat162_rn(blk[F_DW + row / R]);
+                const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
+                uint4 v = *reinterpret_cast<const uint4*>(sX + o);
+                v.x = as_u32(__hmul2(as_bf2(v.x), sc2));
+                v.y = as_u32(__hmul2(as_bf2(v.y), sc2));
+                v.z = as_u32(__hmul2(as_bf2(v.z), sc2));
+                v.w = as_u32(__hmul2(as_bf2(v.w), sc2));
+                *reinterpret_cast<uint4*>(sm + Cfg::XP + o) = v;
             }
-            *reinterpret_cast<uint4*>(sm + OFF_XP + o) = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+        }
+        if (c > 0) {
+            (void)mbar_wait(&bar_m2, (c - 1) & 1);  // thread 0 already saw it complete
+            fence_after_sync();
+            epilogue(c - 1);
         }
         fence_proxy_async();
         fence_before_sync();
@@ -429,56 +592,76 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
         fence_after_sync();
         if (s_abort) break;
 
-        // ---- D. S, Yo, dH ----
-        if (tid == 0) {
+        // ======== I2: S, dH, Yo on the tensor cores; next chunk's scalars meanwhile ========
+        if (warp == 0) {
+            if (elect_one()) {
+                // theta / scalar boxes of chunk c+2 reuse the buffers chunk c has finished with
+                if (c + 2 < nchunks) {
+                    issue_ts(c + 2);
+                    s_issued[1] = c + 2;
+                }
+                constexpr uint32_t hi = desc_hi_sw128(1024);
+                const uint32_t loC = desc_lo(aC, 16), loB = desc_lo(aB, 16);
+                const uint32_t loBt = desc_lo(aB, 8192), loXP = desc_lo(aXP, 8192);
+                const uint32_t loH = desc_lo(aH, 16384);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16(tmem + T_S, sdesc_kmajor(aC, k, 8192), sdesc_kmajor(aB, k, 8192), id_s, k > 0);
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + T_S, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
+                             desc_pack(loB + (kmajor_off(k, 8192) >> 4), hi), id_s, k > 0);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16(tmem + T_YO, sdesc_kmajor(aC, k, 8192), sdesc_mnmajor(aH, k, 16384), id_yo, k > 0);
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + T_DH, desc_pack(loBt + (mnmajor_off(k) >> 4), hi),
+                             desc_pack(loXP + (mnmajor_off(k) >> 4), hi), id_dh, k > 0);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_bf16(tmem + T_DH, sdesc_mnmajor(aB, k, 8192), sdesc_mnmajor(aXP, k, 8192), id_dh, k > 0);
-            mma_commit(smem_u32(&bar_m1));
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
+                             desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
+                mma_commit(smem_u32(&bar_m1));
+                s_issued[2] = c + 1;
+                if (!mbar_wait(&bar_m1, par)) s_abort = 1;
+            }
+            __syncwarp();
         }
-        __syncwarp();
-        if (!mbar_wait(&bar_m1, par)) {
-            if (lane == 0) s_abort = 1;
-        }
+        if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
+        fence_before_sync();
+        __syncthreads();
         fence_after_sync();
+        if (s_abort) break;
+        (void)mbar_try_wait(smem_u32(&bar_m1), par);  // completed: orders the accumulators
 
-        // ---- E. P = S o M  and  H1 = e^{cum_end} H0 + dH ----
+        // ======== I3: P = S o M, H1 = e^{cum_end} H0 + dH, next chunk's scalars ========
         {
             float s[16];
-            const uint32_t ta = tmem + ((32u * q4) << 16) + T_S + 16u * wh;
-            tmem_ld_16x32bx2_x16(ta, s);
-            tmem_wait_ld();
+            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, s);
             const int trow = 16 * q4 + (lane & 15);
             const int col0 = 16 * wh + ((lane >> 4) ? 32 : 0);
             const int t = trow / R;
-            const float cum_t = sf[F_CUM + t], gam_t = sf[F_GAM + t];
-            float pv[16];
+            constexpr int NT = 16 / R;          // tokens covered by the 16 columns
+            const int s0 = col0 / R;
+            float cs_[NT], ws_[NT];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int sidx2 = (col0 + j) / R;
-                float m = 0.f;
-                if (sidx2 < t) m = __expf(cum_t - sf[F_CUM + sidx2]) * sf[F_W + sidx2];
-                else if (sidx2 == t) m = gam_t;
-                pv[j] = s[j] * m;
+            for (int i = 0; i < NT; i += 2) {
+                const float2 a2 = *reinterpret_cast<const float2*>(blk + F_CUM + s0 + i);
+                const float2 w2 = *reinterpret_cast<const float2*>(blk + F_W + s0 + i);
+                cs_[i] = a2.x; cs_[i + 1] = a2.y; ws_[i] = w2.x; ws_[i + 1] = w2.y;
             }
+            const float cum_t = blk[F_CUM + t], gam_t = blk[F_GAM + t];
+            float m[NT];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                uint4 v;
-                v.x = pack_bf16(pv[8 * i + 0], pv[8 * i + 1]);
-                v.y = pack_bf16(pv[8 * i + 2], pv[8 * i + 3]);
-                v.z = pack_bf16(pv[8 * i + 4], pv[8 * i + 5]);
-                v.w = pack_bf16(pv[8 * i + 6], pv[8 * i + 7]);
-                *reinterpret_cast<uint4*>(sm + OFF_P + swz128(trow, col0 + 8 * i)) = v;
+            for (int i = 0; i < NT; ++i) {
+                const int sa = s0 + i;
+                m[i] = (sa < t) ? ex2_approx(fminf(cum_t - cs_[i], 0.f)) * ws_[i] : ((sa == t) ? gam_t : 0.f);
             }
+            tmem_wait_ld();
+            uint32_t pw[8];
+#pragma unroll
+            for (int j = 0; j < 16; j += 2)
+                pw[j / 2] = pack_bf16(s[j] * m[j / R], s[j + 1] * m[(j + 1) / R]);
+            *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
         {
-            const float eend = sf[F_MISC];
+            const float eend = blk[F_MISC];
             const uint32_t ta = tmem + ((32u * q4) << 16) + T_DH + 32u * wh;
             float d0[16], d1[16];
             tmem_ld_32x32b_x16(ta, d0);
@@ -490,56 +673,42 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
                 hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
             }
         }
+        if (c + 1 < nchunks) load_raw(c + 1);
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (s_abort) break;
 
-        // ---- F. Yd = P X ----
-        if (tid == 0) {
+        // ======== I4: Yd = P X (waited for at the next chunk's I1) ========
+        if (warp == 0) {
+            if (elect_one()) {
+                constexpr uint32_t hi = desc_hi_sw128(1024);
+                const uint32_t loP = desc_lo(aP, 16);
+                const uint32_t loX = desc_lo(smem_u32(sm + (st ? Cfg::X1 : Cfg::X0)), 8192);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                mma_bf16(tmem + T_YD, sdesc_kmajor(aP, k, 8192), sdesc_mnmajor(aX, k, 8192), id_yd, k > 0);
-            mma_commit(smem_u32(&bar_m2));
-        }
-        __syncwarp();
-        if (!mbar_wait(&bar_m2, par)) {
-            if (lane == 0) s_abort = 1;
-        }
-        fence_after_sync();
-
-        // ---- G. y = Yd + e^{cum_t} Yo ----
-        {
-            float yd[16], yo[16];
-            const uint32_t lanebase = (32u * q4) << 16;
-            tmem_ld_16x32bx2_x16(tmem + lanebase + T_YD + 16u * wh, yd);
-            tmem_ld_16x32bx2_x16(tmem + lanebase + T_YO + 16u * wh, yo);
-            tmem_wait_ld();
-            const int trow = 16 * q4 + (lane & 15);
-            const int col0 = 16 * wh + ((lane >> 4) ? 32 : 0);
-            const int t = trow / R, r = trow % R;
-            if (t < T) {
-                const float e = sf[F_ECUM + t];
-                __nv_bfloat16* dst = yg + (((bb * L + c0 + t) * p.H + hh) * R + r) * kP + col0;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    uint4 v;
-                    v.x = pack_bf16(fmaf(e, yo[8 * i + 0], yd[8 * i + 0]), fmaf(e, yo[8 * i + 1], yd[8 * i + 1]));
-                    v.y = pack_bf16(fmaf(e, yo[8 * i + 2], yd[8 * i + 2]), fmaf(e, yo[8 * i + 3], yd[8 * i + 3]));
-                    v.z = pack_bf16(fmaf(e, yo[8 * i + 4], yd[8 * i + 4]), fmaf(e, yo[8 * i + 5], yd[8 * i + 5]));
-                    v.w = pack_bf16(fmaf(e, yo[8 * i + 6], yd[8 * i + 6]), fmaf(e, yo[8 * i + 7], yd[8 * i + 7]));
-                    *reinterpret_cast<uint4*>(dst + 8 * i) = v;
-                }
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + T_YD, desc_pack(loP + (kmajor_off(k, 8192) >> 4), hi),
+                             desc_pack(loX + (mnmajor_off(k) >> 4), hi), id_yd, k > 0);
+                mma_commit(smem_u32(&bar_m2));
+                s_issued[3] = c + 1;
             }
+            __syncwarp();
         }
+    }
+    // ---- epilogue of the last chunk ----
+    if (nchunks > 0 && !s_abort) {
+        if (tid == 0 && !mbar_wait(&bar_m2, (nchunks - 1) & 1)) s_abort = 1;  // lane 0 of warp 0
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (s_abort) break;
+        if (!s_abort) {
+            (void)mbar_try_wait(smem_u32(&bar_m2), (nchunks - 1) & 1);
+            epilogue(nchunks - 1);
+        }
     }
 
     // ---------------- final state ----------------
+    __syncthreads();
     if (!s_abort) {
         if (p.h1) {
             float4* dst = reinterpret_cast<float4*>(p.h1 + (u * kN + nrow) * kP + 32 * wh);
@@ -554,17 +723,26 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ CUtensorMap tmx) {
         if (L > 0) {
             if (p.prevB1) {
                 __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevB1) + u * R * kN;
-                const __nv_bfloat16* src = Bg + ((bb * L + L - 1) * p.G + g) * R * kN;
+                const __nv_bfloat16* src = Bu + (L - 1) * tokB;
                 for (int e = tid; e < R * kN; e += kTcThreads) dst[e] = src[e];
             }
             if (p.prevx1) {
                 __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevx1) + u * R * kP;
-                const __nv_bfloat16* src = xg + ((bb * L + L - 1) * p.H + hh) * R * kP;
+                const __nv_bfloat16* src = xu + (L - 1) * tokY;
                 for (int e = tid; e < R * kP; e += kTcThreads) dst[e] = src[e];
             }
         }
     } else if (tid == 0) {
-        set_status(p.status, 1);
+        if (p.status) atomicExch(p.status, 1);
+        // A wait gave up: let this CTA's own TMA copies and MMAs finish (bounded) before the
+        // shared memory and TMEM they target are released.
+        constexpr long long kDrain = 200000000LL;
+        for (int k = s_issued[0] - 1; k <= s_issued[0]; ++k)
+            if (k >= 0) (void)mbar_wait(&bar_x[k & 1], (k >> 1) & 1, kDrain);
+        for (int k = s_issued[1] - 1; k <= s_issued[1]; ++k)
+            if (k >= 0) (void)mbar_wait(&bar_t[k & 1], (k >> 1) & 1, kDrain);
+        if (s_issued[2] > 0) (void)mbar_wait(&bar_m1, (s_issued[2] - 1) & 1, kDrain);
+        if (s_issued[3] > 0) (void)mbar_wait(&bar_m2, (s_issued[3] - 1) & 1, kDrain);
     }
     fence_before_sync();
     __syncthreads();
@@ -584,50 +762,87 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+            const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+            CUtensorMapSwizzle swz) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return enc(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool tc_scan_supported(const ScanParams& p, bool bf16) {
+    // 32-bit element offsets inside one sequence: L * G * R * N and L * H * R * P < 2^31
+    const int64_t lim = 0x7fffffffLL;
     return bf16 && p.N == kN && p.P == kP && p.Q * p.R == 64 &&
-           (p.R == 1 || p.R == 2 || p.R == 4 || p.R == 8) && p.L <= 0x7fffffffLL;
+           (p.R == 1 || p.R == 2 || p.R == 4 || p.R == 8) && p.H % 4 == 0 &&
+           p.L * p.G * p.R * kN < lim && p.L * p.H * p.R * kP < lim && p.b <= lim;
+}
+
+size_t tc_scan_workspace_bytes(const ScanParams& p) {
+    return p.bc_norm ? static_cast<size_t>(p.b * p.L * p.G * p.R) * sizeof(float2) : 0;
 }
 
 template <int R>
-static cudaError_t launch_tc_t(const ScanParams& p, cudaStream_t s) {
-    auto enc = get_encode();
-    if (!enc) return cudaErrorNotSupported;
-    // x viewed as 5D [b][L][H][R][P] (innermost first for the map), box (P, R, 1, Q, 1)
-    CUtensorMap map;
-    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(kP), static_cast<cuuint64_t>(R),
-                                static_cast<cuuint64_t>(p.H), static_cast<cuuint64_t>(p.L),
-                                static_cast<cuuint64_t>(p.b)};
-    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(kP) * 2,
-                                   static_cast<cuuint64_t>(R * kP) * 2,
-                                   static_cast<cuuint64_t>(p.H * R * kP) * 2,
-                                   static_cast<cuuint64_t>(p.L * p.H * R * kP) * 2};
-    const cuuint32_t box[5] = {static_cast<cuuint32_t>(kP), static_cast<cuuint32_t>(R), 1u,
-                               static_cast<cuuint32_t>(64 / R), 1u};
-    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(p.x), dims,
-                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const uint32_t smem = tc_smem_bytes(R);
+static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, cudaStream_t s) {
+    constexpr int Q = 64 / R;
+    TcMaps maps;
+    const cuuint64_t H = p.H, Lq = p.L, b = p.b;
+    {   // x [b][L][H][R][P], box (P, R, 1, Q, 1)
+        const cuuint64_t dims[5] = {kP, static_cast<cuuint64_t>(R), H, Lq, b};
+        const cuuint64_t str[4] = {kP * 2, R * kP * 2, H * R * kP * 2, Lq * H * R * kP * 2};
+        const cuuint32_t box[5] = {kP, static_cast<cuuint32_t>(R), 1, Q, 1};
+        if (!encode(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, p.x, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+    }
+    {   // theta [b][L][H][N/2], box (64, 1, Q, 1)
+        const cuuint64_t dims[4] = {kHalf, H, Lq, b};
+        const cuuint64_t str[3] = {kHalf * 2, H * kHalf * 2, Lq * H * kHalf * 2};
+        const cuuint32_t box[4] = {kHalf, 1, Q, 1};
+        if (!encode(&maps.theta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.theta, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
+    }
+    {   // dt, A, lam [b][L][H] fp32, box (4 heads, Q + 1 tokens, 1)
+        const cuuint64_t dims[3] = {H, Lq, b};
+        const cuuint64_t str[2] = {H * 4, Lq * H * 4};
+        const cuuint32_t box[3] = {4, Q + 1, 1};
+        if (!encode(&maps.dt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.dt, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode(&maps.A, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.A, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+            !encode(&maps.lam, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.lam, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
+    if (rs) {
+        const int64_t rows = p.b * p.L * p.G * R;
+        rms_scale_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
+            p.eps, rs);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    const uint32_t smem = tc_smem_bytes<R>();
     auto k = scan_tc_kernel<R>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k<<<static_cast<unsigned>(p.b * p.H), kTcThreads, smem, s>>>(p, map);
+    k<<<static_cast<unsigned>(p.b * p.H), kTcThreads, smem, s>>>(p, maps, rs);
     return cudaGetLastError();
 }
 
-cudaError_t launch_scan_tc(const ScanParams& p, cudaStream_t s) {
+cudaError_t launch_scan_tc(const ScanParams& p, void* rs_ws, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
+    float2* rs = p.bc_norm ? static_cast<float2*>(rs_ws) : nullptr;
     switch (p.R) {
-        case 1: return launch_tc_t<1>(p, s);
-        case 2: return launch_tc_t<2>(p, s);
-        case 4: return launch_tc_t<4>(p, s);
-        case 8: return launch_tc_t<8>(p, s);
+        case 1: return launch_tc_t<1>(p, rs, s);
+        case 2: return launch_tc_t<2>(p, rs, s);
+        case 4: return launch_tc_t<4>(p, rs, s);
+        case 8: return launch_tc_t<8>(p, rs, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -57,6 +57,37 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// The same descriptors assembled from 32-bit halves: lo = (address >> 4) | (LBO >> 4) << 16,
+// hi = (SBO >> 4) | version | swizzle. With a fixed base, one K step is one add to lo (the
+// 14-bit address field cannot carry: shared memory is below 256 KB).
+__device__ __forceinline__ uint64_t desc_pack(uint32_t lo, uint32_t hi) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+    return d;
+}
+__host__ __device__ constexpr uint32_t desc_hi_sw128(uint32_t sbo_bytes) {
+    return (sbo_bytes >> 4) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+    return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+// Byte offset of K step k inside a K-major tile (slabs of 64 K-columns, slab_bytes apart) and
+// inside an MN-major tile (16 rows of 128 bytes per step).
+__host__ __device__ constexpr uint32_t kmajor_off(int k, uint32_t slab_bytes) {
+    return static_cast<uint32_t>(k >> 2) * slab_bytes + static_cast<uint32_t>(k & 3) * 32u;
+}
+__host__ __device__ constexpr uint32_t mnmajor_off(int k) { return static_cast<uint32_t>(k) * 2048u; }
+
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
@@ -152,8 +183,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// Like mbar_try_wait, but the thread may be suspended (not spinning) for up to hint_ns
+// nanoseconds while the phase is still pending.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
 // Waits for the phase with the given parity to complete, at most ~max_cycles SM clocks.
-// Returns false on timeout.
+// Returns false on timeout. Callers keep the number of waiting threads small (one lane).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           long long max_cycles = 2000000000LL) {
     const uint32_t a = smem_u32(bar);
@@ -183,6 +225,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, uint64_t* bar, int c0,
+                                            int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
 __device__ __forceinline__ void tma_load_5d(void* dst, const void* tmap, uint64_t* bar, int c0,
                                             int c1, int c2, int c3, int c4) {
     asm volatile(
