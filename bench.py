@@ -24,6 +24,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roofline"
+# DRAM bytes (read + write) of one scan launch on this workload from the ncu capture
+# summarised in profiles/scan_tc_siso_prefill_b4_L2048.md; None once the kernel changes.
+SCAN_TRAFFIC_BYTES = 188.3e6
 WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"
 
 
@@ -226,7 +229,7 @@ def run_ours(args):
                    "chunk": d.chunk, "parallelism": f"independent sequences x{world}",
                    "l2": "two alternating input sets of 144 MB each (> 126 MB L2), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm, "traffic": SCAN_TRAFFIC_BYTES,
                      "bytes_per_launch": byts, "launch_ms": launch_ms,
                      "peak_source": peak_kind},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
