@@ -123,6 +123,29 @@ M3_API m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const 
  * header (blocking) so the workspace can be reused. */
 M3_API m3_status m3_scan_check(void* workspace);
 
+/* m3_scan_fwd for callers that cannot allocate device memory when they run the scan: a
+ * serving runtime that fixes all of its device memory before it starts and allows no
+ * allocation afterwards, code running in a step whose memory was planned in advance, or an
+ * embedding with no allocator to hand out. It is m3_scan_fwd without the workspace argument;
+ * the pages define no counterpart, it exists only for those callers.
+ *   Scratch: a 1 MiB array that is part of the library (a __device__ variable, so every GPU
+ *   that loads the library keeps its own copy until the process exits). The call itself
+ *   allocates and frees nothing; the caller still passes inputs, state and y as above.
+ *   First call on a device: looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current and caches it, so make the first call on each device before any
+ *   stream capture.
+ *   Sharing: all calls on a device use the same array, and it keeps what the last call left
+ *   (each call clears the status bytes it needs at zero first). Calls whose work can overlap
+ *   on the GPU (different streams, or different host threads) race on the array: serialise
+ *   them, or use m3_scan_fwd with one workspace each.
+ *   Limit: dims whose m3_scan_workspace_bytes exceeds 1 MiB return M3_ERR_UNSUPPORTED
+ *   (with BC normalisation on, the tensor-core path needs 8 bytes per batch * seqlen *
+ *   ngroups * rank row). A device-side wait that gives up cannot be reported here; use
+ *   m3_scan_fwd and m3_scan_check when that matters. */
+M3_API m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const m3_inputs* in,
+                                     const m3_state* init, const m3_state* final_state,
+                                     void* y, void* stream);
+
 /* Static description of a status code. */
 M3_API const char* m3_status_str(m3_status s);
 

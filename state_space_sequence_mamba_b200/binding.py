@@ -44,7 +44,7 @@ class StateC(ctypes.Structure):
 
 # Symbols include/m3.h declares (checked by the CPU test suite).
 EXPORTS = ("m3_scan_workspace_bytes", "m3_scan_fwd", "m3_decode_step", "m3_scan_check",
-           "m3_status_str", "m3_last_error")
+           "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc")
 
 _lib = None
 
@@ -73,6 +73,9 @@ def load_library(path: str = LIB_PATH):
     lib.m3_status_str.restype = ctypes.c_char_p
     lib.m3_last_error.argtypes = []
     lib.m3_last_error.restype = ctypes.c_char_p
+    lib.m3_scan_fwd_noalloc.argtypes = [P(Dims), P(Inputs), P(StateC), P(StateC),
+                                        ctypes.c_void_p, ctypes.c_void_p]
+    lib.m3_scan_fwd_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 

@@ -127,6 +127,9 @@ m3_status empty_sequence(const m3_dims* d, const m3_state* init, const m3_state*
 }
 
 }  // namespace
+
+m3_status set_error(m3_status s, const char* msg) { return fail(s, "%s", msg); }
+
 }  // namespace m3
 
 using namespace m3;

@@ -48,6 +48,8 @@ bool tc_scan_supported(const ScanParams& p, bool bf16);
 // Workspace bytes the tensor-core scan needs beyond the status header.
 size_t tc_scan_workspace_bytes(const ScanParams& p);
 cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s);
+// Records msg as this thread's m3_last_error() text and returns s.
+m3_status set_error(m3_status s, const char* msg);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 
