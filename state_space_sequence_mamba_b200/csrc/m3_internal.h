@@ -50,6 +50,10 @@ size_t tc_scan_workspace_bytes(const ScanParams& p);
 cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s);
 // Records msg as this thread's m3_last_error() text and returns s.
 m3_status set_error(m3_status s, const char* msg);
+// Persistent decode with bulk asynchronous copies (bf16, N * P <= 8192).
+bool decode_bulk_supported(const ScanParams& p, bool bf16);
+size_t decode_bulk_smem_bytes(const ScanParams& p);
+cudaError_t launch_decode_bulk(const ScanParams& p, cudaStream_t s);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 

@@ -62,13 +62,16 @@ struct TcCfg {
     static constexpr uint32_t SC_SLOT = round_up(SC_ONE, 128);      // 128-byte aligned slots
     static constexpr uint32_t SC_BYTES = 3 * SC_SLOT;
     static constexpr uint32_t SC0 = TH1 + TH_BYTES, SC1 = SC0 + SC_BYTES;  // dt, A, lam boxes
-    static constexpr uint32_t OF = SC1 + SC_BYTES;                  // fp32 scratch
+    static constexpr uint32_t ORS = SC1 + SC_BYTES;                 // RMS scales, 64 float2
+    static constexpr uint32_t OF = ORS + 512;                       // fp32 scratch
+    static constexpr uint32_t BC_TX = 4 * 8192;                     // raw B, C: two slabs each
     static constexpr uint32_t X_TX = 8192;                          // bytes of one X box
     static constexpr uint32_t TS_TX = Q * 128 + 3 * SC_ONE;         // theta + scalar boxes
 };
 // fp32 scratch (float offsets)
 constexpr int F_CUM = 0, F_GAM = 64, F_W = 128, F_ECUM = 192, F_DW = 256, F_DT = 320,
-              F_MISC = 384, F_BLK = 448;   // one block of chunk scalars; two blocks (by parity)
+              F_MISC = 384, F_EROW = 448, F_ECOL = 512,  // tile factors: [64], [4][64]
+              F_BLK = 768;   // one block of chunk scalars; two blocks (by parity)
 constexpr int F_BIAS = 2 * F_BLK;          // then bias_B [R][128], bias_C [R][128], fold scratch
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
@@ -78,17 +81,15 @@ __host__ __device__ constexpr uint32_t tc_smem_bytes() {
     return TcCfg<R>::OF + 4u * (F_BIAS + 2 * R * kN + R * kN + R * kP) + 2u * 2 * R * kN + 1024u;
 }
 
-// Cody-Waite reduction of x by 2*pi (Cody & Waite, "Software Manual for the Elementary
-// Functions", 1980) into [-pi, pi], then the hardware sine/cosine. Absolute error ~1e-6 for
-// |x| < 1e4, far below the bf16 rounding of the rotated operands.
-__device__ __forceinline__ void sincos_2pi_reduced(float x, float* s, float* c) {
+// x reduced by a whole number of turns into [-pi, pi]: Cody-Waite reduction with 2*pi split
+// into an exactly representable head and a tail (Cody & Waite, "Software Manual for the
+// Elementary Functions", 1980). Absolute error ~1e-6 for |x| < 1e4.
+__device__ __forceinline__ float reduce_2pi(float x) {
     constexpr float kInv2Pi = 0.15915494309189535f;
     constexpr float k2PiHi = 6.28125f;                  // exactly representable head of 2*pi
     constexpr float k2PiLo = 1.9353071795864769e-3f;    // 2*pi - 6.28125
     const float k = rintf(x * kInv2Pi);
-    float r = fmaf(-k, k2PiHi, x);
-    r = fmaf(-k, k2PiLo, r);
-    __sincosf(r, s, c);
+    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
 }
 
 // 2^x by the hardware approximation (relative error ~2^-22), x <= 0 here.
@@ -175,17 +176,22 @@ __device__ __forceinline__ uint32_t as_u32(__nv_bfloat162 v) {
 }
 
 struct TcMaps {
-    CUtensorMap x, theta, dt, A, lam;
+    CUtensorMap x, theta, dt, A, lam, B, C;
 };
 
-// RMS scale of every B and C row (shared by all heads): one warp per row of N = 128.
+// RMS scale of every B and C row (shared by all heads): one warp per row of N = 128. Rows
+// (b, l, g, r) are written to out[((b * G + g) * Lpad + l) * R + r] so that the rows of one
+// chunk of one group are contiguous (one bulk copy per chunk); Lpad rounds L up to chunks.
 __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __restrict__ B,
                                                         const __nv_bfloat16* __restrict__ C,
-                                                        int64_t rows, float eps,
-                                                        float2* __restrict__ out) {
+                                                        int64_t rows, int64_t L, int64_t G,
+                                                        int64_t R, int64_t Lpad, float eps,
+                                                        uint2* __restrict__ out) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
+    const int64_t r = row % R, g = (row / R) % G, l = (row / (R * G)) % L, b = row / (R * G * L);
+    const int64_t orow = ((b * G + g) * Lpad + l) * R + r;
     const uint2 ub = __ldg(reinterpret_cast<const uint2*>(B + row * kN) + lane);
     const uint2 uc = __ldg(reinterpret_cast<const uint2*>(C + row * kN) + lane);
     float sb = 0.f, sc = 0.f;
@@ -199,12 +205,17 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
     }
     sb = warp_sum(sb);
     sc = warp_sum(sc);
-    if (lane == 0) out[row] = make_float2(rsqrtf(sb / kN + eps), rsqrtf(sc / kN + eps));
+    if (lane == 0) {  // stored as packed bf16 pairs (rs, rs), the operand form of the rotation
+        const float rb = rsqrtf(sb / kN + eps), rc = rsqrtf(sc / kN + eps);
+        const __nv_bfloat162 vb = __floats2bfloat162_rn(rb, rb), vc = __floats2bfloat162_rn(rc, rc);
+        out[orow] = make_uint2(*reinterpret_cast<const uint32_t*>(&vb),
+                               *reinterpret_cast<const uint32_t*>(&vc));
+    }
 }
 
 template <int R>
 __global__ void __launch_bounds__(kTcThreads, 2)
-scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const float2* __restrict__ rsrow) {
+scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow) {
     using Cfg = TcCfg<R>;
     constexpr int Q = Cfg::Q, TPL = Cfg::TPL, PPL = Cfg::PPL, LPT = Cfg::LPT;
 
@@ -218,11 +229,11 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     float* s_foldx = s_fold + R * kN;     // [R][64]  its x
     __nv_bfloat16* s_biasB2 = reinterpret_cast<__nv_bfloat16*>(s_foldx + R * kP);  // [R][128] bf16
     __nv_bfloat16* s_biasC2 = s_biasB2 + R * kN;
-    __shared__ uint64_t bar_x[2], bar_t[2], bar_m1, bar_m2;
+    __shared__ uint64_t bar_x[2], bar_t[2], bar_bc, bar_m1, bar_m2;
     __shared__ uint32_t tslot;
     __shared__ int s_abort;
     // async work thread 0 has started (for draining it if a wait gives up)
-    __shared__ int s_issued[4];  // last X / TS chunk issued, MMA groups committed (m1, m2)
+    __shared__ int s_issued[5];  // last X / TS chunk issued, MMA groups (m1, m2), B/C loads
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3, wh = warp >> 2;  // TMEM subpartition, column half
@@ -234,7 +245,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     // Per-unit base pointers; offsets below fit in 32 bits (checked on the host).
     const __nv_bfloat16* Bu = static_cast<const __nv_bfloat16*>(p.B) + (bb * p.L * G + g) * R * kN;
     const __nv_bfloat16* Cu = static_cast<const __nv_bfloat16*>(p.C) + (bb * p.L * G + g) * R * kN;
-    const float2* rsu = rsrow ? rsrow + (bb * p.L * G + g) * R : nullptr;
+    const int Lpad = ((L + Q - 1) / Q) * Q;
+    const uint2* rsu = rsrow ? rsrow + (bb * G + g) * static_cast<int64_t>(Lpad) * R : nullptr;
     const __nv_bfloat16* xu = static_cast<const __nv_bfloat16*>(p.x) + (bb * p.L * H + hh) * R * kP;
     __nv_bfloat16* yu = static_cast<__nv_bfloat16*>(p.y) + (bb * p.L * H + hh) * R * kP;
     const int tokB = G * R * kN, tokY = H * R * kP;  // element stride of one token
@@ -299,6 +311,30 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
             blk[F_DT + t] = d[k];
         }
         if (lane == 0) blk[F_MISC] = __expf(cum_end);
+        // Tile factors of the decay mask. Rows come in blocks of 16 (16 / R tokens); with t0 the
+        // first token of t's block, e^{cum_t - cum_s} = 2^(c2_t - c2_t0) * 2^(c2_t0 - c2_s) for
+        // s < t0, both factors <= 1 (cum decreases).
+        constexpr int TB = 16 / R;  // tokens per row block
+        float c2v[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = lane + 32 * k;
+            c2v[k] = ((t < T) ? (k ? c1s : c0s) : cum_end) * kLog2e;
+        }
+        float c2blk[4];
+#pragma unroll
+        for (int qb = 0; qb < 4; ++qb) {
+            const int tq = qb * TB;
+            c2blk[qb] = __shfl_sync(0xffffffffu, tq < 32 ? c2v[0] : c2v[1], tq & 31);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = lane + 32 * k;
+            blk[F_EROW + t] = ex2_approx(c2v[k] - c2blk[t / TB < 4 ? t / TB : 3]);
+#pragma unroll
+            for (int qb = 1; qb < 4; ++qb)
+                blk[F_ECOL + qb * 64 + t] = (t < qb * TB) ? ex2_approx(c2blk[qb] - c2v[k]) * w[k] : 0.f;
+        }
     };
 
     // ---------------- setup ----------------
@@ -307,6 +343,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
         mbar_init(&bar_x[1], 1);
         mbar_init(&bar_t[0], 1);
         mbar_init(&bar_t[1], 1);
+        mbar_init(&bar_bc, 1);
         mbar_init(&bar_m1, 1);
         mbar_init(&bar_m2, 1);
         fence_mbar_init();
@@ -321,7 +358,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     if (tid == 0) {
         s_issued[0] = nchunks > 0 ? 0 : -1;
         s_issued[1] = nchunks > 1 ? 1 : (nchunks > 0 ? 0 : -1);
-        s_issued[2] = s_issued[3] = 0;
+        s_issued[2] = s_issued[3] = s_issued[4] = 0;
     }
     for (int i = tid; i < R * kN; i += kTcThreads) {
         s_biasB[i] = p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f;
@@ -352,9 +389,15 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     // rotation lane mapping: warp -> 8 pairs, lane -> (token group, pair subgroup)
     const int tg = lane / LPT, ps = lane % LPT;
     const int pp0 = 8 * warp + ps * PPL;  // first pair of this lane
-    float carry[PPL];
+    // cumulative angle per pair: carry (as stored in the state) and the same reduced into
+    // [-pi, pi] once per chunk (Cody & Waite's two-constant reduction, "Software Manual for
+    // the Elementary Functions", 1980), so that the per-token angles stay small
+    float carry[PPL], carry_r[PPL];
 #pragma unroll
-    for (int j = 0; j < PPL; ++j) carry[j] = p.phi0 ? p.phi0[u * kHalf + pp0 + j] : 0.f;
+    for (int j = 0; j < PPL; ++j) {
+        carry[j] = p.phi0 ? p.phi0[u * kHalf + pp0 + j] : 0.f;
+        carry_r[j] = reduce_2pi(carry[j]);
+    }
 
     // ---- fold the stored previous token into the primed state ----
     if (p.h0 && L > 0) {
@@ -401,28 +444,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     const uint32_t id_dh = idesc_bf16(128, 64, true, true);   // dH = B^T . X'
     const uint32_t id_yd = idesc_bf16(64, 64, false, true);   // Yd = P . X
 
-    // raw B / C rows of one chunk for this lane (issued a chunk ahead)
-    RawV<PPL> rb0[TPL][R], rb1[TPL][R], rc0[TPL][R], rc1[TPL][R];
-    float2 rsv[TPL][R];
-    auto load_raw = [&](int c) {
-        const int c0 = c * Q;
-        const int T = (L - c0) < Q ? (L - c0) : Q;
-#pragma unroll
-        for (int k = 0; k < TPL; ++k) {
-            const int t = tg * TPL + k;
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                if (t < T) {
-                    const int row = (c0 + t) * G * R + r;
-                    const int off = (c0 + t) * tokB + r * kN + pp0;
-                    rb0[k][r] = ldg_raw<PPL>(Bu + off);
-                    rb1[k][r] = ldg_raw<PPL>(Bu + off + kHalf);
-                    rc0[k][r] = ldg_raw<PPL>(Cu + off);
-                    rc1[k][r] = ldg_raw<PPL>(Cu + off + kHalf);
-                    rsv[k][r] = rsu ? __ldg(rsu + row) : make_float2(1.f, 1.f);
-                }
-            }
-        }
+    // Raw B and C rows of chunk c straight into the Bbar / Cbar operand buffers (two 64-column
+    // slabs each, swizzled as the MMA reads them; the rotation then transforms them in place),
+    // plus the chunk's RMS scales. Only when those buffers are free (their MMAs have finished).
+    uint2* s_rs = reinterpret_cast<uint2*>(sm + Cfg::ORS);
+    auto issue_bc = [&](int c) {
+        const int ic0 = c * Q, ig = static_cast<int>(g), ib = static_cast<int>(bb);
+        mbar_arrive_expect_tx(&bar_bc, Cfg::BC_TX + (rsu ? 512u : 0u));
+        tma_load_5d(sm + Cfg::OB, &maps.B, &bar_bc, 0, 0, ig, ic0, ib);
+        tma_load_5d(sm + Cfg::OB + 8192, &maps.B, &bar_bc, kHalf, 0, ig, ic0, ib);
+        tma_load_5d(sm + Cfg::OC, &maps.C, &bar_bc, 0, 0, ig, ic0, ib);
+        tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_bc, kHalf, 0, ig, ic0, ib);
+        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(ic0) * R, 512u, &bar_bc);
     };
     // y of chunk c from the Yd / Yo accumulators (TMEM): y = Yd + e^{cum_t} Yo
     auto epilogue = [&](int c) {
@@ -452,7 +485,10 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
     };
 
     if (nchunks > 0) {
-        load_raw(0);
+        if (tid == 0) {
+            issue_bc(0);
+            s_issued[4] = 1;
+        }
         if (warp == 1) scalars(0);
     }
     __syncthreads();
@@ -477,7 +513,15 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
             }
             __syncwarp();
         }
+        // work that needs neither this chunk's B / C nor theta first: y of the previous
+        // chunk and the H0 operand, while the B / C tiles finish landing
+        if (c > 0) {
+            (void)mbar_wait(&bar_m2, (c - 1) & 1);  // thread 0 already saw it complete
+            fence_after_sync();
+            epilogue(c - 1);
+        }
         (void)mbar_try_wait(smem_u32(&bar_t[st]), (c >> 1) & 1);  // landed (warp 1 waited)
+        if (!mbar_wait(&bar_bc, par)) s_abort = 1;  // raw B / C of this chunk
         {
             float inc[TPL][PPL];
 #pragma unroll
@@ -501,8 +545,10 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
             }
 #pragma unroll
             for (int j = 0; j < PPL; ++j) {
-                base[j] = carry[j] + incl[j] - inc[TPL - 1][j];
-                carry[j] += __shfl_sync(0xffffffffu, incl[j], 32 - LPT + ps);
+                base[j] = carry_r[j] + incl[j] - inc[TPL - 1][j];
+                const float tot = __shfl_sync(0xffffffffu, incl[j], 32 - LPT + ps);
+                carry[j] += tot;
+                carry_r[j] = reduce_2pi(carry_r[j] + tot);
             }
 #pragma unroll
             for (int k = 0; k < TPL; ++k) {
@@ -511,18 +557,23 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
 #pragma unroll
                 for (int j = 0; j < PPL; j += 2) {
                     float s0, c0v, s1, c1v;
-                    sincos_2pi_reduced(base[j] + inc[k][j], &s0, &c0v);
-                    sincos_2pi_reduced(base[j + 1] + inc[k][j + 1], &s1, &c1v);
+                    __sincosf(base[j] + inc[k][j], &s0, &c0v);
+                    __sincosf(base[j + 1] + inc[k][j + 1], &s1, &c1v);
                     cw[j / 2] = pack_bf16(c0v, c1v);
                     sw[j / 2] = pack_bf16(s0, s1);
                 }
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const int row = t * R + r;
+                    const uint32_t o = swz128(row, pp0);
                     RawV<PPL> ob0, ob1, oc0, oc1;
                     if (t < T) {
-                        const __nv_bfloat162 rb2 = __float2bfloat162_rn(rsv[k][r].x);
-                        const __nv_bfloat162 rc2 = __float2bfloat162_rn(rsv[k][r].y);
+                        const RawV<PPL> rb0 = lds_raw<PPL>(sm + Cfg::OB + o);
+                        const RawV<PPL> rb1 = lds_raw<PPL>(sm + Cfg::OB + 8192 + o);
+                        const RawV<PPL> rc0 = lds_raw<PPL>(sm + Cfg::OC + o);
+                        const RawV<PPL> rc1 = lds_raw<PPL>(sm + Cfg::OC + 8192 + o);
+                        const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
+                        const __nv_bfloat162 rb2 = as_bf2(rsv.x), rc2 = as_bf2(rsv.y);
                         const RawV<PPL> bB0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0));
                         const RawV<PPL> bB1 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0 + kHalf));
                         const RawV<PPL> bC0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasC2 + r * kN + pp0));
@@ -532,12 +583,12 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
                             const __nv_bfloat162 c2 = as_bf2(cw[q]), s2 = as_bf2(sw[q]);
                             // u = rs * raw + bias on both halves of each rotation pair, then
                             // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
-                            __nv_bfloat162 u0 = __hfma2(as_bf2(rb0[k][r].w[q]), rb2, as_bf2(bB0.w[q]));
-                            __nv_bfloat162 u1 = __hfma2(as_bf2(rb1[k][r].w[q]), rb2, as_bf2(bB1.w[q]));
+                            __nv_bfloat162 u0 = __hfma2(as_bf2(rb0.w[q]), rb2, as_bf2(bB0.w[q]));
+                            __nv_bfloat162 u1 = __hfma2(as_bf2(rb1.w[q]), rb2, as_bf2(bB1.w[q]));
                             ob0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
                             ob1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
-                            u0 = __hfma2(as_bf2(rc0[k][r].w[q]), rc2, as_bf2(bC0.w[q]));
-                            u1 = __hfma2(as_bf2(rc1[k][r].w[q]), rc2, as_bf2(bC1.w[q]));
+                            u0 = __hfma2(as_bf2(rc0.w[q]), rc2, as_bf2(bC0.w[q]));
+                            u1 = __hfma2(as_bf2(rc1.w[q]), rc2, as_bf2(bC1.w[q]));
                             oc0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
                             oc1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
                         }
@@ -545,7 +596,6 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
 #pragma unroll
                         for (int q = 0; q < PPL / 2; ++q) ob0.w[q] = ob1.w[q] = oc0.w[q] = oc1.w[q] = 0u;
                     }
-                    const uint32_t o = swz128(row, pp0);
                     sts_raw<PPL>(sm + Cfg::OB + o, ob0);
                     sts_raw<PPL>(sm + Cfg::OB + 8192 + o, ob1);
                     sts_raw<PPL>(sm + Cfg::OC + o, oc0);
@@ -580,11 +630,6 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
                 v.w = as_u32(__hmul2(as_bf2(v.w), sc2));
                 *reinterpret_cast<uint4*>(sm + Cfg::XP + o) = v;
             }
-        }
-        if (c > 0) {
-            (void)mbar_wait(&bar_m2, (c - 1) & 1);  // thread 0 already saw it complete
-            fence_after_sync();
-            epilogue(c - 1);
         }
         fence_proxy_async();
         fence_before_sync();
@@ -629,34 +674,52 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
         if (s_abort) break;
         (void)mbar_try_wait(smem_u32(&bar_m1), par);  // completed: orders the accumulators
 
-        // ======== I3: P = S o M, H1 = e^{cum_end} H0 + dH, next chunk's scalars ========
-        {
-            float s[16];
-            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, s);
-            const int trow = 16 * q4 + (lane & 15);
-            const int col0 = 16 * wh + ((lane >> 4) ? 32 : 0);
-            const int t = trow / R;
-            constexpr int NT = 16 / R;          // tokens covered by the 16 columns
-            const int s0 = col0 / R;
-            float cs_[NT], ws_[NT];
-#pragma unroll
-            for (int i = 0; i < NT; i += 2) {
-                const float2 a2 = *reinterpret_cast<const float2*>(blk + F_CUM + s0 + i);
-                const float2 w2 = *reinterpret_cast<const float2*>(blk + F_W + s0 + i);
-                cs_[i] = a2.x; cs_[i + 1] = a2.y; ws_[i] = w2.x; ws_[i + 1] = w2.y;
+        // ======== I3: P = S o M, H1 = e^{cum_end} H0 + dH ========
+        if (warp == 0) {  // the operand buffers are free again: fetch the next chunk's B / C
+            if (elect_one() && c + 1 < nchunks) {
+                issue_bc(c + 1);
+                s_issued[4] = c + 2;
             }
-            const float cum_t = blk[F_CUM + t], gam_t = blk[F_GAM + t];
+            __syncwarp();
+        }
+        {
+            float sv[16];
+            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, sv);
+            const int trow = 16 * q4 + (lane & 15);   // row block q4
+            const int qc = wh + ((lane >> 4) ? 2 : 0);  // column block of this half-warp
+            const int col0 = 16 * qc;
+            const int t = trow / R;
+            constexpr int NT = 16 / R;                  // tokens covered by the 16 columns
+            const int s0 = col0 / R;
             float m[NT];
+            if (qc < q4) {          // strictly below the diagonal block: factored decay
+                const float er = blk[F_EROW + t];
 #pragma unroll
-            for (int i = 0; i < NT; ++i) {
-                const int sa = s0 + i;
-                m[i] = (sa < t) ? ex2_approx(fminf(cum_t - cs_[i], 0.f)) * ws_[i] : ((sa == t) ? gam_t : 0.f);
+                for (int i = 0; i < NT; i += 2) {
+                    const float2 e2 = *reinterpret_cast<const float2*>(blk + F_ECOL + q4 * 64 + s0 + i);
+                    m[i] = er * e2.x;
+                    m[i + 1] = er * e2.y;
+                }
+            } else if (qc == q4) {  // diagonal block: decay, trapezoid weight and gamma
+                const float cum_t = blk[F_CUM + t], gam_t = blk[F_GAM + t];
+#pragma unroll
+                for (int i = 0; i < NT; i += 2) {
+                    const float2 a2 = *reinterpret_cast<const float2*>(blk + F_CUM + s0 + i);
+                    const float2 w2 = *reinterpret_cast<const float2*>(blk + F_W + s0 + i);
+                    const int sa = s0 + i;
+                    m[i] = (sa < t) ? ex2_approx(fminf(cum_t - a2.x, 0.f)) * w2.x : ((sa == t) ? gam_t : 0.f);
+                    m[i + 1] = (sa + 1 < t) ? ex2_approx(fminf(cum_t - a2.y, 0.f)) * w2.y
+                                            : ((sa + 1 == t) ? gam_t : 0.f);
+                }
+            } else {                // above the diagonal: zero
+#pragma unroll
+                for (int i = 0; i < NT; ++i) m[i] = 0.f;
             }
             tmem_wait_ld();
             uint32_t pw[8];
 #pragma unroll
             for (int j = 0; j < 16; j += 2)
-                pw[j / 2] = pack_bf16(s[j] * m[j / R], s[j + 1] * m[(j + 1) / R]);
+                pw[j / 2] = pack_bf16(sv[j] * m[j / R], sv[j + 1] * m[(j + 1) / R]);
             *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
             *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
@@ -673,7 +736,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
                 hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
             }
         }
-        if (c + 1 < nchunks) load_raw(c + 1);
+
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
@@ -741,6 +804,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
             if (k >= 0) (void)mbar_wait(&bar_x[k & 1], (k >> 1) & 1, kDrain);
         for (int k = s_issued[1] - 1; k <= s_issued[1]; ++k)
             if (k >= 0) (void)mbar_wait(&bar_t[k & 1], (k >> 1) & 1, kDrain);
+        if (s_issued[4] > 0) (void)mbar_wait(&bar_bc, (s_issued[4] - 1) & 1, kDrain);
         if (s_issued[2] > 0) (void)mbar_wait(&bar_m1, (s_issued[2] - 1) & 1, kDrain);
         if (s_issued[3] > 0) (void)mbar_wait(&bar_m2, (s_issued[3] - 1) & 1, kDrain);
     }
@@ -784,11 +848,13 @@ bool tc_scan_supported(const ScanParams& p, bool bf16) {
 }
 
 size_t tc_scan_workspace_bytes(const ScanParams& p) {
-    return p.bc_norm ? static_cast<size_t>(p.b * p.L * p.G * p.R) * sizeof(float2) : 0;
+    const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
+    const int64_t Lpad = (p.L + Q - 1) / Q * Q;
+    return p.bc_norm ? static_cast<size_t>(p.b * Lpad * p.G * p.R) * sizeof(uint2) : 0;
 }
 
 template <int R>
-static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, cudaStream_t s) {
+static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, cudaStream_t s) {
     constexpr int Q = 64 / R;
     TcMaps maps;
     const cuuint64_t H = p.H, Lq = p.L, b = p.b;
@@ -806,6 +872,17 @@ static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, cudaStream_t s) 
         if (!encode(&maps.theta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.theta, dims, str, box,
                     CU_TENSOR_MAP_SWIZZLE_128B)) return cudaErrorInvalidValue;
     }
+    {   // B, C [b][L][G][R][N], box (64 columns, R, 1, Q, 1): one 64-column slab per load
+        const cuuint64_t Gq = p.G;
+        const cuuint64_t dims[5] = {kN, static_cast<cuuint64_t>(R), Gq, Lq, b};
+        const cuuint64_t str[4] = {kN * 2, R * kN * 2, Gq * R * kN * 2, Lq * Gq * R * kN * 2};
+        const cuuint32_t box[5] = {kHalf, static_cast<cuuint32_t>(R), 1, Q, 1};
+        if (!encode(&maps.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, p.B, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode(&maps.C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, p.C, dims, str, box,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     {   // dt, A, lam [b][L][H] fp32, box (4 heads, Q + 1 tokens, 1)
         const cuuint64_t dims[3] = {H, Lq, b};
         const cuuint64_t str[2] = {H * 4, Lq * H * 4};
@@ -820,9 +897,10 @@ static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, cudaStream_t s) 
     }
     if (rs) {
         const int64_t rows = p.b * p.L * p.G * R;
+        const int64_t Lpad = (p.L + Q - 1) / Q * Q;
         rms_scale_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
-            p.eps, rs);
+            p.L, p.G, R, Lpad, p.eps, rs);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -837,7 +915,7 @@ static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, cudaStream_t s) 
 
 cudaError_t launch_scan_tc(const ScanParams& p, void* rs_ws, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
-    float2* rs = p.bc_norm ? static_cast<float2*>(rs_ws) : nullptr;
+    uint2* rs = p.bc_norm ? static_cast<uint2*>(rs_ws) : nullptr;
     switch (p.R) {
         case 1: return launch_tc_t<1>(p, rs, s);
         case 2: return launch_tc_t<2>(p, rs, s);

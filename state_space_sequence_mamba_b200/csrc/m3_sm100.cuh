@@ -194,6 +194,18 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
         : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
     return ok != 0;
 }
+// Like mbar_wait, but the waiting thread is suspended between checks (for up to the hint)
+// instead of spinning: for long waits on memory, where spinning would steal issue slots.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                long long max_cycles = 2000000000LL) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_sleep(a, parity, 1000000u)) return true;
+        if (clock64() - t0 > max_cycles) return false;
+    }
+}
 // Waits for the phase with the given parity to complete, at most ~max_cycles SM clocks.
 // Returns false on timeout. Callers keep the number of waiting threads small (one lane).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
@@ -241,6 +253,13 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const void* tmap, uint64_
         :: "r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
            "r"(c3), "r"(c4)
         : "memory");
+}
+
+// Plain bulk copy global -> shared of `bytes` (multiple of 16, both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
 }  // namespace sm100
