@@ -48,7 +48,9 @@ struct TcCfg {
     static constexpr int TPL = Q >= 16 ? Q / 16 : 1;        // tokens per lane (rotation)
     static constexpr int PPL = (Q / 4) / TPL;               // pairs per lane (rotation)
     static constexpr int LPT = 8 / PPL;                     // lanes per token group
+    static constexpr int NG = 32 / LPT;                     // token groups per warp
     static_assert(LPT * (Q / TPL) == 32, "rotation lane mapping");
+    static_assert(NG * TPL == Q, "interleaved tokens");
     // shared-memory byte layout after 1024-byte alignment
     static constexpr uint32_t X0 = 0, X1 = 8192;             // X chunk (TMA, swizzled), x2
     static constexpr uint32_t XP = 16384;                    // X' = diag(dw) X
@@ -217,7 +219,7 @@ template <int R>
 __global__ void __launch_bounds__(kTcThreads, 2)
 scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow) {
     using Cfg = TcCfg<R>;
-    constexpr int Q = Cfg::Q, TPL = Cfg::TPL, PPL = Cfg::PPL, LPT = Cfg::LPT;
+    constexpr int Q = Cfg::Q, TPL = Cfg::TPL, PPL = Cfg::PPL, LPT = Cfg::LPT, NG = Cfg::NG;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
@@ -523,47 +525,62 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         (void)mbar_try_wait(smem_u32(&bar_t[st]), (c >> 1) & 1);  // landed (warp 1 waited)
         if (!mbar_wait(&bar_bc, par)) s_abort = 1;  // raw B / C of this chunk
         {
+            // Lane (tg, ps) holds tokens tg + NG k (k < TPL): in every access below the lanes of a
+            // half-warp touch consecutive rows, which the 128-byte swizzle spreads over all banks.
             float inc[TPL][PPL];
 #pragma unroll
             for (int k = 0; k < TPL; ++k) {
-                const int t = tg * TPL + k;
+                const int t = tg + NG * k;
                 const RawV<PPL> th = lds_raw<PPL>(sTh + swz128(t, pp0));
                 const float dd = blk[F_DT + t];  // 0 past the end: no rotation there
 #pragma unroll
-                for (int j = 0; j < PPL; ++j) inc[k][j] = fmaf(dd, raw_f<PPL>(th, j), k ? inc[k - 1][j] : 0.f);
+                for (int j = 0; j < PPL; ++j) inc[k][j] = dd * raw_f<PPL>(th, j);
             }
-            float incl[PPL], base[PPL];
+            // cumulative angle: per block k an inclusive scan over the token groups, plus the
+            // totals of the earlier blocks and the carry from earlier chunks
+            float ang[TPL][PPL];
 #pragma unroll
-            for (int j = 0; j < PPL; ++j) incl[j] = inc[TPL - 1][j];
+            for (int k = 0; k < TPL; ++k)
+#pragma unroll
+                for (int j = 0; j < PPL; ++j) ang[k][j] = inc[k][j];
 #pragma unroll
             for (int off = LPT; off < 32; off <<= 1) {
 #pragma unroll
-                for (int j = 0; j < PPL; ++j) {
-                    const float v = __shfl_up_sync(0xffffffffu, incl[j], off);
-                    if (lane >= off) incl[j] += v;
-                }
+                for (int k = 0; k < TPL; ++k)
+#pragma unroll
+                    for (int j = 0; j < PPL; ++j) {
+                        const float v = __shfl_up_sync(0xffffffffu, ang[k][j], off);
+                        if (lane >= off) ang[k][j] += v;
+                    }
             }
 #pragma unroll
             for (int j = 0; j < PPL; ++j) {
-                base[j] = carry_r[j] + incl[j] - inc[TPL - 1][j];
-                const float tot = __shfl_sync(0xffffffffu, incl[j], 32 - LPT + ps);
-                carry[j] += tot;
-                carry_r[j] = reduce_2pi(carry_r[j] + tot);
+                float run = carry_r[j], tot_all = 0.f;
+#pragma unroll
+                for (int k = 0; k < TPL; ++k) {
+                    const float tot = __shfl_sync(0xffffffffu, ang[k][j], 32 - LPT + ps);
+                    ang[k][j] += run;
+                    run += tot;
+                    tot_all += tot;
+                }
+                carry[j] += tot_all;
+                carry_r[j] = reduce_2pi(carry_r[j] + tot_all);
             }
 #pragma unroll
             for (int k = 0; k < TPL; ++k) {
-                const int t = tg * TPL + k;
+                const int t = tg + NG * k;
                 uint32_t cw[PPL / 2], sw[PPL / 2];  // packed bf16 cos / sin of the lane's pairs
 #pragma unroll
                 for (int j = 0; j < PPL; j += 2) {
                     float s0, c0v, s1, c1v;
-                    __sincosf(base[j] + inc[k][j], &s0, &c0v);
-                    __sincosf(base[j + 1] + inc[k][j + 1], &s1, &c1v);
+                    __sincosf(ang[k][j], &s0, &c0v);
+                    __sincosf(ang[k][j + 1], &s1, &c1v);
                     cw[j / 2] = pack_bf16(c0v, c1v);
                     sw[j / 2] = pack_bf16(s0, s1);
                 }
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
+                for (int rr = 0; rr < R; ++rr) {
+                    // rank order rotated by the token group: spreads MIMO rows over more banks
+                    const int r = (rr + tg) & (R - 1);
                     const int row = t * R + r;
                     const uint32_t o = swz128(row, pp0);
                     RawV<PPL> ob0, ob1, oc0, oc1;
