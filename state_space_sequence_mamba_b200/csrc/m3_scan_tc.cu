@@ -45,42 +45,43 @@ __host__ __device__ constexpr uint32_t round_up(uint32_t v, uint32_t a) { return
 template <int R>
 struct TcCfg {
     static constexpr int Q = 64 / R;                        // tokens per chunk
-    static constexpr int TPL = Q >= 16 ? Q / 16 : 1;        // tokens per lane (rotation)
-    static constexpr int PPL = (Q / 4) / TPL;               // pairs per lane (rotation)
-    static constexpr int LPT = 8 / PPL;                     // lanes per token group
-    static constexpr int NG = 32 / LPT;                     // token groups per warp
-    static_assert(LPT * (Q / TPL) == 32, "rotation lane mapping");
-    static_assert(NG * TPL == Q, "interleaved tokens");
+    static constexpr int TPS = Q / 8;                       // tokens per warp (rotation)
+    static_assert(TPS * 8 == Q, "one token segment per warp");
     // shared-memory byte layout after 1024-byte alignment
     static constexpr uint32_t X0 = 0, X1 = 8192;             // X chunk (TMA, swizzled), x2
-    static constexpr uint32_t XP = 16384;                    // X' = diag(dw) X
+    static constexpr uint32_t XP = 16384;                    // X' = diag(dw) X, then P = S o M
     static constexpr uint32_t OB = 24576;                    // Bbar, 2 slabs of 64 x 128 B
-    static constexpr uint32_t OC = 40960;                    // Cbar, 2 slabs
-    static constexpr uint32_t OP = 57344;                    // P = S o M
-    static constexpr uint32_t OH = 65536;                    // H0 bf16, 128 x 128 B
+    static constexpr uint32_t OC = 40960;                    // raw C, rotated in place to Cbar
+    static constexpr uint32_t OH = 57344;                    // H0 bf16, 128 x 128 B
+    static constexpr uint32_t RB = 73728;                    // raw B of the chunk (TMA)
     static constexpr uint32_t TH_BYTES = round_up(Q * 128, 1024);
-    static constexpr uint32_t TH0 = 81920, TH1 = TH0 + TH_BYTES;   // theta (TMA, swizzled)
+    static constexpr uint32_t TH = 90112;                    // theta (TMA, swizzled)
     static constexpr uint32_t SC_ONE = (Q + 1) * 16;                // [Q+1 tokens][4 heads] fp32
     static constexpr uint32_t SC_SLOT = round_up(SC_ONE, 128);      // 128-byte aligned slots
     static constexpr uint32_t SC_BYTES = 3 * SC_SLOT;
-    static constexpr uint32_t SC0 = TH1 + TH_BYTES, SC1 = SC0 + SC_BYTES;  // dt, A, lam boxes
-    static constexpr uint32_t ORS = SC1 + SC_BYTES;                 // RMS scales, 64 float2
+    static constexpr uint32_t SC0 = TH + TH_BYTES, SC1 = SC0 + SC_BYTES;  // dt, A, lam boxes
+    static constexpr uint32_t ORS = SC1 + SC_BYTES;                 // RMS scales, 64 x uint2
     static constexpr uint32_t OF = ORS + 512;                       // fp32 scratch
-    static constexpr uint32_t BC_TX = 4 * 8192;                     // raw B, C: two slabs each
+    static constexpr uint32_t B_TX = 2 * 8192;                      // raw B: two slabs
+    static constexpr uint32_t C_TX = 2 * 8192;                      // raw C: two slabs
     static constexpr uint32_t X_TX = 8192;                          // bytes of one X box
-    static constexpr uint32_t TS_TX = Q * 128 + 3 * SC_ONE;         // theta + scalar boxes
+    static constexpr uint32_t TH_TX = Q * 128;                      // theta box
+    static constexpr uint32_t SC_TX = 3 * SC_ONE;                   // dt, A, lam boxes
 };
-// fp32 scratch (float offsets)
+// fp32 scratch (float offsets): two blocks of chunk scalars (by chunk parity), the angle
+// totals of the eight token segments, then the bf16 biases
 constexpr int F_CUM = 0, F_GAM = 64, F_W = 128, F_ECUM = 192, F_DW = 256, F_DT = 320,
-              F_MISC = 384, F_EROW = 448, F_ECOL = 512,  // tile factors: [64], [4][64]
-              F_BLK = 768;   // one block of chunk scalars; two blocks (by parity)
-constexpr int F_BIAS = 2 * F_BLK;          // then bias_B [R][128], bias_C [R][128], fold scratch
+              F_EROW = 384, F_ECOL = 448,  // tile factors: [64], column blocks 1..3 x [64]
+              F_MISC = 640,                // e^{cum_end}
+              F_BLK = 656;
+constexpr int F_SEG = 2 * F_BLK;           // [8 segments][32 lanes] float2
+constexpr int F_BIAS = F_SEG + 512;        // bias_B [R][128] bf16, bias_C [R][128] bf16
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
 
 template <int R>
 __host__ __device__ constexpr uint32_t tc_smem_bytes() {
-    return TcCfg<R>::OF + 4u * (F_BIAS + 2 * R * kN + R * kN + R * kP) + 2u * 2 * R * kN + 1024u;
+    return TcCfg<R>::OF + 4u * F_BIAS + 2u * 2 * R * kN + 1024u;
 }
 
 // x reduced by a whole number of turns into [-pi, pi]: Cody-Waite reduction with 2*pi split
@@ -106,70 +107,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// PPL consecutive bf16 held as raw words (PPL in {2, 4, 8}).
-template <int PPL>
-struct RawV { uint32_t w[PPL / 2]; };
-
-template <int PPL>
-__device__ __forceinline__ RawV<PPL> ldg_raw(const __nv_bfloat16* src) {
-    RawV<PPL> r;
-    if constexpr (PPL == 8) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
-        r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
-    } else if constexpr (PPL == 4) {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-        r.w[0] = u.x; r.w[1] = u.y;
-    } else {
-        r.w[0] = __ldg(reinterpret_cast<const unsigned int*>(src));
-    }
-    return r;
-}
-template <int PPL>
-__device__ __forceinline__ RawV<PPL> lds_raw(const uint8_t* src) {
-    RawV<PPL> r;
-    if constexpr (PPL == 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(src);
-        r.w[0] = u.x; r.w[1] = u.y; r.w[2] = u.z; r.w[3] = u.w;
-    } else if constexpr (PPL == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(src);
-        r.w[0] = u.x; r.w[1] = u.y;
-    } else {
-        r.w[0] = *reinterpret_cast<const uint32_t*>(src);
-    }
-    return r;
-}
-template <int PPL>
-__device__ __forceinline__ float raw_f(const RawV<PPL>& r, int j) {
-    const uint32_t w = r.w[j >> 1];
-    return __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
-}
-
-template <int PPL>
-__device__ __forceinline__ void st_bf16_smem(uint8_t* dst, const float (&v)[PPL]) {
-    if constexpr (PPL == 8) {
-        uint4 u;
-        u.x = pack_bf16(v[0], v[1]); u.y = pack_bf16(v[2], v[3]);
-        u.z = pack_bf16(v[4], v[5]); u.w = pack_bf16(v[6], v[7]);
-        *reinterpret_cast<uint4*>(dst) = u;
-    } else if constexpr (PPL == 4) {
-        uint2 u;
-        u.x = pack_bf16(v[0], v[1]); u.y = pack_bf16(v[2], v[3]);
-        *reinterpret_cast<uint2*>(dst) = u;
-    } else {
-        *reinterpret_cast<uint32_t*>(dst) = pack_bf16(v[0], v[1]);
-    }
-}
-
-template <int PPL>
-__device__ __forceinline__ void sts_raw(uint8_t* dst, const RawV<PPL>& v) {
-    if constexpr (PPL == 8) {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
-    } else if constexpr (PPL == 4) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(v.w[0], v.w[1]);
-    } else {
-        *reinterpret_cast<uint32_t*>(dst) = v.w[0];
-    }
-}
 __device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) {
     return *reinterpret_cast<const __nv_bfloat162*>(&w);
 }
@@ -219,23 +156,24 @@ template <int R>
 __global__ void __launch_bounds__(kTcThreads, 2)
 scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow) {
     using Cfg = TcCfg<R>;
-    constexpr int Q = Cfg::Q, TPL = Cfg::TPL, PPL = Cfg::PPL, LPT = Cfg::LPT, NG = Cfg::NG;
+    constexpr int Q = Cfg::Q, TPS = Cfg::TPS;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     float* sf = reinterpret_cast<float*>(sm + Cfg::OF);   // two blocks of chunk scalars
-    float* s_biasB = sf + F_BIAS;
-    float* s_biasC = s_biasB + R * kN;
-    float* s_fold = s_biasC + R * kN;     // [R][128] Bbar of the stored previous token
-    float* s_foldx = s_fold + R * kN;     // [R][64]  its x
-    __nv_bfloat16* s_biasB2 = reinterpret_cast<__nv_bfloat16*>(s_foldx + R * kP);  // [R][128] bf16
+    float2* s_seg = reinterpret_cast<float2*>(sf + F_SEG);
+    __nv_bfloat16* s_biasB2 = reinterpret_cast<__nv_bfloat16*>(sf + F_BIAS);  // [R][128] bf16
     __nv_bfloat16* s_biasC2 = s_biasB2 + R * kN;
-    __shared__ uint64_t bar_x[2], bar_t[2], bar_bc, bar_m1, bar_m2;
+    // set-up only: the stored previous token's Bbar and x, in the H0 operand buffer
+    float* s_fold = reinterpret_cast<float*>(sm + Cfg::OH);   // [R][128]
+    float* s_foldx = s_fold + R * kN;                          // [R][64]
+    __shared__ uint64_t bar_x[2], bar_sc[2], bar_th, bar_b, bar_c, bar_m1, bar_m2;
     __shared__ uint32_t tslot;
     __shared__ int s_abort;
-    // async work thread 0 has started (for draining it if a wait gives up)
-    __shared__ int s_issued[5];  // last X / TS chunk issued, MMA groups (m1, m2), B/C loads
+    // async work thread 0 has started, for draining it if a wait gives up: last X and scalar
+    // box chunk issued; theta, raw B, raw C loads issued; MMA groups m1, m2 committed
+    __shared__ int s_issued[7];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3, wh = warp >> 2;  // TMEM subpartition, column half
@@ -246,36 +184,54 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     const int H = static_cast<int>(p.H), G = static_cast<int>(p.G);
     // Per-unit base pointers; offsets below fit in 32 bits (checked on the host).
     const __nv_bfloat16* Bu = static_cast<const __nv_bfloat16*>(p.B) + (bb * p.L * G + g) * R * kN;
-    const __nv_bfloat16* Cu = static_cast<const __nv_bfloat16*>(p.C) + (bb * p.L * G + g) * R * kN;
     const int Lpad = ((L + Q - 1) / Q) * Q;
     const uint2* rsu = rsrow ? rsrow + (bb * G + g) * static_cast<int64_t>(Lpad) * R : nullptr;
     const __nv_bfloat16* xu = static_cast<const __nv_bfloat16*>(p.x) + (bb * p.L * H + hh) * R * kP;
     __nv_bfloat16* yu = static_cast<__nv_bfloat16*>(p.y) + (bb * p.L * H + hh) * R * kP;
     const int tokB = G * R * kN, tokY = H * R * kP;  // element stride of one token
     const int nchunks = (L + Q - 1) / Q;
+    const int ib = static_cast<int>(bb), ih = static_cast<int>(hh), ig = static_cast<int>(g);
+    uint2* s_rs = reinterpret_cast<uint2*>(sm + Cfg::ORS);
 
+    // ---- TMA issue (one thread) ----
     auto issue_x = [&](int c) {
         const int st = c & 1;
         mbar_arrive_expect_tx(&bar_x[st], Cfg::X_TX);
-        tma_load_5d(sm + (st ? Cfg::X1 : Cfg::X0), &maps.x, &bar_x[st], 0, 0,
-                    static_cast<int>(hh), c * Q, static_cast<int>(bb));
+        tma_load_5d(sm + (st ? Cfg::X1 : Cfg::X0), &maps.x, &bar_x[st], 0, 0, ih, c * Q, ib);
+        s_issued[0] = c;
     };
-    auto issue_ts = [&](int c) {  // theta and the dt, A, lam boxes of chunk c
+    auto issue_sc = [&](int c) {  // dt, A, lam boxes of chunk c (4 heads, Q + 1 tokens)
         const int st = c & 1;
-        uint64_t* bar = &bar_t[st];
-        mbar_arrive_expect_tx(bar, Cfg::TS_TX);
-        const int ic0 = c * Q, ih = static_cast<int>(hh), ib = static_cast<int>(bb);
-        tma_load_4d(sm + (st ? Cfg::TH1 : Cfg::TH0), &maps.theta, bar, 0, ih, ic0, ib);
+        mbar_arrive_expect_tx(&bar_sc[st], Cfg::SC_TX);
         uint8_t* sc = sm + (st ? Cfg::SC1 : Cfg::SC0);
         const int h4 = ih & ~3;
-        tma_load_3d(sc, &maps.dt, bar, h4, ic0, ib);
-        tma_load_3d(sc + Cfg::SC_SLOT, &maps.A, bar, h4, ic0, ib);
-        tma_load_3d(sc + 2 * Cfg::SC_SLOT, &maps.lam, bar, h4, ic0, ib);
+        tma_load_3d(sc, &maps.dt, &bar_sc[st], h4, c * Q, ib);
+        tma_load_3d(sc + Cfg::SC_SLOT, &maps.A, &bar_sc[st], h4, c * Q, ib);
+        tma_load_3d(sc + 2 * Cfg::SC_SLOT, &maps.lam, &bar_sc[st], h4, c * Q, ib);
+        s_issued[1] = c;
+    };
+    auto issue_th = [&](int c) {  // theta of chunk c into the (single) theta buffer
+        mbar_arrive_expect_tx(&bar_th, Cfg::TH_TX);
+        tma_load_4d(sm + Cfg::TH, &maps.theta, &bar_th, 0, ih, c * Q, ib);
+        s_issued[2] += 1;
+    };
+    auto issue_b = [&](int c) {   // raw B rows of chunk c (two 64-column slabs) + RMS scales
+        mbar_arrive_expect_tx(&bar_b, Cfg::B_TX + (rsu ? 512u : 0u));
+        tma_load_5d(sm + Cfg::RB, &maps.B, &bar_b, 0, 0, ig, c * Q, ib);
+        tma_load_5d(sm + Cfg::RB + 8192, &maps.B, &bar_b, kHalf, 0, ig, c * Q, ib);
+        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(c) * Q * R, 512u, &bar_b);
+        s_issued[3] += 1;
+    };
+    auto issue_c = [&](int c) {   // raw C rows of chunk c straight into the Cbar operand buffer
+        mbar_arrive_expect_tx(&bar_c, Cfg::C_TX);
+        tma_load_5d(sm + Cfg::OC, &maps.C, &bar_c, 0, 0, ig, c * Q, ib);
+        tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_c, kHalf, 0, ig, c * Q, ib);
+        s_issued[4] += 1;
     };
     // Chunk scalars (one full warp): cumulative log-decay, gamma, trapezoid weight w, ...
     auto scalars = [&](int c) {
         const int st = c & 1;
-        if (!mbar_wait(&bar_t[st], (c >> 1) & 1)) {
+        if (!mbar_wait(&bar_sc[st], (c >> 1) & 1)) {
             if (lane == 0) s_abort = 1;
         }
         const float* sSc = reinterpret_cast<const float*>(sm + (st ? Cfg::SC1 : Cfg::SC0));
@@ -335,7 +291,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             blk[F_EROW + t] = ex2_approx(c2v[k] - c2blk[t / TB < 4 ? t / TB : 3]);
 #pragma unroll
             for (int qb = 1; qb < 4; ++qb)
-                blk[F_ECOL + qb * 64 + t] = (t < qb * TB) ? ex2_approx(c2blk[qb] - c2v[k]) * w[k] : 0.f;
+                blk[F_ECOL + (qb - 1) * 64 + t] = (t < qb * TB) ? ex2_approx(c2blk[qb] - c2v[k]) * w[k] : 0.f;
         }
     };
 
@@ -343,30 +299,30 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     if (tid == 0) {
         mbar_init(&bar_x[0], 1);
         mbar_init(&bar_x[1], 1);
-        mbar_init(&bar_t[0], 1);
-        mbar_init(&bar_t[1], 1);
-        mbar_init(&bar_bc, 1);
+        mbar_init(&bar_sc[0], 1);
+        mbar_init(&bar_sc[1], 1);
+        mbar_init(&bar_th, 1);
+        mbar_init(&bar_b, 1);
+        mbar_init(&bar_c, 1);
         mbar_init(&bar_m1, 1);
         mbar_init(&bar_m2, 1);
         fence_mbar_init();
         s_abort = 0;
+        s_issued[0] = s_issued[1] = -1;
+        for (int i = 2; i < 7; ++i) s_issued[i] = 0;
         if (nchunks > 0) {
             issue_x(0);
-            issue_ts(0);
+            issue_sc(0);
+            issue_th(0);
+            issue_b(0);
+            issue_c(0);
         }
-        if (nchunks > 1) issue_ts(1);
+        if (nchunks > 1) issue_sc(1);
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
-    if (tid == 0) {
-        s_issued[0] = nchunks > 0 ? 0 : -1;
-        s_issued[1] = nchunks > 1 ? 1 : (nchunks > 0 ? 0 : -1);
-        s_issued[2] = s_issued[3] = s_issued[4] = 0;
-    }
     for (int i = tid; i < R * kN; i += kTcThreads) {
-        s_biasB[i] = p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f;
-        s_biasC[i] = p.Cbias ? p.Cbias[hh * R * kN + i] : 0.f;
-        s_biasB2[i] = __float2bfloat16_rn(s_biasB[i]);
-        s_biasC2[i] = __float2bfloat16_rn(s_biasC[i]);
+        s_biasB2[i] = __float2bfloat16_rn(p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f);
+        s_biasC2[i] = __float2bfloat16_rn(p.Cbias ? p.Cbias[hh * R * kN + i] : 0.f);
     }
     fence_before_sync();
     __syncthreads();
@@ -388,17 +344,17 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         for (int j = 0; j < 32; ++j) hreg[j] = 0.f;
     }
 
-    // rotation lane mapping: warp -> 8 pairs, lane -> (token group, pair subgroup)
-    const int tg = lane / LPT, ps = lane % LPT;
-    const int pp0 = 8 * warp + ps * PPL;  // first pair of this lane
-    // cumulative angle per pair: carry (as stored in the state) and the same reduced into
-    // [-pi, pi] once per chunk (Cody & Waite's two-constant reduction, "Software Manual for
-    // the Elementary Functions", 1980), so that the per-token angles stay small
-    float carry[PPL], carry_r[PPL];
+    // Rotation mapping: warp = token segment (TPS consecutive tokens), lane = pair couple
+    // (2 lane, 2 lane + 1) with partners (+ N/2). The cumulative angle of the couple, as stored
+    // in the state (car) and reduced into [-pi, pi] once per chunk (car_r: Cody & Waite's
+    // two-constant reduction, "Software Manual for the Elementary Functions", 1980), so that
+    // the per-token angles stay small.
+    const int jp = 2 * lane;
+    float car[2], car_r[2];
 #pragma unroll
-    for (int j = 0; j < PPL; ++j) {
-        carry[j] = p.phi0 ? p.phi0[u * kHalf + pp0 + j] : 0.f;
-        carry_r[j] = reduce_2pi(carry[j]);
+    for (int j = 0; j < 2; ++j) {
+        car[j] = p.phi0 ? p.phi0[u * kHalf + jp + j] : 0.f;
+        car_r[j] = reduce_2pi(car[j]);
     }
 
     // ---- fold the stored previous token into the primed state ----
@@ -421,8 +377,10 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             float sn, cs;
             sincosf(p.phi0[u * kHalf + i], &sn, &cs);
             const float rs = sf[F_MISC + 8 + r];
-            const float u0 = __bfloat162float(pB[r * kN + i]) * rs + s_biasB[r * kN + i];
-            const float u1 = __bfloat162float(pB[r * kN + i + kHalf]) * rs + s_biasB[r * kN + i + kHalf];
+            const float b0 = p.Bbias ? p.Bbias[hh * R * kN + r * kN + i] : 0.f;
+            const float b1 = p.Bbias ? p.Bbias[hh * R * kN + r * kN + i + kHalf] : 0.f;
+            const float u0 = __bfloat162float(pB[r * kN + i]) * rs + b0;
+            const float u1 = __bfloat162float(pB[r * kN + i + kHalf]) * rs + b1;
             s_fold[r * kN + i] = u0 * cs + u1 * sn;
             s_fold[r * kN + i + kHalf] = u1 * cs - u0 * sn;
         }
@@ -439,26 +397,12 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     }
 
     const uint32_t aB = smem_u32(sm + Cfg::OB), aC = smem_u32(sm + Cfg::OC);
-    const uint32_t aXP = smem_u32(sm + Cfg::XP);
-    const uint32_t aP = smem_u32(sm + Cfg::OP), aH = smem_u32(sm + Cfg::OH);
+    const uint32_t aXP = smem_u32(sm + Cfg::XP), aH = smem_u32(sm + Cfg::OH);
     const uint32_t id_s = idesc_bf16(64, 64, false, false);   // S  = C . B^T
     const uint32_t id_yo = idesc_bf16(64, 64, false, true);   // Yo = C . H
     const uint32_t id_dh = idesc_bf16(128, 64, true, true);   // dH = B^T . X'
     const uint32_t id_yd = idesc_bf16(64, 64, false, true);   // Yd = P . X
 
-    // Raw B and C rows of chunk c straight into the Bbar / Cbar operand buffers (two 64-column
-    // slabs each, swizzled as the MMA reads them; the rotation then transforms them in place),
-    // plus the chunk's RMS scales. Only when those buffers are free (their MMAs have finished).
-    uint2* s_rs = reinterpret_cast<uint2*>(sm + Cfg::ORS);
-    auto issue_bc = [&](int c) {
-        const int ic0 = c * Q, ig = static_cast<int>(g), ib = static_cast<int>(bb);
-        mbar_arrive_expect_tx(&bar_bc, Cfg::BC_TX + (rsu ? 512u : 0u));
-        tma_load_5d(sm + Cfg::OB, &maps.B, &bar_bc, 0, 0, ig, ic0, ib);
-        tma_load_5d(sm + Cfg::OB + 8192, &maps.B, &bar_bc, kHalf, 0, ig, ic0, ib);
-        tma_load_5d(sm + Cfg::OC, &maps.C, &bar_bc, 0, 0, ig, ic0, ib);
-        tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_bc, kHalf, 0, ig, ic0, ib);
-        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(ic0) * R, 512u, &bar_bc);
-    };
     // y of chunk c from the Yd / Yo accumulators (TMEM): y = Yd + e^{cum_t} Yo
     auto epilogue = [&](int c) {
         float yd[16], yo[16];
@@ -486,139 +430,103 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     };
 
-    if (nchunks > 0) {
-        if (tid == 0) {
-            issue_bc(0);
-            s_issued[4] = 1;
-        }
-        if (warp == 1) scalars(0);
-    }
+    if (nchunks > 0 && warp == 1) scalars(0);
     __syncthreads();
 
     for (int c = 0; c < nchunks && !s_abort; ++c) {
-        const int c0 = c * Q;
-        const int T = (L - c0) < Q ? (L - c0) : Q;
         const int st = c & 1;
         const uint32_t par = static_cast<uint32_t>(c & 1);
-        const uint8_t* sTh = sm + (st ? Cfg::TH1 : Cfg::TH0);
         const float* blk = sf + st * F_BLK;
 
-        // ======== I1: rotation(c), H0 and X' operands, epilogue(c-1) ========
+        // ======== I1: rotation(c); then epilogue(c-1), the H0 and X' operands ========
+        if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
+        {
+            // Angle increments dt_t theta_t of the segment's tokens, their sum per pair, and the
+            // segment totals exchanged through shared memory: each lane then walks its own
+            // tokens from carry + the earlier segments' totals.
+            float inc[TPS][2];
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < TPS; ++k) {
+                const int t = warp * TPS + k;
+                const uint32_t th = *reinterpret_cast<const uint32_t*>(sm + Cfg::TH + swz128(t, jp));
+                const float dd = blk[F_DT + t];  // 0 past the sequence end: no rotation there
+                inc[k][0] = dd * __uint_as_float(th << 16);
+                inc[k][1] = dd * __uint_as_float(th & 0xFFFF0000u);
+                sum0 += inc[k][0];
+                sum1 += inc[k][1];
+            }
+            s_seg[warp * 32 + lane] = make_float2(sum0, sum1);
+            __syncthreads();
+            float a0 = car_r[0], a1 = car_r[1], tot0 = 0.f, tot1 = 0.f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float2 v = s_seg[k * 32 + lane];
+                if (k < warp) { a0 += v.x; a1 += v.y; }
+                tot0 += v.x;
+                tot1 += v.y;
+            }
+            car[0] += tot0;
+            car[1] += tot1;
+            car_r[0] = reduce_2pi(car_r[0] + tot0);
+            car_r[1] = reduce_2pi(car_r[1] + tot1);
+            uint32_t cw[TPS], sw[TPS];  // packed bf16 (cos, cos) and (sin, sin) of the couple
+#pragma unroll
+            for (int k = 0; k < TPS; ++k) {
+                a0 += inc[k][0];
+                a1 += inc[k][1];
+                float sn0, cs0, sn1, cs1;
+                __sincosf(a0, &sn0, &cs0);
+                __sincosf(a1, &sn1, &cs1);
+                cw[k] = pack_bf16(cs0, cs1);
+                sw[k] = pack_bf16(sn0, sn1);
+            }
+            if (!mbar_wait(&bar_b, par)) s_abort = 1;   // raw B and the RMS scales
+            if (!mbar_wait(&bar_c, par)) s_abort = 1;   // raw C
+#pragma unroll 1
+            for (int r = 0; r < R; ++r) {
+                // bias words of this rank at the couple, both halves of each pair
+                const __nv_bfloat162 bB0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + jp);
+                const __nv_bfloat162 bB1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + kHalf + jp);
+                const __nv_bfloat162 bC0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + jp);
+                const __nv_bfloat162 bC1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + kHalf + jp);
+#pragma unroll
+                for (int k = 0; k < TPS; ++k) {
+                    const int row = (warp * TPS + k) * R + r;
+                    const uint32_t o = swz128(row, jp);
+                    const uint32_t rb0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + o);
+                    const uint32_t rb1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + 8192 + o);
+                    const uint32_t rc0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + o);
+                    const uint32_t rc1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + 8192 + o);
+                    const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
+                    const __nv_bfloat162 c2 = as_bf2(cw[k]), s2 = as_bf2(sw[k]);
+                    // u = rs * raw + bias on both halves of each pair, then
+                    // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
+                    __nv_bfloat162 u0 = __hfma2(as_bf2(rb0), as_bf2(rsv.x), bB0);
+                    __nv_bfloat162 u1 = __hfma2(as_bf2(rb1), as_bf2(rsv.x), bB1);
+                    *reinterpret_cast<uint32_t*>(sm + Cfg::OB + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
+                    *reinterpret_cast<uint32_t*>(sm + Cfg::OB + 8192 + o) =
+                        as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
+                    u0 = __hfma2(as_bf2(rc0), as_bf2(rsv.y), bC0);
+                    u1 = __hfma2(as_bf2(rc1), as_bf2(rsv.y), bC1);
+                    *reinterpret_cast<uint32_t*>(sm + Cfg::OC + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
+                    *reinterpret_cast<uint32_t*>(sm + Cfg::OC + 8192 + o) =
+                        as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
+                }
+            }
+        }
+        // Yd(c-1) done: its X buffer takes X(c+1), and y(c-1) can be written
         if (warp == 0) {
-            // X of chunk c+1 goes where X of chunk c-1 was: Yd(c-1) must have finished
             if (elect_one()) {
                 if (c > 0 && !mbar_wait(&bar_m2, (c - 1) & 1)) s_abort = 1;
-                if (c + 1 < nchunks) {
-                    issue_x(c + 1);
-                    s_issued[0] = c + 1;
-                }
+                if (c + 1 < nchunks) issue_x(c + 1);
             }
             __syncwarp();
         }
-        // work that needs neither this chunk's B / C nor theta first: y of the previous
-        // chunk and the H0 operand, while the B / C tiles finish landing
         if (c > 0) {
-            (void)mbar_wait(&bar_m2, (c - 1) & 1);  // thread 0 already saw it complete
+            (void)mbar_wait(&bar_m2, (c - 1) & 1);
             fence_after_sync();
             epilogue(c - 1);
-        }
-        (void)mbar_try_wait(smem_u32(&bar_t[st]), (c >> 1) & 1);  // landed (warp 1 waited)
-        if (!mbar_wait(&bar_bc, par)) s_abort = 1;  // raw B / C of this chunk
-        {
-            // Lane (tg, ps) holds tokens tg + NG k (k < TPL): in every access below the lanes of a
-            // half-warp touch consecutive rows, which the 128-byte swizzle spreads over all banks.
-            float inc[TPL][PPL];
-#pragma unroll
-            for (int k = 0; k < TPL; ++k) {
-                const int t = tg + NG * k;
-                const RawV<PPL> th = lds_raw<PPL>(sTh + swz128(t, pp0));
-                const float dd = blk[F_DT + t];  // 0 past the end: no rotation there
-#pragma unroll
-                for (int j = 0; j < PPL; ++j) inc[k][j] = dd * raw_f<PPL>(th, j);
-            }
-            // cumulative angle: per block k an inclusive scan over the token groups, plus the
-            // totals of the earlier blocks and the carry from earlier chunks
-            float ang[TPL][PPL];
-#pragma unroll
-            for (int k = 0; k < TPL; ++k)
-#pragma unroll
-                for (int j = 0; j < PPL; ++j) ang[k][j] = inc[k][j];
-#pragma unroll
-            for (int off = LPT; off < 32; off <<= 1) {
-#pragma unroll
-                for (int k = 0; k < TPL; ++k)
-#pragma unroll
-                    for (int j = 0; j < PPL; ++j) {
-                        const float v = __shfl_up_sync(0xffffffffu, ang[k][j], off);
-                        if (lane >= off) ang[k][j] += v;
-                    }
-            }
-#pragma unroll
-            for (int j = 0; j < PPL; ++j) {
-                float run = carry_r[j], tot_all = 0.f;
-#pragma unroll
-                for (int k = 0; k < TPL; ++k) {
-                    const float tot = __shfl_sync(0xffffffffu, ang[k][j], 32 - LPT + ps);
-                    ang[k][j] += run;
-                    run += tot;
-                    tot_all += tot;
-                }
-                carry[j] += tot_all;
-                carry_r[j] = reduce_2pi(carry_r[j] + tot_all);
-            }
-#pragma unroll
-            for (int k = 0; k < TPL; ++k) {
-                const int t = tg + NG * k;
-                uint32_t cw[PPL / 2], sw[PPL / 2];  // packed bf16 cos / sin of the lane's pairs
-#pragma unroll
-                for (int j = 0; j < PPL; j += 2) {
-                    float s0, c0v, s1, c1v;
-                    __sincosf(ang[k][j], &s0, &c0v);
-                    __sincosf(ang[k][j + 1], &s1, &c1v);
-                    cw[j / 2] = pack_bf16(c0v, c1v);
-                    sw[j / 2] = pack_bf16(s0, s1);
-                }
-                for (int rr = 0; rr < R; ++rr) {
-                    // rank order rotated by the token group: spreads MIMO rows over more banks
-                    const int r = (rr + tg) & (R - 1);
-                    const int row = t * R + r;
-                    const uint32_t o = swz128(row, pp0);
-                    RawV<PPL> ob0, ob1, oc0, oc1;
-                    if (t < T) {
-                        const RawV<PPL> rb0 = lds_raw<PPL>(sm + Cfg::OB + o);
-                        const RawV<PPL> rb1 = lds_raw<PPL>(sm + Cfg::OB + 8192 + o);
-                        const RawV<PPL> rc0 = lds_raw<PPL>(sm + Cfg::OC + o);
-                        const RawV<PPL> rc1 = lds_raw<PPL>(sm + Cfg::OC + 8192 + o);
-                        const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
-                        const __nv_bfloat162 rb2 = as_bf2(rsv.x), rc2 = as_bf2(rsv.y);
-                        const RawV<PPL> bB0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0));
-                        const RawV<PPL> bB1 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasB2 + r * kN + pp0 + kHalf));
-                        const RawV<PPL> bC0 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasC2 + r * kN + pp0));
-                        const RawV<PPL> bC1 = lds_raw<PPL>(reinterpret_cast<const uint8_t*>(s_biasC2 + r * kN + pp0 + kHalf));
-#pragma unroll
-                        for (int q = 0; q < PPL / 2; ++q) {
-                            const __nv_bfloat162 c2 = as_bf2(cw[q]), s2 = as_bf2(sw[q]);
-                            // u = rs * raw + bias on both halves of each rotation pair, then
-                            // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
-                            __nv_bfloat162 u0 = __hfma2(as_bf2(rb0.w[q]), rb2, as_bf2(bB0.w[q]));
-                            __nv_bfloat162 u1 = __hfma2(as_bf2(rb1.w[q]), rb2, as_bf2(bB1.w[q]));
-                            ob0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
-                            ob1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
-                            u0 = __hfma2(as_bf2(rc0.w[q]), rc2, as_bf2(bC0.w[q]));
-                            u1 = __hfma2(as_bf2(rc1.w[q]), rc2, as_bf2(bC1.w[q]));
-                            oc0.w[q] = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
-                            oc1.w[q] = as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < PPL / 2; ++q) ob0.w[q] = ob1.w[q] = oc0.w[q] = oc1.w[q] = 0u;
-                    }
-                    sts_raw<PPL>(sm + Cfg::OB + o, ob0);
-                    sts_raw<PPL>(sm + Cfg::OB + 8192 + o, ob1);
-                    sts_raw<PPL>(sm + Cfg::OC + o, oc0);
-                    sts_raw<PPL>(sm + Cfg::OC + 8192 + o, oc1);
-                }
-            }
         }
         // H0 (bf16) as the Yo operand: row nrow, columns [32 wh, 32 wh + 32)
 #pragma unroll
@@ -630,7 +538,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             v.w = pack_bf16(hreg[8 * i + 6], hreg[8 * i + 7]);
             *reinterpret_cast<uint4*>(sm + Cfg::OH + swz128(nrow, 32 * wh + 8 * i)) = v;
         }
-        // X' = diag(dw) X
+        // X' = diag(dw) X (the XP buffer held P(c-1), read by Yd(c-1), which has finished)
         {
             uint8_t* sX = sm + (st ? Cfg::X1 : Cfg::X0);
             if (!mbar_wait(&bar_x[st], (c >> 1) & 1)) s_abort = 1;
@@ -657,11 +565,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         // ======== I2: S, dH, Yo on the tensor cores; next chunk's scalars meanwhile ========
         if (warp == 0) {
             if (elect_one()) {
-                // theta / scalar boxes of chunk c+2 reuse the buffers chunk c has finished with
-                if (c + 2 < nchunks) {
-                    issue_ts(c + 2);
-                    s_issued[1] = c + 2;
+                // theta and raw B of chunk c+1 (their buffers were read by the rotation), the
+                // scalar boxes of chunk c+2 (chunk c's slot was read by scalars(c))
+                if (c + 1 < nchunks) {
+                    issue_th(c + 1);
+                    issue_b(c + 1);
                 }
+                if (c + 2 < nchunks) issue_sc(c + 2);
                 constexpr uint32_t hi = desc_hi_sw128(1024);
                 const uint32_t loC = desc_lo(aC, 16), loB = desc_lo(aB, 16);
                 const uint32_t loBt = desc_lo(aB, 8192), loXP = desc_lo(aXP, 8192);
@@ -679,7 +589,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                     mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
                              desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
                 mma_commit(smem_u32(&bar_m1));
-                s_issued[2] = c + 1;
+                s_issued[5] = c + 1;
                 if (!mbar_wait(&bar_m1, par)) s_abort = 1;
             }
             __syncwarp();
@@ -692,11 +602,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         (void)mbar_try_wait(smem_u32(&bar_m1), par);  // completed: orders the accumulators
 
         // ======== I3: P = S o M, H1 = e^{cum_end} H0 + dH ========
-        if (warp == 0) {  // the operand buffers are free again: fetch the next chunk's B / C
-            if (elect_one() && c + 1 < nchunks) {
-                issue_bc(c + 1);
-                s_issued[4] = c + 2;
-            }
+        if (warp == 0) {  // the Cbar buffer is free again: fetch the next chunk's raw C
+            if (elect_one() && c + 1 < nchunks) issue_c(c + 1);
             __syncwarp();
         }
         {
@@ -713,7 +620,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 const float er = blk[F_EROW + t];
 #pragma unroll
                 for (int i = 0; i < NT; i += 2) {
-                    const float2 e2 = *reinterpret_cast<const float2*>(blk + F_ECOL + q4 * 64 + s0 + i);
+                    const float2 e2 = *reinterpret_cast<const float2*>(blk + F_ECOL + (q4 - 1) * 64 + s0 + i);
                     m[i] = er * e2.x;
                     m[i + 1] = er * e2.y;
                 }
@@ -737,8 +644,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
 #pragma unroll
             for (int j = 0; j < 16; j += 2)
                 pw[j / 2] = pack_bf16(sv[j] * m[j / R], sv[j + 1] * m[(j + 1) / R]);
-            *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-            *reinterpret_cast<uint4*>(sm + Cfg::OP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+            *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
         {
             const float eend = blk[F_MISC];
@@ -759,18 +666,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         __syncthreads();
         fence_after_sync();
 
-        // ======== I4: Yd = P X (waited for at the next chunk's I1) ========
+        // ======== I4: Yd = P X (waited for in the next chunk's I1) ========
         if (warp == 0) {
             if (elect_one()) {
                 constexpr uint32_t hi = desc_hi_sw128(1024);
-                const uint32_t loP = desc_lo(aP, 16);
+                const uint32_t loP = desc_lo(aXP, 16);
                 const uint32_t loX = desc_lo(smem_u32(sm + (st ? Cfg::X1 : Cfg::X0)), 8192);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tmem + T_YD, desc_pack(loP + (kmajor_off(k, 8192) >> 4), hi),
                              desc_pack(loX + (mnmajor_off(k) >> 4), hi), id_yd, k > 0);
                 mma_commit(smem_u32(&bar_m2));
-                s_issued[3] = c + 1;
+                s_issued[6] = c + 1;
             }
             __syncwarp();
         }
@@ -796,9 +703,9 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             for (int j = 0; j < 8; ++j)
                 dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
         }
-        if (p.phi1 && tg == 0) {
-#pragma unroll
-            for (int j = 0; j < PPL; ++j) p.phi1[u * kHalf + pp0 + j] = carry[j];
+        if (p.phi1 && warp == 0) {
+            p.phi1[u * kHalf + jp] = car[0];
+            p.phi1[u * kHalf + jp + 1] = car[1];
         }
         if (L > 0) {
             if (p.prevB1) {
@@ -820,10 +727,12 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         for (int k = s_issued[0] - 1; k <= s_issued[0]; ++k)
             if (k >= 0) (void)mbar_wait(&bar_x[k & 1], (k >> 1) & 1, kDrain);
         for (int k = s_issued[1] - 1; k <= s_issued[1]; ++k)
-            if (k >= 0) (void)mbar_wait(&bar_t[k & 1], (k >> 1) & 1, kDrain);
-        if (s_issued[4] > 0) (void)mbar_wait(&bar_bc, (s_issued[4] - 1) & 1, kDrain);
-        if (s_issued[2] > 0) (void)mbar_wait(&bar_m1, (s_issued[2] - 1) & 1, kDrain);
-        if (s_issued[3] > 0) (void)mbar_wait(&bar_m2, (s_issued[3] - 1) & 1, kDrain);
+            if (k >= 0) (void)mbar_wait(&bar_sc[k & 1], (k >> 1) & 1, kDrain);
+        if (s_issued[2] > 0) (void)mbar_wait(&bar_th, (s_issued[2] - 1) & 1, kDrain);
+        if (s_issued[3] > 0) (void)mbar_wait(&bar_b, (s_issued[3] - 1) & 1, kDrain);
+        if (s_issued[4] > 0) (void)mbar_wait(&bar_c, (s_issued[4] - 1) & 1, kDrain);
+        if (s_issued[5] > 0) (void)mbar_wait(&bar_m1, (s_issued[5] - 1) & 1, kDrain);
+        if (s_issued[6] > 0) (void)mbar_wait(&bar_m2, (s_issued[6] - 1) & 1, kDrain);
     }
     fence_before_sync();
     __syncthreads();
