@@ -168,15 +168,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // set-up only: the stored previous token's Bbar and x, in the H0 operand buffer
     float* s_fold = reinterpret_cast<float*>(sm + Cfg::OH);   // [R][128]
     float* s_foldx = s_fold + R * kN;                          // [R][64]
-    __shared__ uint64_t bar_x[2], bar_sc[2], bar_th, bar_b, bar_c, bar_m1, bar_m2;
+    __shared__ uint64_t bar_x[2], bar_sc[2], bar_th, bar_b, bar_c, bar_yo, bar_s, bar_dh, bar_m2;
     __shared__ uint32_t tslot;
     __shared__ int s_abort;
     // async work thread 0 has started, for draining it if a wait gives up: last X and scalar
-    // box chunk issued; theta, raw B, raw C loads issued; MMA groups m1, m2 committed
+    // box chunk issued; theta, raw B, raw C loads issued; MMA groups (Yo, S, dH) and Yd committed
     __shared__ int s_issued[7];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q4 = warp & 3, wh = warp >> 2;  // TMEM subpartition, column half
+    // One elected lane of this warp issues every TMA copy and MMA: its share of the masking
+    // (row block 0, column blocks 1 and 3) is all zeros.
+    constexpr int kIssueWarp = 4;
     const int64_t u = blockIdx.x;
     const int64_t bb = u / p.H, hh = u % p.H, g = hh / (p.H / p.G);
     const int hc = static_cast<int>(hh & 3);  // column of this head in the scalar boxes
@@ -296,7 +299,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     };
 
     // ---------------- setup ----------------
-    if (tid == 0) {
+    if (tid == kIssueWarp * 32) {
         mbar_init(&bar_x[0], 1);
         mbar_init(&bar_x[1], 1);
         mbar_init(&bar_sc[0], 1);
@@ -304,7 +307,9 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         mbar_init(&bar_th, 1);
         mbar_init(&bar_b, 1);
         mbar_init(&bar_c, 1);
-        mbar_init(&bar_m1, 1);
+        mbar_init(&bar_yo, 1);
+        mbar_init(&bar_s, 1);
+        mbar_init(&bar_dh, 1);
         mbar_init(&bar_m2, 1);
         fence_mbar_init();
         s_abort = 0;
@@ -430,8 +435,22 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     };
 
+    // H0 (bf16) as the Yo operand: row nrow, columns [32 wh, 32 wh + 32)
+    auto store_h0 = [&]() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint4 v;
+            v.x = pack_bf16(hreg[8 * i + 0], hreg[8 * i + 1]);
+            v.y = pack_bf16(hreg[8 * i + 2], hreg[8 * i + 3]);
+            v.z = pack_bf16(hreg[8 * i + 4], hreg[8 * i + 5]);
+            v.w = pack_bf16(hreg[8 * i + 6], hreg[8 * i + 7]);
+            *reinterpret_cast<uint4*>(sm + Cfg::OH + swz128(nrow, 32 * wh + 8 * i)) = v;
+        }
+    };
+
     if (nchunks > 0 && warp == 1) scalars(0);
-    __syncthreads();
+    __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
+    store_h0();
 
     for (int c = 0; c < nchunks && !s_abort; ++c) {
         const int st = c & 1;
@@ -516,7 +535,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             }
         }
         // Yd(c-1) done: its X buffer takes X(c+1), and y(c-1) can be written
-        if (warp == 0) {
+        if (warp == kIssueWarp) {
             if (elect_one()) {
                 if (c > 0 && !mbar_wait(&bar_m2, (c - 1) & 1)) s_abort = 1;
                 if (c + 1 < nchunks) issue_x(c + 1);
@@ -527,16 +546,6 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             (void)mbar_wait(&bar_m2, (c - 1) & 1);
             fence_after_sync();
             epilogue(c - 1);
-        }
-        // H0 (bf16) as the Yo operand: row nrow, columns [32 wh, 32 wh + 32)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 v;
-            v.x = pack_bf16(hreg[8 * i + 0], hreg[8 * i + 1]);
-            v.y = pack_bf16(hreg[8 * i + 2], hreg[8 * i + 3]);
-            v.z = pack_bf16(hreg[8 * i + 4], hreg[8 * i + 5]);
-            v.w = pack_bf16(hreg[8 * i + 6], hreg[8 * i + 7]);
-            *reinterpret_cast<uint4*>(sm + Cfg::OH + swz128(nrow, 32 * wh + 8 * i)) = v;
         }
         // X' = diag(dw) X (the XP buffer held P(c-1), read by Yd(c-1), which has finished)
         {
@@ -562,8 +571,9 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         fence_after_sync();
         if (s_abort) break;
 
-        // ======== I2: S, dH, Yo on the tensor cores; next chunk's scalars meanwhile ========
-        if (warp == 0) {
+        // ======== I2: Yo, S, dH on the tensor cores; P = S o M and H1 = e^{cum_end} H0 + dH
+        // as their accumulators land; the next chunk's scalars meanwhile ========
+        if (warp == kIssueWarp) {
             if (elect_one()) {
                 // theta and raw B of chunk c+1 (their buffers were read by the rotation), the
                 // scalar boxes of chunk c+2 (chunk c's slot was read by scalars(c))
@@ -578,37 +588,30 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 const uint32_t loH = desc_lo(aH, 16384);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
+                    mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
+                             desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
+                mma_commit(smem_u32(&bar_yo));
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
                     mma_bf16(tmem + T_S, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
                              desc_pack(loB + (kmajor_off(k, 8192) >> 4), hi), id_s, k > 0);
+                mma_commit(smem_u32(&bar_s));
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16(tmem + T_DH, desc_pack(loBt + (mnmajor_off(k) >> 4), hi),
                              desc_pack(loXP + (mnmajor_off(k) >> 4), hi), id_dh, k > 0);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
-                             desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
-                mma_commit(smem_u32(&bar_m1));
+                mma_commit(smem_u32(&bar_dh));
                 s_issued[5] = c + 1;
-                if (!mbar_wait(&bar_m1, par)) s_abort = 1;
+                // Yo and S were the readers of Cbar: fetch the next chunk's raw C in its place
+                if (c + 1 < nchunks) {
+                    if (!mbar_wait(&bar_s, par)) s_abort = 1;
+                    issue_c(c + 1);
+                }
             }
             __syncwarp();
         }
         if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (s_abort) break;
-        (void)mbar_try_wait(smem_u32(&bar_m1), par);  // completed: orders the accumulators
-
-        // ======== I3: P = S o M, H1 = e^{cum_end} H0 + dH ========
-        if (warp == 0) {  // the Cbar buffer is free again: fetch the next chunk's raw C
-            if (elect_one() && c + 1 < nchunks) issue_c(c + 1);
-            __syncwarp();
-        }
         {
-            float sv[16];
-            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, sv);
             const int trow = 16 * q4 + (lane & 15);   // row block q4
             const int qc = wh + ((lane >> 4) ? 2 : 0);  // column block of this half-warp
             const int col0 = 16 * qc;
@@ -639,11 +642,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
 #pragma unroll
                 for (int i = 0; i < NT; ++i) m[i] = 0.f;
             }
+            if (!mbar_wait(&bar_s, par)) s_abort = 1;
+            fence_after_sync();
+            float sv[16];
+            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, sv);
             tmem_wait_ld();
             uint32_t pw[8];
 #pragma unroll
             for (int j = 0; j < 16; j += 2)
                 pw[j / 2] = pack_bf16(sv[j] * m[j / R], sv[j + 1] * m[(j + 1) / R]);
+            // dH has read X': P takes its buffer
+            if (!mbar_wait(&bar_dh, par)) s_abort = 1;
+            fence_after_sync();
             *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
             *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
@@ -660,14 +670,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
             }
         }
+        // Yo(c) has read H0: the next chunk's H0 operand
+        if (!mbar_wait(&bar_yo, par)) s_abort = 1;
+        store_h0();
 
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
+        if (s_abort) break;
 
         // ======== I4: Yd = P X (waited for in the next chunk's I1) ========
-        if (warp == 0) {
+        if (warp == kIssueWarp) {
             if (elect_one()) {
                 constexpr uint32_t hi = desc_hi_sw128(1024);
                 const uint32_t loP = desc_lo(aXP, 16);
@@ -684,7 +698,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     }
     // ---- epilogue of the last chunk ----
     if (nchunks > 0 && !s_abort) {
-        if (tid == 0 && !mbar_wait(&bar_m2, (nchunks - 1) & 1)) s_abort = 1;  // lane 0 of warp 0
+        if (tid == 0 && !mbar_wait(&bar_m2, (nchunks - 1) & 1)) s_abort = 1;
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
@@ -731,7 +745,11 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         if (s_issued[2] > 0) (void)mbar_wait(&bar_th, (s_issued[2] - 1) & 1, kDrain);
         if (s_issued[3] > 0) (void)mbar_wait(&bar_b, (s_issued[3] - 1) & 1, kDrain);
         if (s_issued[4] > 0) (void)mbar_wait(&bar_c, (s_issued[4] - 1) & 1, kDrain);
-        if (s_issued[5] > 0) (void)mbar_wait(&bar_m1, (s_issued[5] - 1) & 1, kDrain);
+        if (s_issued[5] > 0) {
+            (void)mbar_wait(&bar_yo, (s_issued[5] - 1) & 1, kDrain);
+            (void)mbar_wait(&bar_s, (s_issued[5] - 1) & 1, kDrain);
+            (void)mbar_wait(&bar_dh, (s_issued[5] - 1) & 1, kDrain);
+        }
         if (s_issued[6] > 0) (void)mbar_wait(&bar_m2, (s_issued[6] - 1) & 1, kDrain);
     }
     fence_before_sync();
