@@ -26,7 +26,9 @@ sys.path.insert(0, ROOT)
 METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roofline"
 # DRAM bytes (read + write) of one scan launch on this workload from the ncu capture
 # summarised in profiles/scan_tc_siso_prefill_b4_L2048.md; None once the kernel changes.
-SCAN_TRAFFIC_BYTES = None
+SCAN_TRAFFIC_BYTES = 186.9e6
+# kernels one scan launches: the per-token RMS-scale pre-pass of B and C, then the scan
+KERNELS_PER_SCAN = 2
 WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"
 
 
@@ -44,6 +46,26 @@ def parse():
 def dist_env():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
             int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def max_over_ranks(ms, world, dist, device):
+    """The slowest rank's time (every rank calls this at the same point of the run)."""
+    if world == 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_throughput(units_per_rank, world, steps, total_ms):
+    """Whole-job rate when every rank processes its own units_per_rank per step."""
+    return units_per_rank * world * steps / (total_ms / 1e3)
+
+
+def rank_seed(rank, i):
+    """Seed of input set i on a rank: every rank draws its own independent sequences."""
+    return 1 + 100 * rank + i
 
 
 def peaks():
@@ -137,7 +159,7 @@ def run_ours(args):
 
     # two input sets (each > L2) alternate between steps so no step reads the previous
     # step's inputs from L2
-    sets = [make_config(1, device=dev, seed=1 + 100 * rank + i) for i in range(2)]
+    sets = [make_config(1, device=dev, seed=rank_seed(rank, i)) for i in range(2)]
     d = sets[0].dims
     y = torch.empty_like(sets[0].x)
     fin = m3.State.empty(d.batch, d.nheads, d.dstate, d.headdim, d.rank, d.dtype, dev)
@@ -166,14 +188,10 @@ def run_ours(args):
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
     m3.scan_check(ws)
-    total_ms = ev[0].elapsed_time(ev[-1])
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), world, dist, dev)
     per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     tokens = d.batch * d.seqlen
-    value = tokens * world * args.steps / (total_ms / 1e3)
+    value = weak_throughput(tokens, world, args.steps, total_ms)
     byts = scan_bytes(sets[0])
     launch_ms = sum(per_launch) / len(per_launch)
     achieved = byts / (launch_ms / 1e3) / 1e9
@@ -205,12 +223,8 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = tokens * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
+    e2e_val = weak_throughput(tokens, world, e2e_steps, e2e_ms)
     del host, dev_in, y_host
 
     # ---- decode: 1000 consecutive steps in one CUDA graph, SISO and MIMO R=4 ----
@@ -234,7 +248,7 @@ def run_ours(args):
                      "peak_source": peak_kind},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * KERNELS_PER_SCAN,
         "clocks": clk.summary(),
         "decode": decode,
     }
@@ -275,11 +289,7 @@ def bench_decode(m3, dev, R, steps, hbm, world, dist):
         g.replay()
         e1.record(s)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
     us = ms * 1e3 / steps
     units = pr.dims.batch * pr.dims.nheads
     es = 2
@@ -293,20 +303,22 @@ def bench_decode(m3, dev, R, steps, hbm, world, dist):
             "achieved_gbs": ach, "frac_hbm": ach / hbm, "gpu_launches": steps}
 
 
-def cpu_baseline(pr):
-    """The fp64 oracle as it stands, on all host cores, on one of the workload's sequences
-    (batch 0, all heads, full length)."""
+def cpu_baseline(pr, min_s=10.0, max_reps=30):
+    """The fp64 oracle as it stands, on all host cores, on the whole workload (every sequence,
+    head and token), repeated until about min_s seconds of CPU work have been timed."""
     import oracle
-    t = {k: (v[:1].cpu() if (v is not None and k not in ("B_bias", "C_bias")) else
-             (v.cpu() if v is not None else None)) for k, v in pr.tensors().items()}
+    t = {k: (v.cpu() if v is not None else None) for k, v in pr.tensors().items()}
     cores = oracle.max_threads()
-    t0 = time.perf_counter()
-    oracle.scan(**t, bc_norm=True, nthreads=cores)
-    dt = time.perf_counter() - t0
-    tokens = t["x"].shape[1]
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"1 of {pr.dims.batch} sequences (all {pr.dims.nheads} heads, "
-                      f"L={pr.dims.seqlen}), {dt:.2f} s"}
+    reps, el = 0, 0.0
+    while reps < max_reps and (reps == 0 or el < min_s):
+        t0 = time.perf_counter()
+        oracle.scan(**t, bc_norm=True, nthreads=cores)
+        el += time.perf_counter() - t0
+        reps += 1
+    tokens = t["x"].shape[0] * t["x"].shape[1] * reps
+    return {"value": tokens / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"the whole workload ({pr.dims.batch} sequences x {pr.dims.nheads} heads x "
+                      f"L={pr.dims.seqlen}) x {reps} passes, {el:.1f} s"}
 
 
 def run_reference(args):

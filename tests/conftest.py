@@ -19,3 +19,13 @@ def cuda_dev():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With M3_PARITY_REPORT set, write the errors of every GPU comparison to that file."""
+    path = os.environ.get("M3_PARITY_REPORT")
+    gc = sys.modules.get("gpu_common")
+    if path and gc is not None and gc.ERRORS:
+        import json
+        with open(path, "w") as f:
+            json.dump(gc.ERRORS, f, indent=1, sort_keys=True)

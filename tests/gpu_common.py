@@ -4,6 +4,8 @@ stored inputs and compare them with the tolerances of the workloads.
 Tolerance rule: err = max|gpu - oracle| / max|oracle| per output tensor (y, and each field of
 the final state), at most 1e-4 for fp32 inputs and 2e-2 for bf16 inputs with fp32 state.
 """
+import os
+
 import numpy as np
 import torch
 
@@ -11,6 +13,15 @@ import oracle
 from state_space_sequence_mamba_b200 import binding as m3
 
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
+
+# errors measured by every comparison of the run, by test id; written out at the end of the
+# session when M3_PARITY_REPORT names a file (see conftest.py)
+ERRORS: dict = {}
+
+
+def record(errs: dict) -> None:
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    ERRORS.setdefault(test, []).append({k: float(v) for k, v in errs.items()})
 
 
 def rel(g, o) -> float:
@@ -64,6 +75,7 @@ def compare(pr, y, fin, yo, so, heads=None, tol=None):
         errs["prev_B"] = rel(fin.prev_B[:, hs], so.prev_B)
         errs["prev_x"] = rel(fin.prev_x[:, hs], so.prev_x)
         assert errs["prev_B"] == 0.0 and errs["prev_x"] == 0.0, errs
+    record(errs)
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, f"errors above {tol}: {errs}"
     return errs

@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_common import TOL, compare, gpu_scan, oracle_scan, oracle_state, rel
+from gpu_common import TOL, compare, gpu_scan, oracle_scan, oracle_state, record, rel
 from state_space_sequence_mamba_b200 import binding as m3
 from state_space_sequence_mamba_b200.inputs import make_config, make_decode, make_problem
 
@@ -218,5 +218,6 @@ def test_config3_decode_1000_steps_sampled_units(cuda_dev, R):
     e_y = rel(ys, yo)
     e_h = rel(st.h[b_i][:, h_i], so.h)
     e_phi = rel(st.phi[b_i][:, h_i], so.phi)
+    record({"y": e_y, "h": e_h, "phi": e_phi})
     assert e_y <= TOL[torch.bfloat16] and e_h <= TOL[torch.bfloat16] and e_phi <= 2e-2, \
         (e_y, e_h, e_phi)
