@@ -177,16 +177,20 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
         const float al = expf(d * a), be = (1.f - lm) * d * al, ga = lm * d;
 
         // ---- RMS scales of B, C and the stored previous B, one warp per vector ----
-        for (int v = warp; v < 3 * R; v += kWarps) {
-            const __nv_bfloat16* src = (v < R) ? sB + v * N : (v < 2 * R) ? sC + (v - R) * N
-                                                                         : sBp + (v - 2 * R) * N;
-            float ss = 0.f;
-            for (int n = lane; n < N; n += 32) {
-                const float f = __bfloat162float(src[n]);
-                ss = fmaf(f, f, ss);
+        if (p.bc_norm) {
+            for (int v = warp; v < 3 * R; v += kWarps) {
+                const __nv_bfloat16* src = (v < R) ? sB + v * N : (v < 2 * R) ? sC + (v - R) * N
+                                                                             : sBp + (v - 2 * R) * N;
+                float ss = 0.f;
+                for (int n = 2 * lane; n < N; n += 64) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(src + n));
+                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+                ss = warp_sum(ss);
+                if (lane == 0) rs[v] = rsqrtf(ss / static_cast<float>(N) + p.eps);
             }
-            ss = warp_sum(ss);
-            if (lane == 0) rs[v] = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
+        } else if (tid < 3 * R) {
+            rs[tid] = 1.f;
         }
         __syncthreads();
         // ---- angles and rotations, pair i = (i, i + N/2); vectors stored [n][R] ----
@@ -196,43 +200,42 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
             const float* bC = p.Cbias ? p.Cbias + hh * R * N : nullptr;
             const __nv_bfloat16* sth = reinterpret_cast<const __nv_bfloat16*>(base + bl.th);
             const float* sphi = reinterpret_cast<const float*>(base + bl.phi);
-            // threads [0, half) rotate by the new angle (B, C), [half, 2 half) by the old (prev B)
-            for (int k = tid; k < 2 * half; k += kThreads) {
+            // items (k, r): k in [0, half) rotates B and C of rank r by the new angle, k in
+            // [half, 2 half) the stored previous B by the old one
+            for (int it = tid; it < 2 * half * R; it += kThreads) {
+                const int k = it / R, r = it - k * R;
                 const bool cur = k < half;
                 const int i = cur ? k : k - half;
                 const float ph_old = sphi[i];
                 const float ph = cur ? ph_old + d * __bfloat162float(sth[i]) : ph_old;
                 float sn, cn;
                 __sincosf(reduce_turns(ph), &sn, &cn);
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    const int a0 = r * N + i, a1 = a0 + half;
-                    const int o0 = i * R + r, o1 = (i + half) * R + r;
-                    if (cur) {
-                        float u0 = fmaf(__bfloat162float(sB[a0]), rs[r], bB ? bB[a0] : 0.f);
-                        float u1 = fmaf(__bfloat162float(sB[a1]), rs[r], bB ? bB[a1] : 0.f);
-                        vB[o0] = ga * (u0 * cn + u1 * sn);
-                        vB[o1] = ga * (u1 * cn - u0 * sn);
-                        u0 = fmaf(__bfloat162float(sC[a0]), rs[R + r], bC ? bC[a0] : 0.f);
-                        u1 = fmaf(__bfloat162float(sC[a1]), rs[R + r], bC ? bC[a1] : 0.f);
-                        cC[o0] = u0 * cn + u1 * sn;
-                        cC[o1] = u1 * cn - u0 * sn;
-                    } else {
-                        const float u0 = fmaf(__bfloat162float(sBp[a0]), rs[2 * R + r], bB ? bB[a0] : 0.f);
-                        const float u1 = fmaf(__bfloat162float(sBp[a1]), rs[2 * R + r], bB ? bB[a1] : 0.f);
-                        vBp[o0] = be * (u0 * cn + u1 * sn);
-                        vBp[o1] = be * (u1 * cn - u0 * sn);
-                    }
+                const int a0 = r * N + i, a1 = a0 + half;
+                const int o0 = i * R + r, o1 = (i + half) * R + r;
+                if (cur) {
+                    float u0 = fmaf(__bfloat162float(sB[a0]), rs[r], bB ? bB[a0] : 0.f);
+                    float u1 = fmaf(__bfloat162float(sB[a1]), rs[r], bB ? bB[a1] : 0.f);
+                    vB[o0] = ga * (u0 * cn + u1 * sn);
+                    vB[o1] = ga * (u1 * cn - u0 * sn);
+                    u0 = fmaf(__bfloat162float(sC[a0]), rs[R + r], bC ? bC[a0] : 0.f);
+                    u1 = fmaf(__bfloat162float(sC[a1]), rs[R + r], bC ? bC[a1] : 0.f);
+                    cC[o0] = u0 * cn + u1 * sn;
+                    cC[o1] = u1 * cn - u0 * sn;
+                    if (r == 0) phin[i] = ph;
+                } else {
+                    const float u0 = fmaf(__bfloat162float(sBp[a0]), rs[2 * R + r], bB ? bB[a0] : 0.f);
+                    const float u1 = fmaf(__bfloat162float(sBp[a1]), rs[2 * R + r], bB ? bB[a1] : 0.f);
+                    vBp[o0] = be * (u0 * cn + u1 * sn);
+                    vBp[o1] = be * (u1 * cn - u0 * sn);
                 }
-                if (cur) phin[i] = ph;
             }
         }
         __syncthreads();
 
         // ---- state update in place and readout ----
-        float yacc[R][4];
+        float2 y01[R], y23[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) yacc[r][0] = yacc[r][1] = yacc[r][2] = yacc[r][3] = 0.f;
+        for (int r = 0; r < R; ++r) y01[r] = y23[r] = make_float2(0.f, 0.f);
         {
             const __nv_bfloat16* sx = reinterpret_cast<const __nv_bfloat16*>(base + bl.x);
             const __nv_bfloat16* sxp = reinterpret_cast<const __nv_bfloat16*>(base + bl.xp);
@@ -260,27 +263,36 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
                     o[0] = v[n];
                 }
             };
+            // packed fp32 pairs (fma.rn.f32x2): columns (4 pc, 4 pc + 1) and (4 pc + 2, 4 pc + 3)
+            float2 x01[R], x23[R], xp01[R], xp23[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                x01[r] = make_float2(xv[r].x, xv[r].y);
+                x23[r] = make_float2(xv[r].z, xv[r].w);
+                xp01[r] = make_float2(xpv[r].x, xpv[r].y);
+                xp23[r] = make_float2(xpv[r].z, xpv[r].w);
+            }
+            const float2 al2 = make_float2(al, al);
             auto update = [&](int n) {
                 float a2[R], c2[R], cc[R];
                 row_vals(vBp, n, a2);
                 row_vals(vB, n, c2);
                 row_vals(cC, n, cc);
-                float4 h = hs[n * PV + pc];
-                h.x *= al; h.y *= al; h.z *= al; h.w *= al;
+                const float4 h = hs[n * PV + pc];
+                float2 h01 = __fmul2_rn(make_float2(h.x, h.y), al2);
+                float2 h23 = __fmul2_rn(make_float2(h.z, h.w), al2);
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    h.x = fmaf(a2[r], xpv[r].x, fmaf(c2[r], xv[r].x, h.x));
-                    h.y = fmaf(a2[r], xpv[r].y, fmaf(c2[r], xv[r].y, h.y));
-                    h.z = fmaf(a2[r], xpv[r].z, fmaf(c2[r], xv[r].z, h.z));
-                    h.w = fmaf(a2[r], xpv[r].w, fmaf(c2[r], xv[r].w, h.w));
+                    const float2 cr = make_float2(c2[r], c2[r]), ar = make_float2(a2[r], a2[r]);
+                    h01 = __ffma2_rn(ar, xp01[r], __ffma2_rn(cr, x01[r], h01));
+                    h23 = __ffma2_rn(ar, xp23[r], __ffma2_rn(cr, x23[r], h23));
                 }
-                hs[n * PV + pc] = h;
+                hs[n * PV + pc] = make_float4(h01.x, h01.y, h23.x, h23.y);
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    yacc[r][0] = fmaf(h.x, cc[r], yacc[r][0]);
-                    yacc[r][1] = fmaf(h.y, cc[r], yacc[r][1]);
-                    yacc[r][2] = fmaf(h.z, cc[r], yacc[r][2]);
-                    yacc[r][3] = fmaf(h.w, cc[r], yacc[r][3]);
+                    const float2 c = make_float2(cc[r], cc[r]);
+                    y01[r] = __ffma2_rn(h01, c, y01[r]);
+                    y23[r] = __ffma2_rn(h23, c, y23[r]);
                 }
             };
             int n = r0;
@@ -291,6 +303,11 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
             for (; n < N; n += RP) update(n);
         }
         fence_proxy_async();  // the updated state is read by the bulk store
+        float yacc[R][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            yacc[r][0] = y01[r].x; yacc[r][1] = y01[r].y; yacc[r][2] = y23[r].x; yacc[r][3] = y23[r].y;
+        }
         // partial outputs: lanes sharing a column group differ in the bits above log2(PV)
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) {
@@ -324,8 +341,10 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
             const __nv_bfloat16* sx = reinterpret_cast<const __nv_bfloat16*>(base + bl.x);
             __nv_bfloat16* pb1 = static_cast<__nv_bfloat16*>(p.prevB1) + static_cast<int64_t>(u) * R * N;
             __nv_bfloat16* px1 = static_cast<__nv_bfloat16*>(p.prevx1) + static_cast<int64_t>(u) * R * P;
-            for (int e = tid; e < R * N; e += kThreads) pb1[e] = sB[e];
-            for (int e = tid; e < R * P; e += kThreads) px1[e] = sx[e];
+            for (int e = tid; e < R * N / 8; e += kThreads)
+                reinterpret_cast<uint4*>(pb1)[e] = reinterpret_cast<const uint4*>(sB)[e];
+            for (int e = tid; e < R * P / 8; e += kThreads)
+                reinterpret_cast<uint4*>(px1)[e] = reinterpret_cast<const uint4*>(sx)[e];
         }
         if (tid == 0) {
             sc[4 * (b ^ 1) + 0] = snext[0];
