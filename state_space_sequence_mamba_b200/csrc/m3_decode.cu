@@ -248,6 +248,7 @@ static cudaError_t launch_decode_t(const ScanParams& p, cudaStream_t s) {
 
 cudaError_t launch_decode(const ScanParams& p, bool bf16, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
+    if (decode_tc_supported(p, bf16)) return launch_decode_tc(p, s);
     if (decode_bulk_supported(p, bf16)) return launch_decode_bulk(p, s);
     switch (p.R) {
         case 1: return bf16 ? launch_decode_t<1, __nv_bfloat16>(p, s) : launch_decode_t<1, float>(p, s);

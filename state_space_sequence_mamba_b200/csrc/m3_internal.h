@@ -54,6 +54,9 @@ m3_status set_error(m3_status s, const char* msg);
 bool decode_bulk_supported(const ScanParams& p, bool bf16);
 size_t decode_bulk_smem_bytes(const ScanParams& p);
 cudaError_t launch_decode_bulk(const ScanParams& p, cudaStream_t s);
+// Decode with the rank-2R update and the readout on the tensor cores (bf16, N = 128, P = 64).
+bool decode_tc_supported(const ScanParams& p, bool bf16);
+cudaError_t launch_decode_tc(const ScanParams& p, cudaStream_t s);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 
