@@ -24,6 +24,7 @@
 // state lives in registers (row n of the state in lane n of the TMEM datapath, matching the
 // dH accumulator) and is rounded to bf16 only as the Yo operand. All waits are bounded; a
 // timeout sets the status word and the CTA exits cleanly.
+#include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -78,6 +79,9 @@ constexpr int F_SEG = 2 * F_BLK;           // [8 segments][32 lanes] float2
 constexpr int F_BIAS = F_SEG + 512;        // bias_B [R][128] bf16, bias_C [R][128] bf16
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
+// One segment's end state in the workspace (floats): h [N][P], the angle [N/2], the segment's
+// summed log-decay, padding to a multiple of 16 bytes.
+constexpr int kSegStride = kN * kP + kHalf + 4;
 
 template <int R>
 __host__ __device__ constexpr uint32_t tc_smem_bytes() {
@@ -152,9 +156,22 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
     }
 }
 
-template <int R>
+// The sequence-parallel form for few long sequences: the sequence of every unit is cut into
+// nseg segments of seg_chunks chunks (the last may be shorter). A state-only pass computes each
+// segment's end state but the last's; the full pass then runs every segment at once from the
+// state at its start, which it assembles from those end states. nseg = 1 is the plain scan.
+struct SegArgs {
+    int seg_chunks, nseg;
+    float* st;   // [units][nseg - 1][kSegStride]
+};
+
+// One CTA per (unit, segment), CTA index = segment * units + unit. kStateOnly: the segment's
+// end state only (no C, S, Yo, Yd, y); segment 0 starts from the given initial state in the
+// true angle frame, later segments from zero in their own frame (angle 0 at their start).
+template <int R, bool kStateOnly>
 __global__ void __launch_bounds__(kTcThreads, 2)
-scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow) {
+scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow,
+               const SegArgs sa) {
     using Cfg = TcCfg<R>;
     constexpr int Q = Cfg::Q, TPS = Cfg::TPS;
 
@@ -180,7 +197,9 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // One elected lane of this warp issues every TMA copy and MMA: its share of the masking
     // (row block 0, column blocks 1 and 3) is all zeros.
     constexpr int kIssueWarp = 4;
-    const int64_t u = blockIdx.x;
+    const int units32 = static_cast<int>(p.b * p.H);   // < 2^31 (one CTA per unit and segment)
+    const int kseg = static_cast<int>(blockIdx.x) / units32;
+    const int64_t u = static_cast<int>(blockIdx.x) - kseg * units32;
     const int64_t bb = u / p.H, hh = u % p.H, g = hh / (p.H / p.G);
     const int hc = static_cast<int>(hh & 3);  // column of this head in the scalar boxes
     const int L = static_cast<int>(p.L);
@@ -192,7 +211,9 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     const __nv_bfloat16* xu = static_cast<const __nv_bfloat16*>(p.x) + (bb * p.L * H + hh) * R * kP;
     __nv_bfloat16* yu = static_cast<__nv_bfloat16*>(p.y) + (bb * p.L * H + hh) * R * kP;
     const int tokB = G * R * kN, tokY = H * R * kP;  // element stride of one token
-    const int nchunks = (L + Q - 1) / Q;
+    // this segment's chunks: global chunks [cb, cb + nchunks); c below is the local index
+    const int cb = kseg * sa.seg_chunks;
+    const int nchunks = min((L + Q - 1) / Q - cb, sa.seg_chunks);
     const int ib = static_cast<int>(bb), ih = static_cast<int>(hh), ig = static_cast<int>(g);
     uint2* s_rs = reinterpret_cast<uint2*>(sm + Cfg::ORS);
 
@@ -200,7 +221,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     auto issue_x = [&](int c) {
         const int st = c & 1;
         mbar_arrive_expect_tx(&bar_x[st], Cfg::X_TX);
-        tma_load_5d(sm + (st ? Cfg::X1 : Cfg::X0), &maps.x, &bar_x[st], 0, 0, ih, c * Q, ib);
+        tma_load_5d(sm + (st ? Cfg::X1 : Cfg::X0), &maps.x, &bar_x[st], 0, 0, ih, (cb + c) * Q, ib);
         s_issued[0] = c;
     };
     auto issue_sc = [&](int c) {  // dt, A, lam boxes of chunk c (4 heads, Q + 1 tokens)
@@ -208,30 +229,32 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         mbar_arrive_expect_tx(&bar_sc[st], Cfg::SC_TX);
         uint8_t* sc = sm + (st ? Cfg::SC1 : Cfg::SC0);
         const int h4 = ih & ~3;
-        tma_load_3d(sc, &maps.dt, &bar_sc[st], h4, c * Q, ib);
-        tma_load_3d(sc + Cfg::SC_SLOT, &maps.A, &bar_sc[st], h4, c * Q, ib);
-        tma_load_3d(sc + 2 * Cfg::SC_SLOT, &maps.lam, &bar_sc[st], h4, c * Q, ib);
+        tma_load_3d(sc, &maps.dt, &bar_sc[st], h4, (cb + c) * Q, ib);
+        tma_load_3d(sc + Cfg::SC_SLOT, &maps.A, &bar_sc[st], h4, (cb + c) * Q, ib);
+        tma_load_3d(sc + 2 * Cfg::SC_SLOT, &maps.lam, &bar_sc[st], h4, (cb + c) * Q, ib);
         s_issued[1] = c;
     };
     auto issue_th = [&](int c) {  // theta of chunk c into the (single) theta buffer
         mbar_arrive_expect_tx(&bar_th, Cfg::TH_TX);
-        tma_load_4d(sm + Cfg::TH, &maps.theta, &bar_th, 0, ih, c * Q, ib);
+        tma_load_4d(sm + Cfg::TH, &maps.theta, &bar_th, 0, ih, (cb + c) * Q, ib);
         s_issued[2] += 1;
     };
     auto issue_b = [&](int c) {   // raw B rows of chunk c (two 64-column slabs) + RMS scales
         mbar_arrive_expect_tx(&bar_b, Cfg::B_TX + (rsu ? 512u : 0u));
-        tma_load_5d(sm + Cfg::RB, &maps.B, &bar_b, 0, 0, ig, c * Q, ib);
-        tma_load_5d(sm + Cfg::RB + 8192, &maps.B, &bar_b, kHalf, 0, ig, c * Q, ib);
-        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(c) * Q * R, 512u, &bar_b);
+        tma_load_5d(sm + Cfg::RB, &maps.B, &bar_b, 0, 0, ig, (cb + c) * Q, ib);
+        tma_load_5d(sm + Cfg::RB + 8192, &maps.B, &bar_b, kHalf, 0, ig, (cb + c) * Q, ib);
+        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(cb + c) * Q * R, 512u, &bar_b);
         s_issued[3] += 1;
     };
     auto issue_c = [&](int c) {   // raw C rows of chunk c straight into the Cbar operand buffer
         mbar_arrive_expect_tx(&bar_c, Cfg::C_TX);
-        tma_load_5d(sm + Cfg::OC, &maps.C, &bar_c, 0, 0, ig, c * Q, ib);
-        tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_c, kHalf, 0, ig, c * Q, ib);
+        tma_load_5d(sm + Cfg::OC, &maps.C, &bar_c, 0, 0, ig, (cb + c) * Q, ib);
+        tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_c, kHalf, 0, ig, (cb + c) * Q, ib);
         s_issued[4] += 1;
     };
-    // Chunk scalars (one full warp): cumulative log-decay, gamma, trapezoid weight w, ...
+    // Chunk scalars (one full warp): cumulative log-decay, gamma, trapezoid weight w, ...; the
+    // segment's summed log-decay accumulates in lam_acc
+    float lam_acc = 0.f;
     auto scalars = [&](int c) {
         const int st = c & 1;
         if (!mbar_wait(&bar_sc[st], (c >> 1) & 1)) {
@@ -239,7 +262,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
         const float* sSc = reinterpret_cast<const float*>(sm + (st ? Cfg::SC1 : Cfg::SC0));
         float* blk = sf + st * F_BLK;
-        const int T = (L - c * Q) < Q ? (L - c * Q) : Q;
+        const int T = (L - (cb + c) * Q) < Q ? (L - (cb + c) * Q) : Q;
         constexpr int oA = Cfg::SC_SLOT / 4, oL = 2 * Cfg::SC_SLOT / 4;
         float a[2], d[2], ga[2], w[2];
 #pragma unroll
@@ -259,6 +282,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         const float tot0 = __shfl_sync(0xffffffffu, c0s, 31);
         const float c1s = warp_inclusive_scan(a[1]) + tot0;
         const float cum_end = __shfl_sync(0xffffffffu, (T - 1) < 32 ? c0s : c1s, (T - 1) & 31);
+        if constexpr (kStateOnly) lam_acc += cum_end;
         constexpr float kLog2e = 1.4426950408889634f;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
@@ -320,7 +344,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             issue_sc(0);
             issue_th(0);
             issue_b(0);
-            issue_c(0);
+            if constexpr (!kStateOnly) issue_c(0);
         }
         if (nchunks > 1) issue_sc(1);
     }
@@ -337,7 +361,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // state rows owned by this thread: n = 32*q4 + lane, columns [32*wh, 32*wh + 32)
     const int nrow = 32 * q4 + lane;
     float hreg[32];
-    if (p.h0) {
+    if (kseg == 0 && p.h0) {
         const float4* src = reinterpret_cast<const float4*>(p.h0 + (u * kN + nrow) * kP + 32 * wh);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -358,12 +382,12 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     float car[2], car_r[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        car[j] = p.phi0 ? p.phi0[u * kHalf + jp + j] : 0.f;
+        car[j] = (kseg == 0 && p.phi0) ? p.phi0[u * kHalf + jp + j] : 0.f;
         car_r[j] = reduce_2pi(car[j]);
     }
 
     // ---- fold the stored previous token into the primed state ----
-    if (p.h0 && L > 0) {
+    if (kseg == 0 && p.h0 && L > 0) {
         const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(p.prevB0) + u * R * kN;
         const __nv_bfloat16* px = static_cast<const __nv_bfloat16*>(p.prevx0) + u * R * kP;
         if (warp < R) {  // RMS scale of the stored raw B, one warp per rank
@@ -401,6 +425,61 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     }
 
+    // ---- the state at the start of a later segment (full pass) ----
+    // Segment 0's end state is in the true frame. Each later segment j < kseg adds its own
+    // contribution dH_j, computed from zero in its own frame, after decaying the state by its
+    // summed log-decay Lambda_j and rotating dH_j by the angle phi_j at its start:
+    //     h <- e^{Lambda_j} h + R(-phi_j) dH_j,   phi_{j+1} = phi_j + (segment j's angle sum).
+    // The states at segment boundaries are primed (they hold the next token's beta term, as at
+    // every chunk boundary), so no previous token is folded here.
+    if constexpr (!kStateOnly) {
+        if (kseg > 0) {
+            const float* sb = sa.st + u * (sa.nseg - 1) * kSegStride;
+            float* s_phis = reinterpret_cast<float*>(sm + Cfg::OH);   // [kseg][N/2], set-up only
+            if (tid < kHalf) {
+                float acc = sb[kN * kP + tid];
+                s_phis[tid] = acc;
+                for (int j = 1; j < kseg; ++j) {
+                    acc += sb[j * kSegStride + kN * kP + tid];
+                    s_phis[j * kHalf + tid] = acc;
+                }
+            }
+            {
+                const float4* src = reinterpret_cast<const float4*>(sb + nrow * kP + 32 * wh);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 v = src[j];
+                    hreg[4 * j] = v.x; hreg[4 * j + 1] = v.y; hreg[4 * j + 2] = v.z; hreg[4 * j + 3] = v.w;
+                }
+            }
+            __syncthreads();
+            const int prow = nrow ^ kHalf;   // the other half of this row's rotation pair
+            for (int j = 1; j < kseg; ++j) {
+                const float* sj = sb + j * kSegStride;
+                const float e = expf(sj[kN * kP + kHalf]);
+                float sn, cs;
+                sincosf(s_phis[(j - 1) * kHalf + (nrow & (kHalf - 1))], &sn, &cs);
+                // rows n < N/2: v_n cos + v_{n+N/2} sin; rows n >= N/2: v_n cos - v_{n-N/2} sin
+                const float sg = nrow < kHalf ? sn : -sn;
+                const float4* own = reinterpret_cast<const float4*>(sj + nrow * kP + 32 * wh);
+                const float4* oth = reinterpret_cast<const float4*>(sj + prow * kP + 32 * wh);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 a = own[q], b = oth[q];
+                    hreg[4 * q] = fmaf(e, hreg[4 * q], fmaf(a.x, cs, b.x * sg));
+                    hreg[4 * q + 1] = fmaf(e, hreg[4 * q + 1], fmaf(a.y, cs, b.y * sg));
+                    hreg[4 * q + 2] = fmaf(e, hreg[4 * q + 2], fmaf(a.z, cs, b.z * sg));
+                    hreg[4 * q + 3] = fmaf(e, hreg[4 * q + 3], fmaf(a.w, cs, b.w * sg));
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                car[j] = s_phis[(kseg - 1) * kHalf + jp + j];
+                car_r[j] = reduce_2pi(car[j]);
+            }
+        }
+    }
+
     const uint32_t aB = smem_u32(sm + Cfg::OB), aC = smem_u32(sm + Cfg::OC);
     const uint32_t aXP = smem_u32(sm + Cfg::XP), aH = smem_u32(sm + Cfg::OH);
     const uint32_t id_s = idesc_bf16(64, 64, false, false);   // S  = C . B^T
@@ -417,7 +496,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         const int trow = 16 * q4 + (lane & 15);
         const int col0 = 16 * wh + ((lane >> 4) ? 32 : 0);
         const int t = trow / R, r = trow % R;
-        const int c0 = c * Q;
+        const int c0 = (cb + c) * Q;
         const int T = (L - c0) < Q ? (L - c0) : Q;
         const float e = sf[(c & 1) * F_BLK + F_ECUM + t];
         tmem_wait_ld();
@@ -448,84 +527,78 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     };
 
-    if (nchunks > 0 && warp == 1) scalars(0);
-    __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
-    store_h0();
-
-    for (int c = 0; c < nchunks && !s_abort; ++c) {
-        const int st = c & 1;
-        const uint32_t par = static_cast<uint32_t>(c & 1);
-        const float* blk = sf + st * F_BLK;
-
-        // ======== I1: rotation(c); then epilogue(c-1), the H0 and X' operands ========
-        if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
-        {
-            // Angle increments dt_t theta_t of the segment's tokens, their sum per pair, and the
-            // segment totals exchanged through shared memory: each lane then walks its own
-            // tokens from carry + the earlier segments' totals.
-            float inc[TPS][2];
-            float sum0 = 0.f, sum1 = 0.f;
+    // Angles and rotation of chunk c (I1): the cumulative angle of every token, then B and C
+    // (B only in the state-only pass) normalised, biased and rotated into their operand tiles.
+    auto rotate = [&](const float* blk, uint32_t par) {
+        // Angle increments dt_t theta_t of the segment's tokens, their sum per pair, and the
+        // segment totals exchanged through shared memory: each lane then walks its own
+        // tokens from carry + the earlier segments' totals.
+        float inc[TPS][2];
+        float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < TPS; ++k) {
-                const int t = warp * TPS + k;
-                const uint32_t th = *reinterpret_cast<const uint32_t*>(sm + Cfg::TH + swz128(t, jp));
-                const float dd = blk[F_DT + t];  // 0 past the sequence end: no rotation there
-                inc[k][0] = dd * __uint_as_float(th << 16);
-                inc[k][1] = dd * __uint_as_float(th & 0xFFFF0000u);
-                sum0 += inc[k][0];
-                sum1 += inc[k][1];
-            }
-            s_seg[warp * 32 + lane] = make_float2(sum0, sum1);
-            __syncthreads();
-            float a0 = car_r[0], a1 = car_r[1], tot0 = 0.f, tot1 = 0.f;
+        for (int k = 0; k < TPS; ++k) {
+            const int t = warp * TPS + k;
+            const uint32_t th = *reinterpret_cast<const uint32_t*>(sm + Cfg::TH + swz128(t, jp));
+            const float dd = blk[F_DT + t];  // 0 past the sequence end: no rotation there
+            inc[k][0] = dd * __uint_as_float(th << 16);
+            inc[k][1] = dd * __uint_as_float(th & 0xFFFF0000u);
+            sum0 += inc[k][0];
+            sum1 += inc[k][1];
+        }
+        s_seg[warp * 32 + lane] = make_float2(sum0, sum1);
+        __syncthreads();
+        float a0 = car_r[0], a1 = car_r[1], tot0 = 0.f, tot1 = 0.f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float2 v = s_seg[k * 32 + lane];
-                if (k < warp) { a0 += v.x; a1 += v.y; }
-                tot0 += v.x;
-                tot1 += v.y;
-            }
-            car[0] += tot0;
-            car[1] += tot1;
-            car_r[0] = reduce_2pi(car_r[0] + tot0);
-            car_r[1] = reduce_2pi(car_r[1] + tot1);
-            uint32_t cw[TPS], sw[TPS];  // packed bf16 (cos, cos) and (sin, sin) of the couple
+        for (int k = 0; k < 8; ++k) {
+            const float2 v = s_seg[k * 32 + lane];
+            if (k < warp) { a0 += v.x; a1 += v.y; }
+            tot0 += v.x;
+            tot1 += v.y;
+        }
+        car[0] += tot0;
+        car[1] += tot1;
+        car_r[0] = reduce_2pi(car_r[0] + tot0);
+        car_r[1] = reduce_2pi(car_r[1] + tot1);
+        uint32_t cw[TPS], sw[TPS];  // packed bf16 (cos, cos) and (sin, sin) of the couple
 #pragma unroll
-            for (int k = 0; k < TPS; ++k) {
-                a0 += inc[k][0];
-                a1 += inc[k][1];
-                float sn0, cs0, sn1, cs1;
-                __sincosf(a0, &sn0, &cs0);
-                __sincosf(a1, &sn1, &cs1);
-                cw[k] = pack_bf16(cs0, cs1);
-                sw[k] = pack_bf16(sn0, sn1);
-            }
-            if (!mbar_wait(&bar_b, par)) s_abort = 1;   // raw B and the RMS scales
+        for (int k = 0; k < TPS; ++k) {
+            a0 += inc[k][0];
+            a1 += inc[k][1];
+            float sn0, cs0, sn1, cs1;
+            __sincosf(a0, &sn0, &cs0);
+            __sincosf(a1, &sn1, &cs1);
+            cw[k] = pack_bf16(cs0, cs1);
+            sw[k] = pack_bf16(sn0, sn1);
+        }
+        if (!mbar_wait(&bar_b, par)) s_abort = 1;   // raw B and the RMS scales
+        if constexpr (!kStateOnly) {
             if (!mbar_wait(&bar_c, par)) s_abort = 1;   // raw C
+        }
 #pragma unroll 1
-            for (int r = 0; r < R; ++r) {
-                // bias words of this rank at the couple, both halves of each pair
-                const __nv_bfloat162 bB0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + jp);
-                const __nv_bfloat162 bB1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + kHalf + jp);
-                const __nv_bfloat162 bC0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + jp);
-                const __nv_bfloat162 bC1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + kHalf + jp);
+        for (int r = 0; r < R; ++r) {
+            // bias words of this rank at the couple, both halves of each pair
+            const __nv_bfloat162 bB0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + jp);
+            const __nv_bfloat162 bB1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + kHalf + jp);
 #pragma unroll
-                for (int k = 0; k < TPS; ++k) {
-                    const int row = (warp * TPS + k) * R + r;
-                    const uint32_t o = swz128(row, jp);
-                    const uint32_t rb0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + o);
-                    const uint32_t rb1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + 8192 + o);
+            for (int k = 0; k < TPS; ++k) {
+                const int row = (warp * TPS + k) * R + r;
+                const uint32_t o = swz128(row, jp);
+                const uint32_t rb0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + o);
+                const uint32_t rb1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + 8192 + o);
+                const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
+                const __nv_bfloat162 c2 = as_bf2(cw[k]), s2 = as_bf2(sw[k]);
+                // u = rs * raw + bias on both halves of each pair, then
+                // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
+                __nv_bfloat162 u0 = __hfma2(as_bf2(rb0), as_bf2(rsv.x), bB0);
+                __nv_bfloat162 u1 = __hfma2(as_bf2(rb1), as_bf2(rsv.x), bB1);
+                *reinterpret_cast<uint32_t*>(sm + Cfg::OB + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
+                *reinterpret_cast<uint32_t*>(sm + Cfg::OB + 8192 + o) =
+                    as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
+                if constexpr (!kStateOnly) {
+                    const __nv_bfloat162 bC0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + jp);
+                    const __nv_bfloat162 bC1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + kHalf + jp);
                     const uint32_t rc0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + o);
                     const uint32_t rc1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + 8192 + o);
-                    const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
-                    const __nv_bfloat162 c2 = as_bf2(cw[k]), s2 = as_bf2(sw[k]);
-                    // u = rs * raw + bias on both halves of each pair, then
-                    // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
-                    __nv_bfloat162 u0 = __hfma2(as_bf2(rb0), as_bf2(rsv.x), bB0);
-                    __nv_bfloat162 u1 = __hfma2(as_bf2(rb1), as_bf2(rsv.x), bB1);
-                    *reinterpret_cast<uint32_t*>(sm + Cfg::OB + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
-                    *reinterpret_cast<uint32_t*>(sm + Cfg::OB + 8192 + o) =
-                        as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
                     u0 = __hfma2(as_bf2(rc0), as_bf2(rsv.y), bC0);
                     u1 = __hfma2(as_bf2(rc1), as_bf2(rsv.y), bC1);
                     *reinterpret_cast<uint32_t*>(sm + Cfg::OC + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
@@ -534,203 +607,301 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 }
             }
         }
-        // Yd(c-1) done: its X buffer takes X(c+1), and y(c-1) can be written
-        if (warp == kIssueWarp) {
-            if (elect_one()) {
-                if (c > 0 && !mbar_wait(&bar_m2, (c - 1) & 1)) s_abort = 1;
-                if (c + 1 < nchunks) issue_x(c + 1);
-            }
-            __syncwarp();
-        }
-        if (c > 0) {
-            (void)mbar_wait(&bar_m2, (c - 1) & 1);
-            fence_after_sync();
-            epilogue(c - 1);
-        }
-        // X' = diag(dw) X (the XP buffer held P(c-1), read by Yd(c-1), which has finished)
-        {
-            uint8_t* sX = sm + (st ? Cfg::X1 : Cfg::X0);
-            if (!mbar_wait(&bar_x[st], (c >> 1) & 1)) s_abort = 1;
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int e = tid + i * kTcThreads;
-                const int row = e >> 3, ch = e & 7;
-                const __nv_bfloat162 sc2 = __float2bfloat162_rn(blk[F_DW + row / R]);
-                const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
-                uint4 v = *reinterpret_cast<const uint4*>(sX + o);
-                v.x = as_u32(__hmul2(as_bf2(v.x), sc2));
-                v.y = as_u32(__hmul2(as_bf2(v.y), sc2));
-                v.z = as_u32(__hmul2(as_bf2(v.z), sc2));
-                v.w = as_u32(__hmul2(as_bf2(v.w), sc2));
-                *reinterpret_cast<uint4*>(sm + Cfg::XP + o) = v;
-            }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (s_abort) break;
+    };
 
-        // ======== I2: Yo, S, dH on the tensor cores; P = S o M and H1 = e^{cum_end} H0 + dH
-        // as their accumulators land; the next chunk's scalars meanwhile ========
-        if (warp == kIssueWarp) {
-            if (elect_one()) {
-                // theta and raw B of chunk c+1 (their buffers were read by the rotation), the
-                // scalar boxes of chunk c+2 (chunk c's slot was read by scalars(c))
-                if (c + 1 < nchunks) {
-                    issue_th(c + 1);
-                    issue_b(c + 1);
-                }
-                if (c + 2 < nchunks) issue_sc(c + 2);
-                constexpr uint32_t hi = desc_hi_sw128(1024);
-                const uint32_t loC = desc_lo(aC, 16), loB = desc_lo(aB, 16);
-                const uint32_t loBt = desc_lo(aB, 8192), loXP = desc_lo(aXP, 8192);
-                const uint32_t loH = desc_lo(aH, 16384);
+    // X' = diag(dw) X of chunk c into the XP buffer (whose previous readers have finished)
+    auto xprime = [&](int c, const float* blk) {
+        const int st = c & 1;
+        uint8_t* sX = sm + (st ? Cfg::X1 : Cfg::X0);
+        if (!mbar_wait(&bar_x[st], (c >> 1) & 1)) s_abort = 1;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
-                             desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
-                mma_commit(smem_u32(&bar_yo));
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16(tmem + T_S, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
-                             desc_pack(loB + (kmajor_off(k, 8192) >> 4), hi), id_s, k > 0);
-                mma_commit(smem_u32(&bar_s));
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + T_DH, desc_pack(loBt + (mnmajor_off(k) >> 4), hi),
-                             desc_pack(loXP + (mnmajor_off(k) >> 4), hi), id_dh, k > 0);
-                mma_commit(smem_u32(&bar_dh));
-                s_issued[5] = c + 1;
-                // Yo and S were the readers of Cbar: fetch the next chunk's raw C in its place
-                if (c + 1 < nchunks) {
-                    if (!mbar_wait(&bar_s, par)) s_abort = 1;
-                    issue_c(c + 1);
-                }
-            }
-            __syncwarp();
+        for (int i = 0; i < 2; ++i) {
+            const int e = tid + i * kTcThreads;
+            const int row = e >> 3, ch = e & 7;
+            const __nv_bfloat162 sc2 = __float2bfloat162_rn(blk[F_DW + row / R]);
+            const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
+            uint4 v = *reinterpret_cast<const uint4*>(sX + o);
+            v.x = as_u32(__hmul2(as_bf2(v.x), sc2));
+            v.y = as_u32(__hmul2(as_bf2(v.y), sc2));
+            v.z = as_u32(__hmul2(as_bf2(v.z), sc2));
+            v.w = as_u32(__hmul2(as_bf2(v.w), sc2));
+            *reinterpret_cast<uint4*>(sm + Cfg::XP + o) = v;
         }
-        if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
-        {
-            const int trow = 16 * q4 + (lane & 15);   // row block q4
-            const int qc = wh + ((lane >> 4) ? 2 : 0);  // column block of this half-warp
-            const int col0 = 16 * qc;
-            const int t = trow / R;
-            constexpr int NT = 16 / R;                  // tokens covered by the 16 columns
-            const int s0 = col0 / R;
-            float m[NT];
-            if (qc < q4) {          // strictly below the diagonal block: factored decay
-                const float er = blk[F_EROW + t];
-#pragma unroll
-                for (int i = 0; i < NT; i += 2) {
-                    const float2 e2 = *reinterpret_cast<const float2*>(blk + F_ECOL + (q4 - 1) * 64 + s0 + i);
-                    m[i] = er * e2.x;
-                    m[i + 1] = er * e2.y;
-                }
-            } else if (qc == q4) {  // diagonal block: decay, trapezoid weight and gamma
-                const float cum_t = blk[F_CUM + t], gam_t = blk[F_GAM + t];
-#pragma unroll
-                for (int i = 0; i < NT; i += 2) {
-                    const float2 a2 = *reinterpret_cast<const float2*>(blk + F_CUM + s0 + i);
-                    const float2 w2 = *reinterpret_cast<const float2*>(blk + F_W + s0 + i);
-                    const int sa = s0 + i;
-                    m[i] = (sa < t) ? ex2_approx(fminf(cum_t - a2.x, 0.f)) * w2.x : ((sa == t) ? gam_t : 0.f);
-                    m[i + 1] = (sa + 1 < t) ? ex2_approx(fminf(cum_t - a2.y, 0.f)) * w2.y
-                                            : ((sa + 1 == t) ? gam_t : 0.f);
-                }
-            } else {                // above the diagonal: zero
-#pragma unroll
-                for (int i = 0; i < NT; ++i) m[i] = 0.f;
+    };
+
+    if constexpr (kStateOnly) {
+        if (nchunks > 0 && warp == 1) scalars(0);
+        __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
+        for (int c = 0; c < nchunks && !s_abort; ++c) {
+            const int st = c & 1;
+            const uint32_t par = static_cast<uint32_t>(c & 1);
+            const float* blk = sf + st * F_BLK;
+            // ======== I1: angles and rotation of B; X(c+1) (its buffer was last read by X'(c-1));
+            // the X' operand ========
+            if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
+            rotate(blk, par);
+            if (warp == kIssueWarp) {
+                if (elect_one() && c + 1 < nchunks) issue_x(c + 1);
+                __syncwarp();
             }
-            if (!mbar_wait(&bar_s, par)) s_abort = 1;
+            xprime(c, blk);   // XP was last read by dH(c-1), waited for by every thread
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
             fence_after_sync();
-            float sv[16];
-            tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, sv);
-            tmem_wait_ld();
-            uint32_t pw[8];
+            if (s_abort) break;
+            // ======== I2: dH on the tensor cores, the next chunk's scalars meanwhile, then
+            // H1 = e^{cum_end} H0 + dH ========
+            if (warp == kIssueWarp) {
+                if (elect_one()) {
+                    if (c + 1 < nchunks) {
+                        issue_th(c + 1);
+                        issue_b(c + 1);
+                    }
+                    if (c + 2 < nchunks) issue_sc(c + 2);
+                    constexpr uint32_t hi = desc_hi_sw128(1024);
+                    const uint32_t loBt = desc_lo(aB, 8192), loXP = desc_lo(aXP, 8192);
 #pragma unroll
-            for (int j = 0; j < 16; j += 2)
-                pw[j / 2] = pack_bf16(sv[j] * m[j / R], sv[j + 1] * m[(j + 1) / R]);
-            // dH has read X': P takes its buffer
-            if (!mbar_wait(&bar_dh, par)) s_abort = 1;
-            fence_after_sync();
-            *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-            *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-        }
-        {
-            const float eend = blk[F_MISC];
-            const uint32_t ta = tmem + ((32u * q4) << 16) + T_DH + 32u * wh;
-            float d0[16], d1[16];
-            tmem_ld_32x32b_x16(ta, d0);
-            tmem_ld_32x32b_x16(ta + 16, d1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                hreg[j] = fmaf(eend, hreg[j], d0[j]);
-                hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + T_DH, desc_pack(loBt + (mnmajor_off(k) >> 4), hi),
+                                 desc_pack(loXP + (mnmajor_off(k) >> 4), hi), id_dh, k > 0);
+                    mma_commit(smem_u32(&bar_dh));
+                    s_issued[5] = c + 1;
+                }
+                __syncwarp();
             }
+            if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
+            {
+                if (!mbar_wait(&bar_dh, par)) s_abort = 1;
+                fence_after_sync();
+                const float eend = blk[F_MISC];
+                const uint32_t ta = tmem + ((32u * q4) << 16) + T_DH + 32u * wh;
+                float d0[16], d1[16];
+                tmem_ld_32x32b_x16(ta, d0);
+                tmem_ld_32x32b_x16(ta + 16, d1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    hreg[j] = fmaf(eend, hreg[j], d0[j]);
+                    hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
+                }
+            }
+            // the next chunk's scalars are published; dH has been read out of TMEM
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
         }
-        // Yo(c) has read H0: the next chunk's H0 operand
-        if (!mbar_wait(&bar_yo, par)) s_abort = 1;
+    } else {
+        if (nchunks > 0 && warp == 1) scalars(0);
+        __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
         store_h0();
 
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (s_abort) break;
+        for (int c = 0; c < nchunks && !s_abort; ++c) {
+            const int st = c & 1;
+            const uint32_t par = static_cast<uint32_t>(c & 1);
+            const float* blk = sf + st * F_BLK;
 
-        // ======== I4: Yd = P X (waited for in the next chunk's I1) ========
-        if (warp == kIssueWarp) {
-            if (elect_one()) {
-                constexpr uint32_t hi = desc_hi_sw128(1024);
-                const uint32_t loP = desc_lo(aXP, 16);
-                const uint32_t loX = desc_lo(smem_u32(sm + (st ? Cfg::X1 : Cfg::X0)), 8192);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16(tmem + T_YD, desc_pack(loP + (kmajor_off(k, 8192) >> 4), hi),
-                             desc_pack(loX + (mnmajor_off(k) >> 4), hi), id_yd, k > 0);
-                mma_commit(smem_u32(&bar_m2));
-                s_issued[6] = c + 1;
+            // ======== I1: rotation(c); then epilogue(c-1), the H0 and X' operands ========
+            if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
+            rotate(blk, par);
+            // Yd(c-1) done: its X buffer takes X(c+1), and y(c-1) can be written
+            if (warp == kIssueWarp) {
+                if (elect_one()) {
+                    if (c > 0 && !mbar_wait(&bar_m2, (c - 1) & 1)) s_abort = 1;
+                    if (c + 1 < nchunks) issue_x(c + 1);
+                }
+                __syncwarp();
             }
-            __syncwarp();
+            if (c > 0) {
+                (void)mbar_wait(&bar_m2, (c - 1) & 1);
+                fence_after_sync();
+                epilogue(c - 1);
+            }
+            // X' = diag(dw) X (the XP buffer held P(c-1), read by Yd(c-1), which has finished)
+            xprime(c, blk);
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+            if (s_abort) break;
+
+            // ======== I2: Yo, S, dH on the tensor cores; P = S o M and H1 = e^{cum_end} H0 + dH
+            // as their accumulators land; the next chunk's scalars meanwhile ========
+            if (warp == kIssueWarp) {
+                if (elect_one()) {
+                    // theta and raw B of chunk c+1 (their buffers were read by the rotation), the
+                    // scalar boxes of chunk c+2 (chunk c's slot was read by scalars(c))
+                    if (c + 1 < nchunks) {
+                        issue_th(c + 1);
+                        issue_b(c + 1);
+                    }
+                    if (c + 2 < nchunks) issue_sc(c + 2);
+                    constexpr uint32_t hi = desc_hi_sw128(1024);
+                    const uint32_t loC = desc_lo(aC, 16), loB = desc_lo(aB, 16);
+                    const uint32_t loBt = desc_lo(aB, 8192), loXP = desc_lo(aXP, 8192);
+                    const uint32_t loH = desc_lo(aH, 16384);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16(tmem + T_YO, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
+                                 desc_pack(loH + (mnmajor_off(k) >> 4), hi), id_yo, k > 0);
+                    mma_commit(smem_u32(&bar_yo));
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16(tmem + T_S, desc_pack(loC + (kmajor_off(k, 8192) >> 4), hi),
+                                 desc_pack(loB + (kmajor_off(k, 8192) >> 4), hi), id_s, k > 0);
+                    mma_commit(smem_u32(&bar_s));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + T_DH, desc_pack(loBt + (mnmajor_off(k) >> 4), hi),
+                                 desc_pack(loXP + (mnmajor_off(k) >> 4), hi), id_dh, k > 0);
+                    mma_commit(smem_u32(&bar_dh));
+                    s_issued[5] = c + 1;
+                    // Yo and S were the readers of Cbar: fetch the next chunk's raw C in its place
+                    if (c + 1 < nchunks) {
+                        if (!mbar_wait(&bar_s, par)) s_abort = 1;
+                        issue_c(c + 1);
+                    }
+                }
+                __syncwarp();
+            }
+            if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
+            {
+                const int trow = 16 * q4 + (lane & 15);   // row block q4
+                const int qc = wh + ((lane >> 4) ? 2 : 0);  // column block of this half-warp
+                const int col0 = 16 * qc;
+                const int t = trow / R;
+                constexpr int NT = 16 / R;                  // tokens covered by the 16 columns
+                const int s0 = col0 / R;
+                float m[NT];
+                if (qc < q4) {          // strictly below the diagonal block: factored decay
+                    const float er = blk[F_EROW + t];
+#pragma unroll
+                    for (int i = 0; i < NT; i += 2) {
+                        const float2 e2 = *reinterpret_cast<const float2*>(blk + F_ECOL + (q4 - 1) * 64 + s0 + i);
+                        m[i] = er * e2.x;
+                        m[i + 1] = er * e2.y;
+                    }
+                } else if (qc == q4) {  // diagonal block: decay, trapezoid weight and gamma
+                    const float cum_t = blk[F_CUM + t], gam_t = blk[F_GAM + t];
+#pragma unroll
+                    for (int i = 0; i < NT; i += 2) {
+                        const float2 a2 = *reinterpret_cast<const float2*>(blk + F_CUM + s0 + i);
+                        const float2 w2 = *reinterpret_cast<const float2*>(blk + F_W + s0 + i);
+                        const int sa = s0 + i;
+                        m[i] = (sa < t) ? ex2_approx(fminf(cum_t - a2.x, 0.f)) * w2.x : ((sa == t) ? gam_t : 0.f);
+                        m[i + 1] = (sa + 1 < t) ? ex2_approx(fminf(cum_t - a2.y, 0.f)) * w2.y
+                                                : ((sa + 1 == t) ? gam_t : 0.f);
+                    }
+                } else {                // above the diagonal: zero
+#pragma unroll
+                    for (int i = 0; i < NT; ++i) m[i] = 0.f;
+                }
+                if (!mbar_wait(&bar_s, par)) s_abort = 1;
+                fence_after_sync();
+                float sv[16];
+                tmem_ld_16x32bx2_x16(tmem + ((32u * q4) << 16) + T_S + 16u * wh, sv);
+                tmem_wait_ld();
+                uint32_t pw[8];
+#pragma unroll
+                for (int j = 0; j < 16; j += 2)
+                    pw[j / 2] = pack_bf16(sv[j] * m[j / R], sv[j + 1] * m[(j + 1) / R]);
+                // dH has read X': P takes its buffer
+                if (!mbar_wait(&bar_dh, par)) s_abort = 1;
+                fence_after_sync();
+                *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                *reinterpret_cast<uint4*>(sm + Cfg::XP + swz128(trow, col0 + 8)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
+            }
+            {
+                const float eend = blk[F_MISC];
+                const uint32_t ta = tmem + ((32u * q4) << 16) + T_DH + 32u * wh;
+                float d0[16], d1[16];
+                tmem_ld_32x32b_x16(ta, d0);
+                tmem_ld_32x32b_x16(ta + 16, d1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    hreg[j] = fmaf(eend, hreg[j], d0[j]);
+                    hreg[16 + j] = fmaf(eend, hreg[16 + j], d1[j]);
+                }
+            }
+            // Yo(c) has read H0: the next chunk's H0 operand
+            if (!mbar_wait(&bar_yo, par)) s_abort = 1;
+            store_h0();
+
+            fence_proxy_async();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+            if (s_abort) break;
+
+            // ======== I4: Yd = P X (waited for in the next chunk's I1) ========
+            if (warp == kIssueWarp) {
+                if (elect_one()) {
+                    constexpr uint32_t hi = desc_hi_sw128(1024);
+                    const uint32_t loP = desc_lo(aXP, 16);
+                    const uint32_t loX = desc_lo(smem_u32(sm + (st ? Cfg::X1 : Cfg::X0)), 8192);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + T_YD, desc_pack(loP + (kmajor_off(k, 8192) >> 4), hi),
+                                 desc_pack(loX + (mnmajor_off(k) >> 4), hi), id_yd, k > 0);
+                    mma_commit(smem_u32(&bar_m2));
+                    s_issued[6] = c + 1;
+                }
+                __syncwarp();
+            }
         }
-    }
-    // ---- epilogue of the last chunk ----
-    if (nchunks > 0 && !s_abort) {
-        if (tid == 0 && !mbar_wait(&bar_m2, (nchunks - 1) & 1)) s_abort = 1;
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (!s_abort) {
-            (void)mbar_try_wait(smem_u32(&bar_m2), (nchunks - 1) & 1);
-            epilogue(nchunks - 1);
+        // ---- epilogue of the last chunk ----
+        if (nchunks > 0 && !s_abort) {
+            if (tid == 0 && !mbar_wait(&bar_m2, (nchunks - 1) & 1)) s_abort = 1;
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+            if (!s_abort) {
+                (void)mbar_try_wait(smem_u32(&bar_m2), (nchunks - 1) & 1);
+                epilogue(nchunks - 1);
+            }
         }
     }
 
     // ---------------- final state ----------------
     __syncthreads();
-    if (!s_abort) {
-        if (p.h1) {
-            float4* dst = reinterpret_cast<float4*>(p.h1 + (u * kN + nrow) * kP + 32 * wh);
+    if (!s_abort && kStateOnly) {
+        // this segment's end state for the full pass: h, the angle sum (absolute for segment
+        // 0), the summed log-decay
+        float* so = sa.st + (u * (sa.nseg - 1) + kseg) * kSegStride;
+        float4* dst = reinterpret_cast<float4*>(so + nrow * kP + 32 * wh);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
+        for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
+        if (warp == 0) {
+            so[kN * kP + jp] = car[0];
+            so[kN * kP + jp + 1] = car[1];
         }
-        if (p.phi1 && warp == 0) {
-            p.phi1[u * kHalf + jp] = car[0];
-            p.phi1[u * kHalf + jp + 1] = car[1];
-        }
-        if (L > 0) {
-            if (p.prevB1) {
-                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevB1) + u * R * kN;
-                const __nv_bfloat16* src = Bu + (L - 1) * tokB;
-                for (int e = tid; e < R * kN; e += kTcThreads) dst[e] = src[e];
+        if (warp == 1 && lane == 0) so[kN * kP + kHalf] = lam_acc;
+    } else if (!s_abort) {
+        // the sequence's final state, written by its last segment
+        if (kseg == sa.nseg - 1) {
+            if (p.h1) {
+                float4* dst = reinterpret_cast<float4*>(p.h1 + (u * kN + nrow) * kP + 32 * wh);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
             }
-            if (p.prevx1) {
-                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevx1) + u * R * kP;
-                const __nv_bfloat16* src = xu + (L - 1) * tokY;
-                for (int e = tid; e < R * kP; e += kTcThreads) dst[e] = src[e];
+            if (p.phi1 && warp == 0) {
+                p.phi1[u * kHalf + jp] = car[0];
+                p.phi1[u * kHalf + jp + 1] = car[1];
+            }
+            if (L > 0) {
+                if (p.prevB1) {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevB1) + u * R * kN;
+                    const __nv_bfloat16* src = Bu + (L - 1) * tokB;
+                    for (int e = tid; e < R * kN; e += kTcThreads) dst[e] = src[e];
+                }
+                if (p.prevx1) {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.prevx1) + u * R * kP;
+                    const __nv_bfloat16* src = xu + (L - 1) * tokY;
+                    for (int e = tid; e < R * kP; e += kTcThreads) dst[e] = src[e];
+                }
             }
         }
     } else if (tid == 0) {
@@ -746,8 +917,10 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         if (s_issued[3] > 0) (void)mbar_wait(&bar_b, (s_issued[3] - 1) & 1, kDrain);
         if (s_issued[4] > 0) (void)mbar_wait(&bar_c, (s_issued[4] - 1) & 1, kDrain);
         if (s_issued[5] > 0) {
-            (void)mbar_wait(&bar_yo, (s_issued[5] - 1) & 1, kDrain);
-            (void)mbar_wait(&bar_s, (s_issued[5] - 1) & 1, kDrain);
+            if constexpr (!kStateOnly) {
+                (void)mbar_wait(&bar_yo, (s_issued[5] - 1) & 1, kDrain);
+                (void)mbar_wait(&bar_s, (s_issued[5] - 1) & 1, kDrain);
+            }
             (void)mbar_wait(&bar_dh, (s_issued[5] - 1) & 1, kDrain);
         }
         if (s_issued[6] > 0) (void)mbar_wait(&bar_m2, (s_issued[6] - 1) & 1, kDrain);
@@ -791,14 +964,55 @@ bool tc_scan_supported(const ScanParams& p, bool bf16) {
            p.L * p.G * p.R * kN < lim && p.L * p.H * p.R * kP < lim && p.b <= lim;
 }
 
-size_t tc_scan_workspace_bytes(const ScanParams& p) {
+namespace {
+
+int sm_count() {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
+// Segments per sequence. When the (batch, head) units alone would leave SMs idle, each
+// sequence is cut so that units x segments fills every SM twice (two CTAs per SM), keeping at
+// least kMinSegChunks chunks per segment and at most kMaxSeg segments.
+constexpr int64_t kMinSegChunks = 8, kMaxSeg = 16;
+SegArgs seg_plan(const ScanParams& p) {
+    const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
+    const int64_t nch = (p.L + Q - 1) / Q;
+    const int64_t units = p.b * p.H;
+    SegArgs sa{static_cast<int>(nch), 1, nullptr};
+    if (units <= 0 || nch == 0) return sa;
+    int64_t S = 2 * sm_count() / units;
+    S = std::min(S, nch / kMinSegChunks);
+    S = std::min(S, kMaxSeg);
+    if (S < 2) return sa;
+    sa.seg_chunks = static_cast<int>((nch + S - 1) / S);
+    sa.nseg = static_cast<int>((nch + sa.seg_chunks - 1) / sa.seg_chunks);
+    return sa;
+}
+
+size_t rs_bytes(const ScanParams& p) {
     const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
     const int64_t Lpad = (p.L + Q - 1) / Q * Q;
-    return p.bc_norm ? static_cast<size_t>(p.b * Lpad * p.G * p.R) * sizeof(uint2) : 0;
+    const size_t n = p.bc_norm ? static_cast<size_t>(p.b * Lpad * p.G * p.R) * sizeof(uint2) : 0;
+    return (n + 255) / 256 * 256;
+}
+
+}  // namespace
+
+size_t tc_scan_workspace_bytes(const ScanParams& p) {
+    const SegArgs sa = seg_plan(p);
+    const size_t seg = sa.nseg > 1 ? static_cast<size_t>(p.b * p.H) * (sa.nseg - 1) * kSegStride * sizeof(float) : 0;
+    return rs_bytes(p) + seg;
 }
 
 template <int R>
-static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, cudaStream_t s) {
+static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s) {
     constexpr int Q = 64 / R;
     TcMaps maps;
     const cuuint64_t H = p.H, Lq = p.L, b = p.b;
@@ -849,22 +1063,35 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     const uint32_t smem = tc_smem_bytes<R>();
-    auto k = scan_tc_kernel<R>;
+    const int64_t units = p.b * p.H;
+    if (sa.nseg > 1) {   // every segment's end state but the last's
+        auto ks = scan_tc_kernel<R, true>;
+        cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        ks<<<static_cast<unsigned>(units * (sa.nseg - 1)), kTcThreads, smem, s>>>(p, maps, rs, sa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    auto k = scan_tc_kernel<R, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    k<<<static_cast<unsigned>(p.b * p.H), kTcThreads, smem, s>>>(p, maps, rs);
+    k<<<static_cast<unsigned>(units * sa.nseg), kTcThreads, smem, s>>>(p, maps, rs, sa);
     return cudaGetLastError();
 }
 
-cudaError_t launch_scan_tc(const ScanParams& p, void* rs_ws, cudaStream_t s) {
+cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
-    uint2* rs = p.bc_norm ? static_cast<uint2*>(rs_ws) : nullptr;
+    // workspace body: the RMS scales, then the segments' end states
+    uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
+    SegArgs sa = seg_plan(p);
+    if (sa.nseg > 1) sa.st = reinterpret_cast<float*>(static_cast<char*>(ws_body) + rs_bytes(p));
     switch (p.R) {
-        case 1: return launch_tc_t<1>(p, rs, s);
-        case 2: return launch_tc_t<2>(p, rs, s);
-        case 4: return launch_tc_t<4>(p, rs, s);
-        case 8: return launch_tc_t<8>(p, rs, s);
+        case 1: return launch_tc_t<1>(p, rs, sa, s);
+        case 2: return launch_tc_t<2>(p, rs, sa, s);
+        case 4: return launch_tc_t<4>(p, rs, sa, s);
+        case 8: return launch_tc_t<8>(p, rs, sa, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -52,6 +52,32 @@ def test_scan_small(cuda_dev, case):
     compare(pr, y, fin, yo, so)
 
 
+# Few units and long sequences take the sequence-parallel form: each sequence is cut into
+# segments (a state-only pass, then all segments at once from their assembled start states).
+# With 4-8 units on a B200 these lengths give 2-5 segments, the last one ragged.
+SEGMENTED = [
+    # b, L, H, G, R, chunk, state
+    (1, 2543, 4, 1, 1, 64, True),     # 40 chunks -> 5 segments of 8
+    (1, 2543, 4, 1, 1, 64, False),
+    (1, 700, 4, 1, 4, 16, True),      # 44 chunks -> 5 segments of 9
+    (1, 900, 4, 1, 2, 32, True),      # 29 chunks -> 3 segments of 10
+    (1, 333, 4, 1, 8, 8, True),       # 42 chunks -> 5 segments of 9
+    (1, 1100, 4, 2, 1, 64, True),     # 18 chunks, two B/C groups -> 2 segments of 9
+    (2, 1500, 4, 1, 1, 64, True),     # 24 chunks, 8 units -> 3 segments of 8
+]
+
+
+@pytest.mark.parametrize("case", SEGMENTED, ids=lambda c: "b{}L{}H{}G{}R{}Q{}{}".format(
+    *c[:6], "s" if c[6] else ""))
+def test_scan_segmented(cuda_dev, case):
+    b, L, H, G, R, Q, st = case
+    pr = make_problem(b, L, H, G, 64, 128, rank=R, chunk=Q, dtype=torch.bfloat16, bc_norm=True,
+                      bias_std=0.1, seed=7 * L + R, with_state=True)
+    y, fin = gpu_scan(pr, cuda_dev, use_state=st)
+    yo, so = oracle_scan(pr, use_state=st)
+    compare(pr, y, fin, yo, so)
+
+
 def test_final_state_may_alias_init(cuda_dev):
     pr = make_problem(2, 150, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
                       seed=5, with_state=True)
