@@ -91,7 +91,9 @@ typedef struct {
  * step is h_0 = gamma_0 B_0 x_0 (Sec. 3.1.3). */
 
 /* Bytes of device workspace m3_scan_fwd needs for these dims (>= 256), or 0 if the dims are
- * invalid or unsupported. */
+ * invalid or unsupported: a 256-byte status header, the per-token RMS scales of B and C, and
+ * for few long sequences (which the scan cuts into segments that run in parallel) one fp32
+ * end state per sequence and segment but the last. Depends on the current device's SM count. */
 M3_API size_t m3_scan_workspace_bytes(const m3_dims* dims);
 
 /* Chunked parallel prefill scan over a whole sequence (Sec. 3.1.3 parallel form, Sec. 3.3
@@ -100,9 +102,10 @@ M3_API size_t m3_scan_workspace_bytes(const m3_dims* dims);
  *   final     where to write the state after token L-1, or NULL to skip; may alias init.
  *   y         [b, L, H, R, P] in_dtype output, y_t = H_t^T Cbar_t.
  *   workspace device buffer of at least m3_scan_workspace_bytes(dims) bytes, 256-byte
- *             aligned, zero-filled before its first use (e.g. one cudaMemsetAsync). Every
- *             call leaves it zero-filled again, so it is reused without resetting. Two calls
- *             that may run at the same time need separate workspaces.
+ *             aligned, its first 256 bytes (the status header) zero before its first use
+ *             (e.g. one cudaMemsetAsync). A call that does not time out leaves the header
+ *             zero, so the workspace is reused without resetting; the rest is scratch. Two
+ *             calls that may run at the same time need separate workspaces.
  * Asynchronous: returns after launching. A device-side timeout (a wait between CTAs that
  * exceeded its bound) is reported by m3_scan_check after the stream has synchronised. */
 M3_API m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
@@ -138,10 +141,12 @@ M3_API m3_status m3_scan_check(void* workspace);
  *   (each call clears the status bytes it needs at zero first). Calls whose work can overlap
  *   on the GPU (different streams, or different host threads) race on the array: serialise
  *   them, or use m3_scan_fwd with one workspace each.
- *   Limit: dims whose m3_scan_workspace_bytes exceeds 1 MiB return M3_ERR_UNSUPPORTED
- *   (with BC normalisation on, the tensor-core path needs 8 bytes per batch * seqlen *
- *   ngroups * rank row). A device-side wait that gives up cannot be reported here; use
- *   m3_scan_fwd and m3_scan_check when that matters. */
+ *   Limit: dims whose scan cannot run in 1 MiB return M3_ERR_UNSUPPORTED (with BC
+ *   normalisation on, the tensor-core path needs 8 bytes per batch * seqlen * ngroups *
+ *   rank row). Few long sequences, which m3_scan_fwd cuts into parallel segments, use only
+ *   as many segments as the rest of the array holds the end states of (possibly one): the
+ *   results are the same, the time may be longer. A device-side wait that gives up cannot
+ *   be reported here; use m3_scan_fwd and m3_scan_check when that matters. */
 M3_API m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const m3_inputs* in,
                                      const m3_state* init, const m3_state* final_state,
                                      void* y, void* stream);

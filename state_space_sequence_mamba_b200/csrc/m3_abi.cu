@@ -145,9 +145,25 @@ size_t m3_scan_workspace_bytes(const m3_dims* dims) {
     return kWsHeader + (body + 255) / 256 * 256;
 }
 
-m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
-                      const m3_state* final_state, void* y, void* workspace, size_t ws_bytes,
-                      void* stream) {
+}  // extern "C"
+
+namespace m3 {
+
+// The smallest workspace the scan runs in: without the sequence-parallel form's segment
+// states (0 for invalid dims).
+size_t scan_workspace_min_bytes(const m3_dims* dims) {
+    if (check_dims(dims, true) != M3_OK) return 0;
+    const m3_inputs none{};
+    const ScanParams p = make_params(dims, &none, nullptr, nullptr, nullptr);
+    size_t body = 0;
+    if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_min_bytes(p);
+    return kWsHeader + (body + 255) / 256 * 256;
+}
+
+// m3_scan_fwd with the workspace size it must at least have (`need`).
+m3_status scan_fwd_with(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                        const m3_state* final_state, void* y, void* workspace, size_t ws_bytes,
+                        size_t need, void* stream) {
     g_err[0] = 0;
     m3_status st = check_dims(dims, true);
     if (st != M3_OK) return st;
@@ -157,7 +173,6 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
     if ((st = check_state(final_state, "final")) != M3_OK) return st;
     if (any && !y) return fail(M3_ERR_INVALID_ARG, "y is NULL");
     if (y && !aligned16(y)) return fail(M3_ERR_INVALID_ARG, "y is not 16-byte aligned");
-    const size_t need = m3_scan_workspace_bytes(dims);
     if (!workspace) return fail(M3_ERR_INVALID_ARG, "workspace is NULL");
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(M3_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
@@ -174,7 +189,7 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
 
     const bool bf16 = dims->in_dtype == M3_BF16;
     if (tc_scan_supported(p, bf16)) {
-        e = launch_scan_tc(p, static_cast<char*>(workspace) + kWsHeader, s);
+        e = launch_scan_tc(p, static_cast<char*>(workspace) + kWsHeader, ws_bytes - kWsHeader, s);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
         return M3_OK;
     }
@@ -184,6 +199,17 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
     e = launch_scan_simt(p, bf16, s);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return M3_OK;
+}
+
+}  // namespace m3
+
+extern "C" {
+
+m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                      const m3_state* final_state, void* y, void* workspace, size_t ws_bytes,
+                      void* stream) {
+    return scan_fwd_with(dims, in, init, final_state, y, workspace, ws_bytes,
+                         m3_scan_workspace_bytes(dims), stream);
 }
 
 m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,

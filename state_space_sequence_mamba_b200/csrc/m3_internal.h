@@ -45,9 +45,20 @@ size_t simt_scan_smem_bytes(const ScanParams& p);
 cudaError_t launch_scan_simt(const ScanParams& p, bool bf16, cudaStream_t s);
 // Tensor-core scan (bf16, N = 128, P = 64, chunk * R = 64).
 bool tc_scan_supported(const ScanParams& p, bool bf16);
-// Workspace bytes the tensor-core scan needs beyond the status header.
+// Workspace bytes the tensor-core scan needs beyond the status header: with the end states of
+// the sequence-parallel form's segments (preferred), or without them (minimum: one segment).
 size_t tc_scan_workspace_bytes(const ScanParams& p);
-cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s);
+size_t tc_scan_workspace_min_bytes(const ScanParams& p);
+// ws_body: the workspace after the status header, body_bytes long (at least the minimum); the
+// scan uses as many segments as the preferred plan has and body_bytes holds.
+cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s);
+// The smallest workspace m3_scan_fwd's work runs in (one segment per sequence), and the scan
+// entry point with that lower bound instead of m3_scan_workspace_bytes (for the fixed scratch
+// of m3_scan_fwd_noalloc).
+size_t scan_workspace_min_bytes(const m3_dims* dims);
+m3_status scan_fwd_with(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                        const m3_state* final_state, void* y, void* workspace, size_t ws_bytes,
+                        size_t need, void* stream);
 // Records msg as this thread's m3_last_error() text and returns s.
 m3_status set_error(m3_status s, const char* msg);
 // Persistent decode with bulk asynchronous copies (bf16, N * P <= 8192).

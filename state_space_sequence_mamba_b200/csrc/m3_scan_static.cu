@@ -5,8 +5,10 @@
 // runtime that plans all of its device memory up front and forbids allocation while it serves,
 // code that runs inside a step whose memory has been fixed in advance, or an embedding that
 // simply has no allocator to offer. For them this entry point takes its scratch (the status
-// header and the per-token RMS scales of B and C) from one array of fixed size that is part of
-// the library itself, so the call needs nothing beyond its inputs and outputs.
+// header, the per-token RMS scales of B and C and, room permitting, the segment end states of
+// the sequence-parallel form) from one array of fixed size that is part of the library itself,
+// so the call needs nothing beyond its inputs and outputs. Few long sequences then run in as
+// many segments as the array holds the end states of, down to one.
 //
 // The array is a file-scope __device__ variable: every GPU that loads the library holds its
 // own copy of it until the process exits. Host code cannot use the variable's name as a
@@ -44,7 +46,7 @@ extern "C" {
 M3_API m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const m3_inputs* in,
                                      const m3_state* init, const m3_state* final_state,
                                      void* y, void* stream) {
-    const size_t need = m3_scan_workspace_bytes(dims);
+    const size_t need = scan_workspace_min_bytes(dims);
     if (need == 0) {
         // invalid or unsupported dims: let the regular entry point say which, with no launch
         return m3_scan_fwd(dims, in, init, final_state, y, nullptr, 0, stream);
@@ -75,7 +77,7 @@ M3_API m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const m3_inputs* in,
     if (cudaMemsetAsync(scratch, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) !=
         cudaSuccess)
         return static_fail(M3_ERR_CUDA, "m3_scan_fwd_noalloc: clearing the status header failed");
-    return m3_scan_fwd(dims, in, init, final_state, y, scratch, kStaticScratchBytes, stream);
+    return scan_fwd_with(dims, in, init, final_state, y, scratch, kStaticScratchBytes, need, stream);
 }
 
 }  // extern "C"

@@ -979,9 +979,10 @@ int sm_count() {
 
 // Segments per sequence. When the (batch, head) units alone would leave SMs idle, each
 // sequence is cut so that units x segments fills every SM twice (two CTAs per SM), keeping at
-// least kMinSegChunks chunks per segment and at most kMaxSeg segments.
+// least kMinSegChunks chunks per segment and at most kMaxSeg segments, and no more segments
+// than seg_bytes of workspace can hold the end states of.
 constexpr int64_t kMinSegChunks = 8, kMaxSeg = 16;
-SegArgs seg_plan(const ScanParams& p) {
+SegArgs seg_plan(const ScanParams& p, size_t seg_bytes = ~size_t(0)) {
     const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
     const int64_t nch = (p.L + Q - 1) / Q;
     const int64_t units = p.b * p.H;
@@ -990,6 +991,8 @@ SegArgs seg_plan(const ScanParams& p) {
     int64_t S = 2 * sm_count() / units;
     S = std::min(S, nch / kMinSegChunks);
     S = std::min(S, kMaxSeg);
+    const size_t per_seg = static_cast<size_t>(units) * kSegStride * sizeof(float);
+    while (S >= 2 && static_cast<size_t>(S - 1) * per_seg > seg_bytes) --S;
     if (S < 2) return sa;
     sa.seg_chunks = static_cast<int>((nch + S - 1) / S);
     sa.nseg = static_cast<int>((nch + sa.seg_chunks - 1) / sa.seg_chunks);
@@ -1010,6 +1013,8 @@ size_t tc_scan_workspace_bytes(const ScanParams& p) {
     const size_t seg = sa.nseg > 1 ? static_cast<size_t>(p.b * p.H) * (sa.nseg - 1) * kSegStride * sizeof(float) : 0;
     return rs_bytes(p) + seg;
 }
+
+size_t tc_scan_workspace_min_bytes(const ScanParams& p) { return rs_bytes(p); }
 
 template <int R>
 static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s) {
@@ -1081,11 +1086,12 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
     return cudaGetLastError();
 }
 
-cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, cudaStream_t s) {
+cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
     // workspace body: the RMS scales, then the segments' end states
     uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
-    SegArgs sa = seg_plan(p);
+    if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;
+    SegArgs sa = seg_plan(p, body_bytes - rs_bytes(p));
     if (sa.nseg > 1) sa.st = reinterpret_cast<float*>(static_cast<char*>(ws_body) + rs_bytes(p));
     switch (p.R) {
         case 1: return launch_tc_t<1>(p, rs, sa, s);

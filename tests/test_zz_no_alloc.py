@@ -70,3 +70,19 @@ def test_noalloc_rejects_dims_beyond_its_scratch(cuda_dev):
     rc = lib.m3_scan_fwd_noalloc(ctypes.byref(dims), ctypes.byref(ins), None, None, fake, None)
     assert rc == m3.M3_ERR_UNSUPPORTED
     assert b"1 MiB" in lib.m3_last_error()
+
+
+def test_noalloc_runs_long_sequences_in_fewer_segments(cuda_dev):
+    # b1 H4 L2543 is cut into 5 segments by m3_scan_fwd; its 4 stored end states (~0.5 MiB)
+    # plus the RMS scales fit the fixed scratch. For b1 H32 L2543 one segment's 32 end states
+    # alone (~1 MiB) do not: it runs as one segment. Both must match m3_scan_fwd.
+    for H, seed in ((4, 81), (32, 82)):
+        pr = make_problem(1, 2543, H, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
+                          seed=seed, with_state=True)
+        g = pr.to(cuda_dev)
+        y_na, f_na = noalloc_scan(g, 64, True)
+        y_ref, f_ref = reference_scan(g, 64, True)
+        torch.cuda.synchronize()
+        tol = TOL[torch.bfloat16]
+        assert rel(y_na, y_ref.double().cpu().numpy()) <= tol
+        assert rel(f_na.h, f_ref.h.double().cpu().numpy()) <= tol
