@@ -82,6 +82,17 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, float (&v)[8])
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
+// Bulk copy of bytes (a multiple of 16, both addresses 16-byte aligned) from shared to global
+// memory, in this thread's current bulk async-group.
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(gdst), "r"(smem_u32(ssrc)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's bulk copies have read their sources (shared memory reusable) ...
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... or have completed (global writes done).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Byte offset of bf16 element (row, col) in a K-major tile with 32-byte rows and the 32-byte
 // swizzle (16-byte chunk c of row r stored at chunk c ^ ((r / 4) mod 2)).
 __device__ __forceinline__ uint32_t swz32(uint32_t row, uint32_t col) {
@@ -208,6 +219,7 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
             // the other slot held the previous unit, whose readout and copy-out have finished:
             // it takes the next unit, which then streams in while this one computes
             const int un = u + static_cast<int>(gridDim.x);
+            bulk_wait_read();   // the previous unit's stored-token copies have left its slot
             if (un < n_units) {
                 issue(un, s ^ 1);
                 ++issued[s ^ 1];
@@ -373,16 +385,14 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                                                           (((((j >> 1) ^ n) & 3) << 5) | ((j & 1) << 4)));
             }
         }
-        // last token's raw B and x become the stored previous token
-        {
+        // last token's raw B and x become the stored previous token: two bulk copies from the
+        // slot, by one thread (waited for before the slot is refilled)
+        if (tid == 0) {
             if (p.prevB1)
-                for (int e = tid; e < R * kN / 8; e += kThreads)
-                    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.prevB1) + static_cast<int64_t>(u) * R * kN)[e] =
-                        reinterpret_cast<const uint4*>(sB)[e];
+                bulk_store(static_cast<__nv_bfloat16*>(p.prevB1) + static_cast<int64_t>(u) * R * kN, sB, R * kN * 2);
             if (p.prevx1)
-                for (int e = tid; e < R * kP / 8; e += kThreads)
-                    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.prevx1) + static_cast<int64_t>(u) * R * kP)[e] =
-                        reinterpret_cast<const uint4*>(sx)[e];
+                bulk_store(static_cast<__nv_bfloat16*>(p.prevx1) + static_cast<int64_t>(u) * R * kP, sx, R * kP * 2);
+            bulk_commit();
         }
         if (!mbar_wait(&bar_y, mma_phase)) s_abort = 1;
         fence_after_sync();
@@ -412,6 +422,7 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
         fence_after_sync();
     }
     if (tid == 0) {
+        bulk_wait_all();
         if (s_abort && p.status) atomicExch(p.status, 1);
         // inputs requested but never waited for (only after a wait gave up): let them land
         for (int h = 0; h < kRing; ++h)
