@@ -252,7 +252,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         tma_load_5d(sm + Cfg::OC + 8192, &maps.C, &bar_c, kHalf, 0, ig, (cb + c) * Q, ib);
         s_issued[4] += 1;
     };
-    // Chunk scalars (one full warp): cumulative log-decay, gamma, trapezoid weight w, ...; the
+    // Chunk scalars (one full warp, warp 3: its masking share has no diagonal block, so it has
+    // the most slack while the MMAs run): cumulative log-decay, gamma, trapezoid weight w, ...; the
     // segment's summed log-decay accumulates in lam_acc
     float lam_acc = 0.f;
     auto scalars = [&](int c) {
@@ -630,7 +631,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     };
 
     if constexpr (kStateOnly) {
-        if (nchunks > 0 && warp == 1) scalars(0);
+        if (nchunks > 0 && warp == 3) scalars(0);
         __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
         for (int c = 0; c < nchunks && !s_abort; ++c) {
             const int st = c & 1;
@@ -670,7 +671,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 }
                 __syncwarp();
             }
-            if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
+            if (warp == 3 && c + 1 < nchunks) scalars(c + 1);
             {
                 if (!mbar_wait(&bar_dh, par)) s_abort = 1;
                 fence_after_sync();
@@ -692,7 +693,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             fence_after_sync();
         }
     } else {
-        if (nchunks > 0 && warp == 1) scalars(0);
+        if (nchunks > 0 && warp == 3) scalars(0);
         __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
         store_h0();
 
@@ -764,7 +765,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 }
                 __syncwarp();
             }
-            if (warp == 1 && c + 1 < nchunks) scalars(c + 1);
+            if (warp == 3 && c + 1 < nchunks) scalars(c + 1);
             {
                 const int trow = 16 * q4 + (lane & 15);   // row block q4
                 const int qc = wh + ((lane >> 4) ? 2 : 0);  // column block of this half-warp
@@ -877,7 +878,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             so[kN * kP + jp] = car[0];
             so[kN * kP + jp + 1] = car[1];
         }
-        if (warp == 1 && lane == 0) so[kN * kP + kHalf] = lam_acc;
+        if (warp == 3 && lane == 0) so[kN * kP + kHalf] = lam_acc;
     } else if (!s_abort) {
         // the sequence's final state, written by its last segment
         if (kseg == sa.nseg - 1) {
