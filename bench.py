@@ -26,7 +26,7 @@ sys.path.insert(0, ROOT)
 METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roofline"
 # DRAM bytes (read + write) of one scan launch on this workload from the ncu capture
 # summarised in profiles/scan_tc_siso_prefill_b4_L2048.md; None once the kernel changes.
-SCAN_TRAFFIC_BYTES = 186.75e6
+SCAN_TRAFFIC_BYTES = 186.93e6
 # kernels one scan launches: the per-token RMS-scale pre-pass of B and C, then the scan
 KERNELS_PER_SCAN = 2
 WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"
