@@ -93,7 +93,7 @@ typedef struct {
 /* Bytes of device workspace m3_scan_fwd needs for these dims (>= 256), or 0 if the dims are
  * invalid or unsupported: a 256-byte status header, the per-token RMS scales of B and C, and
  * for few long sequences (which the scan cuts into segments that run in parallel) one fp32
- * end state per sequence and segment but the last. Depends on the current device's SM count. */
+ * state per sequence and segment. Depends on the current device's SM count. */
 M3_API size_t m3_scan_workspace_bytes(const m3_dims* dims);
 
 /* Chunked parallel prefill scan over a whole sequence (Sec. 3.1.3 parallel form, Sec. 3.3

@@ -79,8 +79,8 @@ constexpr int F_SEG = 2 * F_BLK;           // [8 segments][32 lanes] float2
 constexpr int F_BIAS = F_SEG + 512;        // bias_B [R][128] bf16, bias_C [R][128] bf16
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
-// One segment's end state in the workspace (floats): h [N][P], the angle [N/2], the segment's
-// summed log-decay, padding to a multiple of 16 bytes.
+// One state slot in the workspace (floats): h [N][P], the angle [N/2], a segment's summed
+// log-decay, padding to a multiple of 16 bytes.
 constexpr int kSegStride = kN * kP + kHalf + 4;
 
 template <int R>
@@ -160,9 +160,12 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
 // nseg segments of seg_chunks chunks (the last may be shorter). A state-only pass computes each
 // segment's end state but the last's; the full pass then runs every segment at once from the
 // state at its start, which it assembles from those end states. nseg = 1 is the plain scan.
+// Per unit, slots 0 .. nseg-2 hold the segments' end states and slot nseg-1 the primed initial
+// state (the given state with the stored token folded in): the full pass reads no caller state,
+// so the final state may overwrite the initial one while other segments still run.
 struct SegArgs {
     int seg_chunks, nseg;
-    float* st;   // [units][nseg - 1][kSegStride]
+    float* st;   // [units][nseg][kSegStride]
 };
 
 // One CTA per (unit, segment), CTA index = segment * units + unit. kStateOnly: the segment's
@@ -362,7 +365,18 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // state rows owned by this thread: n = 32*q4 + lane, columns [32*wh, 32*wh + 32)
     const int nrow = 32 * q4 + lane;
     float hreg[32];
-    if (kseg == 0 && p.h0) {
+    // the full pass of a cut sequence takes every start state from the workspace
+    const bool from_ws = !kStateOnly && sa.nseg > 1;
+    if (from_ws) {
+        // segment 0's primed initial state; later segments assemble theirs below
+        const float4* src = reinterpret_cast<const float4*>(
+            sa.st + (u * sa.nseg + (kseg == 0 ? sa.nseg - 1 : 0)) * kSegStride + nrow * kP + 32 * wh);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 v = src[j];
+            hreg[4 * j] = v.x; hreg[4 * j + 1] = v.y; hreg[4 * j + 2] = v.z; hreg[4 * j + 3] = v.w;
+        }
+    } else if (kseg == 0 && p.h0) {
         const float4* src = reinterpret_cast<const float4*>(p.h0 + (u * kN + nrow) * kP + 32 * wh);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -383,12 +397,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     float car[2], car_r[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        car[j] = (kseg == 0 && p.phi0) ? p.phi0[u * kHalf + jp + j] : 0.f;
+        car[j] = (from_ws && kseg == 0) ? sa.st[(u * sa.nseg + sa.nseg - 1) * kSegStride + kN * kP + jp + j]
+               : (!from_ws && kseg == 0 && p.phi0) ? p.phi0[u * kHalf + jp + j] : 0.f;
         car_r[j] = reduce_2pi(car[j]);
     }
 
     // ---- fold the stored previous token into the primed state ----
-    if (kseg == 0 && p.h0 && L > 0) {
+    if (!from_ws && kseg == 0 && p.h0 && L > 0) {
         const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(p.prevB0) + u * R * kN;
         const __nv_bfloat16* px = static_cast<const __nv_bfloat16*>(p.prevx0) + u * R * kP;
         if (warp < R) {  // RMS scale of the stored raw B, one warp per rank
@@ -426,6 +441,21 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     }
 
+    // ---- the state-only pass keeps segment 0's primed initial state for the full pass ----
+    if constexpr (kStateOnly) {
+        if (kseg == 0) {
+            float* so = sa.st + (u * sa.nseg + sa.nseg - 1) * kSegStride;
+            float4* dst = reinterpret_cast<float4*>(so + nrow * kP + 32 * wh);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
+            if (warp == 0) {
+                so[kN * kP + jp] = car[0];
+                so[kN * kP + jp + 1] = car[1];
+            }
+        }
+    }
+
     // ---- the state at the start of a later segment (full pass) ----
     // Segment 0's end state is in the true frame. Each later segment j < kseg adds its own
     // contribution dH_j, computed from zero in its own frame, after decaying the state by its
@@ -435,7 +465,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // every chunk boundary), so no previous token is folded here.
     if constexpr (!kStateOnly) {
         if (kseg > 0) {
-            const float* sb = sa.st + u * (sa.nseg - 1) * kSegStride;
+            const float* sb = sa.st + u * sa.nseg * kSegStride;
             float* s_phis = reinterpret_cast<float*>(sm + Cfg::OH);   // [kseg][N/2], set-up only
             if (tid < kHalf) {
                 float acc = sb[kN * kP + tid];
@@ -443,14 +473,6 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 for (int j = 1; j < kseg; ++j) {
                     acc += sb[j * kSegStride + kN * kP + tid];
                     s_phis[j * kHalf + tid] = acc;
-                }
-            }
-            {
-                const float4* src = reinterpret_cast<const float4*>(sb + nrow * kP + 32 * wh);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 v = src[j];
-                    hreg[4 * j] = v.x; hreg[4 * j + 1] = v.y; hreg[4 * j + 2] = v.z; hreg[4 * j + 3] = v.w;
                 }
             }
             __syncthreads();
@@ -869,7 +891,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     if (!s_abort && kStateOnly) {
         // this segment's end state for the full pass: h, the angle sum (absolute for segment
         // 0), the summed log-decay
-        float* so = sa.st + (u * (sa.nseg - 1) + kseg) * kSegStride;
+        float* so = sa.st + (u * sa.nseg + kseg) * kSegStride;
         float4* dst = reinterpret_cast<float4*>(so + nrow * kP + 32 * wh);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -993,7 +1015,7 @@ SegArgs seg_plan(const ScanParams& p, size_t seg_bytes = ~size_t(0)) {
     S = std::min(S, nch / kMinSegChunks);
     S = std::min(S, kMaxSeg);
     const size_t per_seg = static_cast<size_t>(units) * kSegStride * sizeof(float);
-    while (S >= 2 && static_cast<size_t>(S - 1) * per_seg > seg_bytes) --S;
+    while (S >= 2 && static_cast<size_t>(S) * per_seg > seg_bytes) --S;   // nseg slots per unit
     if (S < 2) return sa;
     sa.seg_chunks = static_cast<int>((nch + S - 1) / S);
     sa.nseg = static_cast<int>((nch + sa.seg_chunks - 1) / sa.seg_chunks);
@@ -1011,7 +1033,7 @@ size_t rs_bytes(const ScanParams& p) {
 
 size_t tc_scan_workspace_bytes(const ScanParams& p) {
     const SegArgs sa = seg_plan(p);
-    const size_t seg = sa.nseg > 1 ? static_cast<size_t>(p.b * p.H) * (sa.nseg - 1) * kSegStride * sizeof(float) : 0;
+    const size_t seg = sa.nseg > 1 ? static_cast<size_t>(p.b * p.H) * sa.nseg * kSegStride * sizeof(float) : 0;
     return rs_bytes(p) + seg;
 }
 

@@ -66,18 +66,20 @@ def test_workspace_query_validates(lib, kw, ok):
 
 
 def test_workspace_holds_segment_states_for_long_sequences(lib):
-    """Few long sequences run in segments: the workspace grows by one end state per unit and
-    segment but the last (fp32 h [N][P], angle [N/2], log-decay, padding); many short ones do
-    not. Without a GPU the SM count is taken as 148 (two CTAs each: 296 slots)."""
+    """Few long sequences run in segments: the workspace grows by one state slot (fp32 h [N][P],
+    angle [N/2], log-decay, padding) per unit and segment (the segments' end states but the
+    last's, and the primed initial state); many short sequences do not. Without a GPU the SM
+    count is taken as 148 (two CTAs each: 296 slots)."""
     stride = (128 * 64 + 64 + 4) * 4
     def ws(**kw):
         return lib.m3_scan_workspace_bytes(ctypes.byref(dims(bc_norm=0, **kw)))
     base = ws(batch=1, nheads=64, seqlen=64)              # one chunk: never segmented
     assert ws(batch=4, nheads=64, seqlen=2048) == base     # 256 units fill the SMs already
-    # b1 H64 L65536: 296 // 64 = 4 segments of 256 chunks -> 3 stored states per unit
-    assert ws(batch=1, nheads=64, seqlen=65536) == base + 64 * 3 * stride
+    # b1 H64 L65536: 296 // 64 = 4 segments of 256 chunks -> 4 slots per unit
+    r256 = lambda n: (n + 255) // 256 * 256                # the body is 256-byte aligned
+    assert ws(batch=1, nheads=64, seqlen=65536) == base + r256(64 * 4 * stride)
     # b1 H4 L2543: 40 chunks, at least 8 per segment -> 5 segments
-    assert ws(batch=1, nheads=4, seqlen=2543) == base + 4 * 4 * stride
+    assert ws(batch=1, nheads=4, seqlen=2543) == base + r256(4 * 5 * stride)
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any launch

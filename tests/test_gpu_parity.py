@@ -78,6 +78,20 @@ def test_scan_segmented(cuda_dev, case):
     compare(pr, y, fin, yo, so)
 
 
+def test_segmented_final_state_may_alias_init(cuda_dev):
+    """In place with the sequence-parallel form (b1 H4 L2543: 5 segments): the last segment
+    writes the final state while segment 0 runs, so the full pass must not read the caller's
+    initial state; the result must match the oracle from the original state."""
+    pr = make_problem(1, 2543, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
+                      seed=23, with_state=True)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    y, fin = m3.scan_fwd(**g.tensors(), init=st, final=st, chunk=64, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr, use_state=True)
+    compare(pr, y, fin, yo, so)
+
+
 def test_final_state_may_alias_init(cuda_dev):
     pr = make_problem(2, 150, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
                       seed=5, with_state=True)

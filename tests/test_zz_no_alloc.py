@@ -73,9 +73,9 @@ def test_noalloc_rejects_dims_beyond_its_scratch(cuda_dev):
 
 
 def test_noalloc_runs_long_sequences_in_fewer_segments(cuda_dev):
-    # b1 H4 L2543 is cut into 5 segments by m3_scan_fwd; its 4 stored end states (~0.5 MiB)
-    # plus the RMS scales fit the fixed scratch. For b1 H32 L2543 one segment's 32 end states
-    # alone (~1 MiB) do not: it runs as one segment. Both must match m3_scan_fwd.
+    # b1 H4 L2543 is cut into 5 segments by m3_scan_fwd; its 5 state slots per sequence
+    # (~0.6 MiB) plus the RMS scales fit the fixed scratch. For b1 H32 L2543 one slot per
+    # sequence alone (~1 MiB) does not: it runs as one segment. Both must match m3_scan_fwd.
     for H, seed in ((4, 81), (32, 82)):
         pr = make_problem(1, 2543, H, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
                           seed=seed, with_state=True)
