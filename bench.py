@@ -233,6 +233,31 @@ def run_ours(args):
         for R in (1, 4):
             decode[f"R{R}"] = bench_decode(m3, dev, R, args.decode_steps, hbm, world, dist)
 
+    # ---- the fused scalar prologue: dt and lam passed raw, softplus / sigmoid applied in the
+    # kernels (same workloads, one input set each) ----
+    prologue = {}
+    if not args.no_decode:
+        praw = make_config(1, device=dev, seed=rank_seed(rank, 0), raw_scalars=True)
+
+        def step_raw():
+            m3.scan_fwd(**praw.tensors(), **praw.scalar_args(), init=None, final=fin, y=y,
+                        workspace=ws, chunk=d.chunk, bc_norm=True, stream=stream)
+
+        for _ in range(3):
+            step_raw()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(10):
+            step_raw()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        pms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev) / 10
+        prologue["prefill_ms"] = pms
+        prologue["prefill_frac_hbm"] = scan_bytes(praw) / (pms / 1e3) / 1e9 / hbm
+        del praw
+        prologue["decode_R4"] = bench_decode(m3, dev, 4, args.decode_steps, hbm, world, dist,
+                                             raw=True)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -251,6 +276,7 @@ def run_ours(args):
         "gpu_launches": args.steps * KERNELS_PER_SCAN,
         "clocks": clk.summary(),
         "decode": decode,
+        "fused_scalar_prologue": prologue,
     }
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
@@ -260,10 +286,10 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def bench_decode(m3, dev, R, steps, hbm, world, dist):
+def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False):
     import torch
     from state_space_sequence_mamba_b200.inputs import make_decode
-    pr = make_decode(R, steps, device=dev)
+    pr = make_decode(R, steps, device=dev, raw_scalars=raw)
     st = m3.State.from_dict({k: v.clone() for k, v in pr.state.items()})
     yb = torch.empty(pr.dims.batch, pr.dims.nheads, R, pr.dims.headdim, dtype=torch.bfloat16,
                      device=dev)
@@ -273,6 +299,7 @@ def bench_decode(m3, dev, R, steps, hbm, world, dist):
     def run(n):
         for t in range(n):
             m3.decode_step(pr.x[t], pr.B[t], pr.C[t], pr.theta[t], pr.dt[t], pr.A[t], pr.lam[t],
+                           dt_bias=pr.dt_bias, flags=pr.flags,
                            state_in=st, y=yb, stream=s)
 
     with torch.cuda.stream(s):

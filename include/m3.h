@@ -65,7 +65,19 @@ typedef struct {
     int32_t in_dtype; /* m3_dtype                                                   */
     int32_t bc_norm;  /* nonzero: RMS-normalise B and C over N before the bias      */
     float norm_eps;   /* epsilon of the RMS norm (1e-6 is the usual value)          */
+    uint32_t flags;   /* M3_DT_SOFTPLUS | M3_LAM_SIGMOID, or 0                      */
 } m3_dims;
+
+/* m3_dims.flags: the step scalars arrive as the layer's raw projections and the kernels
+ * apply the parameterisation themselves (the fused scalar prologue), per token and head:
+ *   M3_DT_SOFTPLUS: dt holds the raw projection d; the step size is
+ *                   softplus(d + dt_bias[h]) = log(1 + e^{d + dt_bias[h]}) > 0 (the step
+ *                   is a positive projection of the token, Sec. 2 "Mamba-2 parameterisation").
+ *   M3_LAM_SIGMOID: lam holds u; the trapezoid weight is sigma(u) = 1 / (1 + e^{-u})
+ *                   (Appendix F, default parameterisation lambda_t = sigma(u_t)).
+ * Positions past the end of the sequence are not tokens and stay zero. */
+#define M3_DT_SOFTPLUS 1u
+#define M3_LAM_SIGMOID 2u
 
 typedef struct {
     const void* x;        /* [b, L, H, R, P]   in_dtype                                   */
@@ -73,11 +85,14 @@ typedef struct {
     const void* C;        /* [b, L, G, R, N]   in_dtype, raw                              */
     const void* theta;    /* [b, L, H, N/2]    in_dtype: per-step angle rate; the step's
                              rotation angle is dt * theta (Prop. 2)                     */
-    const float* dt;      /* [b, L, H] step size, > 0 (after softplus)                     */
+    const float* dt;      /* [b, L, H] step size, > 0 (raw projection with M3_DT_SOFTPLUS) */
     const float* A;       /* [b, L, H] decay rate, < 0                                     */
-    const float* lam;     /* [b, L, H] trapezoid weight in [0, 1] (lam = 1: Euler)         */
+    const float* lam;     /* [b, L, H] trapezoid weight in [0, 1] (lam = 1: Euler), or the
+                             raw u of sigma(u) with M3_LAM_SIGMOID                         */
     const float* B_bias;  /* [H, R, N] added after the norm, or NULL for zero              */
     const float* C_bias;  /* [H, R, N] or NULL                                             */
+    const float* dt_bias; /* [H] added to dt before the softplus (M3_DT_SOFTPLUS only), or
+                             NULL for zero                                                 */
 } m3_inputs;
 
 /* Recurrent state of every (batch, head) unit. Each unit owns its slice of every field. */

@@ -106,17 +106,41 @@ class State:
         return State(self.h.copy(), self.phi.copy(), self.prev_B.copy(), self.prev_x.copy())
 
 
+DT_SOFTPLUS, LAM_SIGMOID = 1, 2
+
+
+def step_scalars(dt, lam, dt_bias=None, flags: int = 0):
+    """The step scalars from the layer's raw projections, in float64 (dt, lam [..., H];
+    dt_bias [H] or None).
+
+    DT_SOFTPLUS: the step is softplus(dt + dt_bias) = log(1 + e^{dt + dt_bias}). The paper
+    says only that the step is a positive projection of the token (Sec. 2, the Mamba-2
+    parameterisation); softplus is the reading taken. LAM_SIGMOID: the trapezoid weight is
+    sigmoid(u) = 1 / (1 + e^{-u}) (Appendix F, default parameterisation lambda_t = sigma(u_t))."""
+    dt, lam = _f64(dt), _f64(lam)
+    if flags & DT_SOFTPLUS:
+        v = dt + (0.0 if dt_bias is None else _f64(dt_bias))
+        dt = np.logaddexp(0.0, v)
+    if flags & LAM_SIGMOID:
+        e = np.exp(-np.abs(lam))
+        lam = np.where(lam >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return dt, lam
+
+
 def scan(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state: State | None = None,
-         bc_norm: bool = False, norm_eps: float = 1e-6, nthreads: int = 0):
+         bc_norm: bool = False, norm_eps: float = 1e-6, nthreads: int = 0, dt_bias=None,
+         flags: int = 0):
     """Runs the sequential recurrence over a whole sequence.
 
     Shapes: x [b,L,H,R,P]; B, C [b,L,G,R,N]; theta [b,L,H,N/2]; dt, A, lam [b,L,H];
     B_bias, C_bias [H,R,N] or None. ``state`` (float64, not modified) is the state before
-    the first token, or None for a fresh sequence (all zeros).
+    the first token, or None for a fresh sequence (all zeros). ``flags`` and ``dt_bias``:
+    dt and lam are raw projections, see ``step_scalars``.
 
     Returns (y [b,L,H,R,P] float64, final State)."""
     x, B, C, theta = _f64(x), _f64(B), _f64(C), _f64(theta)
-    dt, A, lam = _f64(dt), _f64(A), _f64(lam)
+    dt, lam = step_scalars(dt, lam, dt_bias, flags)
+    A = _f64(A)
     B_bias = None if B_bias is None else _f64(B_bias)
     C_bias = None if C_bias is None else _f64(C_bias)
     b, L, H, R, P = x.shape
@@ -142,7 +166,7 @@ def scan(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state: State | No
 
 def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None,
                 state: State | None = None, bc_norm: bool = False, norm_eps: float = 1e-6,
-                nthreads: int = 0):
+                nthreads: int = 0, dt_bias=None, flags: int = 0):
     """One token: x [b,H,R,P]; B, C [b,G,R,N]; theta [b,H,N/2]; dt, A, lam [b,H].
 
     Exactly one iteration of ``scan``. Returns (y [b,H,R,P], new State)."""
@@ -150,5 +174,5 @@ def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None,
         a = _f64(a)
         return a[:, None]
     y, st = scan(tok(x), tok(B), tok(C), tok(theta), tok(dt), tok(A), tok(lam), B_bias,
-                 C_bias, state, bc_norm, norm_eps, nthreads)
+                 C_bias, state, bc_norm, norm_eps, nthreads, dt_bias, flags)
     return y[:, 0], st

@@ -16,6 +16,8 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
 M3_F32, M3_BF16 = 0, 1
+# m3_dims.flags: the step scalars arrive raw and the kernels apply softplus / sigmoid
+M3_DT_SOFTPLUS, M3_LAM_SIGMOID = 1, 2
 
 
 class M3Error(RuntimeError):
@@ -30,12 +32,12 @@ class Dims(ctypes.Structure):
                 ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64),
                 ("rank", ctypes.c_int64), ("chunk", ctypes.c_int64),
                 ("in_dtype", ctypes.c_int32), ("bc_norm", ctypes.c_int32),
-                ("norm_eps", ctypes.c_float)]
+                ("norm_eps", ctypes.c_float), ("flags", ctypes.c_uint32)]
 
 
 class Inputs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("x", "B", "C", "theta", "dt", "A", "lam", "B_bias", "C_bias")]
+                ("x", "B", "C", "theta", "dt", "A", "lam", "B_bias", "C_bias", "dt_bias")]
 
 
 class StateC(ctypes.Structure):
@@ -129,11 +131,11 @@ class State:
         return StateC(*(_ptr(t) for t in (self.h, self.phi, self.prev_B, self.prev_x)))
 
 
-def make_dims(x, B, chunk, bc_norm, norm_eps):
+def make_dims(x, B, chunk, bc_norm, norm_eps, flags=0):
     b, L, H, R, P = x.shape
     G, N = B.shape[2], B.shape[4]
     return Dims(b, L, H, G, P, N, R, int(chunk), _dtype_code(x.dtype), 1 if bc_norm else 0,
-                float(norm_eps))
+                float(norm_eps), int(flags))
 
 
 def scan_workspace_bytes(dims: Dims) -> int:
@@ -148,13 +150,14 @@ def _stream_handle(stream):
 
 def scan_fwd(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, init: State | None = None,
              final: State | None | bool = True, y=None, workspace=None, chunk=64,
-             bc_norm=False, norm_eps=1e-6, stream=None):
-    """m3_scan_fwd on torch CUDA tensors (shapes as in include/m3.h).
+             bc_norm=False, norm_eps=1e-6, stream=None, dt_bias=None, flags=0):
+    """m3_scan_fwd on torch CUDA tensors (shapes as in include/m3.h). ``flags``
+    (M3_DT_SOFTPLUS | M3_LAM_SIGMOID) passes dt and lam raw, with ``dt_bias`` [H].
 
     ``final=True`` allocates a new State for the result, ``False``/None skips it, or pass a
     State (it may be ``init`` itself). Returns (y, final State or None)."""
     lib = load_library()
-    dims = make_dims(x, B, chunk, bc_norm, norm_eps)
+    dims = make_dims(x, B, chunk, bc_norm, norm_eps, flags)
     dev = x.device
     if y is None:
         y = torch.empty_like(x)
@@ -169,7 +172,7 @@ def scan_fwd(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, init: State |
         need = 256
     if workspace is None:
         workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
-    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias)))
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias, dt_bias)))
     ic = init.c() if init is not None else None
     fc = final.c() if final is not None else None
     rc = lib.m3_scan_fwd(ctypes.byref(dims), ctypes.byref(ins),
@@ -186,18 +189,18 @@ def scan_check(workspace):
 
 def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state_in: State = None,
                 state_out: State | None = None, y=None, bc_norm=False, norm_eps=1e-6,
-                stream=None):
+                stream=None, dt_bias=None, flags=0):
     """m3_decode_step: x [b,1,H,R,P], B, C [b,1,G,R,N], theta [b,1,H,N/2], dt/A/lam [b,1,H].
 
     ``state_out`` defaults to ``state_in`` (in-place). Returns (y [b,H,R,P], state_out)."""
     lib = load_library()
-    dims = make_dims(x, B, 1, bc_norm, norm_eps)
+    dims = make_dims(x, B, 1, bc_norm, norm_eps, flags)
     if state_out is None:
         state_out = state_in
     if y is None:
         y = torch.empty(dims.batch, dims.nheads, dims.rank, dims.headdim, dtype=x.dtype,
                         device=x.device)
-    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias)))
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias, dt_bias)))
     si, so = state_in.c(), state_out.c()
     rc = lib.m3_decode_step(ctypes.byref(dims), ctypes.byref(ins), ctypes.byref(si),
                             ctypes.byref(so), _ptr(y), _stream_handle(stream))

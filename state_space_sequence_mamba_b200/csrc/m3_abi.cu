@@ -42,6 +42,8 @@ m3_status check_dims(const m3_dims* d, bool scan) {
         return fail(M3_ERR_INVALID_ARG, "headdim >= 1, even dstate >= 2 and rank >= 1 required");
     if (!(d->norm_eps >= 0.f) || !std::isfinite(d->norm_eps))
         return fail(M3_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
+    if (d->flags & ~(M3_DT_SOFTPLUS | M3_LAM_SIGMOID))
+        return fail(M3_ERR_INVALID_ARG, "unknown bits in flags (0x%x)", (unsigned)d->flags);
     if (d->headdim != 16 && d->headdim != 32 && d->headdim != 64 && d->headdim != 128)
         return fail(M3_ERR_UNSUPPORTED, "headdim %lld not in {16, 32, 64, 128}",
                     (long long)d->headdim);
@@ -73,6 +75,8 @@ m3_status check_inputs(const m3_inputs* in, bool need) {
     }
     if (in->B_bias && !aligned16(in->B_bias)) return fail(M3_ERR_INVALID_ARG, "B_bias misaligned");
     if (in->C_bias && !aligned16(in->C_bias)) return fail(M3_ERR_INVALID_ARG, "C_bias misaligned");
+    if (in->dt_bias && (reinterpret_cast<uintptr_t>(in->dt_bias) & 3u) != 0)
+        return fail(M3_ERR_INVALID_ARG, "dt_bias misaligned");
     return M3_OK;
 }
 
@@ -96,6 +100,7 @@ ScanParams make_params(const m3_dims* d, const m3_inputs* in, const m3_state* in
     p.bc_norm = d->bc_norm ? 1 : 0; p.eps = d->norm_eps;
     p.x = in->x; p.B = in->B; p.C = in->C; p.theta = in->theta;
     p.dt = in->dt; p.A = in->A; p.lam = in->lam; p.Bbias = in->B_bias; p.Cbias = in->C_bias;
+    p.dt_bias = in->dt_bias; p.flags = d->flags;
     if (init) { p.h0 = init->h; p.phi0 = init->phi; p.prevB0 = init->prev_B; p.prevx0 = init->prev_x; }
     if (fin) { p.h1 = fin->h; p.phi1 = fin->phi; p.prevB1 = fin->prev_B; p.prevx1 = fin->prev_x; }
     p.y = y;

@@ -25,6 +25,30 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
+// The step scalars of one token from what the caller passed (the fused scalar prologue):
+// with the flag, dt holds the raw projection and the step is softplus(raw + bias), and lam
+// holds u and the trapezoid weight is sigmoid(u). Calls only cover real tokens: positions past
+// the end of a sequence keep their zeros. kRaw = false (no flag set) compiles to the identity,
+// so kernels instantiated for plain scalars carry none of this code.
+template <bool kRaw = true>
+__device__ __forceinline__ float step_dt(float raw, float bias, uint32_t flags) {
+    if constexpr (!kRaw) {
+        return raw;
+    } else {
+        if (!(flags & 1u)) return raw;
+        // softplus(v) = max(v, 0) + log(1 + e^{-|v|}): the exponential never overflows and the
+        // logarithm's argument stays in (1, 2]. Below v ~ -16 the log term rounds to zero (an
+        // absolute error of e^v < 1e-7 in a step that is then negligible).
+        const float v = raw + bias;
+        return fmaxf(v, 0.f) + __logf(1.f + __expf(-fabsf(v)));
+    }
+}
+template <bool kRaw = true>
+__device__ __forceinline__ float step_lam(float raw, uint32_t flags) {
+    if constexpr (!kRaw) return raw;
+    else return (flags & 2u) ? __frcp_rn(1.f + __expf(-raw)) : raw;   // e^{-raw} = inf gives 0
+}
+
 // Inclusive prefix sum across the 32 lanes of a warp.
 __device__ __forceinline__ float warp_inclusive_scan(float v) {
     const int lane = threadIdx.x & 31;

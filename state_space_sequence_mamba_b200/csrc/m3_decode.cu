@@ -80,7 +80,8 @@ decode_kernel(const ScanParams p, const int rows_per_pass) {
         xps[i] = to_f(xpin[i]);
     }
     if (tid == 0) {
-        const float d = p.dt[u], a = p.A[u], l = p.lam[u];
+        const float d = step_dt(p.dt[u], p.dt_bias ? p.dt_bias[u % p.H] : 0.f, p.flags);
+        const float a = p.A[u], l = step_lam(p.lam[u], p.flags);
         const float al = expf(d * a);
         scal[0] = al;
         scal[1] = (1.f - l) * d * al;

@@ -82,7 +82,8 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-template <int R>
+// kRaw: dt and lam arrive raw (m3_dims.flags); the step scalars apply softplus / sigmoid.
+template <int R, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_bulk_kernel(const ScanParams p, const int n_units) {
     extern __shared__ uint8_t smem_raw[];
@@ -139,9 +140,10 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
         if (u < n_units) {
             issue(u, 0);
             issued[0] = 1;
-            sc[0] = p.dt[u];
+            sc[0] = step_dt<kRaw>(p.dt[u], (kRaw && p.dt_bias) ? p.dt_bias[u % static_cast<int>(p.H)] : 0.f,
+                                    p.flags);
             sc[1] = p.A[u];
-            sc[2] = p.lam[u];
+            sc[2] = step_lam<kRaw>(p.lam[u], p.flags);
         }
     }
     __syncthreads();
@@ -150,7 +152,7 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
         const int b = i & 1;
         uint8_t* base = sm + b * bl.total;
         const int un = u + gridDim.x;
-        float snext[3] = {0.f, 0.f, 0.f};
+        float snext[4] = {0.f, 0.f, 0.f, 0.f};   // raw dt, A, raw lam, dt bias
         if (tid == 0) {
             // the other half held the previous unit, whose state is being stored from it
             // ...and is free for the next unit once that store has read it: request the next
@@ -162,6 +164,7 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
                 snext[0] = p.dt[un];
                 snext[1] = p.A[un];
                 snext[2] = p.lam[un];
+                if constexpr (kRaw) snext[3] = p.dt_bias ? p.dt_bias[un % static_cast<int>(p.H)] : 0.f;
             }
             if (mbar_wait_sleep(&bar[b], (i >> 1) & 1)) ++waited[b];
             else s_abort = 1;
@@ -303,6 +306,7 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
             for (; n < N; n += RP) update(n);
         }
         fence_proxy_async();  // the updated state is read by the bulk store
+
         float yacc[R][4];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -347,9 +351,9 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
                 reinterpret_cast<uint4*>(px1)[e] = reinterpret_cast<const uint4*>(sx)[e];
         }
         if (tid == 0) {
-            sc[4 * (b ^ 1) + 0] = snext[0];
+            sc[4 * (b ^ 1) + 0] = step_dt<kRaw>(snext[0], snext[3], p.flags);
             sc[4 * (b ^ 1) + 1] = snext[1];
-            sc[4 * (b ^ 1) + 2] = snext[2];
+            sc[4 * (b ^ 1) + 2] = step_lam<kRaw>(snext[2], p.flags);
         }
         __syncthreads();
     }
@@ -385,7 +389,7 @@ static cudaError_t launch_bulk_t(const ScanParams& p, cudaStream_t s) {
             sms = 148;
     }
     const size_t smem = decode_bulk_smem_bytes(p);
-    auto k = decode_bulk_kernel<R>;
+    auto k = p.flags ? decode_bulk_kernel<R, true> : decode_bulk_kernel<R, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;

@@ -138,7 +138,8 @@ __device__ __forceinline__ void store_kvec(uint8_t* tile, int n, int k0, const f
     }
 }
 
-template <int R>
+// kRaw: dt and lam arrive raw (m3_dims.flags); the step scalars apply softplus / sigmoid.
+template <int R, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const int n_units) {
     using Cfg = DecCfg<R>;
@@ -189,9 +190,10 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
         if (u < n_units) {
             issue(u, 0);
             ++issued[0];
-            scal[0] = p.dt[u];
+            scal[0] = step_dt<kRaw>(p.dt[u], (kRaw && p.dt_bias) ? p.dt_bias[u % static_cast<int>(p.H)] : 0.f,
+                                    p.flags);
             scal[1] = p.A[u];
-            scal[2] = p.lam[u];
+            scal[2] = step_lam<kRaw>(p.lam[u], p.flags);
         }
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
@@ -211,8 +213,9 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
     for (int i = 0; u < n_units; ++i, u += gridDim.x) {
         const int s = i % kRing;
         // the next unit's dt, A, lam: loaded into registers now, stored to its slot at the end
-        // of this unit, so the load latency is spent on this unit's work
-        float snext[3] = {0.f, 0.f, 0.f};
+        // of this unit (raw scalars transformed there), so the load latency is spent on this
+        // unit's work
+        float snext[4] = {0.f, 0.f, 0.f, 0.f};   // dt, A, lam, dt bias
         uint8_t* sl = sm + Cfg::SM0 + s * Cfg::S_BYTES;
         uint8_t* hb = sm + Cfg::HB + s * Cfg::H_BYTES;
         if (tid == 0) {
@@ -226,6 +229,7 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                 snext[0] = p.dt[un];
                 snext[1] = p.A[un];
                 snext[2] = p.lam[un];
+                if constexpr (kRaw) snext[3] = p.dt_bias ? p.dt_bias[un % static_cast<int>(p.H)] : 0.f;
             }
             if (mbar_wait_sleep(&bar_full[s], static_cast<uint32_t>((i / kRing) & 1))) ++waited[s];
             else s_abort = 1;
@@ -413,9 +417,9 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
             }
         }
         if (tid == 0) {
-            scal[4 * (s ^ 1) + 0] = snext[0];
+            scal[4 * (s ^ 1) + 0] = step_dt<kRaw>(snext[0], snext[3], p.flags);
             scal[4 * (s ^ 1) + 1] = snext[1];
-            scal[4 * (s ^ 1) + 2] = snext[2];
+            scal[4 * (s ^ 1) + 2] = step_lam<kRaw>(snext[2], p.flags);
         }
         fence_before_sync();
         __syncthreads();
@@ -475,7 +479,7 @@ cudaError_t launch_tc_t(const ScanParams& p, cudaStream_t s) {
     DecMaps maps;
     if (!encode_state(&maps.h0, p.h0, units)) return cudaErrorInvalidValue;
     const uint32_t smem = DecCfg<R>::TOTAL;
-    auto k = decode_tc_kernel<R>;
+    auto k = p.flags ? decode_tc_kernel<R, true> : decode_tc_kernel<R, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;

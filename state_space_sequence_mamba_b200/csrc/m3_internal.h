@@ -22,6 +22,8 @@ struct ScanParams {
     const float* lam;
     const float* Bbias;  // may be null
     const float* Cbias;  // may be null
+    const float* dt_bias;  // [H], may be null; read only with M3_DT_SOFTPLUS
+    uint32_t flags;        // M3_DT_SOFTPLUS | M3_LAM_SIGMOID
     // initial state; all null = zero state
     const float* h0;
     const float* phi0;

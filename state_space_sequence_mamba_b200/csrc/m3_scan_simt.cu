@@ -77,6 +77,9 @@ __global__ void __launch_bounds__(kSimtThreads) scan_simt_kernel(const ScanParam
     const float* biasB = p.Bbias ? p.Bbias + hh * R * N : nullptr;
     const float* biasC = p.Cbias ? p.Cbias + hh * R * N : nullptr;
     auto sidx = [&](int64_t t) { return (bb * L + t) * p.H + hh; };  // dt/A/lam index
+    const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
+    auto dt_at = [&](int64_t t) { return step_dt(p.dt[sidx(t)], dtb, p.flags); };
+    auto lam_at = [&](int64_t t) { return step_lam(p.lam[sidx(t)], p.flags); };
 
     // ---- initial state ----
     for (int64_t e = tid; e < N * P; e += nth) Hs[e] = p.h0 ? p.h0[u * N * P + e] : 0.f;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kSimtThreads) scan_simt_kernel(const ScanParam
             }
         }
         __syncthreads();
-        const float f = (1.f - p.lam[sidx(0)]) * p.dt[sidx(0)];
+        const float f = (1.f - lam_at(0)) * dt_at(0);
         for (int64_t e = tid; e < N * P; e += nth) {
             const int64_t n = e / P, pp = e % P;
             float acc = 0.f;
@@ -125,12 +128,12 @@ __global__ void __launch_bounds__(kSimtThreads) scan_simt_kernel(const ScanParam
             float cum = 0.f;
             for (int64_t t = 0; t < T_; ++t) {
                 const int64_t si = sidx(c0 + t);
-                const float d = p.dt[si], a = p.A[si], l = p.lam[si];
+                const float d = dt_at(c0 + t), a = p.A[si], l = lam_at(c0 + t);
                 cum += d * a;
                 float w = l * d;
                 if (c0 + t + 1 < L) {
                     const int64_t sn = sidx(c0 + t + 1);
-                    w += (1.f - p.lam[sn]) * p.dt[sn];
+                    w += (1.f - lam_at(c0 + t + 1)) * dt_at(c0 + t + 1);
                 }
                 sc[8 * t + 0] = d;
                 sc[8 * t + 1] = cum;

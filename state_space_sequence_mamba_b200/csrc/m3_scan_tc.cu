@@ -171,7 +171,8 @@ struct SegArgs {
 // One CTA per (unit, segment), CTA index = segment * units + unit. kStateOnly: the segment's
 // end state only (no C, S, Yo, Yd, y); segment 0 starts from the given initial state in the
 // true angle frame, later segments from zero in their own frame (angle 0 at their start).
-template <int R, bool kStateOnly>
+// kRaw: dt and lam arrive raw (m3_dims.flags) and the chunk scalars apply softplus / sigmoid.
+template <int R, bool kStateOnly, bool kRaw>
 __global__ void __launch_bounds__(kTcThreads, 2)
 scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow,
                const SegArgs sa) {
@@ -259,6 +260,27 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // the most slack while the MMAs run): cumulative log-decay, gamma, trapezoid weight w, ...; the
     // segment's summed log-decay accumulates in lam_acc
     float lam_acc = 0.f;
+    const float dtb = (kRaw && p.dt_bias) ? p.dt_bias[hh] : 0.f;   // only read with M3_DT_SOFTPLUS
+    // kRaw: the dt and lam boxes of chunk c arrive raw; threads apply softplus(dt + dt_bias) and
+    // sigmoid(lam) in place to this head's column (the box holds 4 heads; the others are not
+    // read), real tokens only (positions past the sequence end stay zero), ahead of scalars(c).
+    auto raw_box = [&](int c) {
+        const int st = c & 1;
+        float* sSc = reinterpret_cast<float*>(sm + (st ? Cfg::SC1 : Cfg::SC0));
+        const int t0 = (cb + c) * Q;
+        constexpr int kCol = Q + 1;   // tokens in the box
+        for (int i = tid; i < 2 * kCol; i += kTcThreads) {
+            const int t = i < kCol ? i : i - kCol;
+            if (t0 + t >= L) continue;
+            if (i < kCol) {
+                float* d = sSc + t * 4 + hc;
+                *d = step_dt<true>(*d, dtb, p.flags);
+            } else {
+                float* lm = sSc + 2 * Cfg::SC_SLOT / 4 + t * 4 + hc;
+                *lm = step_lam<true>(*lm, p.flags);
+            }
+        }
+    };
     auto scalars = [&](int c) {
         const int st = c & 1;
         if (!mbar_wait(&bar_sc[st], (c >> 1) & 1)) {
@@ -431,7 +453,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
         __syncthreads();
         const int64_t s0 = bb * p.L * p.H + hh;
-        const float f = (1.f - p.lam[s0]) * p.dt[s0];
+        const float f = (1.f - step_lam<kRaw>(p.lam[s0], p.flags)) *
+                        step_dt<kRaw>(p.dt[s0], dtb, p.flags);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             float acc = 0.f;
@@ -653,6 +676,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     };
 
     if constexpr (kStateOnly) {
+        if constexpr (kRaw) {
+            if (nchunks > 0) {
+                if (!mbar_wait(&bar_sc[0], 0)) s_abort = 1;
+                raw_box(0);
+                __syncthreads();
+            }
+        }
         if (nchunks > 0 && warp == 3) scalars(0);
         __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
         for (int c = 0; c < nchunks && !s_abort; ++c) {
@@ -661,6 +691,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             const float* blk = sf + st * F_BLK;
             // ======== I1: angles and rotation of B; X(c+1) (its buffer was last read by X'(c-1));
             // the X' operand ========
+            if constexpr (kRaw) {
+                if (c + 1 < nchunks) {   // the next chunk's raw scalars, for scalars(c+1) in I2, while
+                                         // theta(c) lands
+                    if (!mbar_wait(&bar_sc[(c + 1) & 1], ((c + 1) >> 1) & 1)) s_abort = 1;
+                    raw_box(c + 1);
+                }
+            }
             if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
             rotate(blk, par);
             if (warp == kIssueWarp) {
@@ -715,6 +752,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             fence_after_sync();
         }
     } else {
+        if constexpr (kRaw) {
+            if (nchunks > 0) {
+                if (!mbar_wait(&bar_sc[0], 0)) s_abort = 1;
+                raw_box(0);
+                __syncthreads();
+            }
+        }
         if (nchunks > 0 && warp == 3) scalars(0);
         __syncthreads();   // also: the fold's scratch in the H0 buffer has been read
         store_h0();
@@ -725,6 +769,13 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
             const float* blk = sf + st * F_BLK;
 
             // ======== I1: rotation(c); then epilogue(c-1), the H0 and X' operands ========
+            if constexpr (kRaw) {
+                if (c + 1 < nchunks) {   // the next chunk's raw scalars, for scalars(c+1) in I2, while
+                                         // theta(c) lands
+                    if (!mbar_wait(&bar_sc[(c + 1) & 1], ((c + 1) >> 1) & 1)) s_abort = 1;
+                    raw_box(c + 1);
+                }
+            }
             if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
             rotate(blk, par);
             // Yd(c-1) done: its X buffer takes X(c+1), and y(c-1) can be written
@@ -1039,7 +1090,7 @@ size_t tc_scan_workspace_bytes(const ScanParams& p) {
 
 size_t tc_scan_workspace_min_bytes(const ScanParams& p) { return rs_bytes(p); }
 
-template <int R>
+template <int R, bool kRaw>
 static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s) {
     constexpr int Q = 64 / R;
     TcMaps maps;
@@ -1093,7 +1144,7 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
     const uint32_t smem = tc_smem_bytes<R>();
     const int64_t units = p.b * p.H;
     if (sa.nseg > 1) {   // every segment's end state but the last's
-        auto ks = scan_tc_kernel<R, true>;
+        auto ks = scan_tc_kernel<R, true, kRaw>;
         cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
@@ -1101,7 +1152,7 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    auto k = scan_tc_kernel<R, false>;
+    auto k = scan_tc_kernel<R, false, kRaw>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -1116,11 +1167,12 @@ cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes
     if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;
     SegArgs sa = seg_plan(p, body_bytes - rs_bytes(p));
     if (sa.nseg > 1) sa.st = reinterpret_cast<float*>(static_cast<char*>(ws_body) + rs_bytes(p));
+    const bool raw = p.flags != 0;
     switch (p.R) {
-        case 1: return launch_tc_t<1>(p, rs, sa, s);
-        case 2: return launch_tc_t<2>(p, rs, sa, s);
-        case 4: return launch_tc_t<4>(p, rs, sa, s);
-        case 8: return launch_tc_t<8>(p, rs, sa, s);
+        case 1: return raw ? launch_tc_t<1, true>(p, rs, sa, s) : launch_tc_t<1, false>(p, rs, sa, s);
+        case 2: return raw ? launch_tc_t<2, true>(p, rs, sa, s) : launch_tc_t<2, false>(p, rs, sa, s);
+        case 4: return raw ? launch_tc_t<4, true>(p, rs, sa, s) : launch_tc_t<4, false>(p, rs, sa, s);
+        case 8: return raw ? launch_tc_t<8, true>(p, rs, sa, s) : launch_tc_t<8, false>(p, rs, sa, s);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -54,17 +54,24 @@ class Problem:
     B_bias: torch.Tensor | None = None   # [H, R, N] fp32
     C_bias: torch.Tensor | None = None   # [H, R, N] fp32
     state: dict | None = field(default=None)  # h, phi (fp32), prev_B, prev_x (dtype)
+    # raw step scalars: flags = 3 (dt and lam are the raw projections), dt_bias [H] fp32
+    dt_bias: torch.Tensor | None = None
+    flags: int = 0
 
     def tensors(self):
         return dict(x=self.x, B=self.B, C=self.C, theta=self.theta, dt=self.dt, A=self.A,
                     lam=self.lam, B_bias=self.B_bias, C_bias=self.C_bias)
+
+    def scalar_args(self):
+        """How dt and lam are to be read: flags 0 (ready to use) or 3 (raw, with dt_bias)."""
+        return dict(dt_bias=self.dt_bias, flags=self.flags)
 
     def to(self, device) -> "Problem":
         mv = lambda t: None if t is None else t.to(device)
         st = None if self.state is None else {k: mv(v) for k, v in self.state.items()}
         return Problem(self.dims, mv(self.x), mv(self.B), mv(self.C), mv(self.theta),
                        mv(self.dt), mv(self.A), mv(self.lam), mv(self.B_bias),
-                       mv(self.C_bias), st)
+                       mv(self.C_bias), st, mv(self.dt_bias), self.flags)
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -84,9 +91,14 @@ def random_state(batch, nheads, dstate, headdim, rank, dtype, g, device="cpu") -
 
 def make_problem(batch, seqlen, nheads, ngroups, headdim, dstate, rank=1, chunk=64,
                  dtype=torch.bfloat16, bc_norm=False, bias_std=0.0, dt_shift=-2.0,
-                 seed=0, with_state=False, device="cpu", lead=(), input_std=None) -> Problem:
+                 seed=0, with_state=False, device="cpu", lead=(), input_std=None,
+                 raw_scalars=False) -> Problem:
     """Draws one problem. ``lead`` prepends extra leading dims (used for stacks of decode
-    steps: lead=(steps,) gives x [steps, b, 1, H, R, P] and so on)."""
+    steps: lead=(steps,) gives x [steps, b, 1, H, R, P] and so on).
+
+    ``raw_scalars``: dt and lam are stored as their raw N(0,1) draws (the layer's projections
+    before softplus and sigmoid) and a per-head dt_bias ~ N(dt_shift, 0.5^2) is drawn after
+    everything else; the problem's flags ask the consumer to apply the parameterisation."""
     g = _gen(seed, device)
     d = Dims(batch, seqlen, nheads, ngroups, headdim, dstate, rank, chunk, dtype,
              bool(bc_norm), 1e-6)
@@ -101,13 +113,18 @@ def make_problem(batch, seqlen, nheads, ngroups, headdim, dstate, rank=1, chunk=
         C_bias = torch.randn(H, R, N, generator=g, device=device) * bias_std
     else:
         B_bias = C_bias = None
-    dt = torch.nn.functional.softplus(
-        torch.randn(*shp, b, L, H, generator=g, device=device) + dt_shift)
+    dt_raw = torch.randn(*shp, b, L, H, generator=g, device=device)
     A = -torch.exp(torch.rand(*shp, b, L, H, generator=g, device=device) * 2 - 1)
-    lam = torch.sigmoid(torch.randn(*shp, b, L, H, generator=g, device=device))
+    lam_raw = torch.randn(*shp, b, L, H, generator=g, device=device)
     theta = ((torch.rand(*shp, b, L, H, N // 2, generator=g, device=device) * 2 - 1)
              * math.pi).to(dtype)
     st = random_state(b, H, N, P, R, dtype, g, device) if with_state else None
+    if raw_scalars:
+        dt_bias = torch.randn(H, generator=g, device=device) * 0.5 + dt_shift
+        return Problem(d, x, B, C, theta, dt_raw.float(), A.float(), lam_raw.float(), B_bias,
+                       C_bias, st, dt_bias.float(), 3)
+    dt = torch.nn.functional.softplus(dt_raw + dt_shift)
+    lam = torch.sigmoid(lam_raw)
     return Problem(d, x, B, C, theta, dt.float(), A.float(), lam.float(), B_bias, C_bias, st)
 
 
@@ -137,7 +154,7 @@ def make_config(idx: int, device="cpu", **overrides) -> Problem:
 
 
 def make_decode(rank: int, steps: int, batch=128, nheads=64, headdim=64, dstate=128,
-                seed=3, device="cpu"):
+                seed=3, device="cpu", raw_scalars=False):
     """Decode workload: per-step inputs drawn as for the fp32 scan workload (N(0,1) x, B, C;
     no normalisation, zero bias), stored bf16, stacked over ``steps``; initial state drawn
     after them (h ~ N(0,1) fp32, phi ~ U(-pi,pi), prev_B, prev_x ~ N(0,1) bf16).
@@ -146,4 +163,4 @@ def make_decode(rank: int, steps: int, batch=128, nheads=64, headdim=64, dstate=
     return make_problem(batch, 1, nheads, 1, headdim, dstate, rank=rank, chunk=1,
                         dtype=torch.bfloat16, bc_norm=False, bias_std=0.0, dt_shift=-2.0,
                         seed=seed, with_state=True, device=device, lead=(steps,),
-                        input_std=1.0)
+                        input_std=1.0, raw_scalars=raw_scalars)

@@ -41,7 +41,7 @@ def oracle_state(st: dict | None):
 def gpu_scan(pr, dev, use_state=True, chunk=None, final=True):
     g = pr.to(dev)
     init = m3.State.from_dict(g.state) if (use_state and g.state is not None) else None
-    y, fin = m3.scan_fwd(**g.tensors(), init=init, final=final,
+    y, fin = m3.scan_fwd(**g.tensors(), **g.scalar_args(), init=init, final=final,
                          chunk=chunk or pr.dims.chunk, bc_norm=pr.dims.bc_norm)
     torch.cuda.synchronize()
     return y, fin
@@ -49,12 +49,13 @@ def gpu_scan(pr, dev, use_state=True, chunk=None, final=True):
 
 def oracle_scan(pr, use_state=True, heads=None):
     t = pr.tensors()
+    t.update(pr.scalar_args())
     st = pr.state if use_state else None
     if heads is not None:
         hs = torch.as_tensor(heads)
         for k in ("x", "theta", "dt", "A", "lam"):
             t[k] = t[k][:, :, hs]
-        for k in ("B_bias", "C_bias"):
+        for k in ("B_bias", "C_bias", "dt_bias"):
             if t[k] is not None:
                 t[k] = t[k][hs]
         if st is not None:

@@ -44,14 +44,14 @@ def test_status_strings(lib):
 
 def dims(**kw):
     d = dict(batch=2, seqlen=10, nheads=4, ngroups=1, headdim=64, dstate=128, rank=1, chunk=64,
-             in_dtype=bd.M3_BF16, bc_norm=1, norm_eps=1e-6)
+             in_dtype=bd.M3_BF16, bc_norm=1, norm_eps=1e-6, flags=0)
     d.update(kw)
     return bd.Dims(*(d[f] for f, _ in bd.Dims._fields_))
 
 
 def test_struct_layout_matches_header(lib):
-    assert ctypes.sizeof(bd.Dims) == 8 * 8 + 4 + 4 + 4 + 4  # trailing padding to 8
-    assert ctypes.sizeof(bd.Inputs) == 9 * 8 and ctypes.sizeof(bd.StateC) == 4 * 8
+    assert ctypes.sizeof(bd.Dims) == 8 * 8 + 4 + 4 + 4 + 4  # ..., norm_eps, flags
+    assert ctypes.sizeof(bd.Inputs) == 10 * 8 and ctypes.sizeof(bd.StateC) == 4 * 8
 
 
 @pytest.mark.parametrize("kw,ok", [
@@ -59,6 +59,7 @@ def test_struct_layout_matches_header(lib):
     (dict(headdim=48), False), (dict(rank=3), False), (dict(chunk=0), False),
     (dict(chunk=64, rank=4), False), (dict(chunk=16, rank=4), True), (dict(in_dtype=7), False),
     (dict(dstate=272), False), (dict(norm_eps=-1.0), False), (dict(batch=-1), False),
+    (dict(flags=3), True), (dict(flags=4), False),
 ])
 def test_workspace_query_validates(lib, kw, ok):
     n = lib.m3_scan_workspace_bytes(ctypes.byref(dims(**kw)))

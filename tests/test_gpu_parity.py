@@ -261,3 +261,46 @@ def test_config3_decode_1000_steps_sampled_units(cuda_dev, R):
     record({"y": e_y, "h": e_h, "phi": e_phi})
     assert e_y <= TOL[torch.bfloat16] and e_h <= TOL[torch.bfloat16] and e_phi <= 2e-2, \
         (e_y, e_h, e_phi)
+
+
+# ---------------------------------------------------------------- fused scalar prologue
+# dt and lam passed raw (M3_DT_SOFTPLUS | M3_LAM_SIGMOID, per-head dt_bias): every kernel
+# applies softplus / sigmoid to real tokens only.
+RAW = [
+    # b, L, H, P, N, R, chunk, dtype
+    (2, 200, 4, 64, 128, 1, 64, torch.bfloat16),    # tensor-core scan, SISO, ragged tail
+    (2, 100, 4, 64, 128, 4, 16, torch.bfloat16),    # tensor-core scan, MIMO
+    (1, 2543, 4, 64, 128, 1, 64, torch.bfloat16),   # sequence-parallel form, 5 segments
+    (1, 130, 2, 64, 128, 1, 64, torch.float32),     # exact fp32 path
+]
+
+
+@pytest.mark.parametrize("case", RAW, ids=lambda c: "b{}L{}H{}P{}N{}R{}Q{}{}".format(
+    *c[:7], "f32" if c[7] == torch.float32 else "bf16"))
+def test_scan_raw_scalars(cuda_dev, case):
+    b, L, H, P, N, R, Q, dt = case
+    pr = make_problem(b, L, H, 1, P, N, rank=R, chunk=Q, dtype=dt, bc_norm=True,
+                      bias_std=0.1, seed=3 * L + R, with_state=True, raw_scalars=True)
+    assert pr.flags == m3.M3_DT_SOFTPLUS | m3.M3_LAM_SIGMOID
+    y, fin = gpu_scan(pr, cuda_dev)
+    yo, so = oracle_scan(pr)
+    compare(pr, y, fin, yo, so, tol=1e-4 if dt == torch.float32 else None)
+
+
+@pytest.mark.parametrize("R,dt", [(1, torch.bfloat16), (2, torch.bfloat16), (4, torch.bfloat16),
+                                  (2, torch.float32)])
+def test_decode_raw_scalars(cuda_dev, R, dt):
+    steps = 4
+    pr = make_problem(2, steps, 4, 1, 64, 128, rank=R, chunk=1, dtype=dt, bc_norm=True,
+                      bias_std=0.1, seed=50 + R, with_state=True, raw_scalars=True)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    ys = []
+    for t in range(steps):
+        tok = {k: (v[:, t:t + 1].contiguous() if k not in ("B_bias", "C_bias") else v)
+               for k, v in g.tensors().items()}
+        y, st = m3.decode_step(**tok, **g.scalar_args(), state_in=st, bc_norm=True)
+        ys.append(y.clone())
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.stack(ys, 1), st, yo, so, tol=1e-4 if dt == torch.float32 else None)

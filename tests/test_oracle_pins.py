@@ -393,3 +393,65 @@ def test_empty_sequence_keeps_state():
     y, fs = run(p, st)
     assert y.shape[1] == 0
     assert_state_close(fs, st, 0)
+
+
+# ---------------------------------------------------------------- fused scalar prologue
+def test_step_scalars_match_library_softplus_and_sigmoid():
+    """softplus and sigmoid of the raw projections (Sec. 2: a positive step; Appendix F:
+    lambda_t = sigma(u_t)) against torch's own routines in float64, including the far tails
+    where a naive exp overflows."""
+    import torch
+    rng = np.random.default_rng(21)
+    d = np.concatenate([rng.standard_normal((4, 7, 5)).ravel() * 6,
+                        [-800.0, -40.0, -20.0, -1e-9, 0.0, 1e-9, 5.0, 20.0, 25.0, 800.0]]).reshape(-1, 5)
+    u = np.concatenate([rng.standard_normal((4, 7, 5)).ravel() * 6,
+                        [-800.0, -40.0, -20.0, -1e-9, 0.0, 1e-9, 5.0, 20.0, 25.0, 800.0]]).reshape(-1, 5)
+    bias = rng.standard_normal(5) - 2.0
+    dt, lam = oracle.step_scalars(d, u, bias, oracle.DT_SOFTPLUS | oracle.LAM_SIGMOID)
+    v = d + bias
+    ref_dt = torch.nn.functional.softplus(torch.from_numpy(v)).numpy()  # linear above 20
+    ref_lam = torch.sigmoid(torch.from_numpy(u))
+    lin = v > 20   # there the library returns v itself, off by log(1 + e^{-v}) < 2.1e-9
+    np.testing.assert_allclose(dt[~lin], ref_dt[~lin], rtol=1e-14, atol=1e-300)
+    np.testing.assert_allclose(dt[lin], ref_dt[lin], rtol=2.1e-9 / 20, atol=0)
+    np.testing.assert_allclose(lam, ref_lam.numpy(), rtol=1e-14, atol=1e-300)
+    assert np.all(dt >= 0) and np.all(dt[v > -700] > 0)   # e^{-745} underflows fp64
+    assert np.all((lam >= 0) & (lam <= 1))
+    # each flag alone transforms only its own input; no flag is the identity
+    dt1, lam1 = oracle.step_scalars(d, u, bias, oracle.DT_SOFTPLUS)
+    assert np.array_equal(lam1, u) and np.array_equal(dt1, dt)
+    dt2, lam2 = oracle.step_scalars(d, u, bias, 0)
+    assert np.array_equal(dt2, d) and np.array_equal(lam2, u)
+
+
+def test_scan_with_raw_scalars_equals_scan_of_library_transformed():
+    """Wiring of the prologue inside the scan and decode: per-head bias broadcast over [b, L, H]
+    and both flags, against the scan of inputs transformed by torch's softplus / sigmoid."""
+    import torch
+    rng = np.random.default_rng(22)
+    p = rnd_problem(rng, b=2, L=19, H=3, R=2)
+    raw_d = rng.standard_normal((2, 19, 3))
+    raw_u = rng.standard_normal((2, 19, 3)) * 2
+    bias = np.array([-2.0, -0.5, 1.0])
+    st = rand_state(rng, 2, 3, 8, 5, 2)
+    q = dict(p, dt=raw_d, lam=raw_u)
+    y_raw, s_raw = oracle.scan(**{k: v for k, v in q.items() if k != "bc_norm"}, state=st,
+                               bc_norm=q["bc_norm"], dt_bias=bias, flags=3)
+    ref = dict(p, dt=torch.nn.functional.softplus(torch.from_numpy(raw_d + bias)).numpy(),
+               lam=torch.sigmoid(torch.from_numpy(raw_u)).numpy())
+    y_ref, s_ref = oracle.scan(**{k: v for k, v in ref.items() if k != "bc_norm"}, state=st,
+                               bc_norm=ref["bc_norm"])
+    np.testing.assert_allclose(y_raw, y_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s_raw.h, s_ref.h, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s_raw.phi, s_ref.phi, rtol=1e-12, atol=1e-12)
+    # one decode step takes the same parameterisation
+    tok = {k: (v[:, 0] if k in ("x", "B", "C", "theta") else v) for k, v in q.items()
+           if k != "bc_norm"}
+    yd, sd = oracle.decode_step(tok["x"], tok["B"], tok["C"], tok["theta"], raw_d[:, 0],
+                                p["A"][:, 0], raw_u[:, 0], p["B_bias"], p["C_bias"], st,
+                                p["bc_norm"], dt_bias=bias, flags=3)
+    y1, s1 = oracle.scan(**{k: (v[:, :1] if k in ("x", "B", "C", "theta", "dt", "A", "lam")
+                                else v) for k, v in ref.items() if k != "bc_norm"},
+                         state=st, bc_norm=ref["bc_norm"])
+    np.testing.assert_allclose(yd, y1[:, 0], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sd.h, s1.h, rtol=1e-12, atol=1e-12)
