@@ -257,6 +257,8 @@ def run_ours(args):
         del praw
         prologue["decode_R4"] = bench_decode(m3, dev, 4, args.decode_steps, hbm, world, dist,
                                              raw=True)
+        decode["R4_proj"] = bench_decode(m3, dev, 4, args.decode_steps, hbm, world, dist,
+                                         proj=True)
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -286,10 +288,15 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False):
+def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False, proj=False):
     import torch
-    from state_space_sequence_mamba_b200.inputs import make_decode
+    from state_space_sequence_mamba_b200.inputs import make_decode, make_proj
     pr = make_decode(R, steps, device=dev, raw_scalars=raw)
+    if proj:   # MIMO projections fused: x' and z' [P] in, O' [P] out
+        xp, zp, WX, WZ, WO = make_proj(steps, pr.dims.batch, pr.dims.nheads, pr.dims.headdim,
+                                       R, dtype=torch.bfloat16, seed=5, device=dev)
+        ob = torch.empty(pr.dims.batch, pr.dims.nheads, pr.dims.headdim, dtype=torch.bfloat16,
+                         device=dev)
     st = m3.State.from_dict({k: v.clone() for k, v in pr.state.items()})
     yb = torch.empty(pr.dims.batch, pr.dims.nheads, R, pr.dims.headdim, dtype=torch.bfloat16,
                      device=dev)
@@ -298,9 +305,14 @@ def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False):
 
     def run(n):
         for t in range(n):
-            m3.decode_step(pr.x[t], pr.B[t], pr.C[t], pr.theta[t], pr.dt[t], pr.A[t], pr.lam[t],
-                           dt_bias=pr.dt_bias, flags=pr.flags,
-                           state_in=st, y=yb, stream=s)
+            if proj:
+                m3.decode_step_proj(xp[t], zp[t], WX, WZ, WO, pr.B[t], pr.C[t], pr.theta[t],
+                                    pr.dt[t], pr.A[t], pr.lam[t], dt_bias=pr.dt_bias,
+                                    flags=pr.flags, state_in=st, o=ob, stream=s)
+            else:
+                m3.decode_step(pr.x[t], pr.B[t], pr.C[t], pr.theta[t], pr.dt[t], pr.A[t],
+                               pr.lam[t], dt_bias=pr.dt_bias, flags=pr.flags,
+                               state_in=st, y=yb, stream=s)
 
     with torch.cuda.stream(s):
         run(3)  # warm-up outside capture
@@ -321,9 +333,14 @@ def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False):
     units = pr.dims.batch * pr.dims.nheads
     es = 2
     N, P = pr.dims.dstate, pr.dims.headdim
+    # state h and phi read + written, prev_B and prev_x read + written, x and y (or x', z'
+    # and O'), theta, dt/A/lam; B and C once per batch row; the projection weights once
+    io = 3 * P * es if proj else 2 * R * P * es
     per_unit = (2 * N * P * 4 + 2 * (N // 2) * 4 + 2 * R * N * es + 2 * R * P * es
-                + R * P * es + R * P * es + (N // 2) * es + 3 * 4)
+                + io + (N // 2) * es + 3 * 4)
     byts = units * per_unit + pr.dims.batch * 2 * R * N * es
+    if proj:
+        byts += 3 * pr.dims.nheads * R * P * 4
     ach = byts / (us / 1e6) / 1e9
     del g
     return {"us_per_step": us, "steps": steps, "graph": True, "bytes_per_step": byts,

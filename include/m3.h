@@ -102,6 +102,19 @@ typedef struct {
     void* prev_B;  /* [b, H, R, N] in_dtype: raw B of the last token seen (per head copy) */
     void* prev_x;  /* [b, H, R, P] in_dtype: x of the last token seen                     */
 } m3_state;
+/* The MIMO projections around one decode step (Appendix C). The step's input arrives as X'
+ * and is expanded per rank in the kernel, X[r][p] = W_X[h][r][p] X'[p]; the output is gated
+ * and contracted over the ranks, O'[p] = sum_r W_O[h][r][p] Y[r][p] SiLU(W_Z[h][r][p] Z'[p]),
+ * with SiLU(z) = z / (1 + e^{-z}) and Y the SSM output of X. The paper's weights belong to the
+ * layer (P x R); here every head has its own. */
+typedef struct {
+    const void* x_in;   /* [b, H, P] in_dtype: X' of the token                              */
+    const void* z_in;   /* [b, H, P] in_dtype: Z' of the token                              */
+    const float* W_X;   /* [H, R, P]                                                         */
+    const float* W_Z;   /* [H, R, P]                                                         */
+    const float* W_O;   /* [H, R, P]                                                         */
+} m3_proj;
+
 /* An all-zero state is the state of an empty sequence: h_{-1} = 0, x_{-1} = 0, so the first
  * step is h_0 = gamma_0 B_0 x_0 (Sec. 3.1.3). */
 
@@ -134,6 +147,13 @@ M3_API m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_
  *   y         [b, H, R, P] in_dtype. */
 M3_API m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,
                          const m3_state* state_out, void* y, void* stream);
+
+/* m3_decode_step with the MIMO projections fused (Appendix C, m3_proj): in->x is not read
+ * (it may be NULL); the new state's prev_x is the expanded X, rounded to in_dtype; o
+ * [b, H, P] in_dtype receives O'. All of proj's pointers are required, 16-byte aligned. */
+M3_API m3_status m3_decode_step_proj(const m3_dims* dims, const m3_inputs* in,
+                                     const m3_proj* proj, const m3_state* state_in,
+                                     const m3_state* state_out, void* o, void* stream);
 
 /* After the stream that ran m3_scan_fwd has synchronised: M3_OK, or M3_ERR_TIMEOUT if a
  * bounded inter-CTA wait gave up (the outputs of that call are then incomplete). Performs

@@ -176,3 +176,22 @@ def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None,
     y, st = scan(tok(x), tok(B), tok(C), tok(theta), tok(dt), tok(A), tok(lam), B_bias,
                  C_bias, state, bc_norm, norm_eps, nthreads, dt_bias, flags)
     return y[:, 0], st
+
+
+def decode_step_proj(xp, zp, W_X, W_Z, W_O, B, C, theta, dt, A, lam, B_bias=None,
+                     C_bias=None, state: State | None = None, bc_norm: bool = False,
+                     norm_eps: float = 1e-6, nthreads: int = 0, dt_bias=None, flags: int = 0):
+    """One token with the MIMO projections around the SSM (Appendix C):
+        X[r][p] = W_X[h][r][p] X'[p],   Z[r][p] = W_Z[h][r][p] Z'[p],
+        Y = the SSM output of X (decode_step),   Y' = Y * SiLU(Z),
+        O'[p] = sum_r W_O[h][r][p] Y'[r][p],   SiLU(z) = z / (1 + e^{-z}).
+    xp, zp [b,H,P]; W_X, W_Z, W_O [H,R,P] (per head: the reading of the paper's per-layer
+    P x R weights with H heads). The new state's prev_x is X. Returns (O' [b,H,P], State)."""
+    xp, zp = _f64(xp), _f64(zp)
+    W_X, W_Z, W_O = _f64(W_X), _f64(W_Z), _f64(W_O)
+    X = W_X[None] * xp[:, :, None, :]                      # [b,H,R,P]
+    y, st = decode_step(X, B, C, theta, dt, A, lam, B_bias, C_bias, state, bc_norm, norm_eps,
+                        nthreads, dt_bias, flags)
+    Z = W_Z[None] * zp[:, :, None, :]
+    silu = Z / (1.0 + np.exp(-Z))
+    return (W_O[None] * y * silu).sum(axis=2), st

@@ -44,9 +44,13 @@ class StateC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("h", "phi", "prev_B", "prev_x")]
 
 
+class Proj(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("x_in", "z_in", "W_X", "W_Z", "W_O")]
+
+
 # Symbols include/m3.h declares (checked by the CPU test suite).
 EXPORTS = ("m3_scan_workspace_bytes", "m3_scan_fwd", "m3_decode_step", "m3_scan_check",
-           "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc")
+           "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc", "m3_decode_step_proj")
 
 _lib = None
 
@@ -69,6 +73,9 @@ def load_library(path: str = LIB_PATH):
     lib.m3_decode_step.argtypes = [P(Dims), P(Inputs), P(StateC), P(StateC), ctypes.c_void_p,
                                    ctypes.c_void_p]
     lib.m3_decode_step.restype = ctypes.c_int
+    lib.m3_decode_step_proj.argtypes = [P(Dims), P(Inputs), P(Proj), P(StateC), P(StateC),
+                                        ctypes.c_void_p, ctypes.c_void_p]
+    lib.m3_decode_step_proj.restype = ctypes.c_int
     lib.m3_scan_check.argtypes = [ctypes.c_void_p]
     lib.m3_scan_check.restype = ctypes.c_int
     lib.m3_status_str.argtypes = [ctypes.c_int]
@@ -206,3 +213,28 @@ def decode_step(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state_in: 
                             ctypes.byref(so), _ptr(y), _stream_handle(stream))
     _check(rc)
     return y, state_out
+
+
+def decode_step_proj(xp, zp, W_X, W_Z, W_O, B, C, theta, dt, A, lam, B_bias=None, C_bias=None,
+                     state_in: State = None, state_out: State | None = None, o=None,
+                     bc_norm=False, norm_eps=1e-6, stream=None, dt_bias=None, flags=0):
+    """m3_decode_step_proj: one token with the MIMO projections. xp, zp [b,1,H,P] (X', Z');
+    W_X, W_Z, W_O [H,R,P] fp32; B, C [b,1,G,R,N]; theta [b,1,H,N/2]; dt/A/lam [b,1,H].
+    ``state_out`` defaults to ``state_in``. Returns (O' [b,H,P], state_out)."""
+    lib = load_library()
+    b, _, H, P = xp.shape
+    R = W_X.shape[1]
+    dims = make_dims(xp.reshape(b, 1, H, 1, P).expand(b, 1, H, R, P), B, 1, bc_norm, norm_eps,
+                     flags)
+    if state_out is None:
+        state_out = state_in
+    if o is None:
+        o = torch.empty(b, H, P, dtype=xp.dtype, device=xp.device)
+    ins = Inputs(*(_ptr(t) for t in (None, B, C, theta, dt, A, lam, B_bias, C_bias, dt_bias)))
+    pr = Proj(*(_ptr(t) for t in (xp, zp, W_X, W_Z, W_O)))
+    si, so = state_in.c(), state_out.c()
+    rc = lib.m3_decode_step_proj(ctypes.byref(dims), ctypes.byref(ins), ctypes.byref(pr),
+                                 ctypes.byref(si), ctypes.byref(so), _ptr(o),
+                                 _stream_handle(stream))
+    _check(rc)
+    return o, state_out

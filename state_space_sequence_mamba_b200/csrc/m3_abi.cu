@@ -217,25 +217,68 @@ m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
                          m3_scan_workspace_bytes(dims), stream);
 }
 
-m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,
-                         const m3_state* state_out, void* y, void* stream) {
+}  // extern "C"
+
+namespace m3 {
+namespace {
+
+// m3_decode_step, with the MIMO projections when proj is not NULL (x then comes from proj).
+m3_status decode_impl(const m3_dims* dims, const m3_inputs* in, const m3_proj* proj,
+                      const m3_state* state_in, const m3_state* state_out, void* y, void* stream) {
     g_err[0] = 0;
     m3_status st = check_dims(dims, false);
     if (st != M3_OK) return st;
     if (dims->seqlen != 1) return fail(M3_ERR_INVALID_ARG, "decode needs seqlen == 1");
     if (!state_in || !state_out) return fail(M3_ERR_INVALID_ARG, "state_in and state_out are required");
     const bool any = dims->batch > 0;
-    if ((st = check_inputs(in, any)) != M3_OK) return st;
+    if (!in) return fail(M3_ERR_INVALID_ARG, "inputs is NULL");
+    m3_inputs ins = *in;
+    if (proj) {
+        const void* req[] = {proj->x_in, proj->z_in, proj->W_X, proj->W_Z, proj->W_O};
+        const char* names[] = {"x_in", "z_in", "W_X", "W_Z", "W_O"};
+        for (int i = 0; i < 5 && any; ++i) {
+            if (!req[i]) return fail(M3_ERR_INVALID_ARG, "projection %s is NULL", names[i]);
+            if (!aligned16(req[i]))
+                return fail(M3_ERR_INVALID_ARG, "projection %s is not 16-byte aligned", names[i]);
+        }
+        ins.x = proj->x_in;   // checked like x; the kernels read it as [b, H, P]
+    }
+    if ((st = check_inputs(&ins, any)) != M3_OK) return st;
     if ((st = check_state(state_in, "input")) != M3_OK) return st;
     if ((st = check_state(state_out, "output")) != M3_OK) return st;
-    if (any && (!y || !aligned16(y))) return fail(M3_ERR_INVALID_ARG, "y is NULL or misaligned");
+    if (any && (!y || !aligned16(y))) return fail(M3_ERR_INVALID_ARG, "output is NULL or misaligned");
     if (!any) return M3_OK;
-    ScanParams p = make_params(dims, in, state_in, state_out, y);
+    ScanParams p = make_params(dims, &ins, state_in, state_out, y);
+    if (proj) {
+        p.proj = 1;
+        p.xprj = proj->x_in;
+        p.zprj = proj->z_in;
+        p.WX = proj->W_X;
+        p.WZ = proj->W_Z;
+        p.WO = proj->W_O;
+    }
     const size_t smem = decode_smem_bytes(p);
     if (smem > 227 * 1024) return fail(M3_ERR_UNSUPPORTED, "decode shape too large");
     cudaError_t e = launch_decode(p, dims->in_dtype == M3_BF16, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return M3_OK;
+}
+
+}  // namespace
+}  // namespace m3
+
+extern "C" {
+
+m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_state* state_in,
+                         const m3_state* state_out, void* y, void* stream) {
+    return decode_impl(dims, in, nullptr, state_in, state_out, y, stream);
+}
+
+m3_status m3_decode_step_proj(const m3_dims* dims, const m3_inputs* in, const m3_proj* proj,
+                              const m3_state* state_in, const m3_state* state_out, void* o,
+                              void* stream) {
+    if (!proj) return fail(M3_ERR_INVALID_ARG, "proj is NULL");
+    return decode_impl(dims, in, proj, state_in, state_out, o, stream);
 }
 
 m3_status m3_scan_check(void* workspace) {

@@ -76,7 +76,12 @@ decode_kernel(const ScanParams p, const int rows_per_pass) {
         rawBp[i] = to_f(Bpin[i]);
     }
     for (int i = tid; i < R * P; i += blockDim.x) {
-        xs[i] = to_f(xin[i]);
+        if (p.proj) {   // X[r][p] = W_X[h][r][p] X'[p] (Appendix C)
+            const int pp = i % P;
+            xs[i] = p.WX[hh * R * P + i] * to_f(static_cast<const T*>(p.xprj)[u * P + pp]);
+        } else {
+            xs[i] = to_f(xin[i]);
+        }
         xps[i] = to_f(xpin[i]);
     }
     if (tid == 0) {
@@ -202,7 +207,21 @@ decode_kernel(const ScanParams p, const int rows_per_pass) {
             for (int j = 0; j < 4; ++j) ypart[(warp * R + r) * P + lane * 4 + j] = yacc[r][j];
     }
     __syncthreads();
-    {
+    if (p.proj) {
+        // O'[p] = sum_r W_O[h][r][p] Y[r][p] SiLU(W_Z[h][r][p] Z'[p]) (Appendix C)
+        T* oout = static_cast<T*>(p.y) + u * P;
+        for (int col = tid; col < P; col += blockDim.x) {
+            const float zp = to_f(static_cast<const T*>(p.zprj)[u * P + col]);
+            float o = 0.f;
+            for (int r = 0; r < R; ++r) {
+                float acc = 0.f;
+                for (int w = 0; w < nwarps; ++w) acc += ypart[(w * R + r) * P + col];
+                const float z = p.WZ[hh * R * P + r * P + col] * zp;
+                o = fmaf(p.WO[hh * R * P + r * P + col], acc * z / (1.f + __expf(-z)), o);
+            }
+            oout[col] = from_f<T>(o);
+        }
+    } else {
         T* yout = static_cast<T*>(p.y) + u * R * P;
         for (int e = tid; e < R * P; e += blockDim.x) {
             const int r = e / P, col = e % P;
@@ -216,9 +235,9 @@ decode_kernel(const ScanParams p, const int rows_per_pass) {
         T* dst = static_cast<T*>(p.prevB1) + u * R * N;
         for (int i = tid; i < R * N; i += blockDim.x) dst[i] = Bin[i];
     }
-    if (p.prevx1) {
+    if (p.prevx1) {   // with the projections, the expanded X
         T* dst = static_cast<T*>(p.prevx1) + u * R * P;
-        for (int i = tid; i < R * P; i += blockDim.x) dst[i] = xin[i];
+        for (int i = tid; i < R * P; i += blockDim.x) dst[i] = p.proj ? from_f<T>(xs[i]) : xin[i];
     }
 }
 
@@ -250,7 +269,7 @@ static cudaError_t launch_decode_t(const ScanParams& p, cudaStream_t s) {
 cudaError_t launch_decode(const ScanParams& p, bool bf16, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
     if (decode_tc_supported(p, bf16)) return launch_decode_tc(p, s);
-    if (decode_bulk_supported(p, bf16)) return launch_decode_bulk(p, s);
+    if (!p.proj && decode_bulk_supported(p, bf16)) return launch_decode_bulk(p, s);
     switch (p.R) {
         case 1: return bf16 ? launch_decode_t<1, __nv_bfloat16>(p, s) : launch_decode_t<1, float>(p, s);
         case 2: return bf16 ? launch_decode_t<2, __nv_bfloat16>(p, s) : launch_decode_t<2, float>(p, s);

@@ -51,10 +51,14 @@ struct DecCfg {
     static constexpr uint32_t S_X = 0, S_XP = S_X + R * kP * 2, S_B = S_XP + R * kP * 2,
                               S_C = S_B + R * kN * 2, S_BP = S_C + R * kN * 2,
                               S_TH = S_BP + R * kN * 2, S_PHI = S_TH + kHalf * 2,
-                              S_BYTES = (S_PHI + kHalf * 4 + 127) / 128 * 128;
+                              S_Z = S_PHI + kHalf * 4,   // z' [P] (projected decode)
+                              S_W = S_Z + kP * 2,        // the head's W_X, W_Z, W_O [R][P] fp32
+                              S_BYTES = (S_W + 3 * R * kP * 4 + 127) / 128 * 128;
     static constexpr uint32_t SCR = SM0 + kRing * S_BYTES;  // fp32 scratch
     static constexpr uint32_t TOTAL = SCR + 4 * (3 * 8 + 4 * kRing) + 1024;
     static constexpr uint32_t TX = 2 * 16384 + 2 * R * kP * 2 + 3 * R * kN * 2 + kHalf * 2 + kHalf * 4;
+    // projected decode: x' and z' [P] in place of x [R][P]
+    static constexpr uint32_t TX_PROJ = TX - R * kP * 2 + 2 * kP * 2 + 3 * R * kP * 4;
 };
 constexpr uint32_t kTmemCols = 128;
 constexpr uint32_t T_U = 0, T_Y = 64;
@@ -139,7 +143,9 @@ __device__ __forceinline__ void store_kvec(uint8_t* tile, int n, int k0, const f
 }
 
 // kRaw: dt and lam arrive raw (m3_dims.flags); the step scalars apply softplus / sigmoid.
-template <int R, bool kRaw>
+// kProj: the MIMO projections (Appendix C): x' and z' [P] in, X = W_X x' expanded here and
+// kept as the stored previous token, O' = sum_r W_O Y SiLU(W_Z z') out.
+template <int R, bool kRaw, bool kProj>
 __global__ void __launch_bounds__(kThreads, 2)
 decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const int n_units) {
     using Cfg = DecCfg<R>;
@@ -166,10 +172,21 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
         uint8_t* hb = sm + Cfg::HB + s * Cfg::H_BYTES;
         const int64_t bb = u / p.H, hh = u % p.H, g = hh / (p.H / p.G);
         uint64_t* bar = &bar_full[s];
-        mbar_arrive_expect_tx(bar, Cfg::TX);
+        mbar_arrive_expect_tx(bar, kProj ? Cfg::TX_PROJ : Cfg::TX);
         tma_load_3d(hb, &maps.h0, bar, 0, 0, u);
         tma_load_3d(hb + 16384, &maps.h0, bar, 32, 0, u);
-        bulk_load(sl + Cfg::S_X, xg + static_cast<int64_t>(u) * R * kP, R * kP * 2, bar);
+        if constexpr (kProj) {
+            bulk_load(sl + Cfg::S_X, static_cast<const __nv_bfloat16*>(p.xprj) + static_cast<int64_t>(u) * kP,
+                      kP * 2, bar);
+            bulk_load(sl + Cfg::S_Z, static_cast<const __nv_bfloat16*>(p.zprj) + static_cast<int64_t>(u) * kP,
+                      kP * 2, bar);
+            // the head's weights ride with the unit: consecutive units are different heads
+            bulk_load(sl + Cfg::S_W, p.WX + hh * R * kP, R * kP * 4, bar);
+            bulk_load(sl + Cfg::S_W + R * kP * 4, p.WZ + hh * R * kP, R * kP * 4, bar);
+            bulk_load(sl + Cfg::S_W + 2 * R * kP * 4, p.WO + hh * R * kP, R * kP * 4, bar);
+        } else {
+            bulk_load(sl + Cfg::S_X, xg + static_cast<int64_t>(u) * R * kP, R * kP * 2, bar);
+        }
         bulk_load(sl + Cfg::S_XP, pxg + static_cast<int64_t>(u) * R * kP, R * kP * 2, bar);
         bulk_load(sl + Cfg::S_B, Bg + (bb * p.G + g) * R * kN, R * kN * 2, bar);
         bulk_load(sl + Cfg::S_C, Cg + (bb * p.G + g) * R * kN, R * kN * 2, bar);
@@ -306,9 +323,26 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                 // B_U row p = i: columns [0, R) x_prev[r][p], [R, 2R) x[r][p]
                 float vp[R], vx[R];
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    vp[r] = __bfloat162float(sxp[r * kP + i]);
-                    vx[r] = __bfloat162float(sx[r * kP + i]);
+                for (int r = 0; r < R; ++r) vp[r] = __bfloat162float(sxp[r * kP + i]);
+                if constexpr (kProj) {
+                    // X[r][p] = W_X[h][r][p] x'[p]; written over x' (this thread alone reads
+                    // x'[p]) as the stored previous token, which is bulk-copied from there
+                    const float xin = __bfloat162float(sx[i]);
+                    float* sw = reinterpret_cast<float*>(sl + Cfg::S_W) + i;
+                    __nv_bfloat16* sxw = reinterpret_cast<__nv_bfloat16*>(sl + Cfg::S_X);
+                    const float zin = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sl + Cfg::S_Z)[i]);
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        vx[r] = sw[r * kP] * xin;
+                        sxw[r * kP + i] = __float2bfloat16_rn(vx[r]);
+                        // the output weight of Y[r][p], independent of Y: g = W_O SiLU(W_Z z'),
+                        // over W_Z (this thread alone reads column p)
+                        const float z = sw[(R + r) * kP] * zin;
+                        sw[(R + r) * kP] = sw[(2 * R + r) * kP] * z * __frcp_rn(1.f + __expf(-z));
+                    }
+                } else {
+#pragma unroll
+                    for (int r = 0; r < R; ++r) vx[r] = __bfloat162float(sx[r * kP + i]);
                 }
                 store_kvec<R>(sm + Cfg::BU, i, 0, vp);
                 store_kvec<R>(sm + Cfg::BU, i, R, vx);
@@ -411,9 +445,19 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
             for (int r = 0; r < 8; ++r) yv[r] += yw[r];
             if (lane < 16) {
                 const int pcol = 16 * warp + lane;
-                __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(u) * R * kP + pcol;
+                if constexpr (kProj) {
+                    // O'[p] = sum_r W_O[h][r][p] SiLU(W_Z[h][r][p] z'[p]) Y[r][p], the gate
+                    // factors already formed during the rotation
+                    const float* gw = reinterpret_cast<const float*>(sl + Cfg::S_W) + R * kP + pcol;
+                    float o = 0.f;
 #pragma unroll
-                for (int r = 0; r < R; ++r) yo[r * kP] = __float2bfloat16_rn(yv[r]);
+                    for (int r = 0; r < R; ++r) o = fmaf(gw[r * kP], yv[r], o);
+                    static_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(u) * kP + pcol] = __float2bfloat16_rn(o);
+                } else {
+                    __nv_bfloat16* yo = static_cast<__nv_bfloat16*>(p.y) + static_cast<int64_t>(u) * R * kP + pcol;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) yo[r * kP] = __float2bfloat16_rn(yv[r]);
+                }
             }
         }
         if (tid == 0) {
@@ -479,7 +523,8 @@ cudaError_t launch_tc_t(const ScanParams& p, cudaStream_t s) {
     DecMaps maps;
     if (!encode_state(&maps.h0, p.h0, units)) return cudaErrorInvalidValue;
     const uint32_t smem = DecCfg<R>::TOTAL;
-    auto k = p.flags ? decode_tc_kernel<R, true> : decode_tc_kernel<R, false>;
+    auto k = p.proj ? (p.flags ? decode_tc_kernel<R, true, true> : decode_tc_kernel<R, false, true>)
+                    : (p.flags ? decode_tc_kernel<R, true, false> : decode_tc_kernel<R, false, false>);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;

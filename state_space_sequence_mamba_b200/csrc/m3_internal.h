@@ -24,6 +24,14 @@ struct ScanParams {
     const float* Cbias;  // may be null
     const float* dt_bias;  // [H], may be null; read only with M3_DT_SOFTPLUS
     uint32_t flags;        // M3_DT_SOFTPLUS | M3_LAM_SIGMOID
+    // decode with the MIMO projections (m3_decode_step_proj): x' and z' [b,H,P], the per-head
+    // weights [H,R,P]; y then receives O' [b,H,P]
+    int32_t proj;
+    const void* xprj;
+    const void* zprj;
+    const float* WX;
+    const float* WZ;
+    const float* WO;
     // initial state; all null = zero state
     const float* h0;
     const float* phi0;

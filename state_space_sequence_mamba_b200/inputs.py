@@ -164,3 +164,15 @@ def make_decode(rank: int, steps: int, batch=128, nheads=64, headdim=64, dstate=
                         dtype=torch.bfloat16, bc_norm=False, bias_std=0.0, dt_shift=-2.0,
                         seed=seed, with_state=True, device=device, lead=(steps,),
                         input_std=1.0, raw_scalars=raw_scalars)
+
+
+def make_proj(steps: int, batch: int, nheads: int, headdim: int, rank: int,
+              dtype=torch.bfloat16, seed=0, device="cpu"):
+    """Inputs of the MIMO projections around decode steps: X', Z' ~ N(0, 1) per step
+    [steps, b, 1, H, P] in ``dtype``, and per-head weights W_X, W_Z, W_O ~ N(0, 1) [H, R, P]
+    fp32 (drawn in that order)."""
+    g = _gen(seed, device)
+    xp = torch.randn(steps, batch, 1, nheads, headdim, generator=g, device=device).to(dtype)
+    zp = torch.randn(steps, batch, 1, nheads, headdim, generator=g, device=device).to(dtype)
+    W = [torch.randn(nheads, rank, headdim, generator=g, device=device) for _ in range(3)]
+    return xp, zp, W[0], W[1], W[2]

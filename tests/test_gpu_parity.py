@@ -304,3 +304,39 @@ def test_decode_raw_scalars(cuda_dev, R, dt):
     torch.cuda.synchronize()
     yo, so = oracle_scan(pr)
     compare(pr, torch.stack(ys, 1), st, yo, so, tol=1e-4 if dt == torch.float32 else None)
+
+
+# ---------------------------------------------------------------- decode with MIMO projections
+@pytest.mark.parametrize("R,dt", [(1, torch.bfloat16), (2, torch.bfloat16), (4, torch.bfloat16),
+                                  (8, torch.bfloat16), (4, torch.float32)])
+def test_decode_proj(cuda_dev, R, dt):
+    """m3_decode_step_proj over a few steps (X = W_X X' in, O' = sum_r W_O Y SiLU(W_Z Z') out,
+    Appendix C) against the oracle; the stored previous token is the expanded X, rounded to
+    the storage type, so it is compared within the tolerance rather than bit for bit."""
+    from state_space_sequence_mamba_b200.inputs import make_proj
+    steps, b, H, P, N = 3, 2, 4, 64, 128
+    pr = make_problem(b, steps, H, 1, P, N, rank=R, chunk=1, dtype=dt, bc_norm=True,
+                      bias_std=0.1, seed=60 + R, with_state=True)
+    xp, zp, WX, WZ, WO = make_proj(steps, b, H, P, R, dtype=dt, seed=70 + R)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    so = oracle_state(pr.state)
+    tol = TOL[dt]
+    Wd = [w.to(cuda_dev) for w in (WX, WZ, WO)]
+    for t in range(steps):
+        tok = {k: (v[:, t:t + 1].contiguous() if k not in ("B_bias", "C_bias") else v)
+               for k, v in g.tensors().items() if k != "x"}
+        o, st = m3.decode_step_proj(xp[t].to(cuda_dev), zp[t].to(cuda_dev), *Wd, **tok,
+                                    state_in=st, bc_norm=True)
+        oo, so = oracle.decode_step_proj(xp[t][:, 0], zp[t][:, 0], WX, WZ, WO,
+                                         pr.B[:, t], pr.C[:, t], pr.theta[:, t], pr.dt[:, t],
+                                         pr.A[:, t], pr.lam[:, t], pr.B_bias, pr.C_bias, so,
+                                         bc_norm=True)
+        torch.cuda.synchronize()
+        errs = {"o": rel(o, oo)}
+        record(errs)
+        assert errs["o"] <= tol, errs
+    errs = {"h": rel(st.h, so.h), "phi": rel(st.phi, so.phi), "prev_x": rel(st.prev_x, so.prev_x),
+            "prev_B": rel(st.prev_B, so.prev_B)}
+    record(errs)
+    assert errs["prev_B"] == 0.0 and all(v <= tol for v in errs.values()), errs

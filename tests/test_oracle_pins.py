@@ -455,3 +455,44 @@ def test_scan_with_raw_scalars_equals_scan_of_library_transformed():
                          state=st, bc_norm=ref["bc_norm"])
     np.testing.assert_allclose(yd, y1[:, 0], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(sd.h, s1.h, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- MIMO projections (decode)
+def test_decode_step_proj_against_library_gate_and_contraction():
+    """O' = sum_r W_O (Y * SiLU(W_Z Z')) with X = W_X X' (Appendix C): against torch's SiLU and
+    numpy's einsum applied to the plain decode step of the expanded X; with R = 1 and unit
+    weights it is the plain output times SiLU(Z')."""
+    import torch
+    rng = np.random.default_rng(31)
+    for R in (1, 4):
+        b, H, P, N = 2, 3, 5, 8
+        p = rnd_problem(rng, b=b, L=1, H=H, R=R, P=P, N=N)
+        st = rand_state(rng, b, H, N, P, R)
+        xp, zp = rng.standard_normal((b, H, P)), rng.standard_normal((b, H, P)) * 3
+        WX, WZ, WO = (rng.standard_normal((H, R, P)) for _ in range(3))
+        tok = {k: (v[:, 0] if k in ("x", "B", "C", "theta", "dt", "A", "lam") else v)
+               for k, v in p.items() if k != "bc_norm"}
+        o, so = oracle.decode_step_proj(xp, zp, WX, WZ, WO, tok["B"], tok["C"], tok["theta"],
+                                        tok["dt"], tok["A"], tok["lam"], tok["B_bias"],
+                                        tok["C_bias"], st, p["bc_norm"])
+        X = np.einsum("hrp,bhp->bhrp", WX, xp)
+        y, sy = oracle.decode_step(X, tok["B"], tok["C"], tok["theta"], tok["dt"], tok["A"],
+                                   tok["lam"], tok["B_bias"], tok["C_bias"], st, p["bc_norm"])
+        gate = torch.nn.functional.silu(torch.from_numpy(np.einsum("hrp,bhp->bhrp", WZ, zp)))
+        ref = np.einsum("hrp,bhrp->bhp", WO, y * gate.numpy())
+        np.testing.assert_allclose(o, ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(so.h, sy.h, rtol=0, atol=0)
+        np.testing.assert_allclose(so.prev_x, X, rtol=0, atol=0)
+    # R = 1, unit weights: the plain output gated by SiLU(Z')
+    b, H, P, N = 2, 3, 5, 8
+    p = rnd_problem(rng, b=b, L=1, H=H, R=1, P=P, N=N)
+    st = rand_state(rng, b, H, N, P, 1)
+    xp, zp = rng.standard_normal((b, H, P)), rng.standard_normal((b, H, P)) * 3
+    one = np.ones((H, 1, P))
+    args = [p[k][:, 0] for k in ("B", "C", "theta", "dt", "A", "lam")]
+    o1, _ = oracle.decode_step_proj(xp, zp, one, one, one, *args, p["B_bias"], p["C_bias"], st,
+                                    p["bc_norm"])
+    y1, _ = oracle.decode_step(xp[:, :, None, :], *args, p["B_bias"], p["C_bias"], st,
+                               p["bc_norm"])
+    ref1 = y1[:, :, 0, :] * torch.nn.functional.silu(torch.from_numpy(zp)).numpy()
+    np.testing.assert_allclose(o1, ref1, rtol=1e-12, atol=1e-12)
