@@ -155,6 +155,35 @@ M3_API m3_status m3_decode_step_proj(const m3_dims* dims, const m3_inputs* in,
                                      const m3_proj* proj, const m3_state* state_in,
                                      const m3_state* state_out, void* o, void* stream);
 
+/* One segment's end state, for prefill split over devices along the sequence. */
+typedef struct {
+    float* h;        /* [b, H, N, P] fp32                                                    */
+    float* phi;      /* [b, H, N/2]  fp32                                                    */
+    float* lam_sum;  /* [b, H]       fp32: the segment's summed log-decay sum_t dt_t A_t     */
+} m3_seg_state;
+
+/* The recurrence over the tokens of `in` from `init`, without the output y: writes the state
+ * after the last token (h and phi exactly as m3_scan_fwd's final state) and the summed
+ * log-decay. For prefill split along the sequence over devices (context parallelism): each
+ * device runs its own tokens, device 0 from the true initial state and every other one from
+ * h = 0, phi = 0 with the previous device's last token as prev_B (per head) and prev_x; the
+ * results are gathered (stacked over devices) and m3_state_combine gives each device the
+ * state at its start, from which it runs m3_scan_fwd with that token as prev_B, prev_x.
+ * The segments' contributions are exact by linearity (Sec. 3.1.1 Prop. 1) and the rotation
+ * of the frame (Sec. 3.2.2 Prop. 4). Tensor-core shapes only (bf16, N = 128, P = 64,
+ * chunk * R = 64), else M3_ERR_UNSUPPORTED. workspace: at least m3_scan_workspace_bytes. */
+M3_API m3_status m3_scan_state(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                               const m3_seg_state* out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* The state after the last token of segment nseg-1 from the end states of segments
+ * 0 .. nseg-1 stacked in seg (h [nseg, b, H, N, P], phi [nseg, b, H, N/2], lam_sum
+ * [nseg, b, H]), run as m3_scan_state describes: h <- e^{lam_j} h + R(-phi_j) h_j with
+ * phi_j the true angle at segment j's start. Writes h_out [b, H, N, P] and phi_out
+ * [b, H, N/2]. Any supported N, P. */
+M3_API m3_status m3_state_combine(const m3_dims* dims, int nseg, const m3_seg_state* seg,
+                                  float* h_out, float* phi_out, void* stream);
+
 /* After the stream that ran m3_scan_fwd has synchronised: M3_OK, or M3_ERR_TIMEOUT if a
  * bounded inter-CTA wait gave up (the outputs of that call are then incomplete). Performs
  * one blocking 4-byte device-to-host copy; after a timeout it also re-zeroes the workspace

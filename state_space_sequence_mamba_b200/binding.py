@@ -44,13 +44,18 @@ class StateC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("h", "phi", "prev_B", "prev_x")]
 
 
+class SegState(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("h", "phi", "lam_sum")]
+
+
 class Proj(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("x_in", "z_in", "W_X", "W_Z", "W_O")]
 
 
 # Symbols include/m3.h declares (checked by the CPU test suite).
 EXPORTS = ("m3_scan_workspace_bytes", "m3_scan_fwd", "m3_decode_step", "m3_scan_check",
-           "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc", "m3_decode_step_proj")
+           "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc", "m3_decode_step_proj",
+           "m3_scan_state", "m3_state_combine")
 
 _lib = None
 
@@ -76,6 +81,12 @@ def load_library(path: str = LIB_PATH):
     lib.m3_decode_step_proj.argtypes = [P(Dims), P(Inputs), P(Proj), P(StateC), P(StateC),
                                         ctypes.c_void_p, ctypes.c_void_p]
     lib.m3_decode_step_proj.restype = ctypes.c_int
+    lib.m3_scan_state.argtypes = [P(Dims), P(Inputs), P(StateC), P(SegState), ctypes.c_void_p,
+                                  ctypes.c_size_t, ctypes.c_void_p]
+    lib.m3_scan_state.restype = ctypes.c_int
+    lib.m3_state_combine.argtypes = [P(Dims), ctypes.c_int, P(SegState), ctypes.c_void_p,
+                                     ctypes.c_void_p, ctypes.c_void_p]
+    lib.m3_state_combine.restype = ctypes.c_int
     lib.m3_scan_check.argtypes = [ctypes.c_void_p]
     lib.m3_scan_check.restype = ctypes.c_int
     lib.m3_status_str.argtypes = [ctypes.c_int]
@@ -238,3 +249,44 @@ def decode_step_proj(xp, zp, W_X, W_Z, W_O, B, C, theta, dt, A, lam, B_bias=None
                                  _stream_handle(stream))
     _check(rc)
     return o, state_out
+
+
+def scan_state(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, init: State | None = None,
+               chunk=64, bc_norm=False, norm_eps=1e-6, stream=None, dt_bias=None, flags=0,
+               workspace=None):
+    """m3_scan_state: the state after the last token (h [b,H,N,P], phi [b,H,N/2]) and the summed
+    log-decay [b,H], without y. Returns (h, phi, lam_sum)."""
+    lib = load_library()
+    dims = make_dims(x, B, chunk, bc_norm, norm_eps, flags)
+    b, L, H, R, P = x.shape
+    N = B.shape[4]
+    dev = x.device
+    h = torch.empty(b, H, N, P, device=dev)
+    phi = torch.empty(b, H, N // 2, device=dev)
+    lam_sum = torch.empty(b, H, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(max(256, scan_workspace_bytes(dims)), dtype=torch.uint8,
+                                device=dev)
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias, dt_bias)))
+    ic = init.c() if init is not None else None
+    out = SegState(_ptr(h), _ptr(phi), _ptr(lam_sum))
+    rc = lib.m3_scan_state(ctypes.byref(dims), ctypes.byref(ins),
+                           ctypes.byref(ic) if ic is not None else None, ctypes.byref(out),
+                           _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc)
+    return h, phi, lam_sum
+
+
+def state_combine(h, phi, lam_sum, stream=None):
+    """m3_state_combine on stacked segment states h [S,b,H,N,P], phi [S,b,H,N/2], lam_sum
+    [S,b,H]: the state after segment S-1. Returns (h [b,H,N,P], phi [b,H,N/2])."""
+    lib = load_library()
+    S, b, H, N, P = h.shape
+    dims = Dims(b, 1, H, 1, P, N, 1, 1, M3_F32, 0, 1e-6, 0)
+    h_out = torch.empty(b, H, N, P, device=h.device)
+    phi_out = torch.empty(b, H, N // 2, device=h.device)
+    seg = SegState(_ptr(h), _ptr(phi), _ptr(lam_sum))
+    rc = lib.m3_state_combine(ctypes.byref(dims), int(S), ctypes.byref(seg), _ptr(h_out),
+                              _ptr(phi_out), _stream_handle(stream))
+    _check(rc)
+    return h_out, phi_out

@@ -274,6 +274,67 @@ m3_status m3_decode_step(const m3_dims* dims, const m3_inputs* in, const m3_stat
     return decode_impl(dims, in, nullptr, state_in, state_out, y, stream);
 }
 
+m3_status m3_scan_state(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                        const m3_seg_state* out, void* workspace, size_t ws_bytes, void* stream) {
+    g_err[0] = 0;
+    m3_status st = check_dims(dims, true);
+    if (st != M3_OK) return st;
+    const bool any = dims->batch * dims->seqlen * dims->nheads > 0;
+    if ((st = check_inputs(in, any)) != M3_OK) return st;
+    if ((st = check_state(init, "initial")) != M3_OK) return st;
+    if (!out || !out->h || !out->phi || !out->lam_sum)
+        return fail(M3_ERR_INVALID_ARG, "out and its h, phi, lam_sum are required");
+    if (!aligned16(out->h) || !aligned16(out->phi) || !aligned16(out->lam_sum))
+        return fail(M3_ERR_INVALID_ARG, "out fields must be 16-byte aligned");
+    const m3_inputs none{};
+    const ScanParams q = make_params(dims, &none, nullptr, nullptr, nullptr);
+    if (!tc_scan_supported(q, dims->in_dtype == M3_BF16))
+        return fail(M3_ERR_UNSUPPORTED, "m3_scan_state runs the tensor-core shapes only");
+    const size_t need = scan_workspace_min_bytes(dims);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
+        return fail(M3_ERR_INVALID_ARG, "workspace: NULL, misaligned or below %zu bytes", need);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t units = dims->batch * dims->nheads, N = dims->dstate, P = dims->headdim;
+    if (units == 0) return M3_OK;
+    if (dims->seqlen == 0) {   // no token: the initial state, nothing decayed
+        cudaError_t e = init ? cudaMemcpyAsync(out->h, init->h, units * N * P * 4, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(out->h, 0, units * N * P * 4, s);
+        if (e == cudaSuccess)
+            e = init ? cudaMemcpyAsync(out->phi, init->phi, units * (N / 2) * 4, cudaMemcpyDeviceToDevice, s)
+                     : cudaMemsetAsync(out->phi, 0, units * (N / 2) * 4, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(out->lam_sum, 0, units * 4, s);
+        return e == cudaSuccess ? M3_OK : cuda_fail(e, "empty segment copy");
+    }
+    ScanParams p = make_params(dims, in, init, nullptr, nullptr);
+    p.ws = workspace;
+    p.ws_bytes = ws_bytes;
+    p.status = static_cast<int32_t*>(workspace);
+    cudaError_t e = launch_scan_state_tc(p, static_cast<char*>(workspace) + kWsHeader,
+                                         ws_bytes - kWsHeader, out->h, out->phi, out->lam_sum, s);
+    if (e != cudaSuccess) return cuda_fail(e, "state-only scan launch");
+    return M3_OK;
+}
+
+m3_status m3_state_combine(const m3_dims* dims, int nseg, const m3_seg_state* seg, float* h_out,
+                           float* phi_out, void* stream) {
+    g_err[0] = 0;
+    m3_status st = check_dims(dims, false);
+    if (st != M3_OK) return st;
+    if (nseg < 1) return fail(M3_ERR_INVALID_ARG, "nseg must be >= 1");
+    if (!seg || !seg->h || !seg->phi || !seg->lam_sum || !h_out || !phi_out)
+        return fail(M3_ERR_INVALID_ARG, "seg fields, h_out and phi_out are required");
+    const void* ptrs[] = {seg->h, seg->phi, seg->lam_sum, h_out, phi_out};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return fail(M3_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    const int64_t units = dims->batch * dims->nheads, N = dims->dstate, P = dims->headdim;
+    const SegSrc src{seg->h, units * N * P, N * P, seg->phi, units * (N / 2), N / 2,
+                     seg->lam_sum, units, 1};
+    cudaError_t e = launch_state_combine(units, static_cast<int>(N), static_cast<int>(P), nseg, src,
+                                         h_out, phi_out, nullptr, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state combine launch");
+    return M3_OK;
+}
+
 m3_status m3_decode_step_proj(const m3_dims* dims, const m3_inputs* in, const m3_proj* proj,
                               const m3_state* state_in, const m3_state* state_out, void* o,
                               void* stream) {

@@ -62,6 +62,24 @@ size_t tc_scan_workspace_min_bytes(const ScanParams& p);
 // ws_body: the workspace after the status header, body_bytes long (at least the minimum); the
 // scan uses as many segments as the preferred plan has and body_bytes holds.
 cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s);
+// The state-only pass over the whole sequence of every unit (m3_scan_state): the end state h,
+// the angle and the summed log-decay go to out_h [units][N][P], out_phi [units][N/2],
+// out_lam [units].
+cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,
+                                 float* out_h, float* out_phi, float* out_lam, cudaStream_t s);
+// Where the segment states for a combine live: element strides between segments and units.
+struct SegSrc {
+    const float* h;
+    int64_t h_seg, h_unit;
+    const float* phi;
+    int64_t phi_seg, phi_unit;
+    const float* lam;
+    int64_t lam_seg, lam_unit;
+};
+// nseg segment states -> the state after the last of them (h_out [units][N][P], phi_out
+// [units][N/2]) and, if lam_out is set, their summed log-decay [units].
+cudaError_t launch_state_combine(int64_t units, int N, int P, int nseg, const SegSrc& src,
+                                 float* h_out, float* phi_out, float* lam_out, cudaStream_t s);
 // The smallest workspace m3_scan_fwd's work runs in (one segment per sequence), and the scan
 // entry point with that lower bound instead of m3_scan_workspace_bytes (for the fixed scratch
 // of m3_scan_fwd_noalloc).

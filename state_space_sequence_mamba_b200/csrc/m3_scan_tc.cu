@@ -164,8 +164,16 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
 // state (the given state with the stored token folded in): the full pass reads no caller state,
 // so the final state may overwrite the initial one while other segments still run.
 struct SegArgs {
-    int seg_chunks, nseg;
-    float* st;   // [units][nseg][kSegStride]
+    int seg_chunks = 0, nseg = 1;
+    float* st = nullptr;   // [units][nseg][kSegStride]
+    // m3_scan_state in one segment: the end state goes to the caller's buffers instead:
+    // h [units][N][P], phi [units][N/2], the summed log-decay [units]
+    float* out_h = nullptr;
+    float* out_phi = nullptr;
+    float* out_lam = nullptr;
+    // the state-only pass keeps segment 0's primed initial state in slot nseg-1 for the full
+    // pass (not when every segment's end state is wanted, as for m3_scan_state)
+    bool save_init = true;
 };
 
 // One CTA per (unit, segment), CTA index = segment * units + unit. kStateOnly: the segment's
@@ -466,7 +474,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
 
     // ---- the state-only pass keeps segment 0's primed initial state for the full pass ----
     if constexpr (kStateOnly) {
-        if (kseg == 0) {
+        if (kseg == 0 && sa.save_init && !sa.out_h) {
             float* so = sa.st + (u * sa.nseg + sa.nseg - 1) * kSegStride;
             float4* dst = reinterpret_cast<float4*>(so + nrow * kP + 32 * wh);
 #pragma unroll
@@ -940,18 +948,20 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // ---------------- final state ----------------
     __syncthreads();
     if (!s_abort && kStateOnly) {
-        // this segment's end state for the full pass: h, the angle sum (absolute for segment
-        // 0), the summed log-decay
-        float* so = sa.st + (u * sa.nseg + kseg) * kSegStride;
+        // this segment's end state: h, the angle sum (absolute for segment 0), the summed
+        // log-decay; into the workspace for the full pass, or to the caller (m3_scan_state)
+        float* so = sa.out_h ? sa.out_h + u * kN * kP : sa.st + (u * sa.nseg + kseg) * kSegStride;
+        float* sphi = sa.out_h ? sa.out_phi + u * kHalf : so + kN * kP;
+        float* slam = sa.out_h ? sa.out_lam + u : so + kN * kP + kHalf;
         float4* dst = reinterpret_cast<float4*>(so + nrow * kP + 32 * wh);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             dst[j] = make_float4(hreg[4 * j], hreg[4 * j + 1], hreg[4 * j + 2], hreg[4 * j + 3]);
         if (warp == 0) {
-            so[kN * kP + jp] = car[0];
-            so[kN * kP + jp + 1] = car[1];
+            sphi[jp] = car[0];
+            sphi[jp + 1] = car[1];
         }
-        if (warp == 3 && lane == 0) so[kN * kP + kHalf] = lam_acc;
+        if (warp == 3 && lane == 0) *slam = lam_acc;
     } else if (!s_abort) {
         // the sequence's final state, written by its last segment
         if (kseg == sa.nseg - 1) {
@@ -1060,7 +1070,7 @@ SegArgs seg_plan(const ScanParams& p, size_t seg_bytes = ~size_t(0)) {
     const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
     const int64_t nch = (p.L + Q - 1) / Q;
     const int64_t units = p.b * p.H;
-    SegArgs sa{static_cast<int>(nch), 1, nullptr};
+    SegArgs sa{static_cast<int>(nch), 1, nullptr, nullptr, nullptr, nullptr};
     if (units <= 0 || nch == 0) return sa;
     int64_t S = 2 * sm_count() / units;
     S = std::min(S, nch / kMinSegChunks);
@@ -1091,7 +1101,8 @@ size_t tc_scan_workspace_bytes(const ScanParams& p) {
 size_t tc_scan_workspace_min_bytes(const ScanParams& p) { return rs_bytes(p); }
 
 template <int R, bool kRaw>
-static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s) {
+static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s,
+                               bool state_only = false) {
     constexpr int Q = 64 / R;
     TcMaps maps;
     const cuuint64_t H = p.H, Lq = p.L, b = p.b;
@@ -1143,6 +1154,15 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
     }
     const uint32_t smem = tc_smem_bytes<R>();
     const int64_t units = p.b * p.H;
+    if (state_only) {   // m3_scan_state: every segment's end state
+        auto ks = scan_tc_kernel<R, true, kRaw>;
+        cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        const int64_t segs = sa.out_h ? 1 : sa.nseg;
+        ks<<<static_cast<unsigned>(units * segs), kTcThreads, smem, s>>>(p, maps, rs, sa);
+        return cudaGetLastError();
+    }
     if (sa.nseg > 1) {   // every segment's end state but the last's
         auto ks = scan_tc_kernel<R, true, kRaw>;
         cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1158,6 +1178,38 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
     if (e != cudaSuccess) return e;
     k<<<static_cast<unsigned>(units * sa.nseg), kTcThreads, smem, s>>>(p, maps, rs, sa);
     return cudaGetLastError();
+}
+
+cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,
+                                 float* out_h, float* out_phi, float* out_lam, cudaStream_t s) {
+    if (p.b * p.H == 0) return cudaSuccess;
+    uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
+    if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;
+    // few long sequences: the sequence-parallel form, every segment's end state into the
+    // workspace, then their combination; else one segment straight into out
+    SegArgs sa = seg_plan(p, body_bytes - rs_bytes(p));
+    if (sa.nseg > 1) {
+        sa.st = reinterpret_cast<float*>(static_cast<char*>(ws_body) + rs_bytes(p));
+        sa.save_init = false;
+    } else {
+        sa.out_h = out_h;
+        sa.out_phi = out_phi;
+        sa.out_lam = out_lam;
+    }
+    const bool raw = p.flags != 0;
+    cudaError_t e;
+    switch (p.R) {
+        case 1: e = raw ? launch_tc_t<1, true>(p, rs, sa, s, true) : launch_tc_t<1, false>(p, rs, sa, s, true); break;
+        case 2: e = raw ? launch_tc_t<2, true>(p, rs, sa, s, true) : launch_tc_t<2, false>(p, rs, sa, s, true); break;
+        case 4: e = raw ? launch_tc_t<4, true>(p, rs, sa, s, true) : launch_tc_t<4, false>(p, rs, sa, s, true); break;
+        case 8: e = raw ? launch_tc_t<8, true>(p, rs, sa, s, true) : launch_tc_t<8, false>(p, rs, sa, s, true); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess || sa.nseg <= 1) return e;
+    const int64_t S = sa.nseg;
+    const SegSrc src{sa.st, kSegStride, S * kSegStride, sa.st + kN * kP, kSegStride, S * kSegStride,
+                     sa.st + kN * kP + kHalf, kSegStride, S * kSegStride};
+    return launch_state_combine(p.b * p.H, kN, kP, sa.nseg, src, out_h, out_phi, out_lam, s);
 }
 
 cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s) {

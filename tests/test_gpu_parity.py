@@ -340,3 +340,56 @@ def test_decode_proj(cuda_dev, R, dt):
             "prev_B": rel(st.prev_B, so.prev_B)}
     record(errs)
     assert errs["prev_B"] == 0.0 and all(v <= tol for v in errs.values()), errs
+
+
+# ---------------------------------------------------------------- context parallelism
+@pytest.mark.parametrize("b,L,R", [(2, 300, 1), (1, 2543, 1), (1, 700, 4)])
+def test_scan_state_matches_final_state(cuda_dev, b, L, R):
+    """m3_scan_state (no y): its h and phi against the oracle's final state and its summed
+    log-decay against sum_t dt_t A_t, in one segment (8 units: then also equal to
+    m3_scan_fwd's final state to rounding) and in the sequence-parallel form (4 units, 5
+    segments combined on the device, each segment's operands rounded in its own frame)."""
+    pr = make_problem(b, L, 4, 1, 64, 128, rank=R, chunk=64 // R, bc_norm=True, bias_std=0.1,
+                      seed=91 + L, with_state=True)
+    g = pr.to(cuda_dev)
+    init = m3.State.from_dict(g.state)
+    h, phi, lsum = m3.scan_state(**g.tensors(), init=init, chunk=64 // R, bc_norm=True)
+    _, fin = m3.scan_fwd(**g.tensors(), init=init, chunk=64 // R, bc_norm=True)
+    torch.cuda.synchronize()
+    _, so = oracle_scan(pr)
+    errs = {"h": rel(h, so.h), "phi": rel(phi, so.phi),
+            "lam_sum": rel(lsum, (pr.dt.double() * pr.A.double()).sum(1).numpy())}
+    record(errs)
+    assert errs["h"] <= TOL[torch.bfloat16] and errs["phi"] < 1e-5 and errs["lam_sum"] < 1e-5, errs
+    if b * 4 >= 8:   # one segment: the same arithmetic as the scan's own state chain
+        assert rel(h, fin.h.double().cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("world,R,raw", [(2, 1, False), (4, 1, True), (3, 4, False)])
+def test_context_parallel_phases_on_gpu(cuda_dev, world, R, raw):
+    """The context-parallel phases with the library's kernels, the ranks run one after another
+    on one device (no collective: the gathered lists are built locally): the concatenated
+    outputs and the last rank's final state against the oracle's single scan."""
+    from state_space_sequence_mamba_b200 import context_parallel as cp
+    Q = 64 // R
+    pr = make_problem(2, 900 + 7 * world, 4, 1, 64, 128, rank=R, chunk=Q, bc_norm=True,
+                      bias_std=0.1, seed=93 + world, with_state=True, raw_scalars=raw)
+    g = pr.to(cuda_dev)
+    L = pr.dims.seqlen
+    cut = [L * k // world for k in range(world + 1)]
+    ts = [{k: (v[:, cut[r]:cut[r + 1]].contiguous() if k not in ("B_bias", "C_bias") else v)
+           for k, v in g.tensors().items()} for r in range(world)]
+    init = m3.State.from_dict(g.state)
+    scalar = g.scalar_args()
+    ops = cp.DeviceOps()
+    lasts = [cp.last_token(t) for t in ts]
+    prevs = [None] + lasts[:-1]
+    segs = [cp.segment_state(r, ts[r], init, prevs[r], Q, True, scalar, ops) for r in range(world)]
+    seg_h, seg_phi, seg_lam = (torch.stack([s[i] for s in segs]) for i in range(3))
+    outs = [cp.finish(r, world, ts[r], init, prevs[r], seg_h, seg_phi, seg_lam, Q, True,
+                      scalar, ops) for r in range(world)]
+    torch.cuda.synchronize()
+    y = torch.cat([o[0] for o in outs], 1)
+    assert all(o[1] is None for o in outs[:-1])
+    yo, so = oracle_scan(pr)
+    compare(pr, y, outs[-1][1], yo, so)
