@@ -233,6 +233,37 @@ def run_ours(args):
         for R in (1, 4):
             decode[f"R{R}"] = bench_decode(m3, dev, R, args.decode_steps, hbm, world, dist)
 
+    # ---- the other prefill workloads (parity configurations, reported beside the headline):
+    # MIMO R4 (b4 L2048) and the long sequence (b1 L65536, sequence-parallel form) ----
+    others = {}
+    if not args.no_decode:
+        for name, cfg in (("mimo_r4_b4_L2048", 2), ("long_b1_L65536", 4)):
+            po = make_config(cfg, device=dev, seed=rank_seed(rank, cfg))
+            do = po.dims
+            yo = torch.empty_like(po.x)
+            fo = m3.State.empty(do.batch, do.nheads, do.dstate, do.headdim, do.rank, do.dtype, dev)
+            wso = torch.zeros(max(256, m3.scan_workspace_bytes(m3.make_dims(
+                po.x, po.B, do.chunk, True, 1e-6))), dtype=torch.uint8, device=dev)
+
+            def step_o():
+                m3.scan_fwd(**po.tensors(), init=None, final=fo, y=yo, workspace=wso,
+                            chunk=do.chunk, bc_norm=True, stream=stream)
+
+            for _ in range(3):
+                step_o()
+            torch.cuda.synchronize()
+            reps = 3 if cfg == 4 else 10
+            e0.record(stream)
+            for _ in range(reps):
+                step_o()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            oms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev) / reps
+            others[name] = {"ms_per_scan": oms,
+                            "tokens_per_s": do.batch * do.seqlen * world / (oms / 1e3),
+                            "frac_hbm": scan_bytes(po) / (oms / 1e3) / 1e9 / hbm}
+            del po, yo, fo, wso
+
     # ---- the fused scalar prologue: dt and lam passed raw, softplus / sigmoid applied in the
     # kernels (same workloads, one input set each) ----
     prologue = {}
@@ -279,6 +310,7 @@ def run_ours(args):
         "clocks": clk.summary(),
         "decode": decode,
         "fused_scalar_prologue": prologue,
+        "other_prefill": others,
     }
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
