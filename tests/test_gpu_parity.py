@@ -393,3 +393,57 @@ def test_context_parallel_phases_on_gpu(cuda_dev, world, R, raw):
     assert all(o[1] is None for o in outs[:-1])
     yo, so = oracle_scan(pr)
     compare(pr, y, outs[-1][1], yo, so)
+
+
+# ---------------------------------------------------------------- degenerate regimes
+def _degenerate(pr, kind):
+    """Rewrites one problem's step scalars / angles into a limiting regime of the method."""
+    if kind == "euler":            # lam = 1: exponential Euler, no previous-token term
+        pr.lam.fill_(1.0)
+    elif kind == "prev_only":      # lam = 0: only the previous token enters
+        pr.lam.fill_(0.0)
+    elif kind == "no_rotation":    # theta = 0: the real-valued SSM
+        pr.theta.zero_()
+    elif kind == "strong_decay":   # dt A down to about -11 per token: decays underflow within a chunk
+        pr.dt.copy_(pr.dt * 0 + 4.0)
+        pr.A.copy_(pr.A.clamp(max=-2.0))
+    elif kind == "tiny_step":      # dt = 1e-6: alpha = 1, gamma ~ 0
+        pr.dt.fill_(1e-6)
+    elif kind == "fast_angle":     # dt theta up to 3 pi per token: the carried angle wraps often
+        pr.dt.fill_(3.0)
+    return pr
+
+
+@pytest.mark.parametrize("kind", ["euler", "prev_only", "no_rotation", "strong_decay",
+                                  "tiny_step", "fast_angle"])
+@pytest.mark.parametrize("R,L,b", [(1, 333, 2), (4, 150, 2), (1, 2543, 1)])
+def test_scan_degenerate_regimes(cuda_dev, kind, R, L, b):
+    """Limits of the recurrence through the tensor-core scan (SISO, MIMO, and the
+    sequence-parallel form at b1 L2543) against the oracle."""
+    pr = make_problem(b, L, 4, 1, 64, 128, rank=R, chunk=64 // R, bc_norm=True, bias_std=0.1,
+                      seed=101 + L + R, with_state=True)
+    pr = _degenerate(pr, kind)
+    y, fin = gpu_scan(pr, cuda_dev)
+    assert torch.isfinite(y.float()).all() and torch.isfinite(fin.h).all()
+    yo, so = oracle_scan(pr)
+    compare(pr, y, fin, yo, so)
+
+
+@pytest.mark.parametrize("kind", ["euler", "strong_decay", "fast_angle"])
+@pytest.mark.parametrize("R", [1, 4])
+def test_decode_degenerate_regimes(cuda_dev, kind, R):
+    steps = 3
+    pr = make_problem(2, steps, 4, 1, 64, 128, rank=R, chunk=1, bc_norm=True, bias_std=0.1,
+                      seed=121 + R, with_state=True)
+    pr = _degenerate(pr, kind)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    ys = []
+    for t in range(steps):
+        tok = {k: (v[:, t:t + 1].contiguous() if k not in ("B_bias", "C_bias") else v)
+               for k, v in g.tensors().items()}
+        y, st = m3.decode_step(**tok, state_in=st, bc_norm=True)
+        ys.append(y.clone())
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.stack(ys, 1), st, yo, so)
