@@ -65,7 +65,7 @@ typedef struct {
     int32_t in_dtype; /* m3_dtype                                                   */
     int32_t bc_norm;  /* nonzero: RMS-normalise B and C over N before the bias      */
     float norm_eps;   /* epsilon of the RMS norm (1e-6 is the usual value)          */
-    uint32_t flags;   /* M3_DT_SOFTPLUS | M3_LAM_SIGMOID, or 0                      */
+    uint32_t flags;   /* M3_DT_SOFTPLUS | M3_LAM_SIGMOID | M3_DISC_ZOH, or 0        */
 } m3_dims;
 
 /* m3_dims.flags: the step scalars arrive as the layer's raw projections and the kernels
@@ -75,9 +75,14 @@ typedef struct {
  *                   is a positive projection of the token, Sec. 2 "Mamba-2 parameterisation").
  *   M3_LAM_SIGMOID: lam holds u; the trapezoid weight is sigma(u) = 1 / (1 + e^{-u})
  *                   (Appendix F, default parameterisation lambda_t = sigma(u_t)).
- * Positions past the end of the sequence are not tokens and stay zero. */
+ * Positions past the end of the sequence are not tokens and stay zero.
+ *   M3_DISC_ZOH:    the zero-order-hold discretisation of Mamba-1/2 instead of the
+ *                   exponential-trapezoidal one ("Mamba-3：推理优先的状态空间模型", Sec. 1.2):
+ *                   h_t = alpha_t h_{t-1} + gamma_t B_t x_t with gamma_t = (alpha_t - 1) / A_t
+ *                   and no previous-token term; lam is not used. The rotation is unchanged. */
 #define M3_DT_SOFTPLUS 1u
 #define M3_LAM_SIGMOID 2u
+#define M3_DISC_ZOH 4u
 
 typedef struct {
     const void* x;        /* [b, L, H, R, P]   in_dtype                                   */

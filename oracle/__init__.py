@@ -48,6 +48,7 @@ class _Dims(ctypes.Structure):
         ("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
         ("ngroups", ctypes.c_int64), ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64),
         ("rank", ctypes.c_int64), ("bc_norm", ctypes.c_int32), ("norm_eps", ctypes.c_double),
+        ("zoh", ctypes.c_int32),
     ]
 
 
@@ -106,7 +107,7 @@ class State:
         return State(self.h.copy(), self.phi.copy(), self.prev_B.copy(), self.prev_x.copy())
 
 
-DT_SOFTPLUS, LAM_SIGMOID = 1, 2
+DT_SOFTPLUS, LAM_SIGMOID, DISC_ZOH = 1, 2, 4
 
 
 def step_scalars(dt, lam, dt_bias=None, flags: int = 0):
@@ -135,7 +136,8 @@ def scan(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state: State | No
     Shapes: x [b,L,H,R,P]; B, C [b,L,G,R,N]; theta [b,L,H,N/2]; dt, A, lam [b,L,H];
     B_bias, C_bias [H,R,N] or None. ``state`` (float64, not modified) is the state before
     the first token, or None for a fresh sequence (all zeros). ``flags`` and ``dt_bias``:
-    dt and lam are raw projections, see ``step_scalars``.
+    dt and lam are raw projections, see ``step_scalars``; DISC_ZOH: zero-order-hold weights
+    beta = 0, gamma = (e^{dt A} - 1) / A ("Mamba-3：推理优先的状态空间模型", Sec. 1.2).
 
     Returns (y [b,L,H,R,P] float64, final State)."""
     x, B, C, theta = _f64(x), _f64(B), _f64(C), _f64(theta)
@@ -154,7 +156,8 @@ def scan(x, B, C, theta, dt, A, lam, B_bias=None, C_bias=None, state: State | No
     assert st.h.shape == (b, H, N, P) and st.phi.shape == (b, H, N // 2)
     assert st.prev_B.shape == (b, H, R, N) and st.prev_x.shape == (b, H, R, P)
     y = np.zeros((b, L, H, R, P))
-    d = _Dims(b, L, H, G, P, N, R, 1 if bc_norm else 0, float(norm_eps))
+    d = _Dims(b, L, H, G, P, N, R, 1 if bc_norm else 0, float(norm_eps),
+              1 if flags & DISC_ZOH else 0)
     rc = _load().m3o_scan(ctypes.byref(d), _ptr(x), _ptr(B), _ptr(C), _ptr(theta), _ptr(dt),
                           _ptr(A), _ptr(lam), _ptr(B_bias), _ptr(C_bias), _ptr(st.h),
                           _ptr(st.phi), _ptr(st.prev_B), _ptr(st.prev_x), _ptr(y),

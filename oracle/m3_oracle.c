@@ -12,6 +12,8 @@
  *                                             State Space Principles", Sec. 3.4, BC norm
  *                                             and B,C bias)
  *   alpha = exp(dt*A), beta = (1-lam)*dt*alpha, gamma = lam*dt      (Sec. 3.1.1, Prop. 1)
+ *   (zero-order hold instead, when asked: beta = 0, gamma = (alpha - 1)/A, lam unused:
+ *    "Mamba-3：推理优先的状态空间模型", Sec. 1.2; the rotation is unchanged)
  *   Phi  += dt*theta                     cumulative angle of the rotations R_0..R_t
  *                                        (Sec. 3.2.1, Prop. 2: R_t = Block{R(dt_t*theta_t[i])})
  *   Bbar  = R(Phi)^T Bn, Cbar = R(Phi)^T Cn, Bpbar = R(Phi_prev)^T Bpn
@@ -50,6 +52,7 @@ typedef struct {
     int64_t batch, seqlen, nheads, ngroups, headdim, dstate, rank;
     int32_t bc_norm;
     double norm_eps;
+    int32_t zoh; /* nonzero: zero-order-hold weights */
 } m3o_dims;
 
 /* RMS normalisation over the N entries of v (no learnable weight), then add bias. */
@@ -102,8 +105,9 @@ static void scan_unit(const m3o_dims* d, int64_t b, int64_t hh, const double* x,
         const int64_t sc = tok * H + hh; /* index into dt, A, lam */
         const double a_dt = dt[sc] * A[sc];
         const double alpha = exp(a_dt);
-        const double beta = (1.0 - lam[sc]) * dt[sc] * alpha;
-        const double gamma = lam[sc] * dt[sc];
+        const double beta = d->zoh ? 0.0 : (1.0 - lam[sc]) * dt[sc] * alpha;
+        const double gamma = d->zoh ? (a_dt != 0.0 ? expm1(a_dt) / A[sc] : dt[sc])
+                                    : lam[sc] * dt[sc];
 
         memcpy(phi_prev, ph, sizeof(double) * (size_t)half);
         const double* th = theta + sc * half;

@@ -42,7 +42,7 @@ m3_status check_dims(const m3_dims* d, bool scan) {
         return fail(M3_ERR_INVALID_ARG, "headdim >= 1, even dstate >= 2 and rank >= 1 required");
     if (!(d->norm_eps >= 0.f) || !std::isfinite(d->norm_eps))
         return fail(M3_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
-    if (d->flags & ~(M3_DT_SOFTPLUS | M3_LAM_SIGMOID))
+    if (d->flags & ~(M3_DT_SOFTPLUS | M3_LAM_SIGMOID | M3_DISC_ZOH))
         return fail(M3_ERR_INVALID_ARG, "unknown bits in flags (0x%x)", (unsigned)d->flags);
     if (d->headdim != 16 && d->headdim != 32 && d->headdim != 64 && d->headdim != 128)
         return fail(M3_ERR_UNSUPPORTED, "headdim %lld not in {16, 32, 64, 128}",

@@ -49,6 +49,13 @@ __device__ __forceinline__ float step_lam(float raw, uint32_t flags) {
     else return (flags & 2u) ? __frcp_rn(1.f + __expf(-raw)) : raw;   // e^{-raw} = inf gives 0
 }
 
+// The zero-order-hold input weight (e^{dt A} - 1) / A ("Mamba-3：推理优先的状态空间模型",
+// Sec. 1.2), dt in the limit A -> 0; with M3_DISC_ZOH it replaces gamma and beta is 0.
+__device__ __forceinline__ float zoh_gamma(float dt, float A) {
+    const float x = dt * A;
+    return x != 0.f ? expm1f(x) / A : dt;
+}
+
 // Inclusive prefix sum across the 32 lanes of a warp.
 __device__ __forceinline__ float warp_inclusive_scan(float v) {
     const int lane = threadIdx.x & 31;

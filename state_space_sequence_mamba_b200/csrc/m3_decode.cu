@@ -89,8 +89,9 @@ decode_kernel(const ScanParams p, const int rows_per_pass) {
         const float a = p.A[u], l = step_lam(p.lam[u], p.flags);
         const float al = expf(d * a);
         scal[0] = al;
-        scal[1] = (1.f - l) * d * al;
-        scal[2] = l * d;
+        const bool zoh = p.flags & 4u;   // zero-order hold: no previous-token term
+        scal[1] = zoh ? 0.f : (1.f - l) * d * al;
+        scal[2] = zoh ? zoh_gamma(d, a) : l * d;
         scal[3] = d;
     }
     __syncthreads();

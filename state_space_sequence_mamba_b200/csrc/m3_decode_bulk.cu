@@ -177,7 +177,14 @@ decode_bulk_kernel(const ScanParams p, const int n_units) {
         const __nv_bfloat16* sC = reinterpret_cast<const __nv_bfloat16*>(base + bl.c);
         const __nv_bfloat16* sBp = reinterpret_cast<const __nv_bfloat16*>(base + bl.bp);
         const float d = sc[4 * b + 0], a = sc[4 * b + 1], lm = sc[4 * b + 2];
-        const float al = expf(d * a), be = (1.f - lm) * d * al, ga = lm * d;
+        const float al = expf(d * a);
+        float be = (1.f - lm) * d * al, ga = lm * d;
+        if constexpr (kRaw) {
+            if (p.flags & 4u) {   // zero-order hold: no previous-token term
+                be = 0.f;
+                ga = zoh_gamma(d, a);
+            }
+        }
 
         // ---- RMS scales of B, C and the stored previous B, one warp per vector ----
         if (p.bc_norm) {

@@ -261,7 +261,14 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
         const __nv_bfloat16* sx = reinterpret_cast<const __nv_bfloat16*>(sl + Cfg::S_X);
         const __nv_bfloat16* sxp = reinterpret_cast<const __nv_bfloat16*>(sl + Cfg::S_XP);
         const float d = scal[4 * s + 0], a = scal[4 * s + 1], lm = scal[4 * s + 2];
-        const float al = __expf(d * a), be = (1.f - lm) * d * al, ga = lm * d;
+        const float al = __expf(d * a);
+        float be = (1.f - lm) * d * al, ga = lm * d;
+        if constexpr (kRaw) {
+            if (p.flags & 4u) {   // zero-order hold: no previous-token term
+                be = 0.f;
+                ga = zoh_gamma(d, a);
+            }
+        }
         const int64_t hh = u % p.H;
 
         // ---- RMS scales of B, C and the stored previous B, one warp per vector ----

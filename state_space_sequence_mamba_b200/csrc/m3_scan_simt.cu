@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kSimtThreads) scan_simt_kernel(const ScanParam
             }
         }
         __syncthreads();
-        const float f = (1.f - lam_at(0)) * dt_at(0);
+        const float f = (p.flags & 4u) ? 0.f : (1.f - lam_at(0)) * dt_at(0);
         for (int64_t e = tid; e < N * P; e += nth) {
             const int64_t n = e / P, pp = e % P;
             float acc = 0.f;
@@ -130,14 +130,13 @@ __global__ void __launch_bounds__(kSimtThreads) scan_simt_kernel(const ScanParam
                 const int64_t si = sidx(c0 + t);
                 const float d = dt_at(c0 + t), a = p.A[si], l = lam_at(c0 + t);
                 cum += d * a;
-                float w = l * d;
-                if (c0 + t + 1 < L) {
-                    const int64_t sn = sidx(c0 + t + 1);
-                    w += (1.f - lam_at(c0 + t + 1)) * dt_at(c0 + t + 1);
-                }
+                const bool zoh = p.flags & 4u;   // zero-order hold: no previous-token term
+                const float g = zoh ? zoh_gamma(d, a) : l * d;
+                float w = g;
+                if (!zoh && c0 + t + 1 < L) w += (1.f - lam_at(c0 + t + 1)) * dt_at(c0 + t + 1);
                 sc[8 * t + 0] = d;
                 sc[8 * t + 1] = cum;
-                sc[8 * t + 2] = l * d;
+                sc[8 * t + 2] = g;
                 sc[8 * t + 3] = w;
                 sc[8 * t + 4] = expf(cum);
             }

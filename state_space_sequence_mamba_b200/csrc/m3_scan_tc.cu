@@ -310,6 +310,12 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                 ga[k] = lm * dd;
                 // next token (the box holds Q + 1 tokens, zero-filled past the sequence end)
                 w[k] = ga[k] + (1.f - sSc[oL + (t + 1) * 4 + hc]) * sSc[(t + 1) * 4 + hc];
+                if constexpr (kRaw) {
+                    if (p.flags & 4u) {   // zero-order hold: no previous-token term
+                        ga[k] = zoh_gamma(dd, sSc[oA + t * 4 + hc]);
+                        w[k] = ga[k];
+                    }
+                }
             }
         }
         const float c0s = warp_inclusive_scan(a[0]);
@@ -461,8 +467,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
         __syncthreads();
         const int64_t s0 = bb * p.L * p.H + hh;
-        const float f = (1.f - step_lam<kRaw>(p.lam[s0], p.flags)) *
-                        step_dt<kRaw>(p.dt[s0], dtb, p.flags);
+        const float f = (kRaw && (p.flags & 4u)) ? 0.f   // zero-order hold: no beta term
+                        : (1.f - step_lam<kRaw>(p.lam[s0], p.flags)) * step_dt<kRaw>(p.dt[s0], dtb, p.flags);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             float acc = 0.f;

@@ -59,7 +59,7 @@ def test_struct_layout_matches_header(lib):
     (dict(headdim=48), False), (dict(rank=3), False), (dict(chunk=0), False),
     (dict(chunk=64, rank=4), False), (dict(chunk=16, rank=4), True), (dict(in_dtype=7), False),
     (dict(dstate=272), False), (dict(norm_eps=-1.0), False), (dict(batch=-1), False),
-    (dict(flags=3), True), (dict(flags=4), False),
+    (dict(flags=7), True), (dict(flags=8), False),
 ])
 def test_workspace_query_validates(lib, kw, ok):
     n = lib.m3_scan_workspace_bytes(ctypes.byref(dims(**kw)))

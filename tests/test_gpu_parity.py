@@ -447,3 +447,45 @@ def test_decode_degenerate_regimes(cuda_dev, kind, R):
     torch.cuda.synchronize()
     yo, so = oracle_scan(pr)
     compare(pr, torch.stack(ys, 1), st, yo, so)
+
+
+# ---------------------------------------------------------------- zero-order hold
+ZOH = [
+    # b, L, H, P, N, R, chunk, dtype, raw scalars too
+    (2, 333, 4, 64, 128, 1, 64, torch.bfloat16, False),   # tensor-core scan, SISO
+    (2, 150, 4, 64, 128, 4, 16, torch.bfloat16, True),    # tensor-core scan, MIMO, flags 7
+    (1, 2543, 4, 64, 128, 1, 64, torch.bfloat16, False),  # sequence-parallel form
+    (1, 130, 2, 64, 128, 1, 64, torch.float32, False),    # exact fp32 path
+]
+
+
+@pytest.mark.parametrize("case", ZOH, ids=lambda c: "b{}L{}R{}{}{}".format(
+    c[0], c[1], c[5], "f32" if c[7] == torch.float32 else "bf16", "raw" if c[8] else ""))
+def test_scan_zoh(cuda_dev, case):
+    """M3_DISC_ZOH (beta = 0, gamma = (alpha - 1) / A) through every scan path."""
+    b, L, H, P, N, R, Q, dt, raw = case
+    pr = make_problem(b, L, H, 1, P, N, rank=R, chunk=Q, dtype=dt, bc_norm=True,
+                      bias_std=0.1, seed=5 * L + R, with_state=True, raw_scalars=raw)
+    pr.flags |= m3.M3_DISC_ZOH
+    y, fin = gpu_scan(pr, cuda_dev)
+    yo, so = oracle_scan(pr)
+    compare(pr, y, fin, yo, so, tol=1e-4 if dt == torch.float32 else None)
+
+
+@pytest.mark.parametrize("R,dt", [(1, torch.bfloat16), (4, torch.bfloat16), (2, torch.float32)])
+def test_decode_zoh(cuda_dev, R, dt):
+    steps = 4
+    pr = make_problem(2, steps, 4, 1, 64, 128, rank=R, chunk=1, dtype=dt, bc_norm=True,
+                      bias_std=0.1, seed=140 + R, with_state=True)
+    pr.flags |= m3.M3_DISC_ZOH
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    ys = []
+    for t in range(steps):
+        tok = {k: (v[:, t:t + 1].contiguous() if k not in ("B_bias", "C_bias") else v)
+               for k, v in g.tensors().items()}
+        y, st = m3.decode_step(**tok, **g.scalar_args(), state_in=st, bc_norm=True)
+        ys.append(y.clone())
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.stack(ys, 1), st, yo, so, tol=1e-4 if dt == torch.float32 else None)

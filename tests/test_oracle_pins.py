@@ -496,3 +496,30 @@ def test_decode_step_proj_against_library_gate_and_contraction():
                                p["bc_norm"])
     ref1 = y1[:, :, 0, :] * torch.nn.functional.silu(torch.from_numpy(zp)).numpy()
     np.testing.assert_allclose(o1, ref1, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- zero-order hold
+def test_zoh_is_exact_for_piecewise_constant_input():
+    """The zero-order-hold weights ("Mamba-3：推理优先的状态空间模型", Sec. 1.2) are the exact
+    solution of h' = A h + B x when A, B and x are held constant over each step: the oracle
+    with DISC_ZOH against scipy's ODE integrator over the same steps (theta = 0, no norm)."""
+    from scipy.integrate import solve_ivp
+    rng = np.random.default_rng(41)
+    L, N, P = 12, 2, 3
+    x = rng.standard_normal((1, L, 1, 1, P))
+    B = np.zeros((1, L, 1, 1, N)); B[..., 0] = 1.0 + rng.random((1, L, 1, 1))
+    C = np.zeros((1, L, 1, 1, N)); C[..., 0] = 1.0
+    dt = rng.uniform(0.1, 0.6, (1, L, 1))
+    A = -rng.uniform(0.2, 2.5, (1, L, 1))
+    lam = rng.random((1, L, 1))            # unused under zero-order hold
+    y, st = oracle.scan(x, B, C, np.zeros((1, L, 1, N // 2)), dt, A, lam, flags=oracle.DISC_ZOH)
+    h = np.zeros(P)
+    for t in range(L):
+        a, b, xt = A[0, t, 0], B[0, t, 0, 0, 0], x[0, t, 0, 0]
+        sol = solve_ivp(lambda _, v: a * v + b * xt, (0.0, dt[0, t, 0]), h, rtol=1e-12, atol=1e-14)
+        h = sol.y[:, -1]
+        np.testing.assert_allclose(y[0, t, 0, 0], h, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(st.h[0, 0, 0], h, rtol=1e-9, atol=1e-12)
+    # lam does not enter, and the previous token does not either
+    y2, _ = oracle.scan(x, B, C, np.zeros((1, L, 1, N // 2)), dt, A, 1 - lam, flags=oracle.DISC_ZOH)
+    np.testing.assert_array_equal(y, y2)
