@@ -189,6 +189,50 @@ M3_API m3_status m3_scan_state(const m3_dims* dims, const m3_inputs* in, const m
 M3_API m3_status m3_state_combine(const m3_dims* dims, int nseg, const m3_seg_state* seg,
                                   float* h_out, float* phi_out, void* stream);
 
+/* ---- Backward pass of the prefill scan (the training side of the same recurrence) ----
+ * Gradients of  L = sum(y * dy) + <final state, dfinal>  with respect to every input of
+ * m3_scan_fwd and to its initial state, for the forward that m3_scan_fwd computes with the
+ * same dims, inputs and init (Sec. 3.1.1 Prop. 1, Sec. 3.2.2 Prop. 4, Sec. 3.4, Appendix C;
+ * the flags' transforms are differentiated too). All gradients are fp32. */
+typedef struct {
+    float* dx;        /* [b, L, H, R, P]                                                      */
+    float* dB;        /* [b, L, G, R, N] with respect to the raw B (heads of a group summed)  */
+    float* dC;        /* [b, L, G, R, N]                                                      */
+    float* dtheta;    /* [b, L, H, N/2]                                                       */
+    float* ddt;       /* [b, L, H] with respect to dt as passed (the raw projection under
+                         M3_DT_SOFTPLUS)                                                     */
+    float* dA;        /* [b, L, H]                                                            */
+    float* dlam;      /* [b, L, H] with respect to lam as passed (u under M3_LAM_SIGMOID; zero
+                         under M3_DISC_ZOH, which does not use it)                           */
+    float* dB_bias;   /* [H, R, N], or NULL to skip                                           */
+    float* dC_bias;   /* [H, R, N], or NULL                                                   */
+    float* ddt_bias;  /* [H], or NULL; zero unless M3_DT_SOFTPLUS                             */
+} m3_grads;
+
+/* Gradient with respect to a state (all fp32, shapes as m3_state). As an input a NULL field
+ * (or a NULL struct) is zero; as an output a NULL field is not written. */
+typedef struct {
+    float* h;       /* [b, H, N, P] */
+    float* phi;     /* [b, H, N/2]  */
+    float* prev_B;  /* [b, H, R, N] with respect to the raw previous B */
+    float* prev_x;  /* [b, H, R, P] */
+} m3_state_grad;
+
+/* Workspace bytes m3_scan_bwd needs (0 for invalid dims): two fp32 [b, L, H, R, N] buffers
+ * plus O(b H (L + N L / 16)) floats. Any content; it is scratch. */
+M3_API size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims);
+
+/* dims, in, init: as given to m3_scan_fwd (dims->chunk is not used here). dy [b, L, H, R, P]
+ * in_dtype. dfinal: the final state's gradient, or NULL. grads: dx .. dlam are required
+ * (16-byte aligned) and overwritten; the bias gradients are overwritten when not NULL.
+ * dinit: where to write the initial state's gradient, or NULL. workspace: 256-byte aligned,
+ * at least m3_scan_bwd_workspace_bytes. Any supported N, P, R, dtype and flags; asynchronous
+ * on `stream`. */
+M3_API m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                             const void* dy, const m3_state_grad* dfinal,
+                             const m3_grads* grads, const m3_state_grad* dinit,
+                             void* workspace, size_t ws_bytes, void* stream);
+
 /* After the stream that ran m3_scan_fwd has synchronised: M3_OK, or M3_ERR_TIMEOUT if a
  * bounded inter-CTA wait gave up (the outputs of that call are then incomplete). Performs
  * one blocking 4-byte device-to-host copy; after a timeout it also re-zeroes the workspace

@@ -52,10 +52,15 @@ class Proj(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("x_in", "z_in", "W_X", "W_Z", "W_O")]
 
 
+class Grads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dx", "dB", "dC", "dtheta", "ddt", "dA", "dlam",
+                                               "dB_bias", "dC_bias", "ddt_bias")]
+
+
 # Symbols include/m3.h declares (checked by the CPU test suite).
 EXPORTS = ("m3_scan_workspace_bytes", "m3_scan_fwd", "m3_decode_step", "m3_scan_check",
            "m3_status_str", "m3_last_error", "m3_scan_fwd_noalloc", "m3_decode_step_proj",
-           "m3_scan_state", "m3_state_combine")
+           "m3_scan_state", "m3_state_combine", "m3_scan_bwd_workspace_bytes", "m3_scan_bwd")
 
 _lib = None
 
@@ -87,6 +92,12 @@ def load_library(path: str = LIB_PATH):
     lib.m3_state_combine.argtypes = [P(Dims), ctypes.c_int, P(SegState), ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p]
     lib.m3_state_combine.restype = ctypes.c_int
+    lib.m3_scan_bwd_workspace_bytes.argtypes = [P(Dims)]
+    lib.m3_scan_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.m3_scan_bwd.argtypes = [P(Dims), P(Inputs), P(StateC), ctypes.c_void_p, P(StateC),
+                                P(Grads), P(StateC), ctypes.c_void_p, ctypes.c_size_t,
+                                ctypes.c_void_p]
+    lib.m3_scan_bwd.restype = ctypes.c_int
     lib.m3_scan_check.argtypes = [ctypes.c_void_p]
     lib.m3_scan_check.restype = ctypes.c_int
     lib.m3_status_str.argtypes = [ctypes.c_int]
@@ -290,3 +301,50 @@ def state_combine(h, phi, lam_sum, stream=None):
                               _ptr(phi_out), _stream_handle(stream))
     _check(rc)
     return h_out, phi_out
+
+
+def scan_bwd_workspace_bytes(dims: Dims) -> int:
+    return int(load_library().m3_scan_bwd_workspace_bytes(ctypes.byref(dims)))
+
+
+def scan_bwd(x, B, C, theta, dt, A, lam, dy, B_bias=None, C_bias=None, init: State | None = None,
+             dfinal: dict | None = None, bc_norm=False, norm_eps=1e-6, stream=None, dt_bias=None,
+             flags=0, want_init=True, workspace=None):
+    """m3_scan_bwd: gradients of sum(y * dy) + <final state, dfinal> for the forward that
+    scan_fwd runs on the same arguments. ``dfinal``: dict of fp32 h, phi, prev_B, prev_x (any
+    may be missing = 0). Returns a dict of fp32 tensors dx, dB, dC, dtheta, ddt, dA, dlam,
+    dB_bias, dC_bias, ddt_bias and (with want_init) dinit, a dict of the initial state's."""
+    lib = load_library()
+    dims = make_dims(x, B, 1, bc_norm, norm_eps, flags)
+    b, L, H, R, P = x.shape
+    G, N = B.shape[2], B.shape[4]
+    dev = x.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(dx=torch.empty(b, L, H, R, P, **f32), dB=torch.empty(b, L, G, R, N, **f32),
+             dC=torch.empty(b, L, G, R, N, **f32), dtheta=torch.empty(b, L, H, N // 2, **f32),
+             ddt=torch.empty(b, L, H, **f32), dA=torch.empty(b, L, H, **f32),
+             dlam=torch.empty(b, L, H, **f32), dB_bias=torch.empty(H, R, N, **f32),
+             dC_bias=torch.empty(H, R, N, **f32), ddt_bias=torch.empty(H, **f32))
+    gc = Grads(*(_ptr(g[k]) for k in ("dx", "dB", "dC", "dtheta", "ddt", "dA", "dlam",
+                                       "dB_bias", "dC_bias", "ddt_bias")))
+    dinit = None
+    if want_init:
+        dinit = dict(h=torch.empty(b, H, N, P, **f32), phi=torch.empty(b, H, N // 2, **f32),
+                     prev_B=torch.empty(b, H, R, N, **f32), prev_x=torch.empty(b, H, R, P, **f32))
+    if workspace is None:
+        workspace = torch.empty(max(256, scan_bwd_workspace_bytes(dims)), dtype=torch.uint8,
+                                device=dev)
+    ins = Inputs(*(_ptr(t) for t in (x, B, C, theta, dt, A, lam, B_bias, C_bias, dt_bias)))
+    ic = init.c() if init is not None else None
+    df = None
+    if dfinal is not None:
+        df = StateC(*(_ptr(dfinal.get(k)) for k in ("h", "phi", "prev_B", "prev_x")))
+    di = StateC(*(_ptr(dinit[k]) for k in ("h", "phi", "prev_B", "prev_x"))) if dinit else None
+    rc = lib.m3_scan_bwd(ctypes.byref(dims), ctypes.byref(ins),
+                         ctypes.byref(ic) if ic is not None else None, _ptr(dy),
+                         ctypes.byref(df) if df is not None else None, ctypes.byref(gc),
+                         ctypes.byref(di) if di is not None else None, _ptr(workspace),
+                         workspace.numel(), _stream_handle(stream))
+    _check(rc)
+    g["dinit"] = dinit
+    return g

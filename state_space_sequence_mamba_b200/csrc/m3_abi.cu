@@ -368,3 +368,85 @@ const char* m3_status_str(m3_status s) {
 const char* m3_last_error(void) { return g_err; }
 
 }  // extern "C"
+
+extern "C" {
+
+size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims) {
+    if (check_dims(dims, false) != M3_OK) return 0;
+    return sizeof(float) * scan_bwd_workspace_floats(dims->batch, dims->seqlen, dims->nheads,
+                                                     dims->dstate, dims->rank);
+}
+
+m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
+                      const void* dy, const m3_state_grad* dfinal, const m3_grads* grads,
+                      const m3_state_grad* dinit, void* workspace, size_t ws_bytes,
+                      void* stream) {
+    g_err[0] = 0;
+    m3_status st = check_dims(dims, false);
+    if (st != M3_OK) return st;
+    const bool any = dims->batch * dims->seqlen * dims->nheads > 0;
+    if ((st = check_inputs(in, any)) != M3_OK) return st;
+    if ((st = check_state(init, "initial")) != M3_OK) return st;
+    if (!grads) return fail(M3_ERR_INVALID_ARG, "grads is NULL");
+    if (any) {
+        const void* req[] = {dy, grads->dx, grads->dB, grads->dC, grads->dtheta,
+                             grads->ddt, grads->dA, grads->dlam};
+        const char* names[] = {"dy", "dx", "dB", "dC", "dtheta", "ddt", "dA", "dlam"};
+        for (int i = 0; i < 8; ++i) {
+            if (!req[i]) return fail(M3_ERR_INVALID_ARG, "%s is NULL", names[i]);
+            if (!aligned16(req[i]))
+                return fail(M3_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+        }
+    }
+    const void* opt[] = {grads->dB_bias, grads->dC_bias, grads->ddt_bias,
+                         dfinal ? dfinal->h : nullptr, dfinal ? dfinal->phi : nullptr,
+                         dfinal ? dfinal->prev_B : nullptr, dfinal ? dfinal->prev_x : nullptr,
+                         dinit ? dinit->h : nullptr, dinit ? dinit->phi : nullptr,
+                         dinit ? dinit->prev_B : nullptr, dinit ? dinit->prev_x : nullptr};
+    for (const void* q : opt)
+        if (q && !aligned16(q))
+            return fail(M3_ERR_INVALID_ARG, "gradient pointers must be 16-byte aligned");
+    const size_t smem = scan_bwd_smem_bytes(dims->dstate, dims->headdim, dims->rank);
+    if (smem > 227 * 1024)
+        return fail(M3_ERR_UNSUPPORTED, "backward needs %zu bytes of shared memory", smem);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t H = dims->nheads, R = dims->rank, N = dims->dstate, P = dims->headdim;
+    const int64_t units = dims->batch * H;
+    if (!any) {
+        // no token: the biases get nothing and the initial state's gradient is the final one's
+        cudaError_t e = cudaSuccess;
+        if (grads->dB_bias) e = cudaMemsetAsync(grads->dB_bias, 0, H * R * N * 4, s);
+        if (e == cudaSuccess && grads->dC_bias) e = cudaMemsetAsync(grads->dC_bias, 0, H * R * N * 4, s);
+        if (e == cudaSuccess && grads->ddt_bias) e = cudaMemsetAsync(grads->ddt_bias, 0, H * 4, s);
+        float* dst[4] = {dinit ? dinit->h : nullptr, dinit ? dinit->phi : nullptr,
+                         dinit ? dinit->prev_B : nullptr, dinit ? dinit->prev_x : nullptr};
+        const float* src[4] = {dfinal ? dfinal->h : nullptr, dfinal ? dfinal->phi : nullptr,
+                               dfinal ? dfinal->prev_B : nullptr, dfinal ? dfinal->prev_x : nullptr};
+        const size_t bytes[4] = {static_cast<size_t>(units * N * P * 4),
+                                 static_cast<size_t>(units * (N / 2) * 4),
+                                 static_cast<size_t>(units * R * N * 4),
+                                 static_cast<size_t>(units * R * P * 4)};
+        for (int i = 0; i < 4 && e == cudaSuccess; ++i) {
+            if (!dst[i] || bytes[i] == 0) continue;
+            e = src[i] ? cudaMemcpyAsync(dst[i], src[i], bytes[i], cudaMemcpyDeviceToDevice, s)
+                       : cudaMemsetAsync(dst[i], 0, bytes[i], s);
+        }
+        return e == cudaSuccess ? M3_OK : cuda_fail(e, "empty-sequence gradient copy");
+    }
+    const size_t need = m3_scan_bwd_workspace_bytes(dims);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
+        return fail(M3_ERR_INVALID_ARG, "workspace: NULL, misaligned or below %zu bytes", need);
+    const ScanParams p = make_params(dims, in, init, nullptr, nullptr);
+    BwdGrads g{};
+    g.dy = dy;
+    if (dfinal) { g.dh1 = dfinal->h; g.dphi1 = dfinal->phi; g.dprevB1 = dfinal->prev_B; g.dprevx1 = dfinal->prev_x; }
+    g.dx = grads->dx; g.dB = grads->dB; g.dC = grads->dC; g.dtheta = grads->dtheta;
+    g.ddt = grads->ddt; g.dA = grads->dA; g.dlam = grads->dlam;
+    g.dBbias = grads->dB_bias; g.dCbias = grads->dC_bias; g.ddtbias = grads->ddt_bias;
+    if (dinit) { g.dh0 = dinit->h; g.dphi0 = dinit->phi; g.dprevB0 = dinit->prev_B; g.dprevx0 = dinit->prev_x; }
+    cudaError_t e = launch_scan_bwd(p, g, dims->in_dtype == M3_BF16, static_cast<float*>(workspace), s);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+    return M3_OK;
+}
+
+}  // extern "C"

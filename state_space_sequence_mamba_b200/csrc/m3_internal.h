@@ -99,4 +99,36 @@ cudaError_t launch_decode_tc(const ScanParams& p, cudaStream_t s);
 // Size of the decode kernel's dynamic shared memory for these dims.
 size_t decode_smem_bytes(const ScanParams& p);
 
+// Backward pass of the scan (m3_scan_bwd): the output and final-state gradients in, the input
+// and initial-state gradients out (all fp32; the nullable ones as in m3.h).
+struct BwdGrads {
+    const void* dy;
+    const float* dh1;
+    const float* dphi1;
+    const float* dprevB1;
+    const float* dprevx1;
+    float* dx;
+    float* dB;
+    float* dC;
+    float* dtheta;
+    float* ddt;
+    float* dA;
+    float* dlam;
+    float* dBbias;
+    float* dCbias;
+    float* ddtbias;
+    float* dh0;
+    float* dphi0;
+    float* dprevB0;
+    float* dprevx0;
+};
+// Tokens per staged chunk of the backward sweeps, their workspace (floats) and shared memory.
+int bwd_chunk_tokens(int64_t R);
+size_t scan_bwd_workspace_floats(int64_t b, int64_t L, int64_t H, int64_t N, int64_t R);
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t R);
+// f: the forward's inputs and initial state (validated); ws: scan_bwd_workspace_floats floats,
+// 256-byte aligned. L >= 1 and b >= 1.
+cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, float* ws,
+                            cudaStream_t s);
+
 }  // namespace m3

@@ -1,0 +1,884 @@
+// Backward pass of the prefill scan: the gradients of every input and of the initial state,
+// given the gradient dy of the output and of the final state.
+//
+// The forward ("Mamba-3: Improved Sequence Modeling using State Space Principles", Sec. 3.1.1
+// Prop. 1, Sec. 3.2.2 Prop. 4, Sec. 3.4, Appendix C) per (batch, head) unit is
+//   h_t = a_t h_{t-1} + b_t u_{t-1} + g_t u_t,   u_t = sum_r Bbar_t[r] x_t[r]^T,
+//   y_t[r] = h_t^T Cbar_t[r],   Bbar_t = R(Phi_t)^T (norm(B_t) + bias),   Phi_t = Phi_{t-1} + dt_t theta_t.
+// With G_t = dL/dh_t = sum_r Cbar_t[r] dy_t[r]^T + a_{t+1} G_{t+1} the gradients split into
+// two sweeps that never need h and G at the same token:
+//   forward sweep (bwd_fwd_kernel): h_t, hence dCbar_t[r] = h_t dy_t[r] (a contraction over P);
+//   reverse sweep (bwd_rev_kernel): G_t, hence du_t = g_t G_t + b_{t+1} G_{t+1},
+//     dx_t[r] = du_t^T Bbar_t[r], dBbar_t[r] = du_t x_t[r], db_t = <G_t, u_{t-1}>, dg_t = <G_t, u_t>,
+//     and the angle adjoint: Phi_t rotates Bbar_t and Cbar_t, so dPhi_t collects
+//     dBbar x Bbar + dCbar x Cbar (the cross product of each pair) and is summed from the end.
+// The decay's own gradient needs <G_t, h_{t-1}>, which neither sweep has; it follows instead
+// from <G_t, h_t> = dy_t . y_t + a_{t+1} <G_{t+1}, h_t>: with a_t = e^{dt A}, the gradient of
+// the log-decay dt_t A_t through the h_{t-1} term is
+//   D_t = sum_{s >= t} (dy_s . y_s - b_s db_s - g_s dg_s) + <dL/dh_final, h_final>,
+// where dy_s . y_s = sum_r <Cbar_s[r], dCbar_s[r]>. bwd_scalar_kernel takes that suffix sum and
+// the chain rule to dt, A and lam (and to the raw projections under the flags);
+// bwd_norm_kernel undoes the rotation's partner, the RMS norm, and sums heads that share a
+// group's B and C.
+//
+// Thread layout of the sweeps: one CTA per unit with 2N threads; thread = (pair i, quarter q)
+// owns the rows i and i + N/2 (one complex pair, so the rotation is thread-local) and the
+// P/4 columns q*P/4 .. of h or G in registers. Contractions over P finish with two shuffles
+// inside the quad; contractions over N with a butterfly across the warp's eight pairs and a
+// shared-memory add across warps. A chunk of T tokens is staged in shared memory (rotated B and
+// C, x, dy, cos/sin, scalars) before the sequential token loop, so the loop has no barrier.
+#include <cuda_bf16.h>
+
+#include "m3_common.cuh"
+#include "m3_internal.h"
+
+namespace m3 {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+template <typename T>
+__device__ __forceinline__ float4 ld4(const T* p);
+template <>
+__device__ __forceinline__ float4 ld4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <>
+__device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    __nv_bfloat162 lo, hi;
+    memcpy(&lo, &v.x, 4);
+    memcpy(&hi, &v.y, 4);
+    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// Shared-memory layout of one chunk (floats). Slot k = 0..T holds token c0 - 1 + k.
+struct BwdLayout {
+    int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, total;
+};
+__host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P) {
+    BwdLayout l{};
+    int o = 0;
+    const int S = T + 1;
+    l.B = o; o += S * R * N;
+    l.C = o; o += S * R * N;
+    l.X = o; o += S * R * P;
+    l.DY = o; o += S * R * P;
+    l.CS = o; o += S * N;         // [k][i] cos, [k][N/2 + i] sin
+    l.TH = o; o += S * (N / 2);
+    l.DC = o; o += S * R * N;
+    l.DB = o; o += S * R * N;
+    l.DX = o; o += S * R * P;
+    l.DTH = o; o += S * (N / 2);
+    l.SC = o; o += (T + 2) * 4;   // per slot: db (from the step before), dg, dy.y, theta.dPhi
+    l.SCAL = o; o += S * 8;       // per slot: dt, A, lam, alpha, beta, gamma
+    l.total = (o + 3) / 4 * 4;
+    return l;
+}
+
+struct BwdArgs {
+    ScanParams f;
+    const void* dy;
+    const float* dh1;
+    const float* dphi1;
+    const float* dprevB1;
+    const float* dprevx1;
+    float* dx;
+    float* dB;
+    float* dC;
+    float* dtheta;
+    float* ddt;
+    float* dA;
+    float* dlam;
+    float* dBbias;
+    float* dCbias;
+    float* ddtbias;
+    float* dh0;
+    float* dphi0;
+    float* dprevB0;
+    float* dprevx0;
+    float* wdC;    // [b,L,H,R,N] dCbar (forward sweep), then dC after the rotation (reverse)
+    float* wdB;    // [b,L,H,R,N] dB after the rotation
+    float* wphi;   // [units][nchunks][N/2] angle before each chunk
+    float* wF;     // [units] <dL/dh_final, h_final>
+    float* wsc;    // [units][L][4] db, dg, dy.y, theta.dPhi per token
+    float* wprev;  // [units][R][N] gradient of the normalised previous B of the initial state
+    int T;
+    int nchunks;
+};
+
+// Stages the chunk [c0, c0 + Tc) into shared memory: step scalars, angles (continuing from
+// phi_start = the angle before token c0), rotated B (slots 0..Tc) and C (1..Tc), x (0..Tc),
+// dy (1..Tc). Slot 0 is token c0 - 1: the initial state's previous token when c0 = 0.
+template <typename T>
+__device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, int64_t u,
+                            int64_t c0, int Tc, const float* phi_start, bool read_dc) {
+    const ScanParams& p = a.f;
+    const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
+    const int half = N / 2;
+    const int64_t L = p.L, H = p.H;
+    const int64_t bb = u / H, hh = u % H, g = hh / (H / p.G);
+    const int tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
+    const int nwarps = nth >> 5;
+    float* scal = sm + lay.SCAL;
+    float* cs = sm + lay.CS;
+    float* th = sm + lay.TH;
+    const T* thg = static_cast<const T*>(p.theta);
+
+    // scalars and theta
+    const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
+    for (int k = 1 + tid; k <= Tc; k += nth) {
+        const int64_t si = (bb * L + c0 - 1 + k) * H + hh;
+        const float d = step_dt(p.dt[si], dtb, p.flags), A = p.A[si];
+        const float lm = step_lam(p.lam[si], p.flags);
+        const float al = expf(d * A);
+        const bool zoh = p.flags & M3_DISC_ZOH;
+        float* s = scal + 8 * k;
+        s[0] = d; s[1] = A; s[2] = lm; s[3] = al;
+        s[4] = zoh ? 0.f : (1.f - lm) * d * al;
+        s[5] = zoh ? zoh_gamma(d, A) : lm * d;
+    }
+    for (int e = tid; e < Tc * (half / 4); e += nth) {
+        const int k = 1 + e / (half / 4), i4 = (e % (half / 4)) * 4;
+        const float4 v = ld4(thg + ((bb * L + c0 - 1 + k) * H + hh) * half + i4);
+        *reinterpret_cast<float4*>(th + k * half + i4) = v;
+    }
+    // x (slots 0..Tc) and dy (1..Tc), and the forward sweep's dCbar when asked
+    const T* xg = static_cast<const T*>(p.x);
+    const T* dyg = static_cast<const T*>(a.dy);
+    const int RP4 = R * P / 4;
+    for (int e = tid; e < (Tc + 1) * RP4; e += nth) {
+        const int k = e / RP4, o = (e % RP4) * 4;
+        const int64_t t = c0 - 1 + k;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t >= 0) v = ld4(xg + ((bb * L + t) * H + hh) * R * P + o);
+        else if (p.prevx0) v = ld4(static_cast<const T*>(p.prevx0) + u * R * P + o);
+        *reinterpret_cast<float4*>(sm + lay.X + k * R * P + o) = v;
+        if (k > 0)
+            *reinterpret_cast<float4*>(sm + lay.DY + k * R * P + o) =
+                ld4(dyg + ((bb * L + t) * H + hh) * R * P + o);
+    }
+    if (read_dc) {
+        const int RN4 = R * N / 4;
+        for (int e = tid; e < Tc * RN4; e += nth) {
+            const int k = 1 + e / RN4, o = (e % RN4) * 4;
+            *reinterpret_cast<float4*>(sm + lay.DC + k * R * N + o) =
+                *reinterpret_cast<const float4*>(a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o);
+        }
+    }
+    __syncthreads();
+    // angles: one thread per pair walks the chunk
+    for (int i = tid; i < half; i += nth) {
+        float ph = phi_start[i];
+        float s, c;
+        sincosf(ph, &s, &c);
+        cs[i] = c; cs[half + i] = s;
+        for (int k = 1; k <= Tc; ++k) {
+            ph = fmaf(scal[8 * k], th[k * half + i], ph);
+            sincosf(ph, &s, &c);
+            cs[k * N + i] = c; cs[k * N + half + i] = s;
+        }
+    }
+    __syncthreads();
+    // rotated, normalised, biased B (slots 0..Tc) and C (slots 1..Tc): one warp per vector
+    const T* Bg = static_cast<const T*>(p.B);
+    const T* Cg = static_cast<const T*>(p.C);
+    const int nitems = (2 * Tc + 1) * R;
+    for (int it = warp; it < nitems; it += nwarps) {
+        const bool isC = it >= (Tc + 1) * R;
+        const int j = isC ? it - (Tc + 1) * R : it;
+        const int k = isC ? 1 + j / R : j / R, r = j % R;
+        const int64_t t = c0 - 1 + k;
+        const T* src = nullptr;
+        if (t >= 0) src = (isC ? Cg : Bg) + ((bb * L + t) * p.G + g) * R * N + r * N;
+        else if (p.prevB0) src = static_cast<const T*>(p.prevB0) + (u * R + r) * N;
+        const float* bias = isC ? p.Cbias : p.Bbias;
+        if (bias) bias += (hh * R + r) * N;
+        float ss = 0.f;
+        for (int i = lane; i < half; i += 32) {
+            const float v0 = src ? to_f(src[i]) : 0.f, v1 = src ? to_f(src[i + half]) : 0.f;
+            ss = fmaf(v0, v0, fmaf(v1, v1, ss));
+        }
+        ss = warp_sum(ss);
+        const float scale = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
+        float* dst = sm + (isC ? lay.C : lay.B) + (k * R + r) * N;
+        for (int i = lane; i < half; i += 32) {
+            float v0 = src ? to_f(src[i]) : 0.f, v1 = src ? to_f(src[i + half]) : 0.f;
+            v0 = v0 * scale + (bias ? bias[i] : 0.f);
+            v1 = v1 * scale + (bias ? bias[i + half] : 0.f);
+            const float c = cs[k * N + i], s = cs[k * N + half + i];
+            dst[i] = v0 * c + v1 * s;
+            dst[i + half] = v1 * c - v0 * s;
+        }
+    }
+    __syncthreads();
+}
+
+// Sum over the eight lanes of a warp that share the quarter q (lane bits 2..4) of CPQ
+// per-column partials, halving the list at each step; the lane then adds its share into dst
+// (the q-th quarter of a row of P columns in shared memory).
+template <int CPQ>
+__device__ __forceinline__ void add_cols(const float (&v)[CPQ], int lane, float* dst) {
+    constexpr int n1 = CPQ / 2, n2 = n1 / 2;
+    float w1[n1];
+    bool up = lane & 16;
+#pragma unroll
+    for (int j = 0; j < n1; ++j) {
+        const float send = up ? v[j] : v[j + n1];
+        const float keep = up ? v[j + n1] : v[j];
+        w1[j] = keep + __shfl_xor_sync(kFull, send, 16);
+    }
+    int off = up ? n1 : 0;
+    float w2[n2];
+    up = lane & 8;
+#pragma unroll
+    for (int j = 0; j < n2; ++j) {
+        const float send = up ? w1[j] : w1[j + n2];
+        const float keep = up ? w1[j + n2] : w1[j];
+        w2[j] = keep + __shfl_xor_sync(kFull, send, 8);
+    }
+    off += up ? n2 : 0;
+    if constexpr (n2 >= 2) {
+        constexpr int n3 = n2 / 2;
+        up = lane & 4;
+#pragma unroll
+        for (int j = 0; j < n3; ++j) {
+            const float send = up ? w2[j] : w2[j + n3];
+            const float keep = up ? w2[j + n3] : w2[j];
+            atomicAdd(dst + off + (up ? n3 : 0) + j, keep + __shfl_xor_sync(kFull, send, 4));
+        }
+    } else {
+        const float w = w2[0] + __shfl_xor_sync(kFull, w2[0], 4);
+        if (!(lane & 4)) atomicAdd(dst + off, w);
+    }
+}
+
+// Four per-thread partials summed over the warp (halving, then a plain reduction); lanes
+// 0, 8, 16, 24 then hold the sums of v0..v3 in some order, returned with its index.
+__device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v3, int lane,
+                                           int* which) {
+    bool up = lane & 16;
+    const float a0 = (up ? v2 : v0) + __shfl_xor_sync(kFull, up ? v0 : v2, 16);
+    const float a1 = (up ? v3 : v1) + __shfl_xor_sync(kFull, up ? v1 : v3, 16);
+    int w = up ? 2 : 0;
+    up = lane & 8;
+    float b = (up ? a1 : a0) + __shfl_xor_sync(kFull, up ? a0 : a1, 8);
+    w += up ? 1 : 0;
+    b += __shfl_xor_sync(kFull, b, 4);
+    b += __shfl_xor_sync(kFull, b, 2);
+    b += __shfl_xor_sync(kFull, b, 1);
+    *which = w;
+    return b;
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward sweep: h_t token by token; writes dCbar_t = h_t dy_t per token, the angle before
+// every chunk and <dL/dh_final, h_final>.
+template <typename T, int CPQ, int kThreads>
+__global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
+    extern __shared__ float4 smem4[];
+    float* sm = reinterpret_cast<float*>(smem4);
+    const ScanParams& p = a.f;
+    const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
+    const int half = N / 2;
+    const int64_t L = p.L, H = p.H;
+    const int64_t u = blockIdx.x, bb = u / H, hh = u % H;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int i = tid >> 2, q = tid & 3;
+    const BwdLayout lay = bwd_layout(a.T, R, N, P);
+    __shared__ float phi_run[128];
+    __shared__ float red[32];
+
+    float h0[CPQ], h1[CPQ];
+#pragma unroll
+    for (int c = 0; c < CPQ; ++c) {
+        h0[c] = p.h0 ? p.h0[(u * N + i) * P + q * CPQ + c] : 0.f;
+        h1[c] = p.h0 ? p.h0[(u * N + i + half) * P + q * CPQ + c] : 0.f;
+    }
+    for (int e = tid; e < half; e += blockDim.x) phi_run[e] = p.phi0 ? p.phi0[u * half + e] : 0.f;
+    __syncthreads();
+
+    for (int c = 0; c < a.nchunks; ++c) {
+        const int64_t c0 = static_cast<int64_t>(c) * a.T;
+        const int Tc = static_cast<int>(L - c0 < a.T ? L - c0 : a.T);
+        for (int e = tid; e < half; e += blockDim.x)
+            a.wphi[(u * a.nchunks + c) * half + e] = phi_run[e];
+        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_run, false);
+        const float* sB = sm + lay.B;
+        const float* sX = sm + lay.X;
+        const float* sDY = sm + lay.DY;
+        float* sDC = sm + lay.DC;
+        for (int k = 1; k <= Tc; ++k) {
+            const float* s = sm + lay.SCAL + 8 * k;
+            const float al = s[3], be = s[4], ga = s[5];
+#pragma unroll
+            for (int cc = 0; cc < CPQ; ++cc) { h0[cc] *= al; h1[cc] *= al; }
+            for (int r = 0; r < R; ++r) {
+                const float bp0 = be * sB[((k - 1) * R + r) * N + i];
+                const float bp1 = be * sB[((k - 1) * R + r) * N + i + half];
+                const float bc0 = ga * sB[(k * R + r) * N + i];
+                const float bc1 = ga * sB[(k * R + r) * N + i + half];
+                const float* xp = sX + ((k - 1) * R + r) * P + q * CPQ;
+                const float* xc = sX + (k * R + r) * P + q * CPQ;
+#pragma unroll
+                for (int cc = 0; cc < CPQ; cc += 4) {
+                    const float4 vp = *reinterpret_cast<const float4*>(xp + cc);
+                    const float4 vc = *reinterpret_cast<const float4*>(xc + cc);
+                    const float xpv[4] = {vp.x, vp.y, vp.z, vp.w};
+                    const float xcv[4] = {vc.x, vc.y, vc.z, vc.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h0[cc + j] = fmaf(bp0, xpv[j], fmaf(bc0, xcv[j], h0[cc + j]));
+                        h1[cc + j] = fmaf(bp1, xpv[j], fmaf(bc1, xcv[j], h1[cc + j]));
+                    }
+                }
+            }
+            for (int r = 0; r < R; ++r) {
+                const float* dy = sDY + (k * R + r) * P + q * CPQ;
+                float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < CPQ; cc += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(dy + cc);
+                    d0 = fmaf(h0[cc], v.x, fmaf(h0[cc + 1], v.y, fmaf(h0[cc + 2], v.z, fmaf(h0[cc + 3], v.w, d0))));
+                    d1 = fmaf(h1[cc], v.x, fmaf(h1[cc + 1], v.y, fmaf(h1[cc + 2], v.z, fmaf(h1[cc + 3], v.w, d1))));
+                }
+                d0 += __shfl_xor_sync(kFull, d0, 1);
+                d1 += __shfl_xor_sync(kFull, d1, 1);
+                d0 += __shfl_xor_sync(kFull, d0, 2);
+                d1 += __shfl_xor_sync(kFull, d1, 2);
+                if (q == 0) sDC[(k * R + r) * N + i] = d0;
+                if (q == 1) sDC[(k * R + r) * N + i + half] = d1;
+            }
+        }
+        __syncthreads();
+        // the chunk's angle end, and its dCbar rows out
+        for (int e = tid; e < half; e += blockDim.x) {
+            float ph = phi_run[e];
+            for (int k = 1; k <= Tc; ++k) ph = fmaf(sm[lay.SCAL + 8 * k], sm[lay.TH + k * half + e], ph);
+            phi_run[e] = ph;
+        }
+        const int RN4 = R * N / 4;
+        for (int e = tid; e < Tc * RN4; e += blockDim.x) {
+            const int k = 1 + e / RN4, o = (e % RN4) * 4;
+            *reinterpret_cast<float4*>(a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o) =
+                *reinterpret_cast<const float4*>(sDC + k * R * N + o);
+        }
+        __syncthreads();
+    }
+    // <dL/dh_final, h_final>
+    float f = 0.f;
+    if (a.dh1) {
+#pragma unroll
+        for (int c = 0; c < CPQ; ++c) {
+            f = fmaf(a.dh1[(u * N + i) * P + q * CPQ + c], h0[c], f);
+            f = fmaf(a.dh1[(u * N + i + half) * P + q * CPQ + c], h1[c], f);
+        }
+    }
+    f = warp_sum(f);
+    if (lane == 0) red[tid >> 5] = f;
+    __syncthreads();
+    if (tid == 0) {
+        float s = 0.f;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += red[w];
+        a.wF[u] = s;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Reverse sweep: G_t from the end; dx, dtheta, the rotated-back dB and dC per head, the
+// per-token partial sums for the scalars, the bias sums and the initial state's gradients.
+template <typename T, int CPQ, int kThreads>
+__global__ void __launch_bounds__(kThreads) bwd_rev_kernel(const BwdArgs a) {
+    extern __shared__ float4 smem4[];
+    float* sm = reinterpret_cast<float*>(smem4);
+    const ScanParams& p = a.f;
+    const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
+    const int half = N / 2;
+    const int64_t L = p.L, H = p.H;
+    const int64_t u = blockIdx.x, bb = u / H, hh = u % H;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int i = tid >> 2, q = tid & 3;
+    const BwdLayout lay = bwd_layout(a.T, R, N, P);
+    __shared__ float phi_start[128];
+    __shared__ float pend[4];
+
+    float G0[CPQ], G1[CPQ];
+#pragma unroll
+    for (int c = 0; c < CPQ; ++c) {
+        G0[c] = a.dh1 ? a.dh1[(u * N + i) * P + q * CPQ + c] : 0.f;
+        G1[c] = a.dh1 ? a.dh1[(u * N + i + half) * P + q * CPQ + c] : 0.f;
+    }
+    float dphi = a.dphi1 ? a.dphi1[u * half + i] : 0.f;
+    float a_n = 1.f, b_n = 0.f;         // alpha and beta of the token after the current one
+    float accB[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, accC[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+
+    float* sB = sm + lay.B;
+    float* sC = sm + lay.C;
+    float* sX = sm + lay.X;
+    float* sDY = sm + lay.DY;
+    float* sCS = sm + lay.CS;
+    float* sTH = sm + lay.TH;
+    float* sDC = sm + lay.DC;
+    float* sDB = sm + lay.DB;
+    float* sDX = sm + lay.DX;
+    float* sDTH = sm + lay.DTH;
+    float* sSC = sm + lay.SC;
+
+    for (int c = a.nchunks - 1; c >= 0; --c) {
+        const int64_t c0 = static_cast<int64_t>(c) * a.T;
+        const int Tc = static_cast<int>(L - c0 < a.T ? L - c0 : a.T);
+        for (int e = tid; e < half; e += blockDim.x)
+            phi_start[e] = a.wphi[(u * a.nchunks + c) * half + e];
+        for (int e = tid; e < (Tc + 1) * R * P; e += blockDim.x) sDX[e] = 0.f;
+        for (int e = tid; e < (a.T + 2) * 4; e += blockDim.x) sSC[e] = 0.f;
+        __syncthreads();
+        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_start, true);
+
+        for (int k = Tc; k >= 1; --k) {
+            const float* s = sm + lay.SCAL + 8 * k;
+            const float ga = s[5];
+            float go0[CPQ], go1[CPQ];
+#pragma unroll
+            for (int cc = 0; cc < CPQ; ++cc) {
+                go0[cc] = G0[cc]; go1[cc] = G1[cc];
+                G0[cc] *= a_n; G1[cc] *= a_n;
+            }
+            for (int r = 0; r < R; ++r) {
+                const float cb0 = sC[(k * R + r) * N + i], cb1 = sC[(k * R + r) * N + i + half];
+                const float* dy = sDY + (k * R + r) * P + q * CPQ;
+#pragma unroll
+                for (int cc = 0; cc < CPQ; cc += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(dy + cc);
+                    const float dv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        G0[cc + j] = fmaf(cb0, dv[j], G0[cc + j]);
+                        G1[cc + j] = fmaf(cb1, dv[j], G1[cc + j]);
+                    }
+                }
+            }
+            float sg = 0.f, sbn = 0.f, syy = 0.f, dl = 0.f;
+            for (int r = 0; r < R; ++r) {
+                const float bb0 = sB[(k * R + r) * N + i], bb1 = sB[(k * R + r) * N + i + half];
+                const float* x = sX + (k * R + r) * P + q * CPQ;
+                float gA0 = 0.f, gA1 = 0.f, gB0 = 0.f, gB1 = 0.f;
+                float v[CPQ];
+#pragma unroll
+                for (int cc = 0; cc < CPQ; cc += 4) {
+                    const float4 xv4 = *reinterpret_cast<const float4*>(x + cc);
+                    const float xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = cc + j;
+                        gA0 = fmaf(go0[e], xv[j], gA0); gA1 = fmaf(go1[e], xv[j], gA1);
+                        gB0 = fmaf(G0[e], xv[j], gB0); gB1 = fmaf(G1[e], xv[j], gB1);
+                        v[e] = ga * fmaf(bb0, G0[e], bb1 * G1[e]) + b_n * fmaf(bb0, go0[e], bb1 * go1[e]);
+                    }
+                }
+                add_cols<CPQ>(v, lane, sDX + (k * R + r) * P + q * CPQ);
+                sg = fmaf(bb0, gB0, fmaf(bb1, gB1, sg));
+                sbn = fmaf(bb0, gA0, fmaf(bb1, gA1, sbn));
+                float db0 = fmaf(ga, gB0, b_n * gA0), db1 = fmaf(ga, gB1, b_n * gA1);
+                db0 += __shfl_xor_sync(kFull, db0, 1);
+                db1 += __shfl_xor_sync(kFull, db1, 1);
+                db0 += __shfl_xor_sync(kFull, db0, 2);
+                db1 += __shfl_xor_sync(kFull, db1, 2);
+                if (q == (r & 3)) {
+                    const float cb0 = sC[(k * R + r) * N + i], cb1 = sC[(k * R + r) * N + i + half];
+                    float* dcp = sDC + (k * R + r) * N;
+                    const float dc0 = dcp[i], dc1 = dcp[i + half];
+                    const float co = sCS[k * N + i], si = sCS[k * N + half + i];
+                    dl += db0 * bb1 - db1 * bb0 + dc0 * cb1 - dc1 * cb0;
+                    syy = fmaf(cb0, dc0, fmaf(cb1, dc1, syy));
+                    const float nB0 = db0 * co - db1 * si, nB1 = db0 * si + db1 * co;
+                    const float nC0 = dc0 * co - dc1 * si, nC1 = dc0 * si + dc1 * co;
+                    sDB[(k * R + r) * N + i] = nB0;
+                    sDB[(k * R + r) * N + i + half] = nB1;
+                    dcp[i] = nC0;
+                    dcp[i + half] = nC1;
+                    accB[r >> 2][0] += nB0; accB[r >> 2][1] += nB1;
+                    accC[r >> 2][0] += nC0; accC[r >> 2][1] += nC1;
+                }
+            }
+            dl += __shfl_xor_sync(kFull, dl, 1);
+            dl += __shfl_xor_sync(kFull, dl, 2);
+            dphi += dl;
+            float thd = 0.f;
+            if (q == 0) {
+                sDTH[k * half + i] = s[0] * dphi;
+                thd = sTH[k * half + i] * dphi;
+            }
+            int which;
+            const float w = warp_sum4(sbn, sg, syy, thd, lane, &which);
+            if ((lane & 7) == 0) {
+                // which: 0 = db of the next token, 1 = dg, 2 = dy.y, 3 = theta.dPhi
+                if (which == 0) atomicAdd(sSC + (k + 1) * 4 + 0, w);
+                else atomicAdd(sSC + k * 4 + which, w);
+            }
+            a_n = s[3];
+            b_n = s[4];
+        }
+
+        if (c == 0) {
+            // token -1: the initial state's h, previous token and angle
+            if (a.dh0) {
+#pragma unroll
+                for (int cc = 0; cc < CPQ; ++cc) {
+                    a.dh0[(u * N + i) * P + q * CPQ + cc] = a_n * G0[cc];
+                    a.dh0[(u * N + i + half) * P + q * CPQ + cc] = a_n * G1[cc];
+                }
+            }
+            float sbn = 0.f, dl = 0.f;
+            for (int r = 0; r < R; ++r) {
+                const float bb0 = sB[r * N + i], bb1 = sB[r * N + i + half];
+                const float* x = sX + r * P + q * CPQ;
+                float gA0 = 0.f, gA1 = 0.f;
+                float v[CPQ];
+#pragma unroll
+                for (int e = 0; e < CPQ; ++e) {
+                    gA0 = fmaf(G0[e], x[e], gA0);
+                    gA1 = fmaf(G1[e], x[e], gA1);
+                    v[e] = b_n * fmaf(bb0, G0[e], bb1 * G1[e]);
+                }
+                add_cols<CPQ>(v, lane, sDX + r * P + q * CPQ);
+                sbn = fmaf(bb0, gA0, fmaf(bb1, gA1, sbn));
+                float db0 = b_n * gA0, db1 = b_n * gA1;
+                db0 += __shfl_xor_sync(kFull, db0, 1);
+                db1 += __shfl_xor_sync(kFull, db1, 1);
+                db0 += __shfl_xor_sync(kFull, db0, 2);
+                db1 += __shfl_xor_sync(kFull, db1, 2);
+                if (q == (r & 3)) {
+                    const float co = sCS[i], si = sCS[half + i];
+                    dl += db0 * bb1 - db1 * bb0;
+                    const float nB0 = db0 * co - db1 * si, nB1 = db0 * si + db1 * co;
+                    sDB[r * N + i] = nB0;
+                    sDB[r * N + i + half] = nB1;
+                    accB[r >> 2][0] += nB0; accB[r >> 2][1] += nB1;
+                }
+            }
+            dl += __shfl_xor_sync(kFull, dl, 1);
+            dl += __shfl_xor_sync(kFull, dl, 2);
+            if (q == 0 && a.dphi0) a.dphi0[u * half + i] = dphi + dl;
+            int which;
+            const float w = warp_sum4(sbn, 0.f, 0.f, 0.f, lane, &which);
+            if ((lane & 7) == 0 && which == 0) atomicAdd(sSC + 4, w);
+        }
+        __syncthreads();
+
+        // chunk out: dx, dtheta, dB and dC per head, the scalar partials
+        const int RP4 = R * P / 4;
+        for (int e = tid; e < Tc * RP4; e += blockDim.x) {
+            const int k = 1 + e / RP4, o = (e % RP4) * 4;
+            const int64_t t = c0 - 1 + k;
+            float4 v = *reinterpret_cast<const float4*>(sDX + k * R * P + o);
+            if (t == L - 1 && a.dprevx1) {
+                const float4 w = *reinterpret_cast<const float4*>(a.dprevx1 + u * R * P + o);
+                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+            }
+            *reinterpret_cast<float4*>(a.dx + ((bb * L + t) * H + hh) * R * P + o) = v;
+        }
+        const int h4 = half / 4;
+        for (int e = tid; e < Tc * h4; e += blockDim.x) {
+            const int k = 1 + e / h4, o = (e % h4) * 4;
+            *reinterpret_cast<float4*>(a.dtheta + ((bb * L + c0 - 1 + k) * H + hh) * half + o) =
+                *reinterpret_cast<const float4*>(sDTH + k * half + o);
+        }
+        const int RN4 = R * N / 4;
+        for (int e = tid; e < Tc * RN4; e += blockDim.x) {
+            const int k = 1 + e / RN4, o = (e % RN4) * 4;
+            const int64_t off = ((bb * L + c0 - 1 + k) * H + hh) * R * N + o;
+            *reinterpret_cast<float4*>(a.wdB + off) = *reinterpret_cast<const float4*>(sDB + k * R * N + o);
+            *reinterpret_cast<float4*>(a.wdC + off) = *reinterpret_cast<const float4*>(sDC + k * R * N + o);
+        }
+        float* wsc = a.wsc + u * L * 4;
+        for (int e = tid; e < (Tc - 1) * 4; e += blockDim.x) {
+            const int k = 2 + e / 4, j = e % 4;
+            wsc[(c0 - 1 + k) * 4 + j] = sSC[k * 4 + j];
+        }
+        if (tid < 4) {
+            // the token after this chunk got its db from this chunk's last step
+            if (c0 + Tc < L) wsc[(c0 + Tc) * 4 + tid] = pend[tid] + (tid == 0 ? sSC[(Tc + 1) * 4] : 0.f);
+            pend[tid] = sSC[4 + tid];
+            if (c == 0) wsc[tid] = sSC[4 + tid];
+        }
+        if (c == 0) {
+            for (int e = tid; e < RP4; e += blockDim.x)
+                if (a.dprevx0)
+                    *reinterpret_cast<float4*>(a.dprevx0 + u * R * P + e * 4) =
+                        *reinterpret_cast<const float4*>(sDX + e * 4);
+            for (int e = tid; e < RN4; e += blockDim.x)
+                *reinterpret_cast<float4*>(a.wprev + u * R * N + e * 4) =
+                    *reinterpret_cast<const float4*>(sDB + e * 4);
+        }
+        __syncthreads();
+    }
+    // the biases: each unit adds its sums over the sequence
+    for (int rr = 0; rr < 2; ++rr) {
+        const int r = q + 4 * rr;
+        if (r >= R) break;
+        if (a.dBbias) {
+            atomicAdd(a.dBbias + (hh * R + r) * N + i, accB[rr][0]);
+            atomicAdd(a.dBbias + (hh * R + r) * N + i + half, accB[rr][1]);
+        }
+        if (a.dCbias) {
+            atomicAdd(a.dCbias + (hh * R + r) * N + i, accC[rr][0]);
+            atomicAdd(a.dCbias + (hh * R + r) * N + i + half, accC[rr][1]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Step scalars: the suffix sum D_t and the chain rule to dt, A, lam (and the raw
+// projections). One CTA per unit walks the sequence from the end in tiles.
+constexpr int kScalThreads = 256, kScalPer = 4;
+
+__global__ void __launch_bounds__(kScalThreads) bwd_scalar_kernel(const BwdArgs a) {
+    const ScanParams& p = a.f;
+    const int64_t L = p.L, H = p.H;
+    const int64_t u = blockIdx.x, bb = u / H, hh = u % H;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ float wtot[kScalThreads / 32];
+    __shared__ float red[kScalThreads / 32];
+    const float* wsc = a.wsc + u * L * 4;
+    const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
+    const bool zoh = p.flags & M3_DISC_ZOH;
+    float carry = a.wF[u];
+    float bias_sum = 0.f;
+    constexpr int kTile = kScalThreads * kScalPer;
+    for (int64_t t_end = L; t_end > 0; t_end -= kTile) {
+        const int64_t t0 = t_end - kTile;   // may be negative: those tokens are skipped
+        const int blk = kScalThreads - 1 - tid;   // thread 0 takes the last block of the tile
+        float e[kScalPer];
+        float tot = 0.f;
+#pragma unroll
+        for (int j = 0; j < kScalPer; ++j) {
+            const int64_t t = t0 + blk * kScalPer + j;
+            e[j] = 0.f;
+            if (t >= 0) {
+                const int64_t si = (bb * L + t) * H + hh;
+                const float d = step_dt(p.dt[si], dtb, p.flags), A = p.A[si];
+                const float lm = step_lam(p.lam[si], p.flags);
+                const float al = expf(d * A);
+                const float be = zoh ? 0.f : (1.f - lm) * d * al;
+                const float ga = zoh ? zoh_gamma(d, A) : lm * d;
+                e[j] = wsc[t * 4 + 2] - be * wsc[t * 4 + 0] - ga * wsc[t * 4 + 1];
+            }
+            tot += e[j];
+        }
+        // suffix sums over blocks: an inclusive prefix over tid (blocks in reverse order)
+        float incl = warp_inclusive_scan(tot);
+        if (lane == 31) wtot[warp] = incl;
+        __syncthreads();
+        float before = 0.f;
+        for (int w = 0; w < warp; ++w) before += wtot[w];
+        float tile_sum = 0.f;
+        for (int w = 0; w < kScalThreads / 32; ++w) tile_sum += wtot[w];
+        float D = carry + before + incl - tot;   // everything after this block
+        for (int j = kScalPer - 1; j >= 0; --j) {
+            const int64_t t = t0 + blk * kScalPer + j;
+            D += e[j];
+            if (t < 0) continue;
+            const int64_t si = (bb * L + t) * H + hh;
+            const float draw = p.dt[si], A = p.A[si], lraw = p.lam[si];
+            const float d = step_dt(draw, dtb, p.flags), lm = step_lam(lraw, p.flags);
+            const float al = expf(d * A);
+            const float db = wsc[t * 4 + 0], dg = wsc[t * 4 + 1], thd = wsc[t * 4 + 3];
+            float gdt, gA, glam;
+            if (zoh) {
+                // gamma = (e^{dA} - 1) / A: d gamma / d dt = alpha, d gamma / d A = (dt alpha - gamma) / A,
+                // by its series dt^2 (1/2 + x/3 + x^2/8 + x^3/30 + x^4/144) for small x = dt A
+                const float x = d * A;
+                const float dgdA = fabsf(x) < 0.05f
+                    ? d * d * (0.5f + x * (1.f / 3.f + x * (0.125f + x * (1.f / 30.f + x * (1.f / 144.f)))))
+                    : (d * al - zoh_gamma(d, A)) / A;
+                gdt = D * A + dg * al + thd;
+                gA = D * d + dg * dgdA;
+                glam = 0.f;
+            } else {
+                gdt = D * A + db * (1.f - lm) * al * fmaf(d, A, 1.f) + dg * lm + thd;
+                gA = D * d + db * (1.f - lm) * d * d * al;
+                glam = (dg - db * al) * d;
+            }
+            if (p.flags & M3_DT_SOFTPLUS) {
+                const float v = draw + dtb;
+                gdt *= __frcp_rn(1.f + __expf(-v));   // softplus' = sigmoid
+                bias_sum += gdt;
+            }
+            if (p.flags & M3_LAM_SIGMOID) glam *= lm * (1.f - lm);
+            a.ddt[si] = gdt;
+            a.dA[si] = gA;
+            a.dlam[si] = glam;
+        }
+        carry += tile_sum;
+        __syncthreads();
+    }
+    if (a.ddtbias && (p.flags & M3_DT_SOFTPLUS)) {
+        bias_sum = warp_sum(bias_sum);
+        if (lane == 0) red[warp] = bias_sum;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.f;
+            for (int w = 0; w < kScalThreads / 32; ++w) s += red[w];
+            atomicAdd(a.ddtbias + hh, s);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// RMS-norm backward and the sum over the heads of a group: one warp per (token, group, r,
+// B or C), plus one per (unit, r) for the initial state's previous B (per head).
+__global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16) {
+    const ScanParams& p = a.f;
+    const int64_t L = p.L, H = p.H, Gn = p.G, N = p.N, R = p.R;
+    const int64_t hpg = H / Gn;
+    const int lane = threadIdx.x & 31;
+    const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t ntok = p.b * L * Gn * R * 2, nprev = p.b * H * R;
+    if (item >= ntok + nprev) return;
+    auto raw = [&](const void* base, int64_t off) {
+        return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(base)[off])
+                    : static_cast<const float*>(base)[off];
+    };
+    const void* src;
+    int64_t src_off;
+    float* dst;
+    const float* extra = nullptr;   // final state's prev_B gradient, summed over the group
+    int64_t h_first = 0, nh = 0, dn_stride = 0;
+    const float* dn_base;
+    if (item < ntok) {
+        const int isC = static_cast<int>(item & 1);
+        const int64_t rest = item >> 1;
+        const int64_t r = rest % R, g = (rest / R) % Gn, tok = rest / (R * Gn);   // tok = b*L + t
+        const int64_t bb = tok / L, t = tok % L;
+        src = isC ? p.C : p.B;
+        src_off = ((tok * Gn + g) * R + r) * N;
+        dst = (isC ? a.dC : a.dB) + src_off;
+        h_first = g * hpg;
+        nh = hpg;
+        dn_base = (isC ? a.wdC : a.wdB) + ((tok * H + h_first) * R + r) * N;
+        dn_stride = R * N;
+        if (!isC && t == L - 1 && a.dprevB1) extra = a.dprevB1 + ((bb * H + h_first) * R + r) * N;
+    } else {
+        const int64_t j = item - ntok;   // (unit, r)
+        if (!a.dprevB0) return;
+        src = p.prevB0;
+        src_off = j * N;
+        dst = a.dprevB0 + j * N;
+        nh = 1;
+        dn_base = a.wprev + j * N;
+        dn_stride = 0;
+    }
+    float ss = 0.f, dot = 0.f;
+    for (int64_t n = lane; n < N; n += 32) {
+        float dn = 0.f;
+        for (int64_t h = 0; h < nh; ++h) dn += dn_base[h * dn_stride + n];
+        const float v = src ? raw(src, src_off + n) : 0.f;
+        ss = fmaf(v, v, ss);
+        dot = fmaf(v, dn, dot);
+    }
+    ss = warp_sum(ss);
+    dot = warp_sum(dot);
+    const float s = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
+    const float k = p.bc_norm ? s * s * s / static_cast<float>(N) * dot : 0.f;
+    for (int64_t n = lane; n < N; n += 32) {
+        float dn = 0.f;
+        for (int64_t h = 0; h < nh; ++h) dn += dn_base[h * dn_stride + n];
+        const float v = src ? raw(src, src_off + n) : 0.f;
+        float o = s * dn - k * v;
+        if (extra)
+            for (int64_t h = 0; h < nh; ++h) o += extra[h * R * N + n];
+        dst[n] = o;
+    }
+}
+
+template <typename T, int CPQ, int kThreads>
+cudaError_t launch_sweeps(const BwdArgs& a, size_t smem, cudaStream_t s) {
+    const int units = static_cast<int>(a.f.b * a.f.H);
+    const int threads = static_cast<int>(2 * a.f.N);
+    auto kf = bwd_fwd_kernel<T, CPQ, kThreads>;
+    auto kr = bwd_rev_kernel<T, CPQ, kThreads>;
+    cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kf<<<units, threads, smem, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kr<<<units, threads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T, int kThreads>
+cudaError_t launch_sweeps_p(const BwdArgs& a, size_t smem, cudaStream_t s) {
+    switch (a.f.P) {
+        case 16: return launch_sweeps<T, 4, kThreads>(a, smem, s);
+        case 32: return launch_sweeps<T, 8, kThreads>(a, smem, s);
+        case 64: return launch_sweeps<T, 16, kThreads>(a, smem, s);
+        default: return launch_sweeps<T, 32, kThreads>(a, smem, s);
+    }
+}
+
+}  // namespace
+
+int bwd_chunk_tokens(int64_t R) { return static_cast<int>(R >= 16 ? 1 : 16 / R); }
+
+size_t scan_bwd_workspace_floats(int64_t b, int64_t L, int64_t H, int64_t N, int64_t R) {
+    const int64_t T = bwd_chunk_tokens(R), nch = (L + T - 1) / T, units = b * H;
+    auto r64 = [](int64_t v) { return (v + 63) / 64 * 64; };   // 256-byte regions
+    return static_cast<size_t>(2 * r64(b * L * H * R * N) + r64(units * nch * (N / 2)) +
+                               r64(units) + r64(units * L * 4) + r64(units * R * N));
+}
+
+cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, float* ws,
+                            cudaStream_t s) {
+    BwdArgs a{};
+    a.f = f;
+    a.dy = g.dy;
+    a.dh1 = g.dh1; a.dphi1 = g.dphi1; a.dprevB1 = g.dprevB1; a.dprevx1 = g.dprevx1;
+    a.dx = g.dx; a.dB = g.dB; a.dC = g.dC; a.dtheta = g.dtheta;
+    a.ddt = g.ddt; a.dA = g.dA; a.dlam = g.dlam;
+    a.dBbias = g.dBbias; a.dCbias = g.dCbias; a.ddtbias = g.ddtbias;
+    a.dh0 = g.dh0; a.dphi0 = g.dphi0; a.dprevB0 = g.dprevB0; a.dprevx0 = g.dprevx0;
+    a.T = bwd_chunk_tokens(f.R);
+    a.nchunks = static_cast<int>((f.L + a.T - 1) / a.T);
+    const int64_t units = f.b * f.H, nch = a.nchunks;
+    auto r64 = [](int64_t v) { return (v + 63) / 64 * 64; };
+    float* o = ws;
+    a.wdC = o; o += r64(f.b * f.L * f.H * f.R * f.N);
+    a.wdB = o; o += r64(f.b * f.L * f.H * f.R * f.N);
+    a.wphi = o; o += r64(units * nch * (f.N / 2));
+    a.wF = o; o += r64(units);
+    a.wsc = o; o += r64(units * f.L * 4);
+    a.wprev = o;
+
+    cudaError_t e;
+    if (a.dBbias && (e = cudaMemsetAsync(a.dBbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
+    if (a.dCbias && (e = cudaMemsetAsync(a.dCbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
+    if (a.ddtbias && (e = cudaMemsetAsync(a.ddtbias, 0, sizeof(float) * f.H, s)) != cudaSuccess) return e;
+    const BwdLayout lay = bwd_layout(a.T, static_cast<int>(f.R), static_cast<int>(f.N),
+                                     static_cast<int>(f.P));
+    const size_t smem = sizeof(float) * lay.total;
+    if (f.N <= 128)
+        e = bf16 ? launch_sweeps_p<__nv_bfloat16, 256>(a, smem, s)
+                 : launch_sweeps_p<float, 256>(a, smem, s);
+    else
+        e = bf16 ? launch_sweeps_p<__nv_bfloat16, 512>(a, smem, s)
+                 : launch_sweeps_p<float, 512>(a, smem, s);
+    if (e != cudaSuccess) return e;
+    bwd_scalar_kernel<<<static_cast<unsigned>(units), kScalThreads, 0, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t items = f.b * f.L * f.G * f.R * 2 + units * f.R;
+    const int64_t blocks = (items * 32 + 255) / 256;
+    bwd_norm_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, bf16 ? 1 : 0);
+    return cudaGetLastError();
+}
+
+size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t R) {
+    const BwdLayout lay = bwd_layout(bwd_chunk_tokens(R), static_cast<int>(R),
+                                     static_cast<int>(N), static_cast<int>(P));
+    return sizeof(float) * lay.total;
+}
+
+}  // namespace m3

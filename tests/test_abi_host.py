@@ -114,6 +114,35 @@ def test_scan_rejects_bad_arguments_without_launching(lib):
         bd.M3_ERR_INVALID_ARG
 
 
+def test_backward_workspace_and_argument_checks(lib):
+    """m3_scan_bwd_workspace_bytes follows its documented size; m3_scan_bwd rejects bad
+    arguments before anything is launched."""
+    d = dims(batch=2, seqlen=100, nheads=4, dstate=128, rank=1)
+    T = 16
+    r64 = lambda v: (v + 63) // 64 * 64
+    units, nch = 2 * 4, (100 + T - 1) // T
+    want = 4 * (2 * r64(2 * 100 * 4 * 128) + r64(units * nch * 64) + r64(units)
+                + r64(units * 100 * 4) + r64(units * 128))
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d)) == want
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
+    assert ctypes.sizeof(bd.Grads) == 10 * 8
+    ins = fake_inputs()
+    g = bd.Grads(*([FAKE] * 10))
+    ws = ctypes.c_void_p(0x100000)
+    call = lambda dd=d, ii=ins, dy=FAKE, gg=g, w=ws, nb=1 << 40: lib.m3_scan_bwd(
+        ctypes.byref(dd), ctypes.byref(ii), None, dy, None,
+        ctypes.byref(gg) if gg is not None else None, None, w, nb, None)
+    assert call(gg=None) == bd.M3_ERR_INVALID_ARG
+    assert call(dy=None) == bd.M3_ERR_INVALID_ARG
+    assert b"dy" in lib.m3_last_error()
+    assert call(gg=bd.Grads(FAKE, FAKE, None, *([FAKE] * 7))) == bd.M3_ERR_INVALID_ARG
+    assert b"dC" in lib.m3_last_error()
+    assert call(gg=bd.Grads(*([FAKE] * 7), FAKE + 4, FAKE, FAKE)) == bd.M3_ERR_INVALID_ARG
+    assert call(w=None) == bd.M3_ERR_INVALID_ARG
+    assert call(nb=16) == bd.M3_ERR_INVALID_ARG
+    assert call(dd=dims(headdim=48)) == bd.M3_ERR_UNSUPPORTED
+
+
 def test_decode_rejects_bad_arguments_without_launching(lib):
     d = dims(seqlen=1)
     ins = fake_inputs()
