@@ -291,6 +291,14 @@ def run_ours(args):
         decode["R4_proj"] = bench_decode(m3, dev, 4, args.decode_steps, hbm, world, dist,
                                          proj=True)
 
+    # ---- the backward pass of the scan (training side), SISO and MIMO R4 workloads ----
+    backward = {}
+    if not args.no_decode:
+        backward["siso_b4_L2048"] = bench_backward(m3, dev, 1, hbm, world, dist,
+                                                   rank_seed(rank, 11))
+        backward["mimo_r4_b4_L2048"] = bench_backward(m3, dev, 2, hbm, world, dist,
+                                                      rank_seed(rank, 12))
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -311,6 +319,7 @@ def run_ours(args):
         "decode": decode,
         "fused_scalar_prologue": prologue,
         "other_prefill": others,
+        "backward": backward,
     }
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
@@ -318,6 +327,60 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def bwd_bytes(pr) -> int:
+    """Algorithmic HBM bytes of one backward pass: every forward input, dy and the initial
+    state read once; every gradient (fp32) written once."""
+    import torch
+    d = pr.dims
+    es = 2 if d.dtype == torch.bfloat16 else 4
+    b, L, H, G, P, N, R = d.batch, d.seqlen, d.nheads, d.ngroups, d.headdim, d.dstate, d.rank
+    units = b * H
+    reads = (es * (2 * b * L * H * R * P + 2 * b * L * G * R * N + b * L * H * N // 2)
+             + 12 * b * L * H + 8 * H * R * N)
+    writes = 4 * (b * L * H * R * P + 2 * b * L * G * R * N + b * L * H * N // 2 + 3 * b * L * H
+                  + 2 * H * R * N)
+    if pr.state is not None:
+        reads += units * (4 * N * P + 4 * N // 2 + es * R * (N + P))
+        writes += units * 4 * (N * P + N // 2 + R * (N + P))
+    return reads + writes
+
+
+def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5):
+    """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1)."""
+    import torch
+    from state_space_sequence_mamba_b200.inputs import make_config
+    pr = make_config(cfg, device=dev, seed=seed, with_state=True)
+    d = pr.dims
+    g = torch.Generator(device=dev).manual_seed(seed + 1)
+    dy = torch.randn(pr.x.shape, generator=g, device=dev).to(d.dtype)
+    init = m3.State.from_dict(pr.state)
+    ws = torch.empty(m3.scan_bwd_workspace_bytes(m3.make_dims(pr.x, pr.B, 1, True, 1e-6)),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return m3.scan_bwd(**pr.tensors(), dy=dy, init=init, bc_norm=True, workspace=ws,
+                           stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev) / reps
+    byts = bwd_bytes(pr)
+    out = {"ms_per_backward": ms, "tokens_per_s": d.batch * d.seqlen * world / (ms / 1e3),
+           "bytes": byts, "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
+           "kernels_per_call": 4, "workspace_bytes": ws.numel()}
+    del pr, dy, init, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_decode(m3, dev, R, steps, hbm, world, dist, raw=False, proj=False):

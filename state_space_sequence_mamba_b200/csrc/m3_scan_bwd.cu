@@ -53,11 +53,29 @@ __device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
     return make_float4(a.x, a.y, b.x, b.y);
 }
 
-// Shared-memory layout of one chunk (floats). Slot k = 0..T holds token c0 - 1 + k.
+// Asynchronous 16-byte and 4-byte global -> shared copies (sm_80+ cp.async); a 16-byte copy
+// with valid = false writes zeros and reads nothing.
+__device__ __forceinline__ void cp16(void* dst, const void* src, bool valid) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src),
+                 "r"(valid ? 16 : 0));
+}
+__device__ __forceinline__ void cp4(void* dst, const void* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src));
+}
+__device__ __forceinline__ void cp_wait_all() {
+    asm volatile("cp.async.commit_group;\n" ::);
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Shared-memory layout of one chunk (floats). Slot k = 0..T holds token c0 - 1 + k. RAW holds
+// the chunk's inputs as loaded (element size es): B rows (slots 0..T), C, dy and theta rows
+// (slots 1..T at k - 1), x rows (0..T) and the raw dt, A, lam (slots 1..T at k - 1).
 struct BwdLayout {
-    int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, total;
+    int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, BIAS, RAW, total;
 };
-__host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P) {
+__host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P, int es) {
     BwdLayout l{};
     int o = 0;
     const int S = T + 1;
@@ -73,6 +91,11 @@ __host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P) {
     l.DTH = o; o += S * (N / 2);
     l.SC = o; o += (T + 2) * 4;   // per slot: db (from the step before), dg, dy.y, theta.dPhi
     l.SCAL = o; o += S * 8;       // per slot: dt, A, lam, alpha, beta, gamma
+    l.BIAS = o; o += 2 * R * N;   // this head's B and C bias (zeros when absent)
+    o = (o + 3) / 4 * 4;
+    l.RAW = o;
+    o += (S * R * N * es + T * R * N * es + S * R * P * es + T * R * P * es +
+          T * (N / 2) * es + T * 12 + 15) / 16 * 4;
     l.total = (o + 3) / 4 * 4;
     return l;
 }
@@ -109,29 +132,95 @@ struct BwdArgs {
 };
 
 // Stages the chunk [c0, c0 + Tc) into shared memory: step scalars, angles (continuing from
-// phi_start = the angle before token c0), rotated B (slots 0..Tc) and C (1..Tc), x (0..Tc),
-// dy (1..Tc). Slot 0 is token c0 - 1: the initial state's previous token when c0 = 0.
+// phi_start = the angle before token c0; the angle after the chunk goes to phi_end when it is
+// set), rotated B (slots 0..Tc) and C (1..Tc), x (0..Tc), dy (1..Tc), and the forward sweep's
+// dCbar rows when read_dc. Slot 0 is token c0 - 1: the initial state's previous token when
+// c0 = 0. Every global load of the chunk is in flight at once (cp.async); the rest works on
+// shared memory.
 template <typename T>
 __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, int64_t u,
-                            int64_t c0, int Tc, const float* phi_start, bool read_dc) {
+                            int64_t c0, int Tc, const float* phi_start, float* phi_end,
+                            bool read_dc) {
+    constexpr int es = sizeof(T);
     const ScanParams& p = a.f;
     const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
-    const int half = N / 2;
+    const int half = N / 2, Tm = a.T;
     const int64_t L = p.L, H = p.H;
     const int64_t bb = u / H, hh = u % H, g = hh / (H / p.G);
     const int tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
     const int nwarps = nth >> 5;
     float* scal = sm + lay.SCAL;
     float* cs = sm + lay.CS;
-    float* th = sm + lay.TH;
-    const T* thg = static_cast<const T*>(p.theta);
+    const int rowB = R * N * es, rowX = R * P * es, rowT = half * es;   // bytes
+    char* rB = reinterpret_cast<char*>(sm + lay.RAW);
+    char* rC = rB + (Tm + 1) * rowB;
+    char* rX = rC + Tm * rowB;
+    char* rDY = rX + (Tm + 1) * rowX;
+    char* rTH = rDY + Tm * rowX;
+    float* rS = reinterpret_cast<float*>(rTH + Tm * rowT);
 
-    // scalars and theta
+    // ---- one batch of asynchronous loads ----
+    const char* Bg = static_cast<const char*>(p.B);
+    const char* Cg = static_cast<const char*>(p.C);
+    const char* xg = static_cast<const char*>(p.x);
+    const char* dyg = static_cast<const char*>(a.dy);
+    const char* thg = static_cast<const char*>(p.theta);
+    const int vB = rowB / 16, vX = rowX / 16, vT = rowT / 16, vDC = R * N / 4;
+    const int nB = (Tc + 1) * vB, nC = Tc * vB, nX = (Tc + 1) * vX, nDY = Tc * vX;
+    const int nTH = Tc * vT, nDC = read_dc ? Tc * vDC : 0;
+    const int total = nB + nC + nX + nDY + nTH + nDC;
+    for (int e = tid; e < total; e += nth) {
+        int j = e;
+        const void* src = Bg;
+        void* dst;
+        bool valid = true;
+        if (j < nB) {
+            const int k = j / vB, o = (j % vB) * 16;
+            const int64_t t = c0 - 1 + k;
+            if (t >= 0) src = Bg + ((bb * L + t) * p.G + g) * rowB + o;
+            else if (p.prevB0) src = static_cast<const char*>(p.prevB0) + u * rowB + o;
+            else valid = false;
+            dst = rB + k * rowB + o;
+        } else if ((j -= nB) < nC) {
+            const int k = 1 + j / vB, o = (j % vB) * 16;
+            src = Cg + ((bb * L + c0 - 1 + k) * p.G + g) * rowB + o;
+            dst = rC + (k - 1) * rowB + o;
+        } else if ((j -= nC) < nX) {
+            const int k = j / vX, o = (j % vX) * 16;
+            const int64_t t = c0 - 1 + k;
+            if (t >= 0) src = xg + ((bb * L + t) * H + hh) * rowX + o;
+            else if (p.prevx0) src = static_cast<const char*>(p.prevx0) + u * rowX + o;
+            else valid = false;
+            dst = rX + k * rowX + o;
+        } else if ((j -= nX) < nDY) {
+            const int k = 1 + j / vX, o = (j % vX) * 16;
+            src = dyg + ((bb * L + c0 - 1 + k) * H + hh) * rowX + o;
+            dst = rDY + (k - 1) * rowX + o;
+        } else if ((j -= nDY) < nTH) {
+            const int k = 1 + j / vT, o = (j % vT) * 16;
+            src = thg + ((bb * L + c0 - 1 + k) * H + hh) * rowT + o;
+            dst = rTH + (k - 1) * rowT + o;
+        } else {
+            j -= nTH;
+            const int k = 1 + j / vDC, o = (j % vDC) * 4;
+            src = a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o;
+            dst = sm + lay.DC + k * R * N + o;
+        }
+        cp16(dst, src, valid);
+    }
+    for (int e = tid; e < 3 * Tc; e += nth) {
+        const int k = 1 + e / 3, w = e % 3;
+        const int64_t si = (bb * L + c0 - 1 + k) * H + hh;
+        cp4(rS + (k - 1) * 3 + w, (w == 0 ? p.dt : w == 1 ? p.A : p.lam) + si);
+    }
+    cp_wait_all();
+    __syncthreads();
+
+    // ---- step scalars; x and dy to fp32 ----
     const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
     for (int k = 1 + tid; k <= Tc; k += nth) {
-        const int64_t si = (bb * L + c0 - 1 + k) * H + hh;
-        const float d = step_dt(p.dt[si], dtb, p.flags), A = p.A[si];
-        const float lm = step_lam(p.lam[si], p.flags);
+        const float d = step_dt(rS[(k - 1) * 3], dtb, p.flags), A = rS[(k - 1) * 3 + 1];
+        const float lm = step_lam(rS[(k - 1) * 3 + 2], p.flags);
         const float al = expf(d * A);
         const bool zoh = p.flags & M3_DISC_ZOH;
         float* s = scal + 8 * k;
@@ -139,74 +228,65 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
         s[4] = zoh ? 0.f : (1.f - lm) * d * al;
         s[5] = zoh ? zoh_gamma(d, A) : lm * d;
     }
-    for (int e = tid; e < Tc * (half / 4); e += nth) {
-        const int k = 1 + e / (half / 4), i4 = (e % (half / 4)) * 4;
-        const float4 v = ld4(thg + ((bb * L + c0 - 1 + k) * H + hh) * half + i4);
-        *reinterpret_cast<float4*>(th + k * half + i4) = v;
-    }
-    // x (slots 0..Tc) and dy (1..Tc), and the forward sweep's dCbar when asked
-    const T* xg = static_cast<const T*>(p.x);
-    const T* dyg = static_cast<const T*>(a.dy);
-    const int RP4 = R * P / 4;
-    for (int e = tid; e < (Tc + 1) * RP4; e += nth) {
-        const int k = e / RP4, o = (e % RP4) * 4;
-        const int64_t t = c0 - 1 + k;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t >= 0) v = ld4(xg + ((bb * L + t) * H + hh) * R * P + o);
-        else if (p.prevx0) v = ld4(static_cast<const T*>(p.prevx0) + u * R * P + o);
-        *reinterpret_cast<float4*>(sm + lay.X + k * R * P + o) = v;
-        if (k > 0)
-            *reinterpret_cast<float4*>(sm + lay.DY + k * R * P + o) =
-                ld4(dyg + ((bb * L + t) * H + hh) * R * P + o);
-    }
-    if (read_dc) {
-        const int RN4 = R * N / 4;
-        for (int e = tid; e < Tc * RN4; e += nth) {
-            const int k = 1 + e / RN4, o = (e % RN4) * 4;
-            *reinterpret_cast<float4*>(sm + lay.DC + k * R * N + o) =
-                *reinterpret_cast<const float4*>(a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o);
-        }
+    {
+        const T* xr = reinterpret_cast<const T*>(rX);
+        const T* dyr = reinterpret_cast<const T*>(rDY);
+        float* sX = sm + lay.X;
+        float* sDY = sm + lay.DY + R * P;
+        for (int e = tid; e < (Tc + 1) * R * P; e += nth) sX[e] = to_f(xr[e]);
+        for (int e = tid; e < Tc * R * P; e += nth) sDY[e] = to_f(dyr[e]);
+        const T* thr = reinterpret_cast<const T*>(rTH);
+        float* sTH = sm + lay.TH + half;
+        for (int e = tid; e < Tc * half; e += nth) sTH[e] = to_f(thr[e]);
     }
     __syncthreads();
-    // angles: one thread per pair walks the chunk
-    for (int i = tid; i < half; i += nth) {
-        float ph = phi_start[i];
-        float s, c;
-        sincosf(ph, &s, &c);
-        cs[i] = c; cs[half + i] = s;
-        for (int k = 1; k <= Tc; ++k) {
+
+    // ---- angles: the four lanes of a pair's quad walk a quarter of the chunk each ----
+    {
+        const int i = tid >> 2, q = tid & 3;
+        const int nk = (Tc + 3) >> 2;
+        const int klo = 1 + q * nk, khi = min(Tc, klo + nk - 1);
+        const float* th = sm + lay.TH;
+        const float ph0 = phi_start[i];
+        float loc = 0.f;
+        for (int k = klo; k <= khi; ++k) loc = fmaf(scal[8 * k], th[k * half + i], loc);
+        const float e1 = __shfl_up_sync(kFull, loc, 1, 4);
+        const float e2 = __shfl_up_sync(kFull, loc, 2, 4);
+        const float e3 = __shfl_up_sync(kFull, loc, 3, 4);
+        float ph = ph0 + ((q >= 1 ? e1 : 0.f) + (q >= 2 ? e2 : 0.f) + (q >= 3 ? e3 : 0.f));
+        float sn, cn;
+        if (q == 0) {
+            sincosf(ph0, &sn, &cn);
+            cs[i] = cn; cs[half + i] = sn;
+        }
+        for (int k = klo; k <= khi; ++k) {
             ph = fmaf(scal[8 * k], th[k * half + i], ph);
-            sincosf(ph, &s, &c);
-            cs[k * N + i] = c; cs[k * N + half + i] = s;
+            sincosf(ph, &sn, &cn);
+            cs[k * N + i] = cn; cs[k * N + half + i] = sn;
         }
+        if (phi_end && klo <= khi && khi == Tc) phi_end[i] = ph;
     }
     __syncthreads();
-    // rotated, normalised, biased B (slots 0..Tc) and C (slots 1..Tc): one warp per vector
-    const T* Bg = static_cast<const T*>(p.B);
-    const T* Cg = static_cast<const T*>(p.C);
+
+    // ---- rotated, normalised, biased B (slots 0..Tc) and C (1..Tc): one warp per vector ----
     const int nitems = (2 * Tc + 1) * R;
     for (int it = warp; it < nitems; it += nwarps) {
         const bool isC = it >= (Tc + 1) * R;
         const int j = isC ? it - (Tc + 1) * R : it;
         const int k = isC ? 1 + j / R : j / R, r = j % R;
-        const int64_t t = c0 - 1 + k;
-        const T* src = nullptr;
-        if (t >= 0) src = (isC ? Cg : Bg) + ((bb * L + t) * p.G + g) * R * N + r * N;
-        else if (p.prevB0) src = static_cast<const T*>(p.prevB0) + (u * R + r) * N;
-        const float* bias = isC ? p.Cbias : p.Bbias;
-        if (bias) bias += (hh * R + r) * N;
+        const T* src = reinterpret_cast<const T*>(isC ? rC + (k - 1) * rowB : rB + k * rowB) + r * N;
+        const float* bias = sm + lay.BIAS + (isC ? R * N : 0) + r * N;
         float ss = 0.f;
         for (int i = lane; i < half; i += 32) {
-            const float v0 = src ? to_f(src[i]) : 0.f, v1 = src ? to_f(src[i + half]) : 0.f;
+            const float v0 = to_f(src[i]), v1 = to_f(src[i + half]);
             ss = fmaf(v0, v0, fmaf(v1, v1, ss));
         }
         ss = warp_sum(ss);
         const float scale = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
         float* dst = sm + (isC ? lay.C : lay.B) + (k * R + r) * N;
         for (int i = lane; i < half; i += 32) {
-            float v0 = src ? to_f(src[i]) : 0.f, v1 = src ? to_f(src[i + half]) : 0.f;
-            v0 = v0 * scale + (bias ? bias[i] : 0.f);
-            v1 = v1 * scale + (bias ? bias[i + half] : 0.f);
+            const float v0 = to_f(src[i]) * scale + bias[i];
+            const float v1 = to_f(src[i + half]) * scale + bias[i + half];
             const float c = cs[k * N + i], s = cs[k * N + half + i];
             dst[i] = v0 * c + v1 * s;
             dst[i + half] = v1 * c - v0 * s;
@@ -215,11 +295,27 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     __syncthreads();
 }
 
+// Loads this head's B and C biases into shared memory (zeros when absent).
+__device__ __forceinline__ void load_bias(const BwdArgs& a, const BwdLayout& lay, float* sm,
+                                          int64_t hh) {
+    const int RN = static_cast<int>(a.f.R * a.f.N);
+    for (int e = threadIdx.x; e < 2 * RN; e += blockDim.x) {
+        const float* b = e < RN ? a.f.Bbias : a.f.Cbias;
+        sm[lay.BIAS + e] = b ? b[hh * RN + (e % RN)] : 0.f;
+    }
+}
+
+// Column of a thread's e-th register of a row: the quarter q owns the float4 groups
+// 16 m + 4 q .. 16 m + 4 q + 3, so the four quarters of a pair read 64 contiguous bytes
+// (distinct banks) with one 16-byte load each.
+__host__ __device__ __forceinline__ int col_of(int e, int q) { return 16 * (e >> 2) + 4 * q + (e & 3); }
+
 // Sum over the eight lanes of a warp that share the quarter q (lane bits 2..4) of CPQ
-// per-column partials, halving the list at each step; the lane then adds its share into dst
-// (the q-th quarter of a row of P columns in shared memory).
+// per-column partials, halving the list at each step; the lane then adds its share into the
+// shared-memory row of P columns.
 template <int CPQ>
-__device__ __forceinline__ void add_cols(const float (&v)[CPQ], int lane, float* dst) {
+__device__ __forceinline__ void add_cols(const float (&v)[CPQ], int lane, float* row) {
+    const int q = lane & 3;
     constexpr int n1 = CPQ / 2, n2 = n1 / 2;
     float w1[n1];
     bool up = lane & 16;
@@ -246,11 +342,12 @@ __device__ __forceinline__ void add_cols(const float (&v)[CPQ], int lane, float*
         for (int j = 0; j < n3; ++j) {
             const float send = up ? w2[j] : w2[j + n3];
             const float keep = up ? w2[j + n3] : w2[j];
-            atomicAdd(dst + off + (up ? n3 : 0) + j, keep + __shfl_xor_sync(kFull, send, 4));
+            atomicAdd(row + col_of(off + (up ? n3 : 0) + j, q),
+                      keep + __shfl_xor_sync(kFull, send, 4));
         }
     } else {
         const float w = w2[0] + __shfl_xor_sync(kFull, w2[0], 4);
-        if (!(lane & 4)) atomicAdd(dst + off, w);
+        if (!(lane & 4)) atomicAdd(row + col_of(off, q), w);
     }
 }
 
@@ -276,7 +373,7 @@ __device__ __forceinline__ float warp_sum4(float v0, float v1, float v2, float v
 // Forward sweep: h_t token by token; writes dCbar_t = h_t dy_t per token, the angle before
 // every chunk and <dL/dh_final, h_final>.
 template <typename T, int CPQ, int kThreads>
-__global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_fwd_kernel(const BwdArgs a) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     const ScanParams& p = a.f;
@@ -286,17 +383,19 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
     const int64_t u = blockIdx.x, bb = u / H, hh = u % H;
     const int tid = threadIdx.x, lane = tid & 31;
     const int i = tid >> 2, q = tid & 3;
-    const BwdLayout lay = bwd_layout(a.T, R, N, P);
+    const BwdLayout lay = bwd_layout(a.T, R, N, P, sizeof(T));
     __shared__ float phi_run[128];
+    __shared__ float phi_next[128];
     __shared__ float red[32];
 
     float h0[CPQ], h1[CPQ];
 #pragma unroll
     for (int c = 0; c < CPQ; ++c) {
-        h0[c] = p.h0 ? p.h0[(u * N + i) * P + q * CPQ + c] : 0.f;
-        h1[c] = p.h0 ? p.h0[(u * N + i + half) * P + q * CPQ + c] : 0.f;
+        h0[c] = p.h0 ? p.h0[(u * N + i) * P + col_of(c, q)] : 0.f;
+        h1[c] = p.h0 ? p.h0[(u * N + i + half) * P + col_of(c, q)] : 0.f;
     }
     for (int e = tid; e < half; e += blockDim.x) phi_run[e] = p.phi0 ? p.phi0[u * half + e] : 0.f;
+    load_bias(a, lay, sm, hh);
     __syncthreads();
 
     for (int c = 0; c < a.nchunks; ++c) {
@@ -304,7 +403,7 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
         const int Tc = static_cast<int>(L - c0 < a.T ? L - c0 : a.T);
         for (int e = tid; e < half; e += blockDim.x)
             a.wphi[(u * a.nchunks + c) * half + e] = phi_run[e];
-        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_run, false);
+        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_run, phi_next, false);
         const float* sB = sm + lay.B;
         const float* sX = sm + lay.X;
         const float* sDY = sm + lay.DY;
@@ -319,12 +418,12 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
                 const float bp1 = be * sB[((k - 1) * R + r) * N + i + half];
                 const float bc0 = ga * sB[(k * R + r) * N + i];
                 const float bc1 = ga * sB[(k * R + r) * N + i + half];
-                const float* xp = sX + ((k - 1) * R + r) * P + q * CPQ;
-                const float* xc = sX + (k * R + r) * P + q * CPQ;
+                const float* xp = sX + ((k - 1) * R + r) * P + 4 * q;
+                const float* xc = sX + (k * R + r) * P + 4 * q;
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
-                    const float4 vp = *reinterpret_cast<const float4*>(xp + cc);
-                    const float4 vc = *reinterpret_cast<const float4*>(xc + cc);
+                    const float4 vp = *reinterpret_cast<const float4*>(xp + 4 * cc);
+                    const float4 vc = *reinterpret_cast<const float4*>(xc + 4 * cc);
                     const float xpv[4] = {vp.x, vp.y, vp.z, vp.w};
                     const float xcv[4] = {vc.x, vc.y, vc.z, vc.w};
 #pragma unroll
@@ -335,11 +434,11 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
                 }
             }
             for (int r = 0; r < R; ++r) {
-                const float* dy = sDY + (k * R + r) * P + q * CPQ;
+                const float* dy = sDY + (k * R + r) * P + 4 * q;
                 float d0 = 0.f, d1 = 0.f;
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(dy + cc);
+                    const float4 v = *reinterpret_cast<const float4*>(dy + 4 * cc);
                     d0 = fmaf(h0[cc], v.x, fmaf(h0[cc + 1], v.y, fmaf(h0[cc + 2], v.z, fmaf(h0[cc + 3], v.w, d0))));
                     d1 = fmaf(h1[cc], v.x, fmaf(h1[cc + 1], v.y, fmaf(h1[cc + 2], v.z, fmaf(h1[cc + 3], v.w, d1))));
                 }
@@ -353,11 +452,7 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
         }
         __syncthreads();
         // the chunk's angle end, and its dCbar rows out
-        for (int e = tid; e < half; e += blockDim.x) {
-            float ph = phi_run[e];
-            for (int k = 1; k <= Tc; ++k) ph = fmaf(sm[lay.SCAL + 8 * k], sm[lay.TH + k * half + e], ph);
-            phi_run[e] = ph;
-        }
+        for (int e = tid; e < half; e += blockDim.x) phi_run[e] = phi_next[e];
         const int RN4 = R * N / 4;
         for (int e = tid; e < Tc * RN4; e += blockDim.x) {
             const int k = 1 + e / RN4, o = (e % RN4) * 4;
@@ -371,8 +466,8 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
     if (a.dh1) {
 #pragma unroll
         for (int c = 0; c < CPQ; ++c) {
-            f = fmaf(a.dh1[(u * N + i) * P + q * CPQ + c], h0[c], f);
-            f = fmaf(a.dh1[(u * N + i + half) * P + q * CPQ + c], h1[c], f);
+            f = fmaf(a.dh1[(u * N + i) * P + col_of(c, q)], h0[c], f);
+            f = fmaf(a.dh1[(u * N + i + half) * P + col_of(c, q)], h1[c], f);
         }
     }
     f = warp_sum(f);
@@ -388,8 +483,8 @@ __global__ void __launch_bounds__(kThreads) bwd_fwd_kernel(const BwdArgs a) {
 // ---------------------------------------------------------------------------------------
 // Reverse sweep: G_t from the end; dx, dtheta, the rotated-back dB and dC per head, the
 // per-token partial sums for the scalars, the bias sums and the initial state's gradients.
-template <typename T, int CPQ, int kThreads>
-__global__ void __launch_bounds__(kThreads) bwd_rev_kernel(const BwdArgs a) {
+template <typename T, int CPQ, int kThreads, bool kR1>
+__global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_kernel(const BwdArgs a) {
     extern __shared__ float4 smem4[];
     float* sm = reinterpret_cast<float*>(smem4);
     const ScanParams& p = a.f;
@@ -399,15 +494,15 @@ __global__ void __launch_bounds__(kThreads) bwd_rev_kernel(const BwdArgs a) {
     const int64_t u = blockIdx.x, bb = u / H, hh = u % H;
     const int tid = threadIdx.x, lane = tid & 31;
     const int i = tid >> 2, q = tid & 3;
-    const BwdLayout lay = bwd_layout(a.T, R, N, P);
+    const BwdLayout lay = bwd_layout(a.T, R, N, P, sizeof(T));
     __shared__ float phi_start[128];
     __shared__ float pend[4];
 
     float G0[CPQ], G1[CPQ];
 #pragma unroll
     for (int c = 0; c < CPQ; ++c) {
-        G0[c] = a.dh1 ? a.dh1[(u * N + i) * P + q * CPQ + c] : 0.f;
-        G1[c] = a.dh1 ? a.dh1[(u * N + i + half) * P + q * CPQ + c] : 0.f;
+        G0[c] = a.dh1 ? a.dh1[(u * N + i) * P + col_of(c, q)] : 0.f;
+        G1[c] = a.dh1 ? a.dh1[(u * N + i + half) * P + col_of(c, q)] : 0.f;
     }
     float dphi = a.dphi1 ? a.dphi1[u * half + i] : 0.f;
     float a_n = 1.f, b_n = 0.f;         // alpha and beta of the token after the current one
@@ -432,51 +527,95 @@ __global__ void __launch_bounds__(kThreads) bwd_rev_kernel(const BwdArgs a) {
             phi_start[e] = a.wphi[(u * a.nchunks + c) * half + e];
         for (int e = tid; e < (Tc + 1) * R * P; e += blockDim.x) sDX[e] = 0.f;
         for (int e = tid; e < (a.T + 2) * 4; e += blockDim.x) sSC[e] = 0.f;
+        if (c == a.nchunks - 1) load_bias(a, lay, sm, hh);
         __syncthreads();
-        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_start, true);
+        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_start, nullptr, true);
 
         for (int k = Tc; k >= 1; --k) {
             const float* s = sm + lay.SCAL + 8 * k;
             const float ga = s[5];
-            float go0[CPQ], go1[CPQ];
-#pragma unroll
-            for (int cc = 0; cc < CPQ; ++cc) {
-                go0[cc] = G0[cc]; go1[cc] = G1[cc];
-                G0[cc] *= a_n; G1[cc] *= a_n;
-            }
-            for (int r = 0; r < R; ++r) {
-                const float cb0 = sC[(k * R + r) * N + i], cb1 = sC[(k * R + r) * N + i + half];
-                const float* dy = sDY + (k * R + r) * P + q * CPQ;
-#pragma unroll
-                for (int cc = 0; cc < CPQ; cc += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(dy + cc);
-                    const float dv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        G0[cc + j] = fmaf(cb0, dv[j], G0[cc + j]);
-                        G1[cc + j] = fmaf(cb1, dv[j], G1[cc + j]);
-                    }
-                }
-            }
             float sg = 0.f, sbn = 0.f, syy = 0.f, dl = 0.f;
-            for (int r = 0; r < R; ++r) {
-                const float bb0 = sB[(k * R + r) * N + i], bb1 = sB[(k * R + r) * N + i + half];
-                const float* x = sX + (k * R + r) * P + q * CPQ;
-                float gA0 = 0.f, gA1 = 0.f, gB0 = 0.f, gB1 = 0.f;
+            // G_t = a_{t+1} G_{t+1} + sum_r Cbar_t[r] dy_t[r]^T and, per r, the contractions of
+            // G_{t+1} (gA) and G_t (gB) with x_t[r] over this thread's columns and the dx partial
+            // sum over its rows of Bbar_t[r] du_t, du_t = g_t G_t + b_{t+1} G_{t+1}.
+            float gAr[kR1 ? 1 : 8][2], gBr[kR1 ? 1 : 8][2];
+            if constexpr (kR1) {
+                // one pass from G_{t+1}: du = (g a' + b') G_{t+1} + g Cbar dy^T and
+                // G_t x = a' (G_{t+1} x) + Cbar (dy . x)
+                const float cb0 = sC[k * N + i], cb1 = sC[k * N + i + half];
+                const float bb0 = sB[k * N + i], bb1 = sB[k * N + i + half];
+                const float* x = sX + k * P + 4 * q;
+                const float* dy = sDY + k * P + 4 * q;
+                const float coef = fmaf(ga, a_n, b_n);
+                const float gs = ga * fmaf(bb0, cb0, bb1 * cb1);
+                float gA0 = 0.f, gA1 = 0.f, dyx = 0.f;
                 float v[CPQ];
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
-                    const float4 xv4 = *reinterpret_cast<const float4*>(x + cc);
+                    const float4 xv4 = *reinterpret_cast<const float4*>(x + 4 * cc);
+                    const float4 dv4 = *reinterpret_cast<const float4*>(dy + 4 * cc);
                     const float xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+                    const float dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int e = cc + j;
-                        gA0 = fmaf(go0[e], xv[j], gA0); gA1 = fmaf(go1[e], xv[j], gA1);
-                        gB0 = fmaf(G0[e], xv[j], gB0); gB1 = fmaf(G1[e], xv[j], gB1);
-                        v[e] = ga * fmaf(bb0, G0[e], bb1 * G1[e]) + b_n * fmaf(bb0, go0[e], bb1 * go1[e]);
+                        gA0 = fmaf(G0[e], xv[j], gA0);
+                        gA1 = fmaf(G1[e], xv[j], gA1);
+                        dyx = fmaf(dv[j], xv[j], dyx);
+                        v[e] = fmaf(coef, fmaf(bb0, G0[e], bb1 * G1[e]), gs * dv[j]);
+                        G0[e] = fmaf(a_n, G0[e], cb0 * dv[j]);
+                        G1[e] = fmaf(a_n, G1[e], cb1 * dv[j]);
                     }
                 }
-                add_cols<CPQ>(v, lane, sDX + (k * R + r) * P + q * CPQ);
+                add_cols<CPQ>(v, lane, sDX + k * P);
+                gAr[0][0] = gA0; gAr[0][1] = gA1;
+                gBr[0][0] = fmaf(a_n, gA0, cb0 * dyx);
+                gBr[0][1] = fmaf(a_n, gA1, cb1 * dyx);
+            } else {
+                float go0[CPQ], go1[CPQ];
+#pragma unroll
+                for (int cc = 0; cc < CPQ; ++cc) {
+                    go0[cc] = G0[cc]; go1[cc] = G1[cc];
+                    G0[cc] *= a_n; G1[cc] *= a_n;
+                }
+                for (int r = 0; r < R; ++r) {
+                    const float cb0 = sC[(k * R + r) * N + i], cb1 = sC[(k * R + r) * N + i + half];
+                    const float* dy = sDY + (k * R + r) * P + 4 * q;
+#pragma unroll
+                    for (int cc = 0; cc < CPQ; cc += 4) {
+                        const float4 v = *reinterpret_cast<const float4*>(dy + 4 * cc);
+                        const float dv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            G0[cc + j] = fmaf(cb0, dv[j], G0[cc + j]);
+                            G1[cc + j] = fmaf(cb1, dv[j], G1[cc + j]);
+                        }
+                    }
+                }
+                for (int r = 0; r < R; ++r) {
+                    const float bb0 = sB[(k * R + r) * N + i], bb1 = sB[(k * R + r) * N + i + half];
+                    const float* x = sX + (k * R + r) * P + 4 * q;
+                    float gA0 = 0.f, gA1 = 0.f, gB0 = 0.f, gB1 = 0.f;
+                    float v[CPQ];
+#pragma unroll
+                    for (int cc = 0; cc < CPQ; cc += 4) {
+                        const float4 xv4 = *reinterpret_cast<const float4*>(x + 4 * cc);
+                        const float xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int e = cc + j;
+                            gA0 = fmaf(go0[e], xv[j], gA0); gA1 = fmaf(go1[e], xv[j], gA1);
+                            gB0 = fmaf(G0[e], xv[j], gB0); gB1 = fmaf(G1[e], xv[j], gB1);
+                            v[e] = ga * fmaf(bb0, G0[e], bb1 * G1[e]) + b_n * fmaf(bb0, go0[e], bb1 * go1[e]);
+                        }
+                    }
+                    add_cols<CPQ>(v, lane, sDX + (k * R + r) * P);
+                    gAr[r][0] = gA0; gAr[r][1] = gA1; gBr[r][0] = gB0; gBr[r][1] = gB1;
+                }
+            }
+            for (int r = 0; r < (kR1 ? 1 : R); ++r) {
+                const float bb0 = sB[(k * R + r) * N + i], bb1 = sB[(k * R + r) * N + i + half];
+                const float gA0 = gAr[r][0], gA1 = gAr[r][1], gB0 = gBr[r][0], gB1 = gBr[r][1];
                 sg = fmaf(bb0, gB0, fmaf(bb1, gB1, sg));
                 sbn = fmaf(bb0, gA0, fmaf(bb1, gA1, sbn));
                 float db0 = fmaf(ga, gB0, b_n * gA0), db1 = fmaf(ga, gB1, b_n * gA1);
@@ -525,23 +664,24 @@ __global__ void __launch_bounds__(kThreads) bwd_rev_kernel(const BwdArgs a) {
             if (a.dh0) {
 #pragma unroll
                 for (int cc = 0; cc < CPQ; ++cc) {
-                    a.dh0[(u * N + i) * P + q * CPQ + cc] = a_n * G0[cc];
-                    a.dh0[(u * N + i + half) * P + q * CPQ + cc] = a_n * G1[cc];
+                    a.dh0[(u * N + i) * P + col_of(cc, q)] = a_n * G0[cc];
+                    a.dh0[(u * N + i + half) * P + col_of(cc, q)] = a_n * G1[cc];
                 }
             }
             float sbn = 0.f, dl = 0.f;
             for (int r = 0; r < R; ++r) {
                 const float bb0 = sB[r * N + i], bb1 = sB[r * N + i + half];
-                const float* x = sX + r * P + q * CPQ;
+                const float* x = sX + r * P;
                 float gA0 = 0.f, gA1 = 0.f;
                 float v[CPQ];
 #pragma unroll
                 for (int e = 0; e < CPQ; ++e) {
-                    gA0 = fmaf(G0[e], x[e], gA0);
-                    gA1 = fmaf(G1[e], x[e], gA1);
+                    const float xe = x[col_of(e, q)];
+                    gA0 = fmaf(G0[e], xe, gA0);
+                    gA1 = fmaf(G1[e], xe, gA1);
                     v[e] = b_n * fmaf(bb0, G0[e], bb1 * G1[e]);
                 }
-                add_cols<CPQ>(v, lane, sDX + r * P + q * CPQ);
+                add_cols<CPQ>(v, lane, sDX + r * P);
                 sbn = fmaf(bb0, gA0, fmaf(bb1, gA1, sbn));
                 float db0 = b_n * gA0, db1 = b_n * gA1;
                 db0 += __shfl_xor_sync(kFull, db0, 1);
@@ -797,7 +937,8 @@ cudaError_t launch_sweeps(const BwdArgs& a, size_t smem, cudaStream_t s) {
     const int units = static_cast<int>(a.f.b * a.f.H);
     const int threads = static_cast<int>(2 * a.f.N);
     auto kf = bwd_fwd_kernel<T, CPQ, kThreads>;
-    auto kr = bwd_rev_kernel<T, CPQ, kThreads>;
+    auto kr = a.f.R == 1 ? bwd_rev_kernel<T, CPQ, kThreads, true>
+                         : bwd_rev_kernel<T, CPQ, kThreads, false>;
     cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -858,7 +999,7 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
     if (a.dCbias && (e = cudaMemsetAsync(a.dCbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
     if (a.ddtbias && (e = cudaMemsetAsync(a.ddtbias, 0, sizeof(float) * f.H, s)) != cudaSuccess) return e;
     const BwdLayout lay = bwd_layout(a.T, static_cast<int>(f.R), static_cast<int>(f.N),
-                                     static_cast<int>(f.P));
+                                     static_cast<int>(f.P), bf16 ? 2 : 4);
     const size_t smem = sizeof(float) * lay.total;
     if (f.N <= 128)
         e = bf16 ? launch_sweeps_p<__nv_bfloat16, 256>(a, smem, s)
@@ -877,7 +1018,7 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
 
 size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t R) {
     const BwdLayout lay = bwd_layout(bwd_chunk_tokens(R), static_cast<int>(R),
-                                     static_cast<int>(N), static_cast<int>(P));
+                                     static_cast<int>(N), static_cast<int>(P), 4);
     return sizeof(float) * lay.total;
 }
 
