@@ -69,6 +69,27 @@ __device__ __forceinline__ void cp_wait_all() {
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
+// Two-lane fp32 arithmetic of sm_100 (one packed instruction for two columns):
+// fma2 = (a.x b.x + c.x, a.y b.y + c.y), mul2 = (a.x b.x, a.y b.y), round to nearest.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
+
 // Shared-memory layout of one chunk (floats). Slot k = 0..T holds token c0 - 1 + k. RAW holds
 // the chunk's inputs as loaded (element size es): B rows (slots 0..T), C, dy and theta rows
 // (slots 1..T at k - 1), x rows (0..T) and the raw dt, A, lam (slots 1..T at k - 1).
@@ -411,37 +432,48 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_fwd_ker
         for (int k = 1; k <= Tc; ++k) {
             const float* s = sm + lay.SCAL + 8 * k;
             const float al = s[3], be = s[4], ga = s[5];
+            const float2 al2 = dup2(al);
 #pragma unroll
-            for (int cc = 0; cc < CPQ; ++cc) { h0[cc] *= al; h1[cc] *= al; }
+            for (int cc = 0; cc < CPQ; cc += 2) {
+                float2 a0 = mul2(al2, make_float2(h0[cc], h0[cc + 1]));
+                float2 a1 = mul2(al2, make_float2(h1[cc], h1[cc + 1]));
+                h0[cc] = a0.x; h0[cc + 1] = a0.y; h1[cc] = a1.x; h1[cc + 1] = a1.y;
+            }
             for (int r = 0; r < R; ++r) {
-                const float bp0 = be * sB[((k - 1) * R + r) * N + i];
-                const float bp1 = be * sB[((k - 1) * R + r) * N + i + half];
-                const float bc0 = ga * sB[(k * R + r) * N + i];
-                const float bc1 = ga * sB[(k * R + r) * N + i + half];
+                const float2 bp0 = dup2(be * sB[((k - 1) * R + r) * N + i]);
+                const float2 bp1 = dup2(be * sB[((k - 1) * R + r) * N + i + half]);
+                const float2 bc0 = dup2(ga * sB[(k * R + r) * N + i]);
+                const float2 bc1 = dup2(ga * sB[(k * R + r) * N + i + half]);
                 const float* xp = sX + ((k - 1) * R + r) * P + 4 * q;
                 const float* xc = sX + (k * R + r) * P + 4 * q;
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
                     const float4 vp = *reinterpret_cast<const float4*>(xp + 4 * cc);
                     const float4 vc = *reinterpret_cast<const float4*>(xc + 4 * cc);
-                    const float xpv[4] = {vp.x, vp.y, vp.z, vp.w};
-                    const float xcv[4] = {vc.x, vc.y, vc.z, vc.w};
+                    const float2 xpv[2] = {make_float2(vp.x, vp.y), make_float2(vp.z, vp.w)};
+                    const float2 xcv[2] = {make_float2(vc.x, vc.y), make_float2(vc.z, vc.w)};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        h0[cc + j] = fmaf(bp0, xpv[j], fmaf(bc0, xcv[j], h0[cc + j]));
-                        h1[cc + j] = fmaf(bp1, xpv[j], fmaf(bc1, xcv[j], h1[cc + j]));
+                    for (int j = 0; j < 2; ++j) {
+                        const int e = cc + 2 * j;
+                        const float2 n0 = fma2(bp0, xpv[j], fma2(bc0, xcv[j], make_float2(h0[e], h0[e + 1])));
+                        const float2 n1 = fma2(bp1, xpv[j], fma2(bc1, xcv[j], make_float2(h1[e], h1[e + 1])));
+                        h0[e] = n0.x; h0[e + 1] = n0.y; h1[e] = n1.x; h1[e + 1] = n1.y;
                     }
                 }
             }
             for (int r = 0; r < R; ++r) {
                 const float* dy = sDY + (k * R + r) * P + 4 * q;
-                float d0 = 0.f, d1 = 0.f;
+                float2 p0 = make_float2(0.f, 0.f), p1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
                     const float4 v = *reinterpret_cast<const float4*>(dy + 4 * cc);
-                    d0 = fmaf(h0[cc], v.x, fmaf(h0[cc + 1], v.y, fmaf(h0[cc + 2], v.z, fmaf(h0[cc + 3], v.w, d0))));
-                    d1 = fmaf(h1[cc], v.x, fmaf(h1[cc + 1], v.y, fmaf(h1[cc + 2], v.z, fmaf(h1[cc + 3], v.w, d1))));
+                    const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+                    p0 = fma2(make_float2(h0[cc], h0[cc + 1]), v01, p0);
+                    p0 = fma2(make_float2(h0[cc + 2], h0[cc + 3]), v23, p0);
+                    p1 = fma2(make_float2(h1[cc], h1[cc + 1]), v01, p1);
+                    p1 = fma2(make_float2(h1[cc + 2], h1[cc + 3]), v23, p1);
                 }
+                float d0 = p0.x + p0.y, d1 = p1.x + p1.y;
                 d0 += __shfl_xor_sync(kFull, d0, 1);
                 d1 += __shfl_xor_sync(kFull, d1, 1);
                 d0 += __shfl_xor_sync(kFull, d0, 2);
@@ -546,31 +578,38 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
                 const float bb0 = sB[k * N + i], bb1 = sB[k * N + i + half];
                 const float* x = sX + k * P + 4 * q;
                 const float* dy = sDY + k * P + 4 * q;
-                const float coef = fmaf(ga, a_n, b_n);
-                const float gs = ga * fmaf(bb0, cb0, bb1 * cb1);
-                float gA0 = 0.f, gA1 = 0.f, dyx = 0.f;
+                const float2 coef = dup2(fmaf(ga, a_n, b_n));
+                const float2 gs = dup2(ga * fmaf(bb0, cb0, bb1 * cb1));
+                const float2 an2 = dup2(a_n), bb0_2 = dup2(bb0), bb1_2 = dup2(bb1);
+                const float2 cb0_2 = dup2(cb0), cb1_2 = dup2(cb1);
+                float2 gA0 = make_float2(0.f, 0.f), gA1 = gA0, dyx = gA0;
                 float v[CPQ];
 #pragma unroll
                 for (int cc = 0; cc < CPQ; cc += 4) {
                     const float4 xv4 = *reinterpret_cast<const float4*>(x + 4 * cc);
                     const float4 dv4 = *reinterpret_cast<const float4*>(dy + 4 * cc);
-                    const float xv[4] = {xv4.x, xv4.y, xv4.z, xv4.w};
-                    const float dv[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+                    const float2 xv[2] = {make_float2(xv4.x, xv4.y), make_float2(xv4.z, xv4.w)};
+                    const float2 dv[2] = {make_float2(dv4.x, dv4.y), make_float2(dv4.z, dv4.w)};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int e = cc + j;
-                        gA0 = fmaf(G0[e], xv[j], gA0);
-                        gA1 = fmaf(G1[e], xv[j], gA1);
-                        dyx = fmaf(dv[j], xv[j], dyx);
-                        v[e] = fmaf(coef, fmaf(bb0, G0[e], bb1 * G1[e]), gs * dv[j]);
-                        G0[e] = fmaf(a_n, G0[e], cb0 * dv[j]);
-                        G1[e] = fmaf(a_n, G1[e], cb1 * dv[j]);
+                    for (int j = 0; j < 2; ++j) {
+                        const int e = cc + 2 * j;
+                        const float2 g0 = make_float2(G0[e], G0[e + 1]);
+                        const float2 g1 = make_float2(G1[e], G1[e + 1]);
+                        gA0 = fma2(g0, xv[j], gA0);
+                        gA1 = fma2(g1, xv[j], gA1);
+                        dyx = fma2(dv[j], xv[j], dyx);
+                        const float2 w = fma2(coef, fma2(bb0_2, g0, mul2(bb1_2, g1)), mul2(gs, dv[j]));
+                        v[e] = w.x; v[e + 1] = w.y;
+                        const float2 n0 = fma2(an2, g0, mul2(cb0_2, dv[j]));
+                        const float2 n1 = fma2(an2, g1, mul2(cb1_2, dv[j]));
+                        G0[e] = n0.x; G0[e + 1] = n0.y; G1[e] = n1.x; G1[e + 1] = n1.y;
                     }
                 }
                 add_cols<CPQ>(v, lane, sDX + k * P);
-                gAr[0][0] = gA0; gAr[0][1] = gA1;
-                gBr[0][0] = fmaf(a_n, gA0, cb0 * dyx);
-                gBr[0][1] = fmaf(a_n, gA1, cb1 * dyx);
+                const float sA0 = gA0.x + gA0.y, sA1 = gA1.x + gA1.y, sdx = dyx.x + dyx.y;
+                gAr[0][0] = sA0; gAr[0][1] = sA1;
+                gBr[0][0] = fmaf(a_n, sA0, cb0 * sdx);
+                gBr[0][1] = fmaf(a_n, sA1, cb1 * sdx);
             } else {
                 float go0[CPQ], go1[CPQ];
 #pragma unroll
@@ -623,7 +662,27 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
                 db1 += __shfl_xor_sync(kFull, db1, 1);
                 db0 += __shfl_xor_sync(kFull, db0, 2);
                 db1 += __shfl_xor_sync(kFull, db1, 2);
-                if (q == (r & 3)) {
+                if (kR1) {
+                    // B on lane 0 and C on lane 1 of the quad
+                    const float co = sCS[k * N + i], si = sCS[k * N + half + i];
+                    if (q == 0) {
+                        dl += db0 * bb1 - db1 * bb0;
+                        const float nB0 = db0 * co - db1 * si, nB1 = db0 * si + db1 * co;
+                        sDB[k * N + i] = nB0;
+                        sDB[k * N + i + half] = nB1;
+                        accB[0][0] += nB0; accB[0][1] += nB1;
+                    } else if (q == 1) {
+                        const float cb0 = sC[k * N + i], cb1 = sC[k * N + i + half];
+                        float* dcp = sDC + k * N;
+                        const float dc0 = dcp[i], dc1 = dcp[i + half];
+                        dl += dc0 * cb1 - dc1 * cb0;
+                        syy = fmaf(cb0, dc0, fmaf(cb1, dc1, syy));
+                        const float nC0 = dc0 * co - dc1 * si, nC1 = dc0 * si + dc1 * co;
+                        dcp[i] = nC0;
+                        dcp[i + half] = nC1;
+                        accC[0][0] += nC0; accC[0][1] += nC1;
+                    }
+                } else if (q == (r & 3)) {
                     const float cb0 = sC[(k * R + r) * N + i], cb1 = sC[(k * R + r) * N + i + half];
                     float* dcp = sDC + (k * R + r) * N;
                     const float dc0 = dcp[i], dc1 = dcp[i + half];
@@ -754,6 +813,17 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
         __syncthreads();
     }
     // the biases: each unit adds its sums over the sequence
+    if (kR1) {
+        if (q == 0 && a.dBbias) {
+            atomicAdd(a.dBbias + hh * N + i, accB[0][0]);
+            atomicAdd(a.dBbias + hh * N + i + half, accB[0][1]);
+        }
+        if (q == 1 && a.dCbias) {
+            atomicAdd(a.dCbias + hh * N + i, accC[0][0]);
+            atomicAdd(a.dCbias + hh * N + i + half, accC[0][1]);
+        }
+        return;
+    }
     for (int rr = 0; rr < 2; ++rr) {
         const int r = q + 4 * rr;
         if (r >= R) break;
@@ -909,23 +979,30 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
         dn_base = a.wprev + j * N;
         dn_stride = 0;
     }
+    // N <= 256: at most eight elements per lane, kept in registers
+    float dnv[8], vv[8];
     float ss = 0.f, dot = 0.f;
-    for (int64_t n = lane; n < N; n += 32) {
-        float dn = 0.f;
-        for (int64_t h = 0; h < nh; ++h) dn += dn_base[h * dn_stride + n];
-        const float v = src ? raw(src, src_off + n) : 0.f;
-        ss = fmaf(v, v, ss);
-        dot = fmaf(v, dn, dot);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int64_t n = lane + 32 * j;
+        dnv[j] = 0.f;
+        vv[j] = 0.f;
+        if (n < N) {
+            for (int64_t h = 0; h < nh; ++h) dnv[j] += dn_base[h * dn_stride + n];
+            vv[j] = src ? raw(src, src_off + n) : 0.f;
+            ss = fmaf(vv[j], vv[j], ss);
+            dot = fmaf(vv[j], dnv[j], dot);
+        }
     }
     ss = warp_sum(ss);
     dot = warp_sum(dot);
     const float s = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
     const float k = p.bc_norm ? s * s * s / static_cast<float>(N) * dot : 0.f;
-    for (int64_t n = lane; n < N; n += 32) {
-        float dn = 0.f;
-        for (int64_t h = 0; h < nh; ++h) dn += dn_base[h * dn_stride + n];
-        const float v = src ? raw(src, src_off + n) : 0.f;
-        float o = s * dn - k * v;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int64_t n = lane + 32 * j;
+        if (n >= N) break;
+        float o = s * dnv[j] - k * vv[j];
         if (extra)
             for (int64_t h = 0; h < nh; ++h) o += extra[h * R * N + n];
         dst[n] = o;
