@@ -40,6 +40,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward pass (SISO and MIMO R4) and print its numbers")
+    ap.add_argument("--bwd-seqlen", type=int, default=None,
+                    help="sequence length of the --backward-only workloads (default: theirs)")
     return ap.parse_args()
 
 
@@ -156,6 +160,17 @@ def run_ours(args):
     from state_space_sequence_mamba_b200.inputs import make_config, make_decode
     m3.load_library()
     hbm, tc, peak_kind = peaks()
+    if args.backward_only:
+        out = {"backward": {
+            name: bench_backward(m3, dev, cfg, hbm, world, dist, rank_seed(rank, 11 + cfg),
+                                 reps=args.steps, seqlen=args.bwd_seqlen)
+            for name, cfg in (("siso_b4", 1), ("mimo_r4_b4", 2))}, "peak_hbm_gbs": hbm,
+            "seqlen": args.bwd_seqlen or 2048}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     # two input sets (each > L2) alternate between steps so no step reads the previous
     # step's inputs from L2
@@ -347,11 +362,12 @@ def bwd_bytes(pr) -> int:
     return reads + writes
 
 
-def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5):
+def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None):
     """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1)."""
     import torch
     from state_space_sequence_mamba_b200.inputs import make_config
-    pr = make_config(cfg, device=dev, seed=seed, with_state=True)
+    kw = {} if seqlen is None else {"seqlen": seqlen}
+    pr = make_config(cfg, device=dev, seed=seed, with_state=True, **kw)
     d = pr.dims
     g = torch.Generator(device=dev).manual_seed(seed + 1)
     dy = torch.randn(pr.x.shape, generator=g, device=dev).to(d.dtype)
