@@ -56,6 +56,17 @@ __device__ __forceinline__ float zoh_gamma(float dt, float A) {
     return x != 0.f ? expm1f(x) / A : dt;
 }
 
+// x reduced by a whole number of turns into [-pi, pi]: Cody-Waite reduction with 2*pi split
+// into an exactly representable head and a tail (Cody & Waite, "Software Manual for the
+// Elementary Functions", 1980). Absolute error ~1e-6 for |x| < 1e4.
+__device__ __forceinline__ float reduce_2pi(float x) {
+    constexpr float kInv2Pi = 0.15915494309189535f;
+    constexpr float k2PiHi = 6.28125f;                  // exactly representable head of 2*pi
+    constexpr float k2PiLo = 1.9353071795864769e-3f;    // 2*pi - 6.28125
+    const float k = rintf(x * kInv2Pi);
+    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
+}
+
 // Inclusive prefix sum across the 32 lanes of a warp.
 __device__ __forceinline__ float warp_inclusive_scan(float v) {
     const int lane = threadIdx.x & 31;

@@ -64,6 +64,10 @@ __device__ __forceinline__ void cp4(void* dst, const void* src) {
     const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src));
 }
+__device__ __forceinline__ void cp8(void* dst, const void* src) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src));
+}
 __device__ __forceinline__ void cp_wait_all() {
     asm volatile("cp.async.commit_group;\n" ::);
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
@@ -92,7 +96,8 @@ __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 
 // Shared-memory layout of one chunk (floats). Slot k = 0..T holds token c0 - 1 + k. RAW holds
 // the chunk's inputs as loaded (element size es): B rows (slots 0..T), C, dy and theta rows
-// (slots 1..T at k - 1), x rows (0..T) and the raw dt, A, lam (slots 1..T at k - 1).
+// (slots 1..T at k - 1), x rows (0..T), the raw dt, A, lam (slots 1..T at k - 1) and the RMS
+// scales of B and C (slots 0..T, per rank).
 struct BwdLayout {
     int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, BIAS, RAW, total;
 };
@@ -116,7 +121,7 @@ __host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P, int 
     o = (o + 3) / 4 * 4;
     l.RAW = o;
     o += (S * R * N * es + T * R * N * es + S * R * P * es + T * R * P * es +
-          T * (N / 2) * es + T * 12 + 15) / 16 * 4;
+          T * (N / 2) * es + T * 12 + S * R * 8 + 15) / 16 * 4;
     l.total = (o + 3) / 4 * 4;
     return l;
 }
@@ -148,6 +153,8 @@ struct BwdArgs {
     float* wF;     // [units] <dL/dh_final, h_final>
     float* wsc;    // [units][L][4] db, dg, dy.y, theta.dPhi per token
     float* wprev;  // [units][R][N] gradient of the normalised previous B of the initial state
+    float2* wrs;   // [b,L,G,R] RMS scales of B (x) and C (y); null without the norm
+    float* wrsp;   // [units][R] RMS scale of the initial state's previous B
     int T;
     int nchunks;
 };
@@ -180,64 +187,89 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     char* rTH = rDY + Tm * rowX;
     float* rS = reinterpret_cast<float*>(rTH + Tm * rowT);
 
-    // ---- one batch of asynchronous loads ----
+    float2* rRS = reinterpret_cast<float2*>(rS + Tm * 3 + (Tm * 3 & 1));
+    const bool norm = a.wrs != nullptr;
+
+    // ---- one batch of asynchronous loads (region by region; q = j / v by a float
+    // reciprocal, exact for these small integers) ----
     const char* Bg = static_cast<const char*>(p.B);
     const char* Cg = static_cast<const char*>(p.C);
     const char* xg = static_cast<const char*>(p.x);
     const char* dyg = static_cast<const char*>(a.dy);
     const char* thg = static_cast<const char*>(p.theta);
-    const int vB = rowB / 16, vX = rowX / 16, vT = rowT / 16, vDC = R * N / 4;
-    const int nB = (Tc + 1) * vB, nC = Tc * vB, nX = (Tc + 1) * vX, nDY = Tc * vX;
-    const int nTH = Tc * vT, nDC = read_dc ? Tc * vDC : 0;
-    const int total = nB + nC + nX + nDY + nTH + nDC;
-    for (int e = tid; e < total; e += nth) {
-        int j = e;
-        const void* src = Bg;
-        void* dst;
-        bool valid = true;
-        if (j < nB) {
-            const int k = j / vB, o = (j % vB) * 16;
+    auto divq = [](int j, int v, float inv) { return __float2int_rz((j + 0.5f) * inv); };
+    {
+        const int vB = rowB / 16;
+        const float inv = 1.f / vB;
+        for (int j = tid; j < (2 * Tc + 1) * vB; j += nth) {
+            int k = divq(j, vB, inv);
+            const int o = (j - k * vB) * 16;
+            const bool isC = k > Tc;
+            if (isC) k -= Tc;     // C: slots 1..Tc
             const int64_t t = c0 - 1 + k;
-            if (t >= 0) src = Bg + ((bb * L + t) * p.G + g) * rowB + o;
+            const void* src = Bg;
+            bool valid = true;
+            if (isC) src = Cg + ((bb * L + t) * p.G + g) * rowB + o;
+            else if (t >= 0) src = Bg + ((bb * L + t) * p.G + g) * rowB + o;
             else if (p.prevB0) src = static_cast<const char*>(p.prevB0) + u * rowB + o;
             else valid = false;
-            dst = rB + k * rowB + o;
-        } else if ((j -= nB) < nC) {
-            const int k = 1 + j / vB, o = (j % vB) * 16;
-            src = Cg + ((bb * L + c0 - 1 + k) * p.G + g) * rowB + o;
-            dst = rC + (k - 1) * rowB + o;
-        } else if ((j -= nC) < nX) {
-            const int k = j / vX, o = (j % vX) * 16;
+            cp16(isC ? rC + (k - 1) * rowB + o : rB + k * rowB + o, src, valid);
+        }
+    }
+    {
+        const int vX = rowX / 16;
+        const float inv = 1.f / vX;
+        for (int j = tid; j < (2 * Tc + 1) * vX; j += nth) {
+            int k = divq(j, vX, inv);
+            const int o = (j - k * vX) * 16;
+            const bool isDY = k > Tc;
+            if (isDY) k -= Tc;    // dy: slots 1..Tc
             const int64_t t = c0 - 1 + k;
-            if (t >= 0) src = xg + ((bb * L + t) * H + hh) * rowX + o;
+            const void* src = xg;
+            bool valid = true;
+            if (isDY) src = dyg + ((bb * L + t) * H + hh) * rowX + o;
+            else if (t >= 0) src = xg + ((bb * L + t) * H + hh) * rowX + o;
             else if (p.prevx0) src = static_cast<const char*>(p.prevx0) + u * rowX + o;
             else valid = false;
-            dst = rX + k * rowX + o;
-        } else if ((j -= nX) < nDY) {
-            const int k = 1 + j / vX, o = (j % vX) * 16;
-            src = dyg + ((bb * L + c0 - 1 + k) * H + hh) * rowX + o;
-            dst = rDY + (k - 1) * rowX + o;
-        } else if ((j -= nDY) < nTH) {
-            const int k = 1 + j / vT, o = (j % vT) * 16;
-            src = thg + ((bb * L + c0 - 1 + k) * H + hh) * rowT + o;
-            dst = rTH + (k - 1) * rowT + o;
-        } else {
-            j -= nTH;
-            const int k = 1 + j / vDC, o = (j % vDC) * 4;
-            src = a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o;
-            dst = sm + lay.DC + k * R * N + o;
+            cp16(isDY ? rDY + (k - 1) * rowX + o : rX + k * rowX + o, src, valid);
         }
-        cp16(dst, src, valid);
+    }
+    {
+        const int vT = rowT / 16;
+        const float inv = 1.f / vT;
+        for (int j = tid; j < Tc * vT; j += nth) {
+            const int k = 1 + divq(j, vT, inv);
+            const int o = (j - (k - 1) * vT) * 16;
+            cp16(rTH + (k - 1) * rowT + o, thg + ((bb * L + c0 - 1 + k) * H + hh) * rowT + o, true);
+        }
+    }
+    if (read_dc) {
+        const int vDC = R * N / 4;
+        const float inv = 1.f / vDC;
+        for (int j = tid; j < Tc * vDC; j += nth) {
+            const int k = 1 + divq(j, vDC, inv);
+            const int o = (j - (k - 1) * vDC) * 4;
+            cp16(sm + lay.DC + k * R * N + o,
+                 a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o, true);
+        }
     }
     for (int e = tid; e < 3 * Tc; e += nth) {
-        const int k = 1 + e / 3, w = e % 3;
+        const int k = 1 + e / 3, w = e - 3 * (e / 3);
         const int64_t si = (bb * L + c0 - 1 + k) * H + hh;
         cp4(rS + (k - 1) * 3 + w, (w == 0 ? p.dt : w == 1 ? p.A : p.lam) + si);
+    }
+    if (norm) {
+        for (int e = tid; e < (Tc + 1) * R; e += nth) {
+            const int k = e / R, r = e - k * R;
+            const int64_t t = c0 - 1 + k;
+            if (t >= 0) cp8(rRS + e, a.wrs + ((bb * L + t) * p.G + g) * R + r);
+            else cp4(rRS + e, a.wrsp + u * R + r);
+        }
     }
     cp_wait_all();
     __syncthreads();
 
-    // ---- step scalars; x and dy to fp32 ----
+    // ---- step scalars; x, dy and theta to fp32 ----
     const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
     for (int k = 1 + tid; k <= Tc; k += nth) {
         const float d = step_dt(rS[(k - 1) * 3], dtb, p.flags), A = rS[(k - 1) * 3 + 1];
@@ -262,13 +294,14 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     }
     __syncthreads();
 
-    // ---- angles: the four lanes of a pair's quad walk a quarter of the chunk each ----
+    // ---- angles: the four lanes of a pair's quad walk a quarter of the chunk each, from the
+    // chunk-start angle reduced into [-pi, pi], so the hardware sine and cosine stay accurate ----
     {
         const int i = tid >> 2, q = tid & 3;
         const int nk = (Tc + 3) >> 2;
         const int klo = 1 + q * nk, khi = min(Tc, klo + nk - 1);
         const float* th = sm + lay.TH;
-        const float ph0 = phi_start[i];
+        const float ph0 = reduce_2pi(phi_start[i]);
         float loc = 0.f;
         for (int k = klo; k <= khi; ++k) loc = fmaf(scal[8 * k], th[k * half + i], loc);
         const float e1 = __shfl_up_sync(kFull, loc, 1, 4);
@@ -277,43 +310,80 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
         float ph = ph0 + ((q >= 1 ? e1 : 0.f) + (q >= 2 ? e2 : 0.f) + (q >= 3 ? e3 : 0.f));
         float sn, cn;
         if (q == 0) {
-            sincosf(ph0, &sn, &cn);
+            __sincosf(ph0, &sn, &cn);
             cs[i] = cn; cs[half + i] = sn;
         }
         for (int k = klo; k <= khi; ++k) {
             ph = fmaf(scal[8 * k], th[k * half + i], ph);
-            sincosf(ph, &sn, &cn);
+            __sincosf(ph, &sn, &cn);
             cs[k * N + i] = cn; cs[k * N + half + i] = sn;
         }
         if (phi_end && klo <= khi && khi == Tc) phi_end[i] = ph;
     }
     __syncthreads();
 
-    // ---- rotated, normalised, biased B (slots 0..Tc) and C (1..Tc): one warp per vector ----
-    const int nitems = (2 * Tc + 1) * R;
-    for (int it = warp; it < nitems; it += nwarps) {
-        const bool isC = it >= (Tc + 1) * R;
-        const int j = isC ? it - (Tc + 1) * R : it;
-        const int k = isC ? 1 + j / R : j / R, r = j % R;
-        const T* src = reinterpret_cast<const T*>(isC ? rC + (k - 1) * rowB : rB + k * rowB) + r * N;
-        const float* bias = sm + lay.BIAS + (isC ? R * N : 0) + r * N;
-        float ss = 0.f;
-        for (int i = lane; i < half; i += 32) {
-            const float v0 = to_f(src[i]), v1 = to_f(src[i + half]);
-            ss = fmaf(v0, v0, fmaf(v1, v1, ss));
-        }
-        ss = warp_sum(ss);
-        const float scale = p.bc_norm ? rsqrtf(ss / static_cast<float>(N) + p.eps) : 1.f;
-        float* dst = sm + (isC ? lay.C : lay.B) + (k * R + r) * N;
-        for (int i = lane; i < half; i += 32) {
+    // ---- rotated, normalised, biased B (slots 0..Tc) and C (1..Tc): one thread per pair ----
+    {
+        const int RH = R * half;
+        const float inv = 1.f / RH, invh = 1.f / half;
+        const int nBp = (Tc + 1) * RH;
+        for (int e = tid; e < nBp + Tc * RH; e += nth) {
+            const bool isC = e >= nBp;
+            const int j = isC ? e - nBp : e;
+            const int kk = divq(j, RH, inv);
+            const int rem = j - kk * RH;
+            const int r = divq(rem, half, invh), i = rem - r * half;
+            const int k = isC ? kk + 1 : kk;
+            const T* src = reinterpret_cast<const T*>(isC ? rC + (k - 1) * rowB : rB + k * rowB) + r * N;
+            const float* bias = sm + lay.BIAS + (isC ? R * N : 0) + r * N;
+            const float scale = norm ? (isC ? rRS[k * R + r].y : rRS[k * R + r].x) : 1.f;
             const float v0 = to_f(src[i]) * scale + bias[i];
             const float v1 = to_f(src[i + half]) * scale + bias[i + half];
-            const float c = cs[k * N + i], s = cs[k * N + half + i];
-            dst[i] = v0 * c + v1 * s;
-            dst[i + half] = v1 * c - v0 * s;
+            const float c = cs[k * N + i], sn = cs[k * N + half + i];
+            float* dst = sm + (isC ? lay.C : lay.B) + (k * R + r) * N;
+            dst[i] = v0 * c + v1 * sn;
+            dst[i + half] = v1 * c - v0 * sn;
         }
     }
     __syncthreads();
+}
+
+// RMS scales of every B and C row (one warp per (b, t, g, r), both vectors) and of the
+// initial state's previous B (one warp per (unit, r)): 1 / sqrt(mean(v^2) + eps).
+__global__ void __launch_bounds__(256) bwd_rms_kernel(const BwdArgs a, int bf16) {
+    const ScanParams& p = a.f;
+    const int64_t N = p.N;
+    const int lane = threadIdx.x & 31;
+    const int64_t item = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nrow = p.b * p.L * p.G * p.R, nprev = p.b * p.H * p.R;
+    if (item >= nrow + nprev) return;
+    auto ld = [&](const void* base, int64_t off) {
+        return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(base)[off])
+                    : static_cast<const float*>(base)[off];
+    };
+    if (item < nrow) {
+        float sb = 0.f, sc = 0.f;
+        for (int64_t n = lane; n < N; n += 32) {
+            const float vb = ld(p.B, item * N + n), vc = ld(p.C, item * N + n);
+            sb = fmaf(vb, vb, sb);
+            sc = fmaf(vc, vc, sc);
+        }
+        sb = warp_sum(sb);
+        sc = warp_sum(sc);
+        if (lane == 0)
+            a.wrs[item] = make_float2(rsqrtf(sb / static_cast<float>(N) + p.eps),
+                                      rsqrtf(sc / static_cast<float>(N) + p.eps));
+    } else {
+        const int64_t j = item - nrow;
+        float sb = 0.f;
+        if (p.prevB0)
+            for (int64_t n = lane; n < N; n += 32) {
+                const float v = ld(p.prevB0, j * N + n);
+                sb = fmaf(v, v, sb);
+            }
+        sb = warp_sum(sb);
+        if (lane == 0) a.wrsp[j] = rsqrtf(sb / static_cast<float>(N) + p.eps);
+    }
 }
 
 // Loads this head's B and C biases into shared memory (zeros when absent).
@@ -1046,7 +1116,8 @@ size_t scan_bwd_workspace_floats(int64_t b, int64_t L, int64_t H, int64_t N, int
     const int64_t T = bwd_chunk_tokens(R), nch = (L + T - 1) / T, units = b * H;
     auto r64 = [](int64_t v) { return (v + 63) / 64 * 64; };   // 256-byte regions
     return static_cast<size_t>(2 * r64(b * L * H * R * N) + r64(units * nch * (N / 2)) +
-                               r64(units) + r64(units * L * 4) + r64(units * R * N));
+                               r64(units) + r64(units * L * 4) + r64(units * R * N) +
+                               r64(2 * b * L * H * R) + r64(units * R));
 }
 
 cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, float* ws,
@@ -1069,7 +1140,12 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
     a.wphi = o; o += r64(units * nch * (f.N / 2));
     a.wF = o; o += r64(units);
     a.wsc = o; o += r64(units * f.L * 4);
-    a.wprev = o;
+    a.wprev = o; o += r64(units * f.R * f.N);
+    if (f.bc_norm) {
+        a.wrs = reinterpret_cast<float2*>(o);   // G <= H rows: the [b,L,H,R] region holds them
+        o += r64(2 * f.b * f.L * f.H * f.R);
+        a.wrsp = o;
+    }
 
     cudaError_t e;
     if (a.dBbias && (e = cudaMemsetAsync(a.dBbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
@@ -1078,6 +1154,11 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
     const BwdLayout lay = bwd_layout(a.T, static_cast<int>(f.R), static_cast<int>(f.N),
                                      static_cast<int>(f.P), bf16 ? 2 : 4);
     const size_t smem = sizeof(float) * lay.total;
+    if (f.bc_norm) {
+        const int64_t items = f.b * f.L * f.G * f.R + units * f.R;
+        bwd_rms_kernel<<<static_cast<unsigned>((items * 32 + 255) / 256), 256, 0, s>>>(a, bf16 ? 1 : 0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (f.N <= 128)
         e = bf16 ? launch_sweeps_p<__nv_bfloat16, 256>(a, smem, s)
                  : launch_sweeps_p<float, 256>(a, smem, s);

@@ -88,17 +88,6 @@ __host__ __device__ constexpr uint32_t tc_smem_bytes() {
     return TcCfg<R>::OF + 4u * F_BIAS + 2u * 2 * R * kN + 1024u;
 }
 
-// x reduced by a whole number of turns into [-pi, pi]: Cody-Waite reduction with 2*pi split
-// into an exactly representable head and a tail (Cody & Waite, "Software Manual for the
-// Elementary Functions", 1980). Absolute error ~1e-6 for |x| < 1e4.
-__device__ __forceinline__ float reduce_2pi(float x) {
-    constexpr float kInv2Pi = 0.15915494309189535f;
-    constexpr float k2PiHi = 6.28125f;                  // exactly representable head of 2*pi
-    constexpr float k2PiLo = 1.9353071795864769e-3f;    // 2*pi - 6.28125
-    const float k = rintf(x * kInv2Pi);
-    return fmaf(-k, k2PiLo, fmaf(-k, k2PiHi, x));
-}
-
 // 2^x by the hardware approximation (relative error ~2^-22), x <= 0 here.
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;

@@ -122,7 +122,7 @@ def test_backward_workspace_and_argument_checks(lib):
     r64 = lambda v: (v + 63) // 64 * 64
     units, nch = 2 * 4, (100 + T - 1) // T
     want = 4 * (2 * r64(2 * 100 * 4 * 128) + r64(units * nch * 64) + r64(units)
-                + r64(units * 100 * 4) + r64(units * 128))
+                + r64(units * 100 * 4) + r64(units * 128) + r64(2 * 2 * 100 * 4) + r64(units))
     assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d)) == want
     assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
     assert ctypes.sizeof(bd.Grads) == 10 * 8
