@@ -99,7 +99,7 @@ __device__ __forceinline__ float2 dup2(float v) { return make_float2(v, v); }
 // (slots 1..T at k - 1), x rows (0..T), the raw dt, A, lam (slots 1..T at k - 1) and the RMS
 // scales of B and C (slots 0..T, per rank).
 struct BwdLayout {
-    int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, BIAS, RAW, total;
+    int B, C, X, DY, CS, TH, DC, DB, DX, DTH, SC, SCAL, BIAS, RAW, RDC, RPHI, total;
 };
 __host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P, int es) {
     BwdLayout l{};
@@ -122,6 +122,8 @@ __host__ __device__ inline BwdLayout bwd_layout(int T, int R, int N, int P, int 
     l.RAW = o;
     o += (S * R * N * es + T * R * N * es + S * R * P * es + T * R * P * es +
           T * (N / 2) * es + T * 12 + S * R * 8 + 15) / 16 * 4;
+    l.RDC = o; o += T * R * N;    // the reverse sweep's dCbar rows as loaded (slots 1..T)
+    l.RPHI = o; o += N / 2;       // the reverse sweep's chunk-start angle as loaded
     l.total = (o + 3) / 4 * 4;
     return l;
 }
@@ -159,15 +161,10 @@ struct BwdArgs {
     int nchunks;
 };
 
-// Stages the chunk [c0, c0 + Tc) into shared memory: step scalars, angles (continuing from
-// phi_start = the angle before token c0; the angle after the chunk goes to phi_end when it is
-// set), rotated B (slots 0..Tc) and C (1..Tc), x (0..Tc), dy (1..Tc), and the forward sweep's
-// dCbar rows when read_dc. Slot 0 is token c0 - 1: the initial state's previous token when
-// c0 = 0. Every global load of the chunk is in flight at once (cp.async); the rest works on
-// shared memory.
+// Issues every global load of chunk c (cp.async into the RAW, RDC and RPHI areas) as one
+// commit group, without waiting: the loads of the next chunk fly while this one computes.
 template <typename T>
-__device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, int64_t u,
-                            int64_t c0, int Tc, const float* phi_start, float* phi_end,
+__device__ void issue_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, int64_t u, int c,
                             bool read_dc) {
     constexpr int es = sizeof(T);
     const ScanParams& p = a.f;
@@ -177,8 +174,6 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     const int64_t bb = u / H, hh = u % H, g = hh / (H / p.G);
     const int tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
     const int nwarps = nth >> 5;
-    float* scal = sm + lay.SCAL;
-    float* cs = sm + lay.CS;
     const int rowB = R * N * es, rowX = R * P * es, rowT = half * es;   // bytes
     char* rB = reinterpret_cast<char*>(sm + lay.RAW);
     char* rC = rB + (Tm + 1) * rowB;
@@ -190,6 +185,9 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     float2* rRS = reinterpret_cast<float2*>(rS + Tm * 3 + (Tm * 3 & 1));
     const bool norm = a.wrs != nullptr;
 
+    const int64_t c0 = static_cast<int64_t>(c) * Tm;
+    const int Tc = static_cast<int>(L - c0 < Tm ? L - c0 : Tm);
+    (void)warp; (void)lane; (void)nwarps;
     // ---- one batch of asynchronous loads (region by region; q = j / v by a float
     // reciprocal, exact for these small integers) ----
     const char* Bg = static_cast<const char*>(p.B);
@@ -244,12 +242,14 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
         }
     }
     if (read_dc) {
+        for (int j = tid; j < half / 4; j += nth)
+            cp16(sm + lay.RPHI + 4 * j, a.wphi + (u * a.nchunks + c) * half + 4 * j, true);
         const int vDC = R * N / 4;
         const float inv = 1.f / vDC;
         for (int j = tid; j < Tc * vDC; j += nth) {
             const int k = 1 + divq(j, vDC, inv);
             const int o = (j - (k - 1) * vDC) * 4;
-            cp16(sm + lay.DC + k * R * N + o,
+            cp16(sm + lay.RDC + (k - 1) * R * N + o,
                  a.wdC + ((bb * L + c0 - 1 + k) * H + hh) * R * N + o, true);
         }
     }
@@ -266,8 +266,47 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
             else cp4(rRS + e, a.wrsp + u * R + r);
         }
     }
-    cp_wait_all();
+    asm volatile("cp.async.commit_group;\n" ::);
+}
+
+// Stages the chunk [c0, c0 + Tc) into shared memory from what issue_chunk loaded: step
+// scalars, angles (continuing from phi_start = the angle before token c0; the angle after the
+// chunk goes to phi_end when it is set), rotated B (slots 0..Tc) and C (1..Tc), x (0..Tc),
+// dy (1..Tc), and the forward sweep's dCbar rows when read_dc. Slot 0 is token c0 - 1: the
+// initial state's previous token when c0 = 0.
+template <typename T>
+__device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, int64_t u,
+                            int64_t c0, int Tc, const float* phi_start, float* phi_end,
+                            bool read_dc) {
+    constexpr int es = sizeof(T);
+    const ScanParams& p = a.f;
+    const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
+    const int half = N / 2, Tm = a.T;
+    const int64_t L = p.L, H = p.H;
+    const int64_t bb = u / H, hh = u % H, g = hh / (H / p.G);
+    const int tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
+    const int nwarps = nth >> 5;
+    float* scal = sm + lay.SCAL;
+    float* cs = sm + lay.CS;
+    const int rowB = R * N * es, rowX = R * P * es, rowT = half * es;   // bytes
+    char* rB = reinterpret_cast<char*>(sm + lay.RAW);
+    char* rC = rB + (Tm + 1) * rowB;
+    char* rX = rC + Tm * rowB;
+    char* rDY = rX + (Tm + 1) * rowX;
+    char* rTH = rDY + Tm * rowX;
+    float* rS = reinterpret_cast<float*>(rTH + Tm * rowT);
+
+    float2* rRS = reinterpret_cast<float2*>(rS + Tm * 3 + (Tm * 3 & 1));
+    const bool norm = a.wrs != nullptr;
+
+    auto divq = [](int j, int v, float inv) { return __float2int_rz((j + 0.5f) * inv); };
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
+    if (read_dc) {
+        const float4* src = reinterpret_cast<const float4*>(sm + lay.RDC);
+        float4* dst = reinterpret_cast<float4*>(sm + lay.DC + R * N);
+        for (int e = tid; e < Tc * R * N / 4; e += nth) dst[e] = src[e];
+    }
 
     // ---- step scalars; x, dy and theta to fp32 ----
     const float dtb = p.dt_bias ? p.dt_bias[hh] : 0.f;
@@ -487,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_fwd_ker
     }
     for (int e = tid; e < half; e += blockDim.x) phi_run[e] = p.phi0 ? p.phi0[u * half + e] : 0.f;
     load_bias(a, lay, sm, hh);
+    issue_chunk<T>(a, lay, sm, u, 0, false);
     __syncthreads();
 
     for (int c = 0; c < a.nchunks; ++c) {
@@ -495,6 +535,7 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_fwd_ker
         for (int e = tid; e < half; e += blockDim.x)
             a.wphi[(u * a.nchunks + c) * half + e] = phi_run[e];
         stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_run, phi_next, false);
+        if (c + 1 < a.nchunks) issue_chunk<T>(a, lay, sm, u, c + 1, false);
         const float* sB = sm + lay.B;
         const float* sX = sm + lay.X;
         const float* sDY = sm + lay.DY;
@@ -597,7 +638,6 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
     const int tid = threadIdx.x, lane = tid & 31;
     const int i = tid >> 2, q = tid & 3;
     const BwdLayout lay = bwd_layout(a.T, R, N, P, sizeof(T));
-    __shared__ float phi_start[128];
     __shared__ float pend[4];
 
     float G0[CPQ], G1[CPQ];
@@ -625,13 +665,13 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
     for (int c = a.nchunks - 1; c >= 0; --c) {
         const int64_t c0 = static_cast<int64_t>(c) * a.T;
         const int Tc = static_cast<int>(L - c0 < a.T ? L - c0 : a.T);
-        for (int e = tid; e < half; e += blockDim.x)
-            phi_start[e] = a.wphi[(u * a.nchunks + c) * half + e];
+        if (c == a.nchunks - 1) issue_chunk<T>(a, lay, sm, u, c, true);
         for (int e = tid; e < (Tc + 1) * R * P; e += blockDim.x) sDX[e] = 0.f;
         for (int e = tid; e < (a.T + 2) * 4; e += blockDim.x) sSC[e] = 0.f;
         if (c == a.nchunks - 1) load_bias(a, lay, sm, hh);
         __syncthreads();
-        stage_chunk<T>(a, lay, sm, u, c0, Tc, phi_start, nullptr, true);
+        stage_chunk<T>(a, lay, sm, u, c0, Tc, sm + lay.RPHI, nullptr, true);
+        if (c > 0) issue_chunk<T>(a, lay, sm, u, c - 1, true);
 
         for (int k = Tc; k >= 1; --k) {
             const float* s = sm + lay.SCAL + 8 * k;
