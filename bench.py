@@ -393,7 +393,7 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None):
     byts = bwd_bytes(pr)
     out = {"ms_per_backward": ms, "tokens_per_s": d.batch * d.seqlen * world / (ms / 1e3),
            "bytes": byts, "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
-           "kernels_per_call": 4, "workspace_bytes": ws.numel()}
+           "kernels_per_call": 5 if d.bc_norm else 4, "workspace_bytes": ws.numel()}
     del pr, dy, init, ws
     torch.cuda.empty_cache()
     return out

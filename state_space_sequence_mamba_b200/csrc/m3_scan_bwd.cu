@@ -23,10 +23,12 @@
 //
 // Thread layout of the sweeps: one CTA per unit with 2N threads; thread = (pair i, quarter q)
 // owns the rows i and i + N/2 (one complex pair, so the rotation is thread-local) and the
-// P/4 columns q*P/4 .. of h or G in registers. Contractions over P finish with two shuffles
-// inside the quad; contractions over N with a butterfly across the warp's eight pairs and a
-// shared-memory add across warps. A chunk of T tokens is staged in shared memory (rotated B and
-// C, x, dy, cos/sin, scalars) before the sequential token loop, so the loop has no barrier.
+// P/4 columns of h or G in registers (16-byte groups interleaved across the quad). Contractions
+// over P finish with two shuffles inside the quad; contractions over N with a butterfly across
+// the warp's eight pairs and a shared-memory add across warps. A chunk of T tokens is staged in
+// shared memory (rotated B and C, x, dy, cos/sin, scalars) before the sequential token loop,
+// so the loop has no barrier; the next chunk's global loads (cp.async) fly during the loop.
+// bwd_rms_kernel computes the RMS scales of all B and C rows once, before the sweeps.
 #include <cuda_bf16.h>
 
 #include "m3_common.cuh"
@@ -37,24 +39,8 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-template <typename T>
-__device__ __forceinline__ float4 ld4(const T* p);
-template <>
-__device__ __forceinline__ float4 ld4<float>(const float* p) {
-    return *reinterpret_cast<const float4*>(p);
-}
-template <>
-__device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    __nv_bfloat162 lo, hi;
-    memcpy(&lo, &v.x, 4);
-    memcpy(&hi, &v.y, 4);
-    const float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
-    return make_float4(a.x, a.y, b.x, b.y);
-}
-
-// Asynchronous 16-byte and 4-byte global -> shared copies (sm_80+ cp.async); a 16-byte copy
-// with valid = false writes zeros and reads nothing.
+// Asynchronous 16-, 8- and 4-byte global -> shared copies (cp.async); a 16-byte copy with
+// valid = false writes zeros and reads nothing.
 __device__ __forceinline__ void cp16(void* dst, const void* src, bool valid) {
     const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src),
@@ -67,10 +53,6 @@ __device__ __forceinline__ void cp4(void* dst, const void* src) {
 __device__ __forceinline__ void cp8(void* dst, const void* src) {
     const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src));
-}
-__device__ __forceinline__ void cp_wait_all() {
-    asm volatile("cp.async.commit_group;\n" ::);
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
 }
 
 // Two-lane fp32 arithmetic of sm_100 (one packed instruction for two columns):
