@@ -2,9 +2,9 @@
 
 Both sides take the same stored inputs (bf16 inputs are compared after the same rounding),
 so the only difference is the kernels' fp32 arithmetic. Tolerance: for every gradient tensor
-max|gpu - oracle| / max|oracle| <= 2e-3. The bound allows for fp32 sums over L tokens and
-over N * P, and the decay gradient's suffix sum over the sequence; the measured errors are
-recorded (M3_PARITY_REPORT).
+max|gpu - oracle| / max|oracle| <= 1e-4, the bound of the fp32 forward. fp32 sums over L
+tokens and over N * P, and the decay gradient's suffix sum over the sequence, stay near
+1e-6 relative even at L = 2048; the measured errors are recorded (M3_PARITY_REPORT).
 """
 import numpy as np
 import pytest
@@ -18,7 +18,7 @@ from state_space_sequence_mamba_b200.inputs import make_config, make_problem
 
 pytestmark = pytest.mark.gpu
 
-GTOL = 2e-3
+GTOL = 1e-4
 KEYS = ("dx", "dB", "dC", "dtheta", "ddt", "dA", "dlam", "dB_bias", "dC_bias", "ddt_bias")
 PER_HEAD = ("dx", "dtheta", "ddt", "dA", "dlam")
 
@@ -129,6 +129,18 @@ def test_backward_short_sequences(cuda_dev, L):
     dy, _ = draw_grads(pr, seed=L, with_final=False)
     got = gpu_grads(pr, dy, None, cuda_dev)
     compare_grads(got, oracle_grads(pr, dy, None))
+
+
+def test_backward_partial_final_gradient(cuda_dev):
+    """Only the final h has a gradient (NULL phi, prev_B, prev_x count as zero)."""
+    pr = make_problem(2, 40, 2, 1, 64, 128, rank=1, dtype=torch.bfloat16, bc_norm=True,
+                      bias_std=0.1, seed=77, with_state=True, raw_scalars=True)
+    dy, dfin = draw_grads(pr, seed=3)
+    part = {"h": dfin["h"]}
+    got = gpu_grads(pr, dy, part, cuda_dev)
+    zero = {k: torch.zeros_like(v) for k, v in dfin.items()}
+    zero["h"] = dfin["h"]
+    compare_grads(got, oracle_grads(pr, dy, zero))
 
 
 def test_backward_empty_sequence_passes_final_gradient_through(cuda_dev):
