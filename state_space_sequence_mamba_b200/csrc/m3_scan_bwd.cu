@@ -264,10 +264,8 @@ __device__ void stage_chunk(const BwdArgs& a, const BwdLayout& lay, float* sm, i
     const ScanParams& p = a.f;
     const int N = static_cast<int>(p.N), P = static_cast<int>(p.P), R = static_cast<int>(p.R);
     const int half = N / 2, Tm = a.T;
-    const int64_t L = p.L, H = p.H;
-    const int64_t bb = u / H, hh = u % H, g = hh / (H / p.G);
-    const int tid = threadIdx.x, nth = blockDim.x, warp = tid >> 5, lane = tid & 31;
-    const int nwarps = nth >> 5;
+    const int64_t hh = u % p.H;
+    const int tid = threadIdx.x, nth = blockDim.x;
     float* scal = sm + lay.SCAL;
     float* cs = sm + lay.CS;
     const int rowB = R * N * es, rowX = R * P * es, rowT = half * es;   // bytes
@@ -914,18 +912,18 @@ __global__ void __launch_bounds__(kThreads, kThreads <= 256 ? 2 : 1) bwd_rev_ker
             atomicAdd(a.dCbias + hh * N + i, accC[0][0]);
             atomicAdd(a.dCbias + hh * N + i + half, accC[0][1]);
         }
-        return;
-    }
-    for (int rr = 0; rr < 2; ++rr) {
-        const int r = q + 4 * rr;
-        if (r >= R) break;
-        if (a.dBbias) {
-            atomicAdd(a.dBbias + (hh * R + r) * N + i, accB[rr][0]);
-            atomicAdd(a.dBbias + (hh * R + r) * N + i + half, accB[rr][1]);
-        }
-        if (a.dCbias) {
-            atomicAdd(a.dCbias + (hh * R + r) * N + i, accC[rr][0]);
-            atomicAdd(a.dCbias + (hh * R + r) * N + i + half, accC[rr][1]);
+    } else {
+        for (int rr = 0; rr < 2; ++rr) {
+            const int r = q + 4 * rr;
+            if (r >= R) break;
+            if (a.dBbias) {
+                atomicAdd(a.dBbias + (hh * R + r) * N + i, accB[rr][0]);
+                atomicAdd(a.dBbias + (hh * R + r) * N + i + half, accB[rr][1]);
+            }
+            if (a.dCbias) {
+                atomicAdd(a.dCbias + (hh * R + r) * N + i, accC[rr][0]);
+                atomicAdd(a.dCbias + (hh * R + r) * N + i + half, accC[rr][1]);
+            }
         }
     }
 }
