@@ -227,7 +227,8 @@ M3_API size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims);
  * (16-byte aligned) and overwritten; the bias gradients are overwritten when not NULL.
  * dinit: where to write the initial state's gradient, or NULL. workspace: 256-byte aligned,
  * at least m3_scan_bwd_workspace_bytes. Any supported N, P, R, dtype and flags; asynchronous
- * on `stream`. */
+ * on `stream`. Not bitwise reproducible run to run: some sums use atomic adds, whose order
+ * varies in the last bits (m3_scan_fwd and the decode step are reproducible). */
 M3_API m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
                              const void* dy, const m3_state_grad* dfinal,
                              const m3_grads* grads, const m3_state_grad* dinit,

@@ -29,6 +29,11 @@
 // shared memory (rotated B and C, x, dy, cos/sin, scalars) before the sequential token loop,
 // so the loop has no barrier; the next chunk's global loads (cp.async) fly during the loop.
 // bwd_rms_kernel computes the RMS scales of all B and C rows once, before the sweeps.
+//
+// Summation order: the cross-warp sums of dx and of the per-token scalar partials are
+// shared-memory atomic adds, and the bias and dt_bias sums over units are global atomic
+// adds, so the gradients are not bitwise reproducible run to run (they differ in the last
+// bits; the forward scan and the decode step are reproducible).
 #include <cuda_bf16.h>
 
 #include "m3_common.cuh"
