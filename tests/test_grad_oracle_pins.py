@@ -7,6 +7,9 @@
    the norm, the biases, MIMO rank, shared groups, a nonzero initial state and each flag
    (raw step and trapezoid scalars, zero-order hold) switched on. A dropped term, a wrong
    sign or a transposed operand anywhere in the backward fails here.
+3. In the real Euler case (no rotation, lam = 1, no norm or bias) the gradients of x, C and
+   A have closed forms as explicit sums over token pairs, checked without autograd or
+   finite differences.
 
 Page references are to "Mamba-3: Improved Sequence Modeling using State Space Principles".
 """
@@ -124,3 +127,42 @@ def test_gradient_equals_finite_differences_of_c_oracle(flags, bc_norm, R, G, H)
     assert checked > 100
     if flags & oracle.DISC_ZOH:   # lam is not used under the zero-order hold
         assert not np.any(g["dlam"])
+
+
+def test_gradient_closed_form_real_euler_case():
+    """theta = 0, lam = 1 (exponential Euler), no norm, no bias, R = 1, zero initial state:
+    y_t = sum_{s<=t} (prod_{k=s+1..t} alpha_k) dt_s (C_t . B_s) x_s (Sec. 3.1.1 with lam = 1 is
+    the Mamba-2 recurrence). Then, with K(t,s) = prod_{k=s+1..t} alpha_k dt_s,
+        dx_s = sum_{t>=s} K(t,s) (C_t . B_s) dy_t,
+        dC_t = sum_{s<=t} K(t,s) (x_s . dy_t) B_s,
+        dA_k = sum_{s<k<=t} dt_k K(t,s) (C_t . B_s)(x_s . dy_t),
+    written out here as explicit sums (no autograd, no finite differences)."""
+    rng = np.random.default_rng(5)
+    b, L, H, P, N = 1, 7, 1, 3, 4
+    x = rng.standard_normal((b, L, H, 1, P))
+    B = rng.standard_normal((b, L, 1, 1, N))
+    C = rng.standard_normal((b, L, 1, 1, N))
+    dt = np.log1p(np.exp(rng.standard_normal((b, L, H)) - 1.0))
+    A = -np.exp(rng.uniform(-1, 1, (b, L, H)))
+    dy = rng.standard_normal((b, L, H, 1, P))
+    g = og.scan_grad(x, B, C, np.zeros((b, L, H, N // 2)), dt, A, np.ones((b, L, H)),
+                     dy=dy)
+    al = np.exp(dt[0, :, 0] * A[0, :, 0])
+    xs, Bs, Cs, dys, d = x[0, :, 0, 0], B[0, :, 0, 0], C[0, :, 0, 0], dy[0, :, 0, 0], dt[0, :, 0]
+
+    def K(t, s):
+        return np.prod(al[s + 1:t + 1]) * d[s]
+
+    dx = np.zeros((L, P))
+    dC = np.zeros((L, N))
+    dA = np.zeros(L)
+    for t in range(L):
+        for s in range(t + 1):
+            cb, xd = Cs[t] @ Bs[s], xs[s] @ dys[t]
+            dx[s] += K(t, s) * cb * dys[t]
+            dC[t] += K(t, s) * xd * Bs[s]
+            for k in range(s + 1, t + 1):
+                dA[k] += d[k] * K(t, s) * cb * xd
+    np.testing.assert_allclose(g["dx"][0, :, 0, 0], dx, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dC"][0, :, 0, 0], dC, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dA"][0, :, 0], dA, rtol=1e-12, atol=1e-12)
