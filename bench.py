@@ -332,7 +332,8 @@ def run_ours(args):
     backward = {}
     if not args.no_decode:
         backward["siso_b4_L2048"] = bench_backward(m3, dev, 1, hbm, world, dist,
-                                                   rank_seed(rank, 11))
+                                                   rank_seed(rank, 11),
+                                                   cpu=(rank == 0 and world == 1))
         backward["mimo_r4_b4_L2048"] = bench_backward(m3, dev, 2, hbm, world, dist,
                                                       rank_seed(rank, 12))
 
@@ -384,7 +385,7 @@ def bwd_bytes(pr) -> int:
     return reads + writes
 
 
-def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None):
+def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cpu=False):
     """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1)."""
     import torch
     from state_space_sequence_mamba_b200.inputs import make_config
@@ -416,6 +417,11 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None):
     out = {"ms_per_backward": ms, "tokens_per_s": d.batch * d.seqlen * world / (ms / 1e3),
            "bytes": byts, "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
            "kernels_per_call": 5 if d.bc_norm else 4, "workspace_bytes": ws.numel()}
+    if cpu:   # an auxiliary field: a failure here is reported, not fatal to the bench line
+        try:
+            out["cpu_baseline"] = cpu_baseline_backward(pr, dy)
+        except Exception as e:  # noqa: BLE001
+            out["cpu_baseline"] = {"error": f"{type(e).__name__}: {e}"[:200]}
     del pr, dy, init, ws
     torch.cuda.empty_cache()
     return out
@@ -496,6 +502,37 @@ def cpu_baseline(pr, min_s=10.0, max_reps=30):
     return {"value": tokens / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"the whole workload ({pr.dims.batch} sequences x {pr.dims.nheads} heads x "
                       f"L={pr.dims.seqlen}) x {reps} passes, {el:.1f} s"}
+
+
+def cpu_baseline_backward(pr, dy, heads=8):
+    """The gradient oracle (float64 autograd of the plain recurrence) as it stands, on the host
+    cores, on a bounded sample of a backward workload: sequence 0 and its first `heads` heads,
+    every token. The rate counts the sample as that fraction of the workload's tokens."""
+    import torch
+    import oracle
+    from oracle import grad as og
+    hs = torch.arange(heads)
+    t = {}
+    for k, v in pr.tensors().items():
+        if v is None:
+            t[k] = None
+        elif k in ("x", "theta", "dt", "A", "lam"):
+            t[k] = v[:1, :, hs].cpu()
+        elif k in ("B_bias", "C_bias"):
+            t[k] = v[hs].cpu()
+        else:
+            t[k] = v[:1].cpu()
+    st = None if pr.state is None else oracle.State(
+        *(pr.state[k][:1, hs].double().cpu().numpy() for k in ("h", "phi", "prev_B", "prev_x")))
+    t0 = time.perf_counter()
+    og.scan_grad(**t, state=st, dy=dy[:1, :, hs].cpu(), bc_norm=pr.dims.bc_norm,
+                 norm_eps=pr.dims.norm_eps)
+    el = time.perf_counter() - t0
+    tokens = pr.dims.seqlen * heads / pr.dims.nheads
+    return {"value": tokens / el, "unit": "tokens/s", "cores": torch.get_num_threads(),
+            "kind": "oracle",
+            "sample": f"sequence 0, heads 0-{heads - 1} of {pr.dims.nheads}, L={pr.dims.seqlen} "
+                      f"(= {tokens:.0f} workload tokens), {el:.1f} s"}
 
 
 def run_reference(args):
