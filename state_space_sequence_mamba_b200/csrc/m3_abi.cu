@@ -146,7 +146,8 @@ size_t m3_scan_workspace_bytes(const m3_dims* dims) {
     const m3_inputs none{};
     const ScanParams p = make_params(dims, &none, nullptr, nullptr, nullptr);
     size_t body = 0;
-    if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_bytes(p);
+    if (pipe_scan_supported(p, dims->in_dtype == M3_BF16)) body = pipe_scan_workspace_bytes(p);
+    else if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_bytes(p);
     return kWsHeader + (body + 255) / 256 * 256;
 }
 
@@ -161,7 +162,8 @@ size_t scan_workspace_min_bytes(const m3_dims* dims) {
     const m3_inputs none{};
     const ScanParams p = make_params(dims, &none, nullptr, nullptr, nullptr);
     size_t body = 0;
-    if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_min_bytes(p);
+    if (pipe_scan_supported(p, dims->in_dtype == M3_BF16)) body = pipe_scan_workspace_bytes(p);
+    else if (tc_scan_supported(p, dims->in_dtype == M3_BF16)) body = tc_scan_workspace_min_bytes(p);
     return kWsHeader + (body + 255) / 256 * 256;
 }
 
@@ -193,6 +195,11 @@ m3_status scan_fwd_with(const m3_dims* dims, const m3_inputs* in, const m3_state
     if (dims->seqlen == 0 || dims->batch == 0) return empty_sequence(dims, init, final_state, s);
 
     const bool bf16 = dims->in_dtype == M3_BF16;
+    if (pipe_scan_supported(p, bf16)) {
+        e = launch_scan_pipe(p, static_cast<char*>(workspace) + kWsHeader, ws_bytes - kWsHeader, s);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");
+        return M3_OK;
+    }
     if (tc_scan_supported(p, bf16)) {
         e = launch_scan_tc(p, static_cast<char*>(workspace) + kWsHeader, ws_bytes - kWsHeader, s);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core scan launch");

@@ -53,6 +53,11 @@ cudaError_t launch_decode(const ScanParams& p, bool bf16, cudaStream_t s);
 // Shared-memory bytes the SIMT scan needs for these dims (0 = cannot run).
 size_t simt_scan_smem_bytes(const ScanParams& p);
 cudaError_t launch_scan_simt(const ScanParams& p, bool bf16, cudaStream_t s);
+// Warp-specialised tensor-core scan (bf16, N = 128, P = 64, chunk * R = 128, R <= 4): one
+// CTA per (batch, head) unit and SM; its workspace body holds the fp32 RMS scales.
+bool pipe_scan_supported(const ScanParams& p, bool bf16);
+size_t pipe_scan_workspace_bytes(const ScanParams& p);
+cudaError_t launch_scan_pipe(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s);
 // Tensor-core scan (bf16, N = 128, P = 64, chunk * R = 64).
 bool tc_scan_supported(const ScanParams& p, bool bf16);
 // Workspace bytes the tensor-core scan needs beyond the status header: with the end states of
