@@ -24,12 +24,26 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roofline"
-# DRAM bytes (read + write) of one scan launch on this workload from the ncu capture
-# summarised in profiles/scan_tc_siso_prefill_b4_L2048.md; None once the kernel changes.
-SCAN_TRAFFIC_BYTES = 186.93e6
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant
+# scan kernel on this workload, from one ncu capture, keyed by the SHA-256 of the kernel's
+# source file when it was captured: reported while that file is unchanged, else null.
+SCAN_TRAFFIC = {"kernel": "scan_tc_kernel",
+                "source": "state_space_sequence_mamba_b200/csrc/m3_scan_tc.cu",
+                "sha256": None, "bytes": None}
 # kernels one scan launches: the per-token RMS-scale pre-pass of B and C, then the scan
 KERNELS_PER_SCAN = 2
 WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"
+
+
+def scan_traffic():
+    """The captured DRAM bytes per launch, or None when the kernel source has changed since
+    (or no capture is recorded)."""
+    import hashlib
+    if SCAN_TRAFFIC["sha256"] is None:
+        return None
+    with open(os.path.join(ROOT, SCAN_TRAFFIC["source"]), "rb") as f:
+        same = hashlib.sha256(f.read()).hexdigest() == SCAN_TRAFFIC["sha256"]
+    return SCAN_TRAFFIC["bytes"] if same else None
 
 
 def parse():
@@ -211,19 +225,28 @@ def run_ours(args):
     launch_ms = sum(per_launch) / len(per_launch)
     achieved = byts / (launch_ms / 1e3) / 1e9
 
-    # ---- end to end through the public API: pinned host inputs in, y out, every step ----
+    # ---- end to end through the public API: pinned host inputs in, y and the final state
+    # out, every step ----
     # Steps are pipelined over three streams with two buffer sets, as a serving loop would
-    # run them: step i+1's inputs go host -> device while step i's y goes device -> host (the
-    # two directions use separate copy engines). Each step still copies all of its inputs in
-    # and its whole y out inside the timed region.
+    # run them: step i+1's inputs go host -> device while step i's results go device -> host
+    # (the two directions use separate copy engines). Each step still copies all of its
+    # inputs in and its whole y and final state (h, phi, prev_B, prev_x) out inside the timed
+    # region.
     host = {k: (v.cpu().pin_memory() if v is not None else None)
             for k, v in sets[0].tensors().items()}
     y_host = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
     dev_in = [{k: (torch.empty_like(v, device=dev) if v is not None else None)
                for k, v in host.items()} for _ in range(2)]
     y_dev = [torch.empty_like(y) for _ in range(2)]
+    fin_dev = [m3.State.empty(d.batch, d.nheads, d.dstate, d.headdim, d.rank, d.dtype, dev)
+               for _ in range(2)]
+    fin_fields = ("h", "phi", "prev_B", "prev_x")
+    fin_host = [{k: torch.empty(getattr(fin_dev[0], k).shape,
+                                dtype=getattr(fin_dev[0], k).dtype).pin_memory()
+                 for k in fin_fields} for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-    d2h = y_host[0].numel() * y_host[0].element_size()
+    d2h = y_host[0].numel() * y_host[0].element_size() + sum(
+        v.numel() * v.element_size() for v in fin_host[0].values())
     s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     in_done = [torch.cuda.Event() for _ in range(2)]
     comp_done = [torch.cuda.Event() for _ in range(2)]
@@ -242,12 +265,14 @@ def run_ours(args):
             in_done[j].record(s_in)
         stream.wait_event(in_done[j])
         stream.wait_event(out_done[j])            # y of step i-2 has left the device
-        m3.scan_fwd(**dev_in[j], init=None, final=fin, y=y_dev[j], workspace=ws,
+        m3.scan_fwd(**dev_in[j], init=None, final=fin_dev[j], y=y_dev[j], workspace=ws,
                     chunk=d.chunk, bc_norm=True, stream=stream)
         comp_done[j].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(comp_done[j])
             y_host[j].copy_(y_dev[j], non_blocking=True)
+            for k in fin_fields:
+                fin_host[j][k].copy_(getattr(fin_dev[j], k), non_blocking=True)
             out_done[j].record(s_out)
 
     e2e_steps = max(3, min(args.steps, 10))
@@ -262,7 +287,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev)
     e2e_val = weak_throughput(tokens, world, e2e_steps, e2e_ms)
-    del host, dev_in, y_host, y_dev
+    del host, dev_in, y_host, y_dev, fin_dev, fin_host
 
     # ---- decode: 1000 consecutive steps in one CUDA graph, SISO and MIMO R=4 ----
     decode = {}
@@ -347,7 +372,7 @@ def run_ours(args):
                    "chunk": d.chunk, "parallelism": f"independent sequences x{world}",
                    "l2": "two alternating input sets of 144 MB each (> 126 MB L2), no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": SCAN_TRAFFIC_BYTES,
+                     "frac": achieved / hbm, "traffic": scan_traffic(),
                      "bytes_per_launch": byts, "launch_ms": launch_ms,
                      "peak_source": peak_kind},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -395,13 +420,14 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cp
     g = torch.Generator(device=dev).manual_seed(seed + 1)
     dy = torch.randn(pr.x.shape, generator=g, device=dev).to(d.dtype)
     init = m3.State.from_dict(pr.state)
-    ws = torch.empty(m3.scan_bwd_workspace_bytes(m3.make_dims(pr.x, pr.B, 1, True, 1e-6)),
-                     dtype=torch.uint8, device=dev)
+    ws = torch.empty(m3.scan_bwd_workspace_bytes(
+        m3.make_dims(pr.x, pr.B, 1, d.bc_norm, d.norm_eps, pr.flags)), dtype=torch.uint8,
+        device=dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        return m3.scan_bwd(**pr.tensors(), dy=dy, init=init, bc_norm=True, workspace=ws,
-                           stream=stream)
+    def step():   # the config's own BC norm, eps and scalar form, as the CPU baseline reads them
+        return m3.scan_bwd(**pr.tensors(), dy=dy, init=init, bc_norm=d.bc_norm,
+                           norm_eps=d.norm_eps, workspace=ws, stream=stream, **pr.scalar_args())
 
     for _ in range(3):
         step()

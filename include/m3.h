@@ -145,7 +145,13 @@ M3_API m3_status m3_scan_fwd(const m3_dims* dims, const m3_inputs* in, const m3_
                       const m3_state* final_state, void* y, void* workspace,
                       size_t ws_bytes, void* stream);
 
-/* One-token decode step: exactly one iteration of the recurrence for every unit.
+/* One-token decode step: exactly one iteration of the recurrence for every unit, as
+ * "Mamba-3: Improved Sequence Modeling using State Space Principles" states it for
+ * inference: the trapezoidal update h_t = alpha_t h_{t-1} + beta_t Bbar_{t-1} x_{t-1}^T +
+ * gamma_t Bbar_t x_t^T (Sec. 3.1.1 Prop. 1) with B and C rotated by the cumulative angle
+ * carried in phi (Sec. 3.2.2 Prop. 4), then y_t = h_t^T Cbar_t; MIMO as in Appendix C
+ * (H_t = a_t H_{t-1} + B_t X_t^T, Y_t = H_t^T C_t). prev_B and prev_x carry the token that
+ * the beta term of the next step reads.
  *   dims->seqlen must be 1; `in` points at one token: x [b,1,H,R,P], B, C [b,1,G,R,N] ...
  *   state_in  the state before the token (required).
  *   state_out where to write the state after it; may be the same buffers as state_in.
@@ -255,9 +261,12 @@ M3_API m3_status m3_scan_check(void* workspace);
  *   (each call clears the status bytes it needs at zero first). Calls whose work can overlap
  *   on the GPU (different streams, or different host threads) race on the array: serialise
  *   them, or use m3_scan_fwd with one workspace each.
- *   Limit: dims whose scan cannot run in 1 MiB return M3_ERR_UNSUPPORTED (with BC
- *   normalisation on, the tensor-core path needs 8 bytes per batch * seqlen * ngroups *
- *   rank row). Few long sequences, which m3_scan_fwd cuts into parallel segments, use only
+ *   Limit: dims whose scan cannot run in 1 MiB return M3_ERR_UNSUPPORTED. With BC
+ *   normalisation on, the tensor-core paths keep 8 bytes of RMS scales per row and the
+ *   array holds 131040 rows (1 MiB less a 256-byte status header), so the call runs when
+ *   batch * ceil(seqlen / chunk) * chunk * ngroups * rank <= 131040 (seqlen padded up to
+ *   whole chunks) and is rejected above that. With BC normalisation off, or on the fp32
+ *   path, there is no such limit. Few long sequences, which m3_scan_fwd cuts into parallel segments, use only
  *   as many segments as the rest of the array holds the end states of (possibly one): the
  *   results are the same, the time may be longer. A device-side wait that gives up cannot
  *   be reported here; use m3_scan_fwd and m3_scan_check when that matters. */

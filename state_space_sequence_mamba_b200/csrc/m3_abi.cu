@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/m3.h: argument validation, workspace layout and
 // dispatch to the kernels. Nothing here allocates device memory or synchronises a stream
 // (m3_scan_check excepted, which is documented to block).
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -134,6 +135,20 @@ m3_status empty_sequence(const m3_dims* d, const m3_state* init, const m3_state*
 }  // namespace
 
 m3_status set_error(m3_status s, const char* msg) { return fail(s, "%s", msg); }
+
+int device_sm_count() {
+    constexpr int kSlots = 64, kDefault = 148;
+    static std::atomic<int> cached[kSlots];   // 0 until the device's count is known
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSlots) return kDefault;
+    int sms = cached[dev].load(std::memory_order_relaxed);
+    if (sms > 0) return sms;
+    // two threads may both look it up; they store the same value
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return kDefault;
+    cached[dev].store(sms, std::memory_order_relaxed);
+    return sms;
+}
 
 }  // namespace m3
 

@@ -388,13 +388,7 @@ size_t decode_bulk_smem_bytes(const ScanParams& p) {
 
 template <int R>
 static cudaError_t launch_bulk_t(const ScanParams& p, cudaStream_t s) {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
+    const int sms = device_sm_count();
     const size_t smem = decode_bulk_smem_bytes(p);
     auto k = p.flags ? decode_bulk_kernel<R, true> : decode_bulk_kernel<R, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -519,13 +519,7 @@ bool encode_state(CUtensorMap* m, const float* base, int64_t units) {
 
 template <int R>
 cudaError_t launch_tc_t(const ScanParams& p, cudaStream_t s) {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
+    const int sms = device_sm_count();
     const int64_t units = p.b * p.H;
     DecMaps maps;
     if (!encode_state(&maps.h0, p.h0, units)) return cudaErrorInvalidValue;

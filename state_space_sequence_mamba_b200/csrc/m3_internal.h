@@ -94,6 +94,9 @@ m3_status scan_fwd_with(const m3_dims* dims, const m3_inputs* in, const m3_state
                         size_t need, void* stream);
 // Records msg as this thread's m3_last_error() text and returns s.
 m3_status set_error(m3_status s, const char* msg);
+// SM count of the calling thread's current device, looked up once per device (148, the
+// B200's count, when no device answers). Safe to call from several host threads.
+int device_sm_count();
 // Persistent decode with bulk asynchronous copies (bf16, N * P <= 8192).
 bool decode_bulk_supported(const ScanParams& p, bool bf16);
 size_t decode_bulk_smem_bytes(const ScanParams& p);

@@ -54,8 +54,9 @@ M3_API m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const m3_inputs* in,
     if (need > kStaticScratchBytes)
         return static_fail(M3_ERR_UNSUPPORTED,
                            "m3_scan_fwd_noalloc: these dims need more scratch than the "
-                           "library's fixed 1 MiB (batch * seqlen * ngroups * rank must stay "
-                           "below 131040 with BC normalisation on); use m3_scan_fwd");
+                           "library's fixed 1 MiB (with BC normalisation on, batch * "
+                           "ceil(seqlen / chunk) * chunk * ngroups * rank must be <= 131040); "
+                           "use m3_scan_fwd");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return static_fail(M3_ERR_CUDA, "m3_scan_fwd_noalloc: no usable current device");

@@ -1045,17 +1045,6 @@ bool tc_scan_supported(const ScanParams& p, bool bf16) {
 
 namespace {
 
-int sm_count() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    return sms;
-}
-
 // Segments per sequence. When the (batch, head) units alone would leave SMs idle, each
 // sequence is cut so that units x segments fills every SM twice (two CTAs per SM), keeping at
 // least kMinSegChunks chunks per segment and at most kMaxSeg segments, and no more segments
@@ -1067,7 +1056,7 @@ SegArgs seg_plan(const ScanParams& p, size_t seg_bytes = ~size_t(0)) {
     const int64_t units = p.b * p.H;
     SegArgs sa{static_cast<int>(nch), 1, nullptr, nullptr, nullptr, nullptr};
     if (units <= 0 || nch == 0) return sa;
-    int64_t S = 2 * sm_count() / units;
+    int64_t S = 2 * device_sm_count() / units;
     S = std::min(S, nch / kMinSegChunks);
     S = std::min(S, kMaxSeg);
     const size_t per_seg = static_cast<size_t>(units) * kSegStride * sizeof(float);

@@ -165,3 +165,32 @@ def test_missing_library_fails_loudly(tmp_path):
             bd.load_library(str(tmp_path / "nope.so"))
         finally:
             bd._lib = bd._lib_backup
+
+
+@pytest.mark.parametrize("kw,fits", [
+    # rows = batch * ceil(seqlen / chunk) * chunk * ngroups * rank; chunks hold 64 or 128 rows,
+    # so the largest count that fits is 130944 or 131008 (131040 is not a multiple of 64)
+    (dict(batch=1, seqlen=131008, chunk=64), True),     # 2047 chunks: 131008 rows
+    (dict(batch=1, seqlen=131009, chunk=64), False),    # 2048 chunks: 131072 rows
+    (dict(batch=2, seqlen=65472, chunk=64), True),      # 2 * 1023 chunks: 130944 rows
+    (dict(batch=2, seqlen=65473, chunk=64), False),     # 130946 tokens, padded to 131072 rows
+    (dict(batch=2, seqlen=65500, chunk=64), False),     # 131000 tokens, padded to 131072 rows
+    (dict(batch=1, seqlen=130944, chunk=128), True),    # 1023 chunks of 128
+    (dict(batch=1, seqlen=130945, chunk=128), False),   # 1024 chunks: 131072 rows
+    (dict(batch=1, seqlen=32736, chunk=32, rank=4), True),    # 1023 chunks of 32 tokens x 4
+    (dict(batch=1, seqlen=32737, chunk=32, rank=4), False),
+    (dict(batch=2, seqlen=65521, chunk=64, bc_norm=0), True),  # no scales: no limit
+])
+def test_noalloc_limit_on_both_sides(lib, kw, fits):
+    """m3_scan_fwd_noalloc runs when batch * ceil(seqlen / chunk) * chunk * ngroups * rank
+    <= 131040 with BC norm on, and returns M3_ERR_UNSUPPORTED above it. x is null, so a call
+    within the bound stops at argument validation (or at the missing device) and never
+    launches."""
+    d = dims(nheads=4, **kw)
+    ins = fake_inputs(x=None)
+    st = lib.m3_scan_fwd_noalloc(ctypes.byref(d), ctypes.byref(ins), None, None, FAKE, None)
+    if fits:
+        assert st in (bd.M3_ERR_INVALID_ARG, bd.M3_ERR_CUDA), st
+    else:
+        assert st == bd.M3_ERR_UNSUPPORTED
+        assert b"131040" in lib.m3_last_error()
