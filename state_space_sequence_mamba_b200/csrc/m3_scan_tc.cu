@@ -25,6 +25,8 @@
 // dH accumulator) and is rounded to bf16 only as the Yo operand. All waits are bounded; a
 // timeout sets the status word and the CTA exits cleanly.
 #include <algorithm>
+#include <cstdlib>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -809,7 +811,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
                     // theta and raw B of chunk c+1 (their buffers were read by the rotation), the
                     // scalar boxes of chunk c+2 (chunk c's slot was read by scalars(c))
                     if (c + 1 < nchunks) {
-                        issue_th(c + 1);
+                        if (!(blockIdx.x == 0 && c + 1 == p.test_skip_theta)) issue_th(c + 1);
                         issue_b(c + 1);
                     }
                     if (c + 2 < nchunks) issue_sc(c + 2);
@@ -1196,8 +1198,10 @@ cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body
     return launch_state_combine(p.b * p.H, kN, kP, sa.nseg, src, out_h, out_phi, out_lam, s);
 }
 
-cudaError_t launch_scan_tc(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s) {
-    if (p.b * p.H == 0) return cudaSuccess;
+cudaError_t launch_scan_tc(const ScanParams& p_in, void* ws_body, size_t body_bytes, cudaStream_t s) {
+    if (p_in.b * p_in.H == 0) return cudaSuccess;
+    ScanParams p = p_in;
+    if (const char* e = std::getenv("M3_TEST_SKIP_THETA_LOAD")) p.test_skip_theta = std::atoi(e);
     // workspace body: the RMS scales, then the segments' end states
     uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
     if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;

@@ -47,10 +47,17 @@ def gpu_scan(pr, dev, use_state=True, chunk=None, final=True):
     return y, fin
 
 
-def oracle_scan(pr, use_state=True, heads=None):
+def oracle_scan(pr, use_state=True, heads=None, batches=None):
+    """The oracle on problem pr, optionally on some heads and / or batch rows only."""
     t = pr.tensors()
     t.update(pr.scalar_args())
     st = pr.state if use_state else None
+    if batches is not None:
+        bs = torch.as_tensor(batches)
+        for k in ("x", "B", "C", "theta", "dt", "A", "lam"):
+            t[k] = t[k][bs]
+        if st is not None:
+            st = {k: v[bs] for k, v in st.items()}
     if heads is not None:
         hs = torch.as_tensor(heads)
         for k in ("x", "theta", "dt", "A", "lam"):
@@ -65,9 +72,14 @@ def oracle_scan(pr, use_state=True, heads=None):
                        norm_eps=pr.dims.norm_eps)
 
 
-def compare(pr, y, fin, yo, so, heads=None, tol=None):
+def compare(pr, y, fin, yo, so, heads=None, tol=None, batches=None):
     tol = tol or TOL[pr.dims.dtype]
     hs = slice(None) if heads is None else torch.as_tensor(heads)
+    if batches is not None:
+        bs = torch.as_tensor(batches, device=y.device)
+        y = y[bs]
+        if fin is not None:
+            fin = type(fin)(*(getattr(fin, k)[bs] for k in ("h", "phi", "prev_B", "prev_x")))
     errs = {"y": rel(y[:, :, hs], yo)}
     if fin is not None:
         errs["h"] = rel(fin.h[:, hs], so.h)

@@ -192,23 +192,108 @@ def test_decode_out_of_place_and_fp32(cuda_dev):
         assert torch.equal(getattr(sin, k), g.state[k])  # input state untouched
 
 
+# ---------------------------------------------------------------- 128-row chunks
+# The warp-specialised scan takes chunks of 128 (token, rank) rows: chunk 128 / R. Cases span
+# several chunks with a ragged tail; dt_shift > 0 makes chunks decay by more than 60 nats,
+# which that kernel computes in its exact (unscaled) form, dt_shift 0 mixes both forms.
+PIPE = [
+    # b, L, H, G, R, norm, bias, state, dt_shift, raw scalars, zoh
+    (1, 300, 4, 1, 1, True, 0.1, True, -2.0, False, False),
+    (2, 130, 4, 1, 2, False, 0.0, False, -2.0, False, False),
+    (2, 77, 4, 1, 4, True, 0.1, True, -2.0, False, False),
+    (1, 1, 4, 1, 1, True, 0.1, True, -2.0, False, False),
+    (2, 128, 4, 2, 1, True, 0.1, False, -2.0, False, False),
+    (1, 257, 8, 4, 2, True, 0.1, True, -2.0, False, False),
+    (1, 400, 4, 1, 1, True, 0.1, True, 1.5, False, False),
+    (1, 300, 4, 1, 2, True, 0.1, True, 1.5, False, False),
+    (1, 300, 4, 1, 4, False, 0.0, True, 1.0, False, False),
+    (2, 700, 4, 1, 1, True, 0.1, True, 0.0, False, False),
+    (2, 333, 4, 1, 1, True, 0.1, True, -2.0, True, False),
+    (2, 150, 4, 1, 4, True, 0.1, True, -2.0, True, True),
+    (1, 260, 4, 1, 2, True, 0.1, True, -2.0, False, True),
+]
+
+
+@pytest.mark.parametrize("case", PIPE, ids=lambda c: "b{}L{}H{}G{}R{}{}{}d{}{}{}".format(
+    *c[:5], "n" if c[5] else "", "s" if c[7] else "", c[8], "raw" if c[9] else "",
+    "zoh" if c[10] else ""))
+def test_scan_128_row_chunks(cuda_dev, case):
+    b, L, H, G, R, norm, bias, st, dts, raw, zoh = case
+    pr = make_problem(b, L, H, G, 64, 128, rank=R, chunk=128 // R, bc_norm=norm,
+                      bias_std=bias, seed=11 * L + R, with_state=True, dt_shift=dts,
+                      raw_scalars=raw)
+    if zoh:
+        pr.flags |= m3.M3_DISC_ZOH
+    y, fin = gpu_scan(pr, cuda_dev, use_state=st)
+    yo, so = oracle_scan(pr, use_state=st)
+    compare(pr, y, fin, yo, so)
+
+
+@pytest.mark.parametrize("R", [1, 4])
+def test_128_row_chunks_final_state_may_alias_init(cuda_dev, R):
+    pr = make_problem(2, 290, 4, 1, 64, 128, rank=R, chunk=128 // R, bc_norm=True,
+                      bias_std=0.1, seed=17 + R, with_state=True)
+    g = pr.to(cuda_dev)
+    st = m3.State.from_dict({k: v.clone() for k, v in g.state.items()})
+    y, fin = m3.scan_fwd(**g.tensors(), init=st, final=st, chunk=128 // R, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, y, fin, yo, so)
+
+
+def test_128_row_chunks_deterministic_and_split(cuda_dev):
+    """Two runs are bit-identical; scan(L1) -> state -> scan(L2) matches the oracle's
+    single scan over L1 + L2 with the cut inside a chunk."""
+    pr = make_problem(2, 300, 4, 1, 64, 128, rank=1, chunk=128, bc_norm=True, bias_std=0.1,
+                      seed=29, with_state=True)
+    y1, f1 = gpu_scan(pr, cuda_dev)
+    y2, f2 = gpu_scan(pr, cuda_dev)
+    assert torch.equal(y1, y2) and torch.equal(f1.h, f2.h) and torch.equal(f1.phi, f2.phi)
+    g = pr.to(cuda_dev)
+    t = g.tensors()
+    cut = 170
+    part = lambda sl: {k: (v[:, sl].contiguous() if k not in ("B_bias", "C_bias") else v)
+                       for k, v in t.items()}
+    ya, sa = m3.scan_fwd(**part(slice(0, cut)), init=m3.State.from_dict(g.state), chunk=128,
+                         bc_norm=True)
+    yb, sb = m3.scan_fwd(**part(slice(cut, None)), init=sa, chunk=128, bc_norm=True)
+    torch.cuda.synchronize()
+    yo, so = oracle_scan(pr)
+    compare(pr, torch.cat([ya, yb], 1), sb, yo, so)
+
+
 # ---------------------------------------------------------------- full-size workloads
 @pytest.mark.slow
-def test_config1_full_size_sampled_heads(cuda_dev):
+def test_config1_full_size_all_heads_of_one_sequence(cuda_dev):
+    """The SISO prefill workload as the benchmark launches it (chunk 64): all 64 heads of
+    sequence 2 against the oracle."""
     pr = make_config(1)
     y, fin = gpu_scan(pr, cuda_dev, use_state=False)
-    heads = [0, 17, 38, 63]
-    yo, so = oracle_scan(pr, use_state=False, heads=heads)
-    compare(pr, y, fin, yo, so, heads=heads)
+    yo, so = oracle_scan(pr, use_state=False, batches=[2])
+    compare(pr, y, fin, yo, so, batches=[2])
 
 
 @pytest.mark.slow
 def test_config2_mimo_full_size_sampled_heads(cuda_dev):
+    """MIMO R4 as the benchmark launches it (chunk 16): 8 heads of sequences 0 and 3."""
     pr = make_config(2)
     y, fin = gpu_scan(pr, cuda_dev, use_state=False)
-    heads = [5, 44]
-    yo, so = oracle_scan(pr, use_state=False, heads=heads)
-    compare(pr, y, fin, yo, so, heads=heads)
+    heads = [1, 9, 18, 27, 36, 45, 54, 63]
+    yo, so = oracle_scan(pr, use_state=False, heads=heads, batches=[0, 3])
+    compare(pr, y, fin, yo, so, heads=heads, batches=[0, 3])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_full_size_128_row_chunks(cuda_dev, cfg):
+    """The two b4 L2048 prefill workloads with 128-row chunks (chunk 128 and 32): 16 heads of
+    sequence 1 (SISO), 8 heads of sequence 2 (MIMO R4)."""
+    pr = make_config(cfg)
+    y, fin = gpu_scan(pr, cuda_dev, use_state=False, chunk=128 // pr.dims.rank)
+    heads = list(range(3, 64, 4)) if cfg == 1 else [0, 8, 16, 24, 32, 40, 48, 56]
+    bsel = [1] if cfg == 1 else [2]
+    yo, so = oracle_scan(pr, use_state=False, heads=heads, batches=bsel)
+    compare(pr, y, fin, yo, so, heads=heads, batches=bsel)
 
 
 @pytest.mark.slow
@@ -416,11 +501,12 @@ def _degenerate(pr, kind):
 
 @pytest.mark.parametrize("kind", ["euler", "prev_only", "no_rotation", "strong_decay",
                                   "tiny_step", "fast_angle"])
-@pytest.mark.parametrize("R,L,b", [(1, 333, 2), (4, 150, 2), (1, 2543, 1)])
-def test_scan_degenerate_regimes(cuda_dev, kind, R, L, b):
-    """Limits of the recurrence through the tensor-core scan (SISO, MIMO, and the
-    sequence-parallel form at b1 L2543) against the oracle."""
-    pr = make_problem(b, L, 4, 1, 64, 128, rank=R, chunk=64 // R, bc_norm=True, bias_std=0.1,
+@pytest.mark.parametrize("R,L,b,rows", [(1, 333, 2, 64), (4, 150, 2, 64), (1, 2543, 1, 64),
+                                        (1, 333, 2, 128), (4, 150, 2, 128)])
+def test_scan_degenerate_regimes(cuda_dev, kind, R, L, b, rows):
+    """Limits of the recurrence through the tensor-core scans (SISO, MIMO, the
+    sequence-parallel form at b1 L2543, and 128-row chunks) against the oracle."""
+    pr = make_problem(b, L, 4, 1, 64, 128, rank=R, chunk=rows // R, bc_norm=True, bias_std=0.1,
                       seed=101 + L + R, with_state=True)
     pr = _degenerate(pr, kind)
     y, fin = gpu_scan(pr, cuda_dev)

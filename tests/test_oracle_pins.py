@@ -498,6 +498,65 @@ def test_decode_step_proj_against_library_gate_and_contraction():
     np.testing.assert_allclose(o1, ref1, rtol=1e-12, atol=1e-12)
 
 
+def test_decode_step_proj_structural_cases_by_hand():
+    """Two cases of the projected decode step (Appendix C) fixed without the oracle's own
+    contraction code, by plain loops over a tiny problem with no rotation (theta = 0 and a
+    zero carried angle), no norm and no bias:
+      - W_X = 0: the new token enters nothing, so h' = alpha h + beta sum_r prevB_r prevx_r^T
+        (Prop. 1 with x_t = 0), Y[r][p] = sum_n C[r][n] h'[n][p], and O' is the W_O-weighted,
+        SiLU(W_Z Z')-gated sum of Y over the ranks; the stored prev_x is 0;
+      - W_O one-hot on rank q: O' is rank q's gated output alone, so the outputs of the R
+        one-hot choices add up to the output with every weight of W_O at 1 (linear in W_O)."""
+    rng = np.random.default_rng(77)
+    b, H, R, N, P = 1, 2, 2, 4, 3
+    st = oracle.State(rng.standard_normal((b, H, N, P)), np.zeros((b, H, N // 2)),
+                      rng.standard_normal((b, H, R, N)), rng.standard_normal((b, H, R, P)))
+    B = rng.standard_normal((b, 1, R, N))
+    C = rng.standard_normal((b, 1, R, N))
+    theta = np.zeros((b, H, N // 2))
+    dt = np.array([[0.7, 0.2]])
+    A = np.array([[-0.5, -1.3]])
+    lam = np.array([[0.3, 0.8]])
+    xp, zp = rng.standard_normal((b, H, P)), rng.standard_normal((b, H, P))
+    WZ, WO = rng.standard_normal((H, R, P)), rng.standard_normal((H, R, P))
+    WX0 = np.zeros((H, R, P))
+    o, so = oracle.decode_step_proj(xp, zp, WX0, WZ, WO, B, C, theta, dt, A, lam, state=st)
+    for h in range(H):
+        al = math.exp(dt[0, h] * A[0, h])
+        be = (1.0 - lam[0, h]) * dt[0, h] * al
+        hn = [[al * st.h[0, h, n, p] + be * sum(st.prev_B[0, h, r, n] * st.prev_x[0, h, r, p]
+                                              for r in range(R))
+               for p in range(P)] for n in range(N)]
+        for n in range(N):
+            for p in range(P):
+                assert abs(so.h[0, h, n, p] - hn[n][p]) < 1e-12
+        for p in range(P):
+            want = 0.0
+            for r in range(R):
+                y = sum(C[0, 0, r, n] * hn[n][p] for n in range(N))
+                z = WZ[h, r, p] * zp[0, h, p]
+                want += WO[h, r, p] * y * (z / (1.0 + math.exp(-z)))
+            assert abs(o[0, h, p] - want) < 1e-12 * max(1.0, abs(want))
+    assert np.all(so.prev_x == 0.0)
+    # one-hot W_O: rank q alone, and the ranks add up to W_O = 1
+    WX = rng.standard_normal((H, R, P))
+    ones = np.ones((H, R, P))
+    o_all, _ = oracle.decode_step_proj(xp, zp, WX, WZ, ones, B, C, theta, dt, A, lam, state=st)
+    y_all, _ = oracle.decode_step(WX[None] * xp[:, :, None, :], B, C, theta, dt, A, lam,
+                                  state=st)
+    total = np.zeros_like(o_all)
+    for q in range(R):
+        e = np.zeros((H, R, P))
+        e[:, q, :] = 1.0
+        oq, _ = oracle.decode_step_proj(xp, zp, WX, WZ, e, B, C, theta, dt, A, lam, state=st)
+        for h in range(H):
+            for p in range(P):
+                z = WZ[h, q, p] * zp[0, h, p]
+                assert abs(oq[0, h, p] - y_all[0, h, q, p] * z / (1.0 + math.exp(-z))) < 1e-12
+        total += oq
+    np.testing.assert_allclose(total, o_all, rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- zero-order hold
 def test_zoh_is_exact_for_piecewise_constant_input():
     """The zero-order-hold weights ("Mamba-3：推理优先的状态空间模型", Sec. 1.2) are the exact
