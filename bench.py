@@ -8,8 +8,10 @@ captured in one CUDA graph, the end-to-end prefill through the public API with h
 the roofline of the dominant kernel, SM clocks during the timed region, and the CPU oracle.
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-decode]
-For N > 1 launch under torch.distributed.run; every rank runs its own copy of the workload
-(independent sequences: weak scaling, no collective on the data path).
+For N > 1 it runs under torch.distributed.run (started by itself when no launcher set
+WORLD_SIZE); every rank runs its own copy of the workload (independent sequences: weak
+scaling, no collective on the data path) and the reported time is the slowest rank's.
+--context-parallel adds the long-sequence prefill split along the sequence over the ranks.
 """
 from __future__ import annotations
 
@@ -58,7 +60,57 @@ def parse():
                     help="time only the backward pass (SISO and MIMO R4) and print its numbers")
     ap.add_argument("--bwd-seqlen", type=int, default=None,
                     help="sequence length of the --backward-only workloads (default: theirs)")
+    ap.add_argument("--context-parallel", action="store_true",
+                    help="also time the long-sequence prefill (b1 H64 L65536) split along the "
+                         "sequence over the ranks (N > 1)")
+    ap.add_argument("--host-plumbing", action="store_true",
+                    help="check the multi-rank launch, max-over-ranks timing and report on "
+                         "CPU ranks (gloo), with a fixed per-rank wait as the step: no GPU")
     return ap.parse_args()
+
+
+def spawn_ranks(args) -> int:
+    """`--gpus N` (N > 1) started without a launcher: run this script again under
+    torch.distributed.run with N processes on this node, one per GPU, rendezvous on
+    127.0.0.1. Rank 0 prints the line; returns the launcher's exit code."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def run_host_plumbing(args):
+    """The multi-rank path of the report without a GPU: gloo ranks whose step is a fixed
+    wait (10 + 5 * rank ms), timed on each rank, maximised over the ranks, turned into the
+    whole-job rate of `units` per rank and step, and printed by rank 0."""
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    wait = 0.010 + 0.005 * rank
+    units = 8192
+    for _ in range(args.warmup):
+        time.sleep(wait)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(wait)
+    local_ms = (time.perf_counter() - t0) * 1e3
+    total_ms = max_over_ranks(local_ms, world, dist, "cpu")
+    if rank == 0:
+        print(json.dumps({"check": "host-plumbing", "n_gpus": world, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                          "value": weak_throughput(units, world, args.steps, total_ms),
+                          "units_per_rank_step": units, "scaling": "weak"}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def dist_env():
@@ -362,6 +414,10 @@ def run_ours(args):
         backward["mimo_r4_b4_L2048"] = bench_backward(m3, dev, 2, hbm, world, dist,
                                                       rank_seed(rank, 12))
 
+    cp_leg = None
+    if args.context_parallel:
+        cp_leg = (bench_context_parallel(m3, dev, hbm, world, dist, stream) if world > 1 else
+                  {"skipped": "needs more than one rank"})
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
@@ -384,12 +440,50 @@ def run_ours(args):
         "other_prefill": others,
         "backward": backward,
     }
+    if cp_leg is not None:
+        line["context_parallel"] = cp_leg
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def bench_context_parallel(m3, dev, hbm, world, dist, stream, reps=3):
+    """The long-sequence prefill (b1 H64 L65536) split along the sequence over the ranks:
+    rank k scans tokens [k L / N, (k + 1) L / N) of the same sequence after one exchange of
+    the last tokens and the segments' end states (two NCCL all-gathers, no peer loads), and
+    the time is the slowest rank's. Strong scaling: the sequence is fixed."""
+    import torch
+    from state_space_sequence_mamba_b200 import context_parallel as cp
+    from state_space_sequence_mamba_b200.inputs import make_config
+    rank = dist.get_rank()
+    pr = make_config(4, device=dev, seed=rank_seed(0, 40))   # the same sequence on every rank
+    d = pr.dims
+    L = d.seqlen
+    lo, hi = L * rank // world, L * (rank + 1) // world
+    t = {k: (v[:, lo:hi].contiguous() if k not in ("B_bias", "C_bias") else v)
+         for k, v in pr.tensors().items()}
+    del pr
+
+    def run():
+        return cp.scan_context_parallel(**t, chunk=d.chunk, bc_norm=True)
+
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dist, dev) / reps
+    return {"workload": "long SISO prefill b1 H64 L65536 split over the ranks", "world": world,
+            "ms_per_scan": ms, "tokens_per_s": d.batch * L / (ms / 1e3), "scaling": "strong",
+            "exchange": "two all-gathers of last tokens and end states (NCCL)"}
 
 
 def bwd_bytes(pr) -> int:
@@ -594,7 +688,13 @@ def run_reference(args):
 
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(a))
+    if int(os.environ.get("WORLD_SIZE", 1)) != a.gpus:
+        sys.exit(f"--gpus {a.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE')}")
+    if a.host_plumbing:
+        run_host_plumbing(a)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_ours(a)

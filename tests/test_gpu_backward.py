@@ -168,6 +168,20 @@ def test_backward_full_size_prefill_sampled_heads(cuda_dev):
         assert torch.isfinite(got[k]).all(), k
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg,kw", [(1, dict(batch=1, nheads=8)),
+                                    (2, dict(batch=1, nheads=4, seqlen=1024))])
+def test_backward_full_length_every_gradient(cuda_dev, cfg, kw):
+    """Every gradient, dB, dC and the bias gradients (sums over all heads and tokens) too,
+    element by element at the workloads' full sequence length on a reduced head count: SISO
+    b1 H8 L2048 and MIMO R4 b1 H4 L1024, with a carried state."""
+    pr = make_config(cfg, with_state=True, **kw)
+    dy, dfin = draw_grads(pr, seed=13 + cfg)
+    got = gpu_grads(pr, dy, dfin, cuda_dev)
+    ref = oracle_grads(pr, dy, dfin)
+    compare_grads(got, ref)
+
+
 def test_backward_full_size_mimo_sampled_heads(cuda_dev):
     pr = make_config(2, seqlen=512, with_state=True)
     dy, dfin = draw_grads(pr, seed=12)

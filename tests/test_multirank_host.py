@@ -79,3 +79,31 @@ def test_weak_throughput_counts_every_rank():
     eight = bench.weak_throughput(8192, 8, 10, 2.0)
     assert eight == pytest.approx(8 * one)
     assert bench.rank_seed(0, 0) != bench.rank_seed(1, 0) != bench.rank_seed(0, 1)
+
+
+def test_bench_spawns_its_ranks_and_reports_the_slowest():
+    """`bench.py --gpus 2` without a launcher starts two ranks under torch.distributed.run
+    (rendezvous on 127.0.0.1). With --host-plumbing the ranks are gloo CPU processes whose
+    step is a fixed wait (rank 1's is the longer, 15 ms): rank 0 alone prints one line whose
+    n_gpus is 2, whose step time is the slowest rank's and whose rate counts both ranks."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("WORLD_SIZE", None)
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--steps", "4", "--warmup", "1", "--host-plumbing"],
+                         capture_output=True, text=True, timeout=240, env=env, cwd=ROOT)
+    assert out.returncode == 0, out.stdout[-2000:] + out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    r = lines[0]
+    assert r["n_gpus"] == 2 and r["steps"] == 4 and r["scaling"] == "weak"
+    assert r["ms_per_step"] >= 15.0                     # rank 1's wait, not rank 0's 10 ms
+    want = r["units_per_rank_step"] * 2 * 4 / (r["ms_per_step"] * 4 / 1e3)
+    assert abs(r["value"] - want) <= 1e-9 * want
+
+
+def test_bench_rejects_a_rank_count_that_disagrees_with_the_launcher():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2",
+                          "--host-plumbing"], capture_output=True, text=True, timeout=120,
+                         env=env, cwd=ROOT)
+    assert out.returncode != 0 and "WORLD_SIZE=3" in out.stderr
