@@ -444,6 +444,8 @@ def run_ours(args):
         line["context_parallel"] = cp_leg
     if rank == 0:
         line["cpu_baseline"] = cpu_baseline(sets[0]) if world == 1 else None
+        if world == 1 and not args.no_decode:
+            line["cpu_baselines"] = cpu_baselines()
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -622,6 +624,89 @@ def cpu_baseline(pr, min_s=10.0, max_reps=30):
     return {"value": tokens / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"the whole workload ({pr.dims.batch} sequences x {pr.dims.nheads} heads x "
                       f"L={pr.dims.seqlen}) x {reps} passes, {el:.1f} s"}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _timed_oracle(make, start, limit, target_s, nthreads):
+    """The oracle scan on samples of growing size (`make(k)` builds one of k units) until one
+    takes at least target_s or k reaches limit. Returns (k, seconds)."""
+    import oracle
+    k = start
+    while True:
+        t = make(k)
+        t0 = time.perf_counter()
+        oracle.scan(**t, nthreads=nthreads)
+        el = time.perf_counter() - t0
+        if el >= target_s or k >= limit:
+            return k, el
+        k = min(limit, max(2 * k, int(k * target_s / max(el, 1e-3) * 1.2)))
+
+
+def cpu_baselines(target_s=1.5):
+    """The fp64 oracle as it stands on every workload of the measurement: one thread and all
+    host cores, each on a bounded sample (reduced head count, or reduced batch for the
+    decode steps, at full length), scaled to the workload's unit. Prefill: tokens/s of the
+    whole workload (a sample of k of H heads runs k/H of its work). Decode: us per step of
+    the whole batch over 1000 consecutive steps, from a sample of heads of one sequence (the
+    oracle's scan over those steps is the same recurrence)."""
+    import oracle
+    from state_space_sequence_mamba_b200.inputs import make_config, make_decode
+    cores = oracle.max_threads()
+    out = {"cpu_model": cpu_model(), "nproc": os.cpu_count(), "kind": "oracle"}
+
+    def prefill(cfg):
+        H = 64
+
+        def make(k):
+            pr = make_config(cfg, batch=1, nheads=k)
+            t = {kk: v for kk, v in pr.tensors().items()}
+            t.update(bc_norm=True)
+            return t
+        L = make_config(cfg, batch=1, nheads=1).dims.seqlen
+        res = {}
+        for name, nt, start in (("one_thread", 1, 1), ("all_cores", cores, min(H, cores))):
+            k, el = _timed_oracle(make, start, H, target_s, nt)
+            res[name] = {"value": L * k / H / el, "unit": "tokens/s", "threads": nt,
+                         "sample": f"1 sequence, {k} of {H} heads, L={L}, {el:.2f} s"}
+        return res
+
+    def decode(R, steps=1000, batch=128, H=64):
+        def make(k):
+            pr = make_decode(R, steps, batch=1, nheads=k)
+            sq = lambda v: v[:, :, 0].transpose(0, 1).contiguous()
+            st = oracle.State(*(pr.state[f].double().numpy()
+                                for f in ("h", "phi", "prev_B", "prev_x")))
+            return dict(x=sq(pr.x), B=sq(pr.B), C=sq(pr.C), theta=sq(pr.theta), dt=sq(pr.dt),
+                        A=sq(pr.A), lam=sq(pr.lam), state=st)
+        res = {}
+        for name, nt, start in (("one_thread", 1, 1), ("all_cores", cores, min(H, cores))):
+            k, el = _timed_oracle(make, start, H, target_s, nt)
+            res[name] = {"value": el / steps * batch * H / k * 1e6, "unit": "us/step",
+                         "threads": nt, "sample": f"1 of {batch} sequences, {k} of {H} heads, "
+                                                  f"{steps} steps, {el:.2f} s"}
+        return res
+
+    for key, fn in (("siso_prefill_b4_L2048", lambda: prefill(1)),
+                    ("mimo_r4_prefill_b4_L2048", lambda: prefill(2)),
+                    ("decode_siso_b128_1000_steps", lambda: decode(1)),
+                    ("decode_mimo_r4_b128_1000_steps", lambda: decode(4)),
+                    ("long_prefill_b1_L65536", lambda: prefill(4))):
+        try:
+            out[key] = fn()
+        except Exception as e:  # noqa: BLE001  (an auxiliary field: reported, not fatal)
+            out[key] = {"error": f"{type(e).__name__}: {e}"[:200]}
+    return out
 
 
 def cpu_baseline_backward(pr, dy, heads=8):
