@@ -63,7 +63,7 @@ struct TcCfg {
     static constexpr uint32_t SC_SLOT = round_up(SC_ONE, 128);      // 128-byte aligned slots
     static constexpr uint32_t SC_BYTES = 3 * SC_SLOT;
     static constexpr uint32_t SC0 = TH + TH_BYTES, SC1 = SC0 + SC_BYTES;  // dt, A, lam boxes
-    static constexpr uint32_t ORS = SC1 + SC_BYTES;                 // RMS scales, 64 x uint2
+    static constexpr uint32_t ORS = SC1 + SC_BYTES;                 // RMS scales, 64 x float2
     static constexpr uint32_t OF = ORS + 512;                       // fp32 scratch
     static constexpr uint32_t B_TX = 2 * 8192;                      // raw B: two slabs
     static constexpr uint32_t C_TX = 2 * 8192;                      // raw C: two slabs
@@ -78,7 +78,7 @@ constexpr int F_CUM = 0, F_GAM = 64, F_W = 128, F_ECUM = 192, F_DW = 256, F_DT =
               F_MISC = 640,                // e^{cum_end}
               F_BLK = 656;
 constexpr int F_SEG = 2 * F_BLK;           // [8 segments][32 lanes] float2
-constexpr int F_BIAS = F_SEG + 512;        // bias_B [R][128] bf16, bias_C [R][128] bf16
+constexpr int F_BIAS = F_SEG + 512;        // bias_B [R][128] fp32, bias_C [R][128] fp32
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t T_S = 0, T_YO = 64, T_YD = 128, T_DH = 192;
 // One state slot in the workspace (floats): h [N][P], the angle [N/2], a segment's summed
@@ -87,7 +87,7 @@ constexpr int kSegStride = kN * kP + kHalf + 4;
 
 template <int R>
 __host__ __device__ constexpr uint32_t tc_smem_bytes() {
-    return TcCfg<R>::OF + 4u * F_BIAS + 2u * 2 * R * kN + 1024u;
+    return TcCfg<R>::OF + 4u * F_BIAS + 4u * 2 * R * kN + 1024u;
 }
 
 // 2^x by the hardware approximation (relative error ~2^-22), x <= 0 here.
@@ -101,6 +101,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+
+// (low, high) bf16 halves of a word as exact fp32, and two floats rounded to a bf16 pair
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) { return pack_bf16(v.x, v.y); }
 
 __device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) {
     return *reinterpret_cast<const __nv_bfloat162*>(&w);
@@ -120,7 +126,7 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
                                                         const __nv_bfloat16* __restrict__ C,
                                                         int64_t rows, int64_t L, int64_t G,
                                                         int64_t R, int64_t Lpad, float eps,
-                                                        uint2* __restrict__ out) {
+                                                        float2* __restrict__ out) {
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -139,12 +145,7 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
     }
     sb = warp_sum(sb);
     sc = warp_sum(sc);
-    if (lane == 0) {  // stored as packed bf16 pairs (rs, rs), the operand form of the rotation
-        const float rb = rsqrtf(sb / kN + eps), rc = rsqrtf(sc / kN + eps);
-        const __nv_bfloat162 vb = __floats2bfloat162_rn(rb, rb), vc = __floats2bfloat162_rn(rc, rc);
-        out[orow] = make_uint2(*reinterpret_cast<const uint32_t*>(&vb),
-                               *reinterpret_cast<const uint32_t*>(&vc));
-    }
+    if (lane == 0) out[orow] = make_float2(rsqrtf(sb / kN + eps), rsqrtf(sc / kN + eps));
 }
 
 // The sequence-parallel form for few long sequences: the sequence of every unit is cut into
@@ -173,7 +174,7 @@ struct SegArgs {
 // kRaw: dt and lam arrive raw (m3_dims.flags) and the chunk scalars apply softplus / sigmoid.
 template <int R, bool kStateOnly, bool kRaw>
 __global__ void __launch_bounds__(kTcThreads, 2)
-scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const uint2* __restrict__ rsrow,
+scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const float2* __restrict__ rsrow,
                const SegArgs sa) {
     using Cfg = TcCfg<R>;
     constexpr int Q = Cfg::Q, TPS = Cfg::TPS;
@@ -183,8 +184,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     float* sf = reinterpret_cast<float*>(sm + Cfg::OF);   // two blocks of chunk scalars
     float2* s_seg = reinterpret_cast<float2*>(sf + F_SEG);
-    __nv_bfloat16* s_biasB2 = reinterpret_cast<__nv_bfloat16*>(sf + F_BIAS);  // [R][128] bf16
-    __nv_bfloat16* s_biasC2 = s_biasB2 + R * kN;
+    float* s_biasB = sf + F_BIAS;              // [R][128]
+    float* s_biasC = s_biasB + R * kN;
     // set-up only: the stored previous token's Bbar and x, in the H0 operand buffer
     float* s_fold = reinterpret_cast<float*>(sm + Cfg::OH);   // [R][128]
     float* s_foldx = s_fold + R * kN;                          // [R][64]
@@ -210,7 +211,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     // Per-unit base pointers; offsets below fit in 32 bits (checked on the host).
     const __nv_bfloat16* Bu = static_cast<const __nv_bfloat16*>(p.B) + (bb * p.L * G + g) * R * kN;
     const int Lpad = ((L + Q - 1) / Q) * Q;
-    const uint2* rsu = rsrow ? rsrow + (bb * G + g) * static_cast<int64_t>(Lpad) * R : nullptr;
+    const float2* rsu = rsrow ? rsrow + (bb * G + g) * static_cast<int64_t>(Lpad) * R : nullptr;
     const __nv_bfloat16* xu = static_cast<const __nv_bfloat16*>(p.x) + (bb * p.L * H + hh) * R * kP;
     __nv_bfloat16* yu = static_cast<__nv_bfloat16*>(p.y) + (bb * p.L * H + hh) * R * kP;
     const int tokB = G * R * kN, tokY = H * R * kP;  // element stride of one token
@@ -218,7 +219,7 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     const int cb = kseg * sa.seg_chunks;
     const int nchunks = min((L + Q - 1) / Q - cb, sa.seg_chunks);
     const int ib = static_cast<int>(bb), ih = static_cast<int>(hh), ig = static_cast<int>(g);
-    uint2* s_rs = reinterpret_cast<uint2*>(sm + Cfg::ORS);
+    float2* s_rs = reinterpret_cast<float2*>(sm + Cfg::ORS);
 
     // ---- TMA issue (one thread) ----
     auto issue_x = [&](int c) {
@@ -381,8 +382,8 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     for (int i = tid; i < R * kN; i += kTcThreads) {
-        s_biasB2[i] = __float2bfloat16_rn(p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f);
-        s_biasC2[i] = __float2bfloat16_rn(p.Cbias ? p.Cbias[hh * R * kN + i] : 0.f);
+        s_biasB[i] = p.Bbias ? p.Bbias[hh * R * kN + i] : 0.f;
+        s_biasC[i] = p.Cbias ? p.Cbias[hh * R * kN + i] : 0.f;
     }
     fence_before_sync();
     __syncthreads();
@@ -578,6 +579,20 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         }
     };
 
+    // One couple of rotation pairs (jp, jp + 1) of one operand row: byte offset o in the two
+    // 64-column slabs of src (raw, bf16) and dst (rotated, bf16); bias at [jp] and [jp + 64].
+    auto rotate_couple = [&](const uint8_t* src, uint8_t* dst, uint32_t o, float rs,
+                             const float* bias, float2 c, float2 s) {
+        const float2 r2 = make_float2(rs, rs);
+        const float2 u0 = __ffma2_rn(bf2_to_f2(*reinterpret_cast<const uint32_t*>(src + o)), r2,
+                                     *reinterpret_cast<const float2*>(bias));
+        const float2 u1 = __ffma2_rn(bf2_to_f2(*reinterpret_cast<const uint32_t*>(src + 8192 + o)),
+                                     r2, *reinterpret_cast<const float2*>(bias + kHalf));
+        *reinterpret_cast<uint32_t*>(dst + o) = f2_to_bf2(__ffma2_rn(u0, c, __fmul2_rn(u1, s)));
+        *reinterpret_cast<uint32_t*>(dst + 8192 + o) =
+            f2_to_bf2(__ffma2_rn(u1, c, __fmul2_rn(make_float2(-u0.x, -u0.y), s)));
+    };
+
     // Angles and rotation of chunk c (I1): the cumulative angle of every token, then B and C
     // (B only in the state-only pass) normalised, biased and rotated into their operand tiles.
     auto rotate = [&](const float* blk, uint32_t par) {
@@ -610,52 +625,45 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         car[1] += tot1;
         car_r[0] = reduce_2pi(car_r[0] + tot0);
         car_r[1] = reduce_2pi(car_r[1] + tot1);
-        uint32_t cw[TPS], sw[TPS];  // packed bf16 (cos, cos) and (sin, sin) of the couple
+        // Each token's angle, then its cos and sin: before the raw B and C have landed when
+        // they fit in registers (two tokens or fewer per warp), else token by token below.
+        constexpr bool kEarly = TPS <= 2;
+        float2 cse[kEarly ? TPS : 1], sne[kEarly ? TPS : 1];
+        if constexpr (kEarly) {
 #pragma unroll
-        for (int k = 0; k < TPS; ++k) {
-            a0 += inc[k][0];
-            a1 += inc[k][1];
-            float sn0, cs0, sn1, cs1;
-            __sincosf(a0, &sn0, &cs0);
-            __sincosf(a1, &sn1, &cs1);
-            cw[k] = pack_bf16(cs0, cs1);
-            sw[k] = pack_bf16(sn0, sn1);
+            for (int k = 0; k < TPS; ++k) {
+                a0 += inc[k][0];
+                a1 += inc[k][1];
+                __sincosf(a0, &sne[k].x, &cse[k].x);
+                __sincosf(a1, &sne[k].y, &cse[k].y);
+            }
         }
         if (!mbar_wait(&bar_b, par)) s_abort = 1;   // raw B and the RMS scales
         if constexpr (!kStateOnly) {
             if (!mbar_wait(&bar_c, par)) s_abort = 1;   // raw C
         }
-#pragma unroll 1
-        for (int r = 0; r < R; ++r) {
-            // bias words of this rank at the couple, both halves of each pair
-            const __nv_bfloat162 bB0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + jp);
-            const __nv_bfloat162 bB1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasB2 + r * kN + kHalf + jp);
+        // Every rank's B (and C) row at the couple: u = rs raw + bias on both halves of each
+        // pair, (u0, u1) -> (u0 c + u1 s, u1 c - u0 s), all in fp32 with one rounding to bf16.
 #pragma unroll
-            for (int k = 0; k < TPS; ++k) {
+        for (int k = 0; k < TPS; ++k) {
+            float2 cs, sn;
+            if constexpr (kEarly) {
+                cs = cse[k];
+                sn = sne[k];
+            } else {
+                a0 += inc[k][0];
+                a1 += inc[k][1];
+                __sincosf(a0, &sn.x, &cs.x);
+                __sincosf(a1, &sn.y, &cs.y);
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
                 const int row = (warp * TPS + k) * R + r;
                 const uint32_t o = swz128(row, jp);
-                const uint32_t rb0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + o);
-                const uint32_t rb1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::RB + 8192 + o);
-                const uint2 rsv = rsu ? s_rs[row] : make_uint2(0x3F803F80u, 0x3F803F80u);
-                const __nv_bfloat162 c2 = as_bf2(cw[k]), s2 = as_bf2(sw[k]);
-                // u = rs * raw + bias on both halves of each pair, then
-                // (u0, u1) -> (u0 c + u1 s, u1 c - u0 s)
-                __nv_bfloat162 u0 = __hfma2(as_bf2(rb0), as_bf2(rsv.x), bB0);
-                __nv_bfloat162 u1 = __hfma2(as_bf2(rb1), as_bf2(rsv.x), bB1);
-                *reinterpret_cast<uint32_t*>(sm + Cfg::OB + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
-                *reinterpret_cast<uint32_t*>(sm + Cfg::OB + 8192 + o) =
-                    as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
-                if constexpr (!kStateOnly) {
-                    const __nv_bfloat162 bC0 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + jp);
-                    const __nv_bfloat162 bC1 = *reinterpret_cast<const __nv_bfloat162*>(s_biasC2 + r * kN + kHalf + jp);
-                    const uint32_t rc0 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + o);
-                    const uint32_t rc1 = *reinterpret_cast<const uint32_t*>(sm + Cfg::OC + 8192 + o);
-                    u0 = __hfma2(as_bf2(rc0), as_bf2(rsv.y), bC0);
-                    u1 = __hfma2(as_bf2(rc1), as_bf2(rsv.y), bC1);
-                    *reinterpret_cast<uint32_t*>(sm + Cfg::OC + o) = as_u32(__hfma2(u0, c2, __hmul2(u1, s2)));
-                    *reinterpret_cast<uint32_t*>(sm + Cfg::OC + 8192 + o) =
-                        as_u32(__hfma2(u1, c2, __hneg2(__hmul2(u0, s2))));
-                }
+                const float2 rsv = rsu ? s_rs[row] : make_float2(1.f, 1.f);
+                rotate_couple(sm + Cfg::RB, sm + Cfg::OB, o, rsv.x, s_biasB + r * kN + jp, cs, sn);
+                if constexpr (!kStateOnly)
+                    rotate_couple(sm + Cfg::OC, sm + Cfg::OC, o, rsv.y, s_biasC + r * kN + jp, cs, sn);
             }
         }
     };
@@ -669,13 +677,14 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const ui
         for (int i = 0; i < 2; ++i) {
             const int e = tid + i * kTcThreads;
             const int row = e >> 3, ch = e & 7;
-            const __nv_bfloat162 sc2 = __float2bfloat162_rn(blk[F_DW + row / R]);
+            const float dw = blk[F_DW + row / R];
+            const float2 dw2 = make_float2(dw, dw);
             const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
-            uint4 v = *reinterpret_cast<const uint4*>(sX + o);
-            v.x = as_u32(__hmul2(as_bf2(v.x), sc2));
-            v.y = as_u32(__hmul2(as_bf2(v.y), sc2));
-            v.z = as_u32(__hmul2(as_bf2(v.z), sc2));
-            v.w = as_u32(__hmul2(as_bf2(v.w), sc2));
+            uint4 v = *reinterpret_cast<const uint4*>(sX + o);   // x dw in fp32, one rounding
+            v.x = f2_to_bf2(__fmul2_rn(bf2_to_f2(v.x), dw2));
+            v.y = f2_to_bf2(__fmul2_rn(bf2_to_f2(v.y), dw2));
+            v.z = f2_to_bf2(__fmul2_rn(bf2_to_f2(v.z), dw2));
+            v.w = f2_to_bf2(__fmul2_rn(bf2_to_f2(v.w), dw2));
             *reinterpret_cast<uint4*>(sm + Cfg::XP + o) = v;
         }
     };
@@ -1072,7 +1081,7 @@ SegArgs seg_plan(const ScanParams& p, size_t seg_bytes = ~size_t(0)) {
 size_t rs_bytes(const ScanParams& p) {
     const int64_t Q = 64 / (p.R > 0 ? p.R : 1);
     const int64_t Lpad = (p.L + Q - 1) / Q * Q;
-    const size_t n = p.bc_norm ? static_cast<size_t>(p.b * Lpad * p.G * p.R) * sizeof(uint2) : 0;
+    const size_t n = p.bc_norm ? static_cast<size_t>(p.b * Lpad * p.G * p.R) * sizeof(float2) : 0;
     return (n + 255) / 256 * 256;
 }
 
@@ -1087,7 +1096,7 @@ size_t tc_scan_workspace_bytes(const ScanParams& p) {
 size_t tc_scan_workspace_min_bytes(const ScanParams& p) { return rs_bytes(p); }
 
 template <int R, bool kRaw>
-static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa, cudaStream_t s,
+static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, const SegArgs& sa, cudaStream_t s,
                                bool state_only = false) {
     constexpr int Q = 64 / R;
     TcMaps maps;
@@ -1169,7 +1178,7 @@ static cudaError_t launch_tc_t(const ScanParams& p, uint2* rs, const SegArgs& sa
 cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,
                                  float* out_h, float* out_phi, float* out_lam, cudaStream_t s) {
     if (p.b * p.H == 0) return cudaSuccess;
-    uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
+    float2* rs = p.bc_norm ? static_cast<float2*>(ws_body) : nullptr;
     if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;
     // few long sequences: the sequence-parallel form, every segment's end state into the
     // workspace, then their combination; else one segment straight into out
@@ -1203,7 +1212,7 @@ cudaError_t launch_scan_tc(const ScanParams& p_in, void* ws_body, size_t body_by
     ScanParams p = p_in;
     if (const char* e = std::getenv("M3_TEST_SKIP_THETA_LOAD")) p.test_skip_theta = std::atoi(e);
     // workspace body: the RMS scales, then the segments' end states
-    uint2* rs = p.bc_norm ? static_cast<uint2*>(ws_body) : nullptr;
+    float2* rs = p.bc_norm ? static_cast<float2*>(ws_body) : nullptr;
     if (body_bytes < rs_bytes(p)) return cudaErrorInvalidValue;
     SegArgs sa = seg_plan(p, body_bytes - rs_bytes(p));
     if (sa.nseg > 1) sa.st = reinterpret_cast<float*>(static_cast<char*>(ws_body) + rs_bytes(p));
