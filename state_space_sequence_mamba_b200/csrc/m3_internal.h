@@ -44,7 +44,7 @@ struct ScanParams {
     void* prevx1;
     void* y;
     int32_t* status;  // device status word (workspace), may be null for decode
-    // Test hook of the tensor-core scan: > 0 makes CTA 0 skip the theta load of that chunk,
+    // Test hook of the tensor-core scans: > 0 makes CTA 0 skip the theta load of that chunk,
     // so that its bounded wait runs out and the timeout path (status word, drain, TMEM
     // release) is exercised. Set only from the M3_TEST_SKIP_THETA_LOAD environment variable.
     int32_t test_skip_theta;

@@ -40,6 +40,8 @@
 // rotation and TMEM groups one leader thread waits and a named barrier releases the group. All
 // waits are bounded, and a wait that gives up records the status word and lets every role
 // leave its loop.
+#include <cstdlib>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -789,10 +791,12 @@ scan_pipe_kernel(const ScanParams p, const __grid_constant__ PMaps maps,
                 if (c >= 2 && (!pwait(&bars[B_TH_EMPTY + st], (c >> 1) - 1, &s_abort) ||
                                !pwait(&bars[B_XP_EMPTY + st], (c >> 1) - 1, &s_abort)))
                     break;
-                mbar_arrive_expect_tx(&bars[B_TH_FULL + st], Cfg::TH_TX);
-                tma_load_4d(sm + Cfg::TH0 + st * Cfg::TH_STAGE, &maps.theta, &bars[B_TH_FULL + st], 0,
-                            ih, c * Q, ib);
-                if (st) ++n_th1; else ++n_th0;
+                if (!(blockIdx.x == 0 && c > 0 && c == p.test_skip_theta)) {   // (test hook)
+                    mbar_arrive_expect_tx(&bars[B_TH_FULL + st], Cfg::TH_TX);
+                    tma_load_4d(sm + Cfg::TH0 + st * Cfg::TH_STAGE, &maps.theta,
+                                &bars[B_TH_FULL + st], 0, ih, c * Q, ib);
+                    if (st) ++n_th1; else ++n_th0;
+                }
                 if (c >= 2 && !pwait(&bars[B_BC_EMPTY + st], (c >> 1) - 1, &s_abort)) break;
                 uint64_t* bar = &bars[B_BC_FULL + st];
                 mbar_arrive_expect_tx(bar, Cfg::BC_TX + (rsu ? kRows * 8u : 0u));
@@ -810,7 +814,8 @@ scan_pipe_kernel(const ScanParams p, const __grid_constant__ PMaps maps,
                             ih, c * Q, ib);
                 if (st) ++n_x1; else ++n_x0;
             }
-            if (s_abort) {   // let this CTA's copies land before the CTA exits
+            {   // every copy issued has landed before the CTA exits (at once unless a wait
+                // elsewhere gave up while copies were in flight)
                 constexpr long long kDrain = 200000000LL;
                 if (n_th0 > 0) (void)mbar_wait(&bars[B_TH_FULL], (n_th0 - 1) & 1, kDrain);
                 if (n_th1 > 0) (void)mbar_wait(&bars[B_TH_FULL1], (n_th1 - 1) & 1, kDrain);
@@ -1035,8 +1040,10 @@ bool pipe_scan_supported(const ScanParams& p, bool bf16) {
 
 size_t pipe_scan_workspace_bytes(const ScanParams& p) { return pipe_rs_bytes(p); }
 
-cudaError_t launch_scan_pipe(const ScanParams& p, void* ws_body, size_t body_bytes, cudaStream_t s) {
-    if (p.b * p.H == 0 || p.L == 0) return cudaSuccess;
+cudaError_t launch_scan_pipe(const ScanParams& p_in, void* ws_body, size_t body_bytes, cudaStream_t s) {
+    if (p_in.b * p_in.H == 0 || p_in.L == 0) return cudaSuccess;
+    ScanParams p = p_in;
+    if (const char* e = std::getenv("M3_TEST_SKIP_THETA_LOAD")) p.test_skip_theta = std::atoi(e);
     float2* rs = p.bc_norm ? static_cast<float2*>(ws_body) : nullptr;
     if (body_bytes < pipe_rs_bytes(p)) return cudaErrorInvalidValue;
     const bool raw = p.flags != 0;

@@ -22,17 +22,19 @@ from state_space_sequence_mamba_b200.inputs import make_problem
 pytestmark = pytest.mark.gpu
 
 
-def test_timeout_is_reported_and_the_workspace_reusable(cuda_dev):
-    pr = make_problem(2, 300, 4, 1, 64, 128, rank=1, chunk=64, bc_norm=True, bias_std=0.1,
-                      seed=151, with_state=True)
+@pytest.mark.parametrize("R,chunk", [(1, 64), (1, 128), (4, 32)])
+def test_timeout_is_reported_and_the_workspace_reusable(cuda_dev, R, chunk):
+    """Through the 64-row (chunk 64) and the 128-row (chunk 128 / R) tensor-core scans."""
+    pr = make_problem(2, 300, 4, 1, 64, 128, rank=R, chunk=chunk, bc_norm=True, bias_std=0.1,
+                      seed=151 + R, with_state=True)
     g = pr.to(cuda_dev)
     t = g.tensors()
-    dims = m3.make_dims(t["x"], t["B"], 64, True, 1e-6)
+    dims = m3.make_dims(t["x"], t["B"], chunk, True, 1e-6)
     ws = torch.zeros(m3.scan_workspace_bytes(dims), dtype=torch.uint8, device=cuda_dev)
     init = m3.State.from_dict(g.state)
     os.environ["M3_TEST_SKIP_THETA_LOAD"] = "1"
     try:
-        m3.scan_fwd(**t, init=init, chunk=64, bc_norm=True, workspace=ws)
+        m3.scan_fwd(**t, init=init, chunk=chunk, bc_norm=True, workspace=ws)
         torch.cuda.synchronize()
     finally:
         del os.environ["M3_TEST_SKIP_THETA_LOAD"]
@@ -41,7 +43,7 @@ def test_timeout_is_reported_and_the_workspace_reusable(cuda_dev):
     assert ei.value.status == m3.M3_ERR_TIMEOUT
     assert int(ws[:256].count_nonzero()) == 0          # the header is zero again
     # the same workspace, the same stream, right after: a normal call, checked exactly
-    y, fin = m3.scan_fwd(**t, init=init, chunk=64, bc_norm=True, workspace=ws)
+    y, fin = m3.scan_fwd(**t, init=init, chunk=chunk, bc_norm=True, workspace=ws)
     torch.cuda.synchronize()
     m3.scan_check(ws)
     yo, so = oracle_scan(pr)
