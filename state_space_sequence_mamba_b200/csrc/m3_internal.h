@@ -4,6 +4,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "../../include/m3.h"
 
 namespace m3 {
@@ -98,6 +100,28 @@ m3_status scan_fwd_with(const m3_dims* dims, const m3_inputs* in, const m3_state
                         size_t need, void* stream);
 // Records msg as this thread's m3_last_error() text and returns s.
 m3_status set_error(m3_status s, const char* msg);
+// The per-token RMS scales of B and C for the tensor-core scans: out[((b * G + g) * Lpad + l)
+// * R + r] = (1 / rms(B row), 1 / rms(C row)), Lpad = L rounded up to whole chunks of Q tokens.
+// The kernel lets a scan launched with launch_after_rms start before it finishes.
+cudaError_t launch_rms_scales(const ScanParams& p, int64_t Q, float2* out, cudaStream_t s);
+// Launches kernel<<<grid, block, smem, s>>>(args...) so that it may start while the kernel
+// before it in the stream (the RMS scales) finishes; the kernel must call grid_dep_wait()
+// before it reads that kernel's output.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after_rms(void (*kernel)(KArgs...), unsigned grid, unsigned block,
+                             size_t smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 // SM count of the calling thread's current device, looked up once per device (148, the
 // B200's count, when no device answers). Safe to call from several host threads.
 int device_sm_count();

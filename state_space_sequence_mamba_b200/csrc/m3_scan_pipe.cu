@@ -169,34 +169,6 @@ struct PMaps {
     CUtensorMap x, theta, B, C;
 };
 
-// RMS scale of every B and C row (shared by all heads), fp32: one warp per row of N = 128.
-// Rows (b, l, g, r) go to out[((b * G + g) * Lpad + l) * R + r], so one chunk's rows of one
-// group are contiguous (one bulk copy per chunk); Lpad rounds L up to whole chunks.
-__global__ void __launch_bounds__(256) rms_scale_f32_kernel(const __nv_bfloat16* __restrict__ B,
-                                                            const __nv_bfloat16* __restrict__ C,
-                                                            int64_t rows, int64_t L, int64_t G,
-                                                            int64_t R, int64_t Lpad, float eps,
-                                                            float2* __restrict__ out) {
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const int64_t r = row % R, g = (row / R) % G, l = (row / (R * G)) % L, b = row / (R * G * L);
-    const uint2 ub = __ldg(reinterpret_cast<const uint2*>(B + row * kN) + lane);
-    const uint2 uc = __ldg(reinterpret_cast<const uint2*>(C + row * kN) + lane);
-    float sb = 0.f, sc = 0.f;
-    const uint32_t wb[2] = {ub.x, ub.y}, wc[2] = {uc.x, uc.y};
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float2 b2 = unpack2(wb[i]), c2 = unpack2(wc[i]);
-        sb = fmaf(b2.x, b2.x, fmaf(b2.y, b2.y, sb));
-        sc = fmaf(c2.x, c2.x, fmaf(c2.y, c2.y, sc));
-    }
-    sb = warp_sum(sb);
-    sc = warp_sum(sc);
-    if (lane == 0)
-        out[((b * G + g) * Lpad + l) * R + r] = make_float2(rsqrtf(sb / kN + eps), rsqrtf(sc / kN + eps));
-}
-
 // Waits for the phase of `bar` with the given parity, giving up when another role has
 // recorded an abort or after ~max_cycles SM clocks (then records the abort itself). Between
 // checks the warp is suspended in the wait instruction itself (up to kSuspendNs, or until the
@@ -805,6 +777,7 @@ scan_pipe_kernel(const ScanParams p, const __grid_constant__ PMaps maps,
                 tma_load_5d(base + Cfg::SLAB, &maps.B, bar, kHalf, 0, ig, c * Q, ib);
                 tma_load_5d(base + Cfg::C_OFF, &maps.C, bar, 0, 0, ig, c * Q, ib);
                 tma_load_5d(base + Cfg::C_OFF + Cfg::SLAB, &maps.C, bar, kHalf, 0, ig, c * Q, ib);
+                if (rsu && c == 0) grid_dep_wait();   // the scales' kernel may still run
                 if (rsu) bulk_load(sm + Cfg::RS + st * (kRows * 8), rsu + static_cast<int64_t>(c) * Q * R,
                                    kRows * 8u, bar);
                 if (st) ++n_bc1; else ++n_bc0;
@@ -1011,12 +984,7 @@ cudaError_t launch_pipe_t(const ScanParams& p, float2* rs, cudaStream_t s) {
             return cudaErrorInvalidValue;
     }
     if (rs) {
-        const int64_t rows = p.b * p.L * p.G * R;
-        const int64_t Lpad = (p.L + Q - 1) / Q * Q;
-        rms_scale_f32_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
-            p.L, p.G, R, Lpad, p.eps, rs);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_rms_scales(p, Q, rs, s);
         if (e != cudaSuccess) return e;
     }
     auto k = scan_pipe_kernel<R, kRaw>;
@@ -1024,6 +992,9 @@ cudaError_t launch_pipe_t(const ScanParams& p, float2* rs, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    if (rs)   // may start while the scales' kernel finishes (the TMA lane waits for it)
+        return launch_after_rms(k, static_cast<unsigned>(p.b * p.H), kThreads, smem, s, p, maps,
+                                static_cast<const float2*>(rs));
     k<<<static_cast<unsigned>(p.b * p.H), kThreads, smem, s>>>(p, maps, rs);
     return cudaGetLastError();
 }

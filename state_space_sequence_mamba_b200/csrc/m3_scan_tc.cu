@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
                                                         int64_t rows, int64_t L, int64_t G,
                                                         int64_t R, int64_t Lpad, float eps,
                                                         float2* __restrict__ out) {
+    grid_dep_launch_dependents();   // the scan's set-up may overlap this kernel
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -247,7 +248,10 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
         mbar_arrive_expect_tx(&bar_b, Cfg::B_TX + (rsu ? 512u : 0u));
         tma_load_5d(sm + Cfg::RB, &maps.B, &bar_b, 0, 0, ig, (cb + c) * Q, ib);
         tma_load_5d(sm + Cfg::RB + 8192, &maps.B, &bar_b, kHalf, 0, ig, (cb + c) * Q, ib);
-        if (rsu) bulk_load(s_rs, rsu + static_cast<int64_t>(cb + c) * Q * R, 512u, &bar_b);
+        if (rsu) {
+            if (c == 0) grid_dep_wait();   // the scales' kernel may still be running
+            bulk_load(s_rs, rsu + static_cast<int64_t>(cb + c) * Q * R, 512u, &bar_b);
+        }
         s_issued[3] += 1;
     };
     auto issue_c = [&](int c) {   // raw C rows of chunk c straight into the Cbar operand buffer
@@ -1087,6 +1091,16 @@ size_t rs_bytes(const ScanParams& p) {
 
 }  // namespace
 
+cudaError_t launch_rms_scales(const ScanParams& p, int64_t Q, float2* out, cudaStream_t s) {
+    const int64_t rows = p.b * p.L * p.G * p.R;
+    if (rows == 0) return cudaSuccess;
+    const int64_t Lpad = (p.L + Q - 1) / Q * Q;
+    rms_scale_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
+        p.L, p.G, p.R, Lpad, p.eps, out);
+    return cudaGetLastError();
+}
+
 size_t tc_scan_workspace_bytes(const ScanParams& p) {
     const SegArgs sa = seg_plan(p);
     const size_t seg = sa.nseg > 1 ? static_cast<size_t>(p.b * p.H) * sa.nseg * kSegStride * sizeof(float) : 0;
@@ -1139,40 +1153,33 @@ static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, const SegArgs& s
             return cudaErrorInvalidValue;
     }
     if (rs) {
-        const int64_t rows = p.b * p.L * p.G * R;
-        const int64_t Lpad = (p.L + Q - 1) / Q * Q;
-        rms_scale_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
-            p.L, p.G, R, Lpad, p.eps, rs);
-        cudaError_t e = cudaGetLastError();
+        cudaError_t e = launch_rms_scales(p, Q, rs, s);
         if (e != cudaSuccess) return e;
     }
     const uint32_t smem = tc_smem_bytes<R>();
     const int64_t units = p.b * p.H;
-    if (state_only) {   // m3_scan_state: every segment's end state
-        auto ks = scan_tc_kernel<R, true, kRaw>;
-        cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    // the first scan kernel after the scales' kernel may start while that one finishes (it
+    // waits for it only before its first load of the scales)
+    bool first = rs != nullptr;
+    auto launch = [&](auto kern, int64_t grid) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
-        const int64_t segs = sa.out_h ? 1 : sa.nseg;
-        ks<<<static_cast<unsigned>(units * segs), kTcThreads, smem, s>>>(p, maps, rs, sa);
+        if (first) {
+            first = false;
+            return launch_after_rms(kern, static_cast<unsigned>(grid), kTcThreads, smem, s, p,
+                                    maps, static_cast<const float2*>(rs), sa);
+        }
+        kern<<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(p, maps, rs, sa);
         return cudaGetLastError();
-    }
+    };
+    if (state_only)   // m3_scan_state: every segment's end state
+        return launch(scan_tc_kernel<R, true, kRaw>, units * (sa.out_h ? 1 : sa.nseg));
     if (sa.nseg > 1) {   // every segment's end state but the last's
-        auto ks = scan_tc_kernel<R, true, kRaw>;
-        cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        ks<<<static_cast<unsigned>(units * (sa.nseg - 1)), kTcThreads, smem, s>>>(p, maps, rs, sa);
-        e = cudaGetLastError();
+        cudaError_t e = launch(scan_tc_kernel<R, true, kRaw>, units * (sa.nseg - 1));
         if (e != cudaSuccess) return e;
     }
-    auto k = scan_tc_kernel<R, false, kRaw>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    k<<<static_cast<unsigned>(units * sa.nseg), kTcThreads, smem, s>>>(p, maps, rs, sa);
-    return cudaGetLastError();
+    return launch(scan_tc_kernel<R, false, kRaw>, units * sa.nseg);
 }
 
 cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,
