@@ -61,7 +61,8 @@ typedef struct {
     int64_t headdim;  /* P in {16, 32, 64, 128}                                    */
     int64_t dstate;   /* N, a multiple of 16, <= 256                               */
     int64_t rank;     /* R in {1, 2, 4, 8}; 1 = SISO                                */
-    int64_t chunk;    /* tokens per chunk of the prefill scan (chunk * R <= 128)    */
+    int64_t chunk;    /* tokens per chunk of the prefill scan (chunk * R <= 128;
+                         64 or 128 rows run on the tensor cores, see m3_scan_fwd)  */
     int32_t in_dtype; /* m3_dtype                                                   */
     int32_t bc_norm;  /* nonzero: RMS-normalise B and C over N before the bias      */
     float norm_eps;   /* epsilon of the RMS norm (1e-6 is the usual value)          */
@@ -130,7 +131,11 @@ typedef struct {
 M3_API size_t m3_scan_workspace_bytes(const m3_dims* dims);
 
 /* Chunked parallel prefill scan over a whole sequence (Sec. 3.1.3 parallel form, Sec. 3.3
- * chunked algorithm).
+ * chunked algorithm). The chunk length is a tile size: the result does not depend on it
+ * beyond rounding. bf16 inputs with N = 128 and P = 64 run on the tensor cores when
+ * chunk * R = 64 (any R) or chunk * R = 128 (R <= 4, a warp-specialised kernel with one CTA
+ * per (batch, head) and per SM); other shapes, other chunk lengths and fp32 run on the
+ * CUDA cores in exact fp32.
  *   init      state before token 0, or NULL for a fresh sequence (all zeros).
  *   final     where to write the state after token L-1, or NULL to skip; may alias init.
  *   y         [b, L, H, R, P] in_dtype output, y_t = H_t^T Cbar_t.
