@@ -229,9 +229,9 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
     uint32_t mma_phase = 0;
     for (int i = 0; u < n_units; ++i, u += gridDim.x) {
         const int s = i % kRing;
-        // the next unit's dt, A, lam: loaded into registers now, stored to its slot at the end
-        // of this unit (raw scalars transformed there), so the load latency is spent on this
-        // unit's work
+        // the next unit's dt, A, lam: loaded into registers now, stored to its slot after this
+        // unit's state update (raw scalars transformed there), so the load latency is spent on
+        // this unit's work
         float snext[4] = {0.f, 0.f, 0.f, 0.f};   // dt, A, lam, dt bias
         uint8_t* sl = sm + Cfg::SM0 + s * Cfg::S_BYTES;
         uint8_t* hb = sm + Cfg::HB + s * Cfg::H_BYTES;
@@ -418,6 +418,14 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
             }
             __syncwarp();
         }
+        // the next unit's step scalars (softplus / sigmoid of raw ones) into its slot, which no
+        // one reads during this unit; here their loads have long landed and the work overlaps
+        // the copy-out and the readout instead of delaying the unit's last barrier
+        if (tid == 0) {
+            scal[4 * (s ^ 1) + 0] = step_dt<kRaw>(snext[0], snext[3], p.flags);
+            scal[4 * (s ^ 1) + 1] = snext[1];
+            scal[4 * (s ^ 1) + 2] = step_lam<kRaw>(snext[2], p.flags);
+        }
         // ---- the updated state to HBM: consecutive threads take consecutive 16-byte pieces of
         // the [N][P] row-major state (piece c of row n: box c / 8, 32-byte chunk (c mod 8) / 2)
         {
@@ -466,11 +474,6 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                     for (int r = 0; r < R; ++r) yo[r * kP] = __float2bfloat16_rn(yv[r]);
                 }
             }
-        }
-        if (tid == 0) {
-            scal[4 * (s ^ 1) + 0] = step_dt<kRaw>(snext[0], snext[3], p.flags);
-            scal[4 * (s ^ 1) + 1] = snext[1];
-            scal[4 * (s ^ 1) + 2] = step_lam<kRaw>(snext[2], p.flags);
         }
         fence_before_sync();
         __syncthreads();
