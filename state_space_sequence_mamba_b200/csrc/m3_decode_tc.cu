@@ -335,17 +335,12 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                     // X[r][p] = W_X[h][r][p] x'[p]; written over x' (this thread alone reads
                     // x'[p]) as the stored previous token, which is bulk-copied from there
                     const float xin = __bfloat162float(sx[i]);
-                    float* sw = reinterpret_cast<float*>(sl + Cfg::S_W) + i;
+                    const float* sw = reinterpret_cast<const float*>(sl + Cfg::S_W) + i;
                     __nv_bfloat16* sxw = reinterpret_cast<__nv_bfloat16*>(sl + Cfg::S_X);
-                    const float zin = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sl + Cfg::S_Z)[i]);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         vx[r] = sw[r * kP] * xin;
                         sxw[r * kP + i] = __float2bfloat16_rn(vx[r]);
-                        // the output weight of Y[r][p], independent of Y: g = W_O SiLU(W_Z z'),
-                        // over W_Z (this thread alone reads column p)
-                        const float z = sw[(R + r) * kP] * zin;
-                        sw[(R + r) * kP] = sw[(2 * R + r) * kP] * z * __frcp_rn(1.f + __expf(-z));
                     }
                 } else {
 #pragma unroll
@@ -368,6 +363,18 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                 mma_commit(smem_u32(&bar_u));
             }
             __syncwarp();
+        }
+        if constexpr (kProj) {
+            // the output weights of Y[r][p], independent of Y: g = W_O SiLU(W_Z z'), written
+            // over W_Z by all threads while the update MMA runs (read after the next barrier)
+            float* sw = reinterpret_cast<float*>(sl + Cfg::S_W);
+            const __nv_bfloat16* sz = reinterpret_cast<const __nv_bfloat16*>(sl + Cfg::S_Z);
+#pragma unroll
+            for (int e = tid; e < R * kP; e += kThreads) {
+                const int r = e / kP, pc = e % kP;
+                const float z = sw[(R + r) * kP + pc] * __bfloat162float(sz[pc]);
+                sw[(R + r) * kP + pc] = sw[(2 * R + r) * kP + pc] * z * __frcp_rn(1.f + __expf(-z));
+            }
         }
         if (!mbar_wait(&bar_u, mma_phase)) s_abort = 1;
         fence_after_sync();
@@ -462,7 +469,7 @@ decode_tc_kernel(const ScanParams p, const __grid_constant__ DecMaps maps, const
                 const int pcol = 16 * warp + lane;
                 if constexpr (kProj) {
                     // O'[p] = sum_r W_O[h][r][p] SiLU(W_Z[h][r][p] z'[p]) Y[r][p], the gate
-                    // factors already formed during the rotation
+                    // factors formed while the update MMA ran
                     const float* gw = reinterpret_cast<const float*>(sl + Cfg::S_W) + R * kP + pcol;
                     float o = 0.f;
 #pragma unroll
