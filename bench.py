@@ -230,8 +230,9 @@ def run_ours(args):
     if args.backward_only:
         out = {"backward": {
             name: bench_backward(m3, dev, cfg, hbm, world, dist, rank_seed(rank, 11 + cfg),
-                                 reps=args.steps, seqlen=args.bwd_seqlen)
-            for name, cfg in (("siso_b4", 1), ("mimo_r4_b4", 2))}, "peak_hbm_gbs": hbm,
+                                 reps=args.steps, seqlen=args.bwd_seqlen, exact=exact)
+            for name, cfg, exact in (("siso_b4", 1, False), ("siso_b4_fp32", 1, True),
+                                     ("mimo_r4_b4", 2, False))}, "peak_hbm_gbs": hbm,
             "seqlen": args.bwd_seqlen or 2048}
         if rank == 0:
             print(json.dumps(out), flush=True)
@@ -412,6 +413,8 @@ def run_ours(args):
         backward["siso_b4_L2048"] = bench_backward(m3, dev, 1, hbm, world, dist,
                                                    rank_seed(rank, 11),
                                                    cpu=(rank == 0 and world == 1))
+        backward["siso_b4_L2048_fp32"] = bench_backward(m3, dev, 1, hbm, world, dist,
+                                                        rank_seed(rank, 11), exact=True)
         backward["mimo_r4_b4_L2048"] = bench_backward(m3, dev, 2, hbm, world, dist,
                                                       rank_seed(rank, 12))
 
@@ -507,8 +510,10 @@ def bwd_bytes(pr) -> int:
     return reads + writes
 
 
-def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cpu=False):
-    """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1)."""
+def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cpu=False,
+                   exact=False):
+    """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1); with
+    exact, the fp32 sequential sweeps (M3_BWD_FP32) instead of the path the call picks."""
     import torch
     from state_space_sequence_mamba_b200.inputs import make_config
     kw = {} if seqlen is None else {"seqlen": seqlen}
@@ -517,14 +522,18 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cp
     g = torch.Generator(device=dev).manual_seed(seed + 1)
     dy = torch.randn(pr.x.shape, generator=g, device=dev).to(d.dtype)
     init = m3.State.from_dict(pr.state)
-    ws = torch.empty(m3.scan_bwd_workspace_bytes(
-        m3.make_dims(pr.x, pr.B, 1, d.bc_norm, d.norm_eps, pr.flags)), dtype=torch.uint8,
-        device=dev)
+    sa = pr.scalar_args()
+    if exact:
+        sa["flags"] = sa["flags"] | m3.BWD_FP32
+    dims = m3.make_dims(pr.x, pr.B, 1, d.bc_norm, d.norm_eps, sa["flags"])
+    ws = torch.empty(m3.scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
+    tc = (not exact and d.dtype == torch.bfloat16 and d.rank == 1 and d.dstate == 128
+          and d.headdim == 64 and d.nheads % 4 == 0)
     stream = torch.cuda.current_stream()
 
     def step():   # the config's own BC norm, eps and scalar form, as the CPU baseline reads them
         return m3.scan_bwd(**pr.tensors(), dy=dy, init=init, bc_norm=d.bc_norm,
-                           norm_eps=d.norm_eps, workspace=ws, stream=stream, **pr.scalar_args())
+                           norm_eps=d.norm_eps, workspace=ws, stream=stream, **sa)
 
     for _ in range(3):
         step()
@@ -539,7 +548,11 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cp
     byts = bwd_bytes(pr)
     out = {"ms_per_backward": ms, "tokens_per_s": d.batch * d.seqlen * world / (ms / 1e3),
            "bytes": byts, "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm,
-           "kernels_per_call": 5 if d.bc_norm else 4, "workspace_bytes": ws.numel()}
+           # chunked: [RMS scales], state pass, chunk kernel, bias sums, scalar, norm;
+           # sequential: [RMS scales], two sweeps, scalar, norm
+           "form": "tensor-core chunked" if tc else "fp32 sequential sweeps",
+           "kernels_per_call": (5 if tc else 4) + (1 if d.bc_norm else 0),
+           "workspace_bytes": ws.numel()}
     if cpu:   # an auxiliary field: a failure here is reported, not fatal to the bench line
         try:
             out["cpu_baseline"] = cpu_baseline_backward(pr, dy)

@@ -84,6 +84,10 @@ typedef struct {
 #define M3_DT_SOFTPLUS 1u
 #define M3_LAM_SIGMOID 2u
 #define M3_DISC_ZOH 4u
+/* m3_scan_bwd only: compute every product of the backward in fp32 on the CUDA cores (the
+ * sequential sweeps), also where the chunked tensor-core backward applies. Other entry points
+ * ignore it. */
+#define M3_BWD_FP32 8u
 
 typedef struct {
     const void* x;        /* [b, L, H, R, P]   in_dtype                                   */
@@ -229,23 +233,37 @@ typedef struct {
     float* prev_x;  /* [b, H, R, P] */
 } m3_state_grad;
 
-/* Workspace bytes m3_scan_bwd needs (0 for invalid dims): two fp32 [b, L, H, R, N] buffers
- * plus O(b H (L + N L / 16)) floats. Any content; it is scratch. */
+/* Workspace bytes m3_scan_bwd needs (0 for invalid dims): a 256-byte status header, two
+ * fp32 [b, L, H, R, N] buffers plus O(b H (L + N L / 16)) floats, and where the chunked
+ * tensor-core form runs (see m3_scan_bwd) 16 KB per unit and 64-token chunk for the chunk
+ * states plus O(b H N P) floats. Any content: the call resets the status word itself. */
 M3_API size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims);
 
-/* dims, in, init: as given to m3_scan_fwd (dims->chunk is not used here). dy [b, L, H, R, P]
+/* Gradients of the prefill scan ("Mamba-3: Improved Sequence Modeling using State Space
+ * Principles", the recurrence of Sec. 3.1.1 Prop. 1 with the rotation of Sec. 3.2.2 Prop. 4,
+ * differentiated; Sec. 3.3 for the chunked form).
+ * dims, in, init: as given to m3_scan_fwd (dims->chunk is not used here). dy [b, L, H, R, P]
  * in_dtype. dfinal: the final state's gradient, or NULL. grads: dx .. dlam are required
  * (16-byte aligned) and overwritten; the bias gradients are overwritten when not NULL.
  * dinit: where to write the initial state's gradient, or NULL. workspace: 256-byte aligned,
  * at least m3_scan_bwd_workspace_bytes. Any supported N, P, R, dtype and flags; asynchronous
- * on `stream`. Not bitwise reproducible run to run: some sums use atomic adds, whose order
- * varies in the last bits (m3_scan_fwd and the decode step are reproducible). */
+ * on `stream`.
+ * Two forms compute the same gradients:
+ *  - bf16 inputs with R = 1, N = 128, P = 64 and H a multiple of 4 run the chunked form on the
+ *    tensor cores (64-token chunks, bf16 operands with fp32 accumulators, fp32 state
+ *    adjoint), bitwise reproducible run to run except the dt_bias gradient (an atomic sum
+ *    over units). Its bounded waits report a timeout through the workspace's status word,
+ *    which m3_scan_check reads after the stream has synchronised.
+ *  - every other shape, and any shape with M3_BWD_FP32 in dims->flags, runs two sequential
+ *    sweeps in fp32 on the CUDA cores; not bitwise reproducible run to run (some sums use
+ *    atomic adds, whose order varies in the last bits). */
 M3_API m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
                              const void* dy, const m3_state_grad* dfinal,
                              const m3_grads* grads, const m3_state_grad* dinit,
                              void* workspace, size_t ws_bytes, void* stream);
 
-/* After the stream that ran m3_scan_fwd has synchronised: M3_OK, or M3_ERR_TIMEOUT if a
+/* After the stream that ran m3_scan_fwd (or m3_scan_bwd, on its workspace) has synchronised:
+ * M3_OK, or M3_ERR_TIMEOUT if a
  * bounded inter-CTA wait gave up (the outputs of that call are then incomplete). Performs
  * one blocking 4-byte device-to-host copy; after a timeout it also re-zeroes the workspace
  * header (blocking) so the workspace can be reused. */

@@ -16,8 +16,10 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 
 M3_OK, M3_ERR_INVALID_ARG, M3_ERR_UNSUPPORTED, M3_ERR_CUDA, M3_ERR_TIMEOUT = range(5)
 M3_F32, M3_BF16 = 0, 1
-# m3_dims.flags: the step scalars arrive raw and the kernels apply softplus / sigmoid
-M3_DT_SOFTPLUS, M3_LAM_SIGMOID, M3_DISC_ZOH = 1, 2, 4
+# m3_dims.flags: the step scalars arrive raw and the kernels apply softplus / sigmoid; the
+# zero-order-hold discretisation; the backward in fp32 on the CUDA cores
+M3_DT_SOFTPLUS, M3_LAM_SIGMOID, M3_DISC_ZOH, M3_BWD_FP32 = 1, 2, 4, 8
+BWD_FP32 = M3_BWD_FP32
 
 
 class M3Error(RuntimeError):

@@ -43,7 +43,7 @@ m3_status check_dims(const m3_dims* d, bool scan) {
         return fail(M3_ERR_INVALID_ARG, "headdim >= 1, even dstate >= 2 and rank >= 1 required");
     if (!(d->norm_eps >= 0.f) || !std::isfinite(d->norm_eps))
         return fail(M3_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
-    if (d->flags & ~(M3_DT_SOFTPLUS | M3_LAM_SIGMOID | M3_DISC_ZOH))
+    if (d->flags & ~(M3_DT_SOFTPLUS | M3_LAM_SIGMOID | M3_DISC_ZOH | M3_BWD_FP32))
         return fail(M3_ERR_INVALID_ARG, "unknown bits in flags (0x%x)", (unsigned)d->flags);
     if (d->headdim != 16 && d->headdim != 32 && d->headdim != 64 && d->headdim != 128)
         return fail(M3_ERR_UNSUPPORTED, "headdim %lld not in {16, 32, 64, 128}",
@@ -101,7 +101,7 @@ ScanParams make_params(const m3_dims* d, const m3_inputs* in, const m3_state* in
     p.bc_norm = d->bc_norm ? 1 : 0; p.eps = d->norm_eps;
     p.x = in->x; p.B = in->B; p.C = in->C; p.theta = in->theta;
     p.dt = in->dt; p.A = in->A; p.lam = in->lam; p.Bbias = in->B_bias; p.Cbias = in->C_bias;
-    p.dt_bias = in->dt_bias; p.flags = d->flags;
+    p.dt_bias = in->dt_bias; p.flags = d->flags & ~M3_BWD_FP32;   // a choice of path, not of scalars
     if (init) { p.h0 = init->h; p.phi0 = init->phi; p.prevB0 = init->prev_B; p.prevx0 = init->prev_x; }
     if (fin) { p.h1 = fin->h; p.phi1 = fin->phi; p.prevB1 = fin->prev_B; p.prevx1 = fin->prev_x; }
     p.y = y;
@@ -393,10 +393,23 @@ const char* m3_last_error(void) { return g_err; }
 
 extern "C" {
 
-size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims) {
-    if (check_dims(dims, false) != M3_OK) return 0;
+// The backward's workspace: the status header, the sequential form's intermediate buffers,
+// then (where the chunked tensor-core form runs) its chunk states.
+static size_t bwd_simt_bytes(const m3_dims* dims) {
     return sizeof(float) * scan_bwd_workspace_floats(dims->batch, dims->seqlen, dims->nheads,
                                                      dims->dstate, dims->rank);
+}
+static bool bwd_uses_tc(const m3_dims* dims, const m3::ScanParams& p) {
+    return !(dims->flags & M3_BWD_FP32) && bwd_tc_supported(p, dims->in_dtype == M3_BF16);
+}
+
+size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims) {
+    if (check_dims(dims, false) != M3_OK) return 0;
+    m3_inputs none{};
+    const ScanParams p = make_params(dims, &none, nullptr, nullptr, nullptr);
+    size_t n = kWsHeader + (bwd_simt_bytes(dims) + 255) / 256 * 256;
+    if (bwd_uses_tc(dims, p)) n += bwd_tc_workspace_bytes(p);
+    return n;
 }
 
 m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* init,
@@ -458,7 +471,7 @@ m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
     const size_t need = m3_scan_bwd_workspace_bytes(dims);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
         return fail(M3_ERR_INVALID_ARG, "workspace: NULL, misaligned or below %zu bytes", need);
-    const ScanParams p = make_params(dims, in, init, nullptr, nullptr);
+    ScanParams p = make_params(dims, in, init, nullptr, nullptr);
     BwdGrads g{};
     g.dy = dy;
     if (dfinal) { g.dh1 = dfinal->h; g.dphi1 = dfinal->phi; g.dprevB1 = dfinal->prev_B; g.dprevx1 = dfinal->prev_x; }
@@ -466,7 +479,15 @@ m3_status m3_scan_bwd(const m3_dims* dims, const m3_inputs* in, const m3_state* 
     g.ddt = grads->ddt; g.dA = grads->dA; g.dlam = grads->dlam;
     g.dBbias = grads->dB_bias; g.dCbias = grads->dC_bias; g.ddtbias = grads->ddt_bias;
     if (dinit) { g.dh0 = dinit->h; g.dphi0 = dinit->phi; g.dprevB0 = dinit->prev_B; g.dprevx0 = dinit->prev_x; }
-    cudaError_t e = launch_scan_bwd(p, g, dims->in_dtype == M3_BF16, static_cast<float*>(workspace), s);
+    char* ws = static_cast<char*>(workspace);
+    int32_t* status = reinterpret_cast<int32_t*>(ws);
+    void* tc_ws = bwd_uses_tc(dims, p) ? ws + kWsHeader + (bwd_simt_bytes(dims) + 255) / 256 * 256
+                                       : nullptr;
+    p.status = status;
+    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess)
+        e = launch_scan_bwd(p, g, dims->in_dtype == M3_BF16,
+                            reinterpret_cast<float*>(ws + kWsHeader), tc_ws, status, s);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
     return M3_OK;
 }

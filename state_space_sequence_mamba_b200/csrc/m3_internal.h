@@ -163,8 +163,49 @@ int bwd_chunk_tokens(int64_t R);
 size_t scan_bwd_workspace_floats(int64_t b, int64_t L, int64_t H, int64_t N, int64_t R);
 size_t scan_bwd_smem_bytes(int64_t N, int64_t P, int64_t R);
 // f: the forward's inputs and initial state (validated); ws: scan_bwd_workspace_floats floats,
-// 256-byte aligned. L >= 1 and b >= 1.
+// 256-byte aligned. L >= 1 and b >= 1. tc_ws: bwd_tc_workspace_bytes more (256-byte aligned)
+// when bwd_tc_supported, which then runs the chunked tensor-core backward; status: the
+// device status word the tensor-core kernels set when a bounded wait gives up.
 cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, float* ws,
-                            cudaStream_t s);
+                            void* tc_ws, int32_t* status, cudaStream_t s);
+
+// Chunked backward on the tensor cores (bf16, R = 1, N = 128, P = 64, H % 4 == 0, without
+// M3_BWD_FP32): the forward state pass, then one CTA per unit over its chunks in reverse.
+bool bwd_tc_supported(const ScanParams& p, bool bf16);
+size_t bwd_tc_workspace_bytes(const ScanParams& p);
+// Where the chunked backward writes: the sequential backward's intermediate buffers (wdB,
+// wdC [b,L,H,N], wsc [units][L][4], wprev [units][N], wF [units]) and the gradients it
+// produces itself.
+struct BwdTcOut {
+    const void* dy;
+    const float* dh1;
+    const float* dphi1;
+    const float* dprevx1;
+    float* dx;
+    float* dtheta;
+    float* wdB;
+    float* wdC;
+    float* wsc;
+    float* wprev;
+    float* wF;
+    float* dh0;
+    float* dphi0;
+    float* dprevx0;
+    float* dBbias;
+    float* dCbias;
+    int32_t* status;
+};
+cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cudaStream_t s);
+// The tensor-core scan's state-only pass over whole sequences, for the backward: per unit
+// and chunk, e^{cum_0} H0' (bf16 in the swizzled [n][p] operand layout, 16384 bytes) into
+// chunk_h and the angle before the chunk into chunk_phi [64]; the final state into hfin
+// [units][N][P], phifin [units][N/2], lamfin [units]. rs: the RMS-scale buffer or null.
+cudaError_t launch_bwd_states_tc(const ScanParams& p, float2* rs, uint8_t* chunk_h,
+                                 float* chunk_phi, float* hfin, float* phifin, float* lamfin,
+                                 cudaStream_t s);
+// cuTensorMapEncodeTiled for a bf16 (else fp32) tensor, 128-byte swizzle (else none), unit
+// element strides; map points at a CUtensorMap.
+bool encode_tmap(void* map, bool bf16, int rank, const void* base, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, bool swizzle128);
 
 }  // namespace m3

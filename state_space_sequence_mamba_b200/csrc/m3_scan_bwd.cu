@@ -1146,7 +1146,7 @@ size_t scan_bwd_workspace_floats(int64_t b, int64_t L, int64_t H, int64_t N, int
 }
 
 cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, float* ws,
-                            cudaStream_t s) {
+                            void* tc_ws, int32_t* status, cudaStream_t s) {
     BwdArgs a{};
     a.f = f;
     a.dy = g.dy;
@@ -1173,24 +1173,39 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
     }
 
     cudaError_t e;
-    if (a.dBbias && (e = cudaMemsetAsync(a.dBbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
-    if (a.dCbias && (e = cudaMemsetAsync(a.dCbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
     if (a.ddtbias && (e = cudaMemsetAsync(a.ddtbias, 0, sizeof(float) * f.H, s)) != cudaSuccess) return e;
-    const BwdLayout lay = bwd_layout(a.T, static_cast<int>(f.R), static_cast<int>(f.N),
-                                     static_cast<int>(f.P), bf16 ? 2 : 4);
-    const size_t smem = sizeof(float) * lay.total;
-    if (f.bc_norm) {
-        const int64_t items = f.b * f.L * f.G * f.R + units * f.R;
-        bwd_rms_kernel<<<static_cast<unsigned>((items * 32 + 255) / 256), 256, 0, s>>>(a, bf16 ? 1 : 0);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (tc_ws) {
+        // the chunked tensor-core form writes dx, dtheta, the initial state's h, phi and
+        // prev_x gradients, the bias gradients and the intermediate buffers of the two kernels
+        // below in place of the sweeps
+        BwdTcOut o{};
+        o.dy = g.dy;
+        o.dh1 = g.dh1; o.dphi1 = g.dphi1; o.dprevx1 = g.dprevx1;
+        o.dx = g.dx; o.dtheta = g.dtheta;
+        o.wdB = a.wdB; o.wdC = a.wdC; o.wsc = a.wsc; o.wprev = a.wprev; o.wF = a.wF;
+        o.dh0 = g.dh0; o.dphi0 = g.dphi0; o.dprevx0 = g.dprevx0;
+        o.dBbias = g.dBbias; o.dCbias = g.dCbias;
+        o.status = status;
+        if ((e = launch_bwd_tc(f, o, tc_ws, s)) != cudaSuccess) return e;
+    } else {
+        if (a.dBbias && (e = cudaMemsetAsync(a.dBbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
+        if (a.dCbias && (e = cudaMemsetAsync(a.dCbias, 0, sizeof(float) * f.H * f.R * f.N, s)) != cudaSuccess) return e;
+        const BwdLayout lay = bwd_layout(a.T, static_cast<int>(f.R), static_cast<int>(f.N),
+                                         static_cast<int>(f.P), bf16 ? 2 : 4);
+        const size_t smem = sizeof(float) * lay.total;
+        if (f.bc_norm) {
+            const int64_t items = f.b * f.L * f.G * f.R + units * f.R;
+            bwd_rms_kernel<<<static_cast<unsigned>((items * 32 + 255) / 256), 256, 0, s>>>(a, bf16 ? 1 : 0);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+        if (f.N <= 128)
+            e = bf16 ? launch_sweeps_p<__nv_bfloat16, 256>(a, smem, s)
+                     : launch_sweeps_p<float, 256>(a, smem, s);
+        else
+            e = bf16 ? launch_sweeps_p<__nv_bfloat16, 512>(a, smem, s)
+                     : launch_sweeps_p<float, 512>(a, smem, s);
+        if (e != cudaSuccess) return e;
     }
-    if (f.N <= 128)
-        e = bf16 ? launch_sweeps_p<__nv_bfloat16, 256>(a, smem, s)
-                 : launch_sweeps_p<float, 256>(a, smem, s);
-    else
-        e = bf16 ? launch_sweeps_p<__nv_bfloat16, 512>(a, smem, s)
-                 : launch_sweeps_p<float, 512>(a, smem, s);
-    if (e != cudaSuccess) return e;
     bwd_scalar_kernel<<<static_cast<unsigned>(units), kScalThreads, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t items = f.b * f.L * f.G * f.R * 2 + units * f.R;

@@ -130,7 +130,17 @@ __global__ void __launch_bounds__(256) rms_scale_kernel(const __nv_bfloat16* __r
     grid_dep_launch_dependents();   // the scan's set-up may overlap this kernel
     const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
+    if (row >= rows) {
+        // the rows past the sequence end in the last chunk: zero scales (their B and C rows are
+        // zero-filled loads, so the scaled value is 0 whatever the workspace held before)
+        const int64_t pr = row - rows, pad = Lpad - L;
+        if (lane == 0 && pad > 0 && pr < (rows / (L * G * R)) * G * pad * R) {
+            const int64_t r = pr % R, g = (pr / R) % G, l = L + (pr / (R * G)) % pad;
+            const int64_t b = pr / (R * G * pad);
+            out[((b * G + g) * Lpad + l) * R + r] = make_float2(0.f, 0.f);
+        }
+        return;
+    }
     const int64_t r = row % R, g = (row / R) % G, l = (row / (R * G)) % L, b = row / (R * G * L);
     const int64_t orow = ((b * G + g) * Lpad + l) * R + r;
     const uint2 ub = __ldg(reinterpret_cast<const uint2*>(B + row * kN) + lane);
@@ -167,6 +177,10 @@ struct SegArgs {
     // the state-only pass keeps segment 0's primed initial state in slot nseg-1 for the full
     // pass (not when every segment's end state is wanted, as for m3_scan_state)
     bool save_init = true;
+    // one segment, for the backward: per unit and chunk, e^{cum_0} H0' as bf16 in the swizzled
+    // [n][p] operand layout (16384 bytes) and the angle before the chunk (64 floats)
+    uint8_t* chunk_h = nullptr;
+    float* chunk_phi = nullptr;
 };
 
 // One CTA per (unit, segment), CTA index = segment * units + unit. kStateOnly: the segment's
@@ -716,6 +730,24 @@ scan_tc_kernel(const ScanParams p, const __grid_constant__ TcMaps maps, const fl
                     raw_box(c + 1);
                 }
             }
+            if (sa.chunk_h) {
+                // the primed state before this chunk, scaled by its first token's decay, and the
+                // angle before it, for the backward's per-chunk products
+                const float e0 = blk[F_ECUM];
+                uint8_t* dst = sa.chunk_h + (u * nchunks + c) * 16384;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint4 v;
+                    v.x = pack_bf16(e0 * hreg[8 * i + 0], e0 * hreg[8 * i + 1]);
+                    v.y = pack_bf16(e0 * hreg[8 * i + 2], e0 * hreg[8 * i + 3]);
+                    v.z = pack_bf16(e0 * hreg[8 * i + 4], e0 * hreg[8 * i + 5]);
+                    v.w = pack_bf16(e0 * hreg[8 * i + 6], e0 * hreg[8 * i + 7]);
+                    *reinterpret_cast<uint4*>(dst + swz128(nrow, 32 * wh + 8 * i)) = v;
+                }
+                if (warp == 0)
+                    *reinterpret_cast<float2*>(sa.chunk_phi + (u * nchunks + c) * kHalf + jp) =
+                        make_float2(car[0], car[1]);
+            }
             if (!mbar_wait(&bar_th, par)) s_abort = 1;   // theta of this chunk
             rotate(blk, par);
             if (warp == kIssueWarp) {
@@ -1095,7 +1127,8 @@ cudaError_t launch_rms_scales(const ScanParams& p, int64_t Q, float2* out, cudaS
     const int64_t rows = p.b * p.L * p.G * p.R;
     if (rows == 0) return cudaSuccess;
     const int64_t Lpad = (p.L + Q - 1) / Q * Q;
-    rms_scale_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+    const int64_t all = rows + p.b * p.G * (Lpad - p.L) * p.R;   // padded rows get zero scales
+    rms_scale_kernel<<<static_cast<unsigned>((all + 7) / 8), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(p.B), static_cast<const __nv_bfloat16*>(p.C), rows,
         p.L, p.G, p.R, Lpad, p.eps, out);
     return cudaGetLastError();
@@ -1180,6 +1213,38 @@ static cudaError_t launch_tc_t(const ScanParams& p, float2* rs, const SegArgs& s
         if (e != cudaSuccess) return e;
     }
     return launch(scan_tc_kernel<R, false, kRaw>, units * sa.nseg);
+}
+
+bool encode_tmap(void* map, bool bf16, int rank, const void* base, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, bool swizzle128) {
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    return encode(static_cast<CUtensorMap*>(map),
+                  bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank,
+                  base, d, st, bx, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+cudaError_t launch_bwd_states_tc(const ScanParams& p_in, float2* rs, uint8_t* chunk_h,
+                                 float* chunk_phi, float* hfin, float* phifin, float* lamfin,
+                                 cudaStream_t s) {
+    if (p_in.b * p_in.H == 0 || p_in.R != 1) return cudaErrorInvalidValue;
+    ScanParams p = p_in;
+    p.Q = 64;
+    SegArgs sa;
+    sa.seg_chunks = static_cast<int>((p.L + 63) / 64);
+    sa.nseg = 1;
+    sa.out_h = hfin;
+    sa.out_phi = phifin;
+    sa.out_lam = lamfin;
+    sa.save_init = false;
+    sa.chunk_h = chunk_h;
+    sa.chunk_phi = chunk_phi;
+    return p.flags ? launch_tc_t<1, true>(p, rs, sa, s, true) : launch_tc_t<1, false>(p, rs, sa, s, true);
 }
 
 cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,

@@ -59,7 +59,7 @@ def test_struct_layout_matches_header(lib):
     (dict(headdim=48), False), (dict(rank=3), False), (dict(chunk=0), False),
     (dict(chunk=64, rank=4), False), (dict(chunk=16, rank=4), True), (dict(in_dtype=7), False),
     (dict(dstate=272), False), (dict(norm_eps=-1.0), False), (dict(batch=-1), False),
-    (dict(flags=7), True), (dict(flags=8), False),
+    (dict(flags=7), True), (dict(flags=8), True), (dict(flags=16), False),
 ])
 def test_workspace_query_validates(lib, kw, ok):
     n = lib.m3_scan_workspace_bytes(ctypes.byref(dims(**kw)))
@@ -121,9 +121,20 @@ def test_backward_workspace_and_argument_checks(lib):
     T = 16
     r64 = lambda v: (v + 63) // 64 * 64
     units, nch = 2 * 4, (100 + T - 1) // T
-    want = 4 * (2 * r64(2 * 100 * 4 * 128) + r64(units * nch * 64) + r64(units)
+    simt = 4 * (2 * r64(2 * 100 * 4 * 128) + r64(units * nch * 64) + r64(units)
                 + r64(units * 100 * 4) + r64(units * 128) + r64(2 * 2 * 100 * 4) + r64(units))
-    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d)) == want
+    r256 = lambda v: (v + 255) // 256 * 256
+    base = 256 + r256(simt)   # status header, the sequential sweeps' buffers
+    # bf16, R = 1, N = 128, P = 64, H % 4 == 0: the chunked tensor-core form's chunk states
+    # (16 KB and the chunk's angle per unit and 64-token chunk), final state, bias sums, scales
+    n64 = (100 + 63) // 64
+    tc = (r256(units * n64 * 16384) + r256(units * n64 * 64 * 4) + r256(units * 128 * 64 * 4)
+          + r256(units * 65 * 4) + r256(units * 2 * 128 * 4) + r256(2 * n64 * 64 * 1 * 8))
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d)) == base + tc
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(batch=2, seqlen=100, nheads=4,
+                                                             flags=bd.M3_BWD_FP32))) == base
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(batch=2, seqlen=100, nheads=4,
+                                                             in_dtype=bd.M3_F32))) == base
     assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
     assert ctypes.sizeof(bd.Grads) == 10 * 8
     ins = fake_inputs()

@@ -35,10 +35,15 @@ def draw_grads(pr, seed, with_final=True):
     return dy, dfin
 
 
-def gpu_grads(pr, dy, dfin, dev):
+def gpu_grads(pr, dy, dfin, dev, exact=True):
+    """exact: the fp32 sequential sweeps (M3_BWD_FP32); else the path m3_scan_bwd picks, the
+    chunked tensor-core form where it applies."""
     g = pr.to(dev)
     init = m3.State.from_dict(g.state) if g.state is not None else None
-    out = m3.scan_bwd(**g.tensors(), dy=dy.to(dev), **g.scalar_args(), init=init,
+    sa = g.scalar_args()
+    if exact:
+        sa["flags"] = sa["flags"] | m3.BWD_FP32
+    out = m3.scan_bwd(**g.tensors(), dy=dy.to(dev), **sa, init=init,
                       dfinal=None if dfin is None else {k: v.to(dev) for k, v in dfin.items()},
                       bc_norm=pr.dims.bc_norm, norm_eps=pr.dims.norm_eps)
     torch.cuda.synchronize()
