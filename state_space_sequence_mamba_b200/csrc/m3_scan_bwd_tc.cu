@@ -177,10 +177,14 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     float* s_cu = reinterpret_cast<float*>(sm + S_CU);
     float* s_tok = reinterpret_cast<float*>(sm + S_TOK);
     float* sphi = reinterpret_cast<float*>(sm + S_PHI);
-    __shared__ uint64_t bar_ld, bar_m1, bar_g, bar_m2;
+    // loads in four groups, each issued as soon as the previous chunk has released its buffers:
+    // A (scalar boxes, raw B, RMS scales, the chunk's start angle), X, H (the chunk-start state),
+    // B (theta, dY, raw C)
+    __shared__ uint64_t bar_a, bar_x, bar_h, bar_b, bar_m1, bar_g, bar_m2;
     __shared__ uint32_t tslot;
     __shared__ int s_abort;
-    __shared__ int s_cnt[4];   // loads issued, and MMA groups m1, g, m2 committed
+    __shared__ int s_cnt[4];   // MMA groups m1, g, m2 committed (index 1..3)
+    __shared__ int s_lcnt[4];  // load groups A, X, H, B issued
     __shared__ float s_wred[8];
     __shared__ float s_t4[8];
     __shared__ float s_dnext;   // D'_t of the first token of the chunk after the current one
@@ -197,37 +201,58 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     const bool zoh = kRaw && (p.flags & M3_DISC_ZOH);
     const float2* rsu = a.rs ? a.rs + (bb * p.G + g) * Lpad : nullptr;
 
-    auto issue_loads = [&](int c) {
-        const uint32_t tx = 3 * 8192 + 2 * 16384 + 3 * SC_ONE + (rsu ? 512u : 0u) + 16384 + 256;
-        mbar_arrive_expect_tx(&bar_ld, tx);
+    auto issue_a = [&](int c) {
         const int t0 = c * kQ;
-        tma_load_5d(sm + S_XT, &maps.x, &bar_ld, 0, 0, ih, t0, ib);
-        tma_load_5d(sm + S_DT, &maps.dy, &bar_ld, 0, 0, ih, t0, ib);
-        tma_load_4d(sm + S_TH, &maps.theta, &bar_ld, 0, ih, t0, ib);
-        tma_load_5d(sm + S_RB, &maps.B, &bar_ld, 0, 0, ig, t0, ib);
-        tma_load_5d(sm + S_RB + 8192, &maps.B, &bar_ld, kHalf, 0, ig, t0, ib);
-        tma_load_5d(sm + S_CT, &maps.C, &bar_ld, 0, 0, ig, t0, ib);
-        tma_load_5d(sm + S_CT + 8192, &maps.C, &bar_ld, kHalf, 0, ig, t0, ib);
+        mbar_arrive_expect_tx(&bar_a, 3 * SC_ONE + 16384 + (rsu ? 512u : 0u) + 256);
         const int h4 = ih & ~3;
-        tma_load_3d(sm + S_SC, &maps.dt, &bar_ld, h4, t0, ib);
-        tma_load_3d(sm + S_SC + SC_SLOT, &maps.A, &bar_ld, h4, t0, ib);
-        tma_load_3d(sm + S_SC + 2 * SC_SLOT, &maps.lam, &bar_ld, h4, t0, ib);
-        if (rsu) bulk_load(sm + S_RS, rsu + t0, 512u, &bar_ld);
-        bulk_load(sm + S_HS, a.chunk_h + (u * nch + c) * 16384, 16384u, &bar_ld);
-        bulk_load(sm + S_PHI0, a.chunk_phi + (u * nch + c) * kHalf, 256u, &bar_ld);
-        s_cnt[0] += 1;
+        tma_load_3d(sm + S_SC, &maps.dt, &bar_a, h4, t0, ib);
+        tma_load_3d(sm + S_SC + SC_SLOT, &maps.A, &bar_a, h4, t0, ib);
+        tma_load_3d(sm + S_SC + 2 * SC_SLOT, &maps.lam, &bar_a, h4, t0, ib);
+        tma_load_5d(sm + S_RB, &maps.B, &bar_a, 0, 0, ig, t0, ib);
+        tma_load_5d(sm + S_RB + 8192, &maps.B, &bar_a, kHalf, 0, ig, t0, ib);
+        if (rsu) bulk_load(sm + S_RS, rsu + t0, 512u, &bar_a);
+        bulk_load(sm + S_PHI0, a.chunk_phi + (u * nch + c) * kHalf, 256u, &bar_a);
+        s_lcnt[0] += 1;
+    };
+    auto issue_x = [&](int c) {
+        mbar_arrive_expect_tx(&bar_x, 8192);
+        tma_load_5d(sm + S_XT, &maps.x, &bar_x, 0, 0, ih, c * kQ, ib);
+        s_lcnt[1] += 1;
+    };
+    auto issue_h = [&](int c) {
+        mbar_arrive_expect_tx(&bar_h, 16384);
+        bulk_load(sm + S_HS, a.chunk_h + (u * nch + c) * 16384, 16384u, &bar_h);
+        s_lcnt[2] += 1;
+    };
+    auto issue_b = [&](int c) {
+        const int t0 = c * kQ;
+        mbar_arrive_expect_tx(&bar_b, 8192 + 8192 + 16384);
+        tma_load_4d(sm + S_TH, &maps.theta, &bar_b, 0, ih, t0, ib);
+        tma_load_5d(sm + S_DT, &maps.dy, &bar_b, 0, 0, ih, t0, ib);
+        tma_load_5d(sm + S_CT, &maps.C, &bar_b, 0, 0, ig, t0, ib);
+        tma_load_5d(sm + S_CT + 8192, &maps.C, &bar_b, kHalf, 0, ig, t0, ib);
+        s_lcnt[3] += 1;
     };
 
     // ---------------- set-up ----------------
     if (tid == 0) {
-        mbar_init(&bar_ld, 1);
+        mbar_init(&bar_a, 1);
+        mbar_init(&bar_x, 1);
+        mbar_init(&bar_h, 1);
+        mbar_init(&bar_b, 1);
         mbar_init(&bar_m1, 1);
         mbar_init(&bar_g, 1);
         mbar_init(&bar_m2, 1);
         fence_mbar_init();
         s_abort = 0;
         s_cnt[0] = s_cnt[1] = s_cnt[2] = s_cnt[3] = 0;
-        if (nch > 0) issue_loads(nch - 1);
+        s_lcnt[0] = s_lcnt[1] = s_lcnt[2] = s_lcnt[3] = 0;
+        if (nch > 0) {
+            issue_a(nch - 1);
+            issue_b(nch - 1);
+            issue_x(nch - 1);
+            issue_h(nch - 1);
+        }
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
     for (int i = tid; i < 2 * kN; i += kThreads) {
@@ -304,7 +329,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         const uint32_t par = static_cast<uint32_t>(it & 1);
         const int t0 = c * kQ;
         const int T = (L - t0) < kQ ? (L - t0) : kQ;
-        if (!mbar_wait(&bar_ld, par)) s_abort = 1;
+        if (!mbar_wait(&bar_a, par)) s_abort = 1;   // scalar boxes, raw B, scales, start angle
         if constexpr (kRaw) {
             // this head's column of the dt and lam boxes: softplus / sigmoid in place
             float* sSc = reinterpret_cast<float*>(sm + S_SC);
@@ -381,25 +406,10 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             }
         }
         __syncthreads();
-        {
-            // <G_n, e^{cum_0} H0'> (this thread's 32 elements; summed per warp)
-            float t4 = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 hv = *reinterpret_cast<const uint4*>(sm + S_HS + swz128(nrow, 32 * wh + 8 * i));
-                const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = bf2_to_f2(hw[j]);
-                    t4 = fmaf(gr[8 * i + 2 * j], f.x, fmaf(gr[8 * i + 2 * j + 1], f.y, t4));
-                }
-            }
-            t4 = warp_sum(t4);
-            if (lane == 0) s_t4[warp] = t4;
-        }
 
         // ---- angles of the chunk and the rotation of B and C (warp = 8 tokens, lane = pair
         // couple (2 lane, 2 lane + 1), partners + N/2) ----
+        if (!mbar_wait(&bar_b, par)) s_abort = 1;   // theta, dY, raw C
         {
             const int jp = 2 * lane;
             constexpr int TPS = kQ / 8;
@@ -466,6 +476,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             }
         }
         // ---- Xs = diag(vn) X and Ds = diag(e^{cum - cum_0}) dY (rows keep their swizzle) ----
+        if (!mbar_wait(&bar_x, par)) s_abort = 1;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int e = tid + i * kThreads;
@@ -521,6 +532,8 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             mma_commit(smem_u32(&bar_g));
             s_cnt[1] += 1;
             s_cnt[2] += 1;
+            // the rotation and the scalars have read their inputs: the earlier chunk's group A
+            if (c > 0) issue_a(c - 1);
         }
         __syncwarp();
 
@@ -603,6 +616,23 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             }
         }
         // ---- G_0 = Cbar^T Ds + e^{cx_T - cum_0} G_n: the next (earlier) chunk's G_n ----
+        if (!mbar_wait(&bar_h, par)) s_abort = 1;   // e^{cum_0} H0'
+        {   // before G_n is replaced
+            // <G_n, e^{cum_0} H0'> (this thread's 32 elements; summed per warp)
+            float t4 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 hv = *reinterpret_cast<const uint4*>(sm + S_HS + swz128(nrow, 32 * wh + 8 * i));
+                const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = bf2_to_f2(hw[j]);
+                    t4 = fmaf(gr[8 * i + 2 * j], f.x, fmaf(gr[8 * i + 2 * j + 1], f.y, t4));
+                }
+            }
+            t4 = warp_sum(t4);
+            if (lane == 0) s_t4[warp] = t4;
+        }
         {
             if (!mbar_wait(&bar_g, par)) s_abort = 1;
             fence_after_sync();
@@ -676,6 +706,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                          desc_pack(loHm + (mnmajor_off(k) >> 4), hi), id64, k > 0);
             mma_commit(smem_u32(&bar_m2));
             s_cnt[3] += 1;
+            if (c > 0) issue_x(c - 1);   // X was last read by Z, Xs and the q sums
         }
         __syncwarp();
         // per-token dg and the next token's db (threads 0..63, fixed summation order)
@@ -702,6 +733,15 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         {
             if (!mbar_wait(&bar_m2, par)) s_abort = 1;
             fence_after_sync();
+            if (tid == 0 && c > 0) issue_h(c - 1);   // its readers (T4, dCbar, Yo) are done
+            {   // theta into the Ps buffer (read by dx, done): its own buffer takes the next load
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int e = tid + i * kThreads;
+                    *reinterpret_cast<uint4*>(sm + S_PS + 16 * e) =
+                        *reinterpret_cast<const uint4*>(sm + S_TH + 16 * e);
+                }
+            }
             const int t = trow;
             const bool real = t < T;
             const int64_t tok = static_cast<int64_t>(t0) + t;
@@ -772,6 +812,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         __syncthreads();
         fence_after_sync();
         if (s_abort) break;
+        if (tid == 0 && c > 0) issue_b(c - 1);   // theta copied, dY and Cbar read
 
         // ---- the angle adjoint's suffix sum over the sequence: dPhi_t = carry + sum_{s>=t} dl_s;
         // dtheta = dt dPhi; theta . dPhi per token (4 segments of 16 tokens per pair) ----
@@ -791,7 +832,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 if (t < T) {
                     const int64_t tok = static_cast<int64_t>(t0) + t;
                     a.dtheta[((bb * L + tok) * H + hh) * kHalf + i] = sf[F_DT + t] * acc;
-                    const uint16_t thb = *reinterpret_cast<const uint16_t*>(sm + S_TH + swz128(t, i));
+                    const uint16_t thb = *reinterpret_cast<const uint16_t*>(sm + S_PS + swz128(t, i));
                     thd = __uint_as_float(static_cast<uint32_t>(thb) << 16) * acc;
                 }
                 sphi[t * kPhiStride + i] = thd;
@@ -873,7 +914,6 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             if (lane == 0) s_dnext = dp[0];
         }
         __syncthreads();
-        if (tid == 0 && c > 0) issue_loads(c - 1);
     }
 
     // ---------------- the initial state's gradients (token -1) ----------------
@@ -988,7 +1028,10 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         if (a.status) atomicExch(a.status, 1);
         // let this CTA's own copies and MMAs finish (bounded) before TMEM is released
         constexpr long long kDrain = 200000000LL;
-        if (s_cnt[0] > 0) (void)mbar_wait(&bar_ld, (s_cnt[0] - 1) & 1, kDrain);
+        if (s_lcnt[0] > 0) (void)mbar_wait(&bar_a, (s_lcnt[0] - 1) & 1, kDrain);
+        if (s_lcnt[1] > 0) (void)mbar_wait(&bar_x, (s_lcnt[1] - 1) & 1, kDrain);
+        if (s_lcnt[2] > 0) (void)mbar_wait(&bar_h, (s_lcnt[2] - 1) & 1, kDrain);
+        if (s_lcnt[3] > 0) (void)mbar_wait(&bar_b, (s_lcnt[3] - 1) & 1, kDrain);
         if (s_cnt[1] > 0) (void)mbar_wait(&bar_m1, (s_cnt[1] - 1) & 1, kDrain);
         if (s_cnt[2] > 0) (void)mbar_wait(&bar_g, (s_cnt[2] - 1) & 1, kDrain);
         if (s_cnt[3] > 0) (void)mbar_wait(&bar_m2, (s_cnt[3] - 1) & 1, kDrain);
