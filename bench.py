@@ -527,8 +527,8 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cp
         sa["flags"] = sa["flags"] | m3.BWD_FP32
     dims = m3.make_dims(pr.x, pr.B, 1, d.bc_norm, d.norm_eps, sa["flags"])
     ws = torch.empty(m3.scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
-    tc = (not exact and d.dtype == torch.bfloat16 and d.rank == 1 and d.dstate == 128
-          and d.headdim == 64 and d.nheads % 4 == 0)
+    tc = (not exact and d.dtype == torch.bfloat16 and d.rank in (1, 2, 4, 8)
+          and d.dstate == 128 and d.headdim == 64 and d.nheads % 4 == 0)
     stream = torch.cuda.current_stream()
 
     def step():   # the config's own BC norm, eps and scalar form, as the CPU baseline reads them

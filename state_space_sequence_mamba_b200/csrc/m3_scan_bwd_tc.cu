@@ -62,7 +62,7 @@ constexpr uint32_t S_RB = 98304;      // raw B (TMA)
 constexpr uint32_t S_GN = 114688;     // G_n bf16 [n][p], two buffers of 16384
 constexpr uint32_t S_HS = 147456;     // e^{cum_0} H0' bf16 [n][p] (bulk copy)
 constexpr uint32_t S_TH = 163840;     // theta [t][i] (TMA)
-constexpr uint32_t SC_ONE = (kQ + 1) * 16, SC_SLOT = 1152;   // [Q + 1 tokens][4 heads] fp32
+constexpr uint32_t SC_SLOT = 1152;   // room for [Q + 1 tokens][4 heads] fp32, Q <= 64
 constexpr uint32_t S_SC = 172032;     // dt, A, lam boxes
 constexpr uint32_t S_RS = S_SC + 3 * SC_SLOT;            // RMS scales, 64 float2
 constexpr uint32_t S_PHI0 = S_RS + 512;                  // angle before the chunk, 64 floats
@@ -72,16 +72,15 @@ constexpr uint32_t S_RED = S_F + 4 * 800;                // row partials [5 kind
 constexpr uint32_t S_CU = S_RED + 4 * 5 * 4 * 64;        // column partials [4 row blocks][64]
 constexpr uint32_t S_TOK = S_CU + 4 * 4 * 64;            // per-token dg, db_{t+1}: [2][64]
 constexpr uint32_t S_SEG = S_TOK + 4 * 2 * 64;           // angle walk: [8 segments][32] float2
-constexpr uint32_t S_BIAS = S_SEG + 2048;                // bias_B, bias_C fp32 [2][128]
-constexpr uint32_t S_SUF = S_BIAS + 1024;                // suffix-scan segment sums [4][64]
+constexpr uint32_t S_BIAS = S_SEG + 2048;                // bias_B, bias_C fp32 [2][R][128]
+constexpr uint32_t S_SUF = S_BIAS + 8192;                // suffix-scan segment sums [4][64]
 constexpr uint32_t S_CAR = S_SUF + 1024;                 // angle-adjoint carry [64]
-constexpr uint32_t S_PREV = S_CAR + 256;                 // token -1 work area, 1024 floats
-constexpr uint32_t S_END = S_PREV + 4096;
+constexpr uint32_t S_END = S_CAR + 256;
 constexpr uint32_t kSmemBytes = S_END + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // chunk scalars (float offsets into S_F)
-constexpr int F_C2 = 0;      // [65] log2e * cum_t (t < 64), log2e * cx_T at [64]
+constexpr int F_C2 = 0;      // [65] log2e * cum_t (t < Q), log2e * cx_T at [Q]
 constexpr int F_GAM = 80;    // gamma_t
 constexpr int F_W = 144;     // w_t
 constexpr int F_VN = 208;    // w_t e^{cx_T - cum_t}
@@ -89,7 +88,7 @@ constexpr int F_EE = 272;    // e^{cx_T - cum_t}
 constexpr int F_EB = 336;    // e^{cx_T - cum_{t+1}} (1 for the chunk's last token)
 constexpr int F_DS = 400;    // e^{cum_t - cum_0}
 constexpr int F_DT = 464;    // dt_t
-constexpr int F_BETA = 528;  // [65] beta_t; beta of the next chunk's first token at [64]
+constexpr int F_BETA = 528;  // [65] beta_t; beta of the next chunk's first token at [Q]
 constexpr int F_MISC = 600;  // e^{cx_T - cum_0}, alpha_0, beta_0
 // row-partial kinds
 constexpr int R_KG = 0, R_KB = 1, R_Q = 2, R_RU = 3, R_V = 4;
@@ -132,21 +131,21 @@ __device__ __forceinline__ void load_row16(const uint8_t* tile, int row, int c, 
 
 struct BwdTcArgs {
     ScanParams p;
-    const float2* rs;          // RMS scales [b][G][Lpad] (x: B, y: C), null without the norm
+    const float2* rs;          // RMS scales [b][G][Lpad][R] (x: B, y: C), null without the norm
     const uint8_t* chunk_h;    // [units][nch][16384]: e^{cum_0} H0' bf16, swizzled [n][p]
     const float* chunk_phi;    // [units][nch][64]: the angle before each chunk
     const float* hfin;         // [units][N][P]: the final state
     const float* dh1;          // gradients of the final state (nullable)
     const float* dphi1;
     const float* dprevx1;
-    float* dx;                 // [b, L, H, P]
+    float* dx;                 // [b, L, H, R, P]
     float* dtheta;             // [b, L, H, N/2]
-    float* wdB;                // [b, L, H, N]: dBbar rotated back (per head)
+    float* wdB;                // [b, L, H, R, N]: dBbar rotated back (per head)
     float* wdC;
-    float* wsc;                // [units][L][4]: db, dg, dy.y, theta.dPhi per token
-    float* wprev;              // [units][N]: the same for the initial state's previous B
+    float* wsc;                // [units][L][4]: db, dg, decay term, theta.dPhi per token
+    float* wprev;              // [units][R][N]: the same for the initial state's previous B
     float* wF;                 // [units]: <dL/dh_final, h_final>
-    float* wbias;              // [units][2][N]: this unit's bias sums (B, C)
+    float* wbias;              // [units][2][R][N]: this unit's bias sums (B, C)
     float* dh0;                // initial-state gradients (nullable)
     float* dphi0;
     float* dprevx0;
@@ -160,9 +159,13 @@ struct BwdMaps {
 
 namespace {
 
-template <bool kRaw>
+// R: the rank; a chunk is Q = 64 / R tokens, its 64 operand rows are (token, rank) pairs,
+// row = token * R + rank, and the token mask acts on full R x R blocks.
+template <int R, bool kRaw>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
+    constexpr int Q = kQ / R;                      // tokens per chunk
+    constexpr uint32_t SC_ONE = (Q + 1) * 16;      // bytes of one scalar box
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -173,7 +176,6 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     float* s_bias = reinterpret_cast<float*>(sm + S_BIAS);
     float* s_suf = reinterpret_cast<float*>(sm + S_SUF);
     float* s_car = reinterpret_cast<float*>(sm + S_CAR);
-    float* s_prev = reinterpret_cast<float*>(sm + S_PREV);
     float* s_cu = reinterpret_cast<float*>(sm + S_CU);
     float* s_tok = reinterpret_cast<float*>(sm + S_TOK);
     float* sphi = reinterpret_cast<float*>(sm + S_PHI);
@@ -196,13 +198,13 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     const int ib = static_cast<int>(bb), ih = static_cast<int>(hh), ig = static_cast<int>(g);
     const int hc = ih & 3;
     const int64_t H = p.H;
-    const int64_t Lpad = static_cast<int64_t>(nch) * kQ;
+    const int64_t Lpad = static_cast<int64_t>(nch) * Q;
     const float dtb = (kRaw && p.dt_bias) ? p.dt_bias[hh] : 0.f;
     const bool zoh = kRaw && (p.flags & M3_DISC_ZOH);
-    const float2* rsu = a.rs ? a.rs + (bb * p.G + g) * Lpad : nullptr;
+    const float2* rsu = a.rs ? a.rs + (bb * p.G + g) * Lpad * R : nullptr;
 
     auto issue_a = [&](int c) {
-        const int t0 = c * kQ;
+        const int t0 = c * Q;
         mbar_arrive_expect_tx(&bar_a, 3 * SC_ONE + 16384 + (rsu ? 512u : 0u) + 256);
         const int h4 = ih & ~3;
         tma_load_3d(sm + S_SC, &maps.dt, &bar_a, h4, t0, ib);
@@ -210,13 +212,13 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         tma_load_3d(sm + S_SC + 2 * SC_SLOT, &maps.lam, &bar_a, h4, t0, ib);
         tma_load_5d(sm + S_RB, &maps.B, &bar_a, 0, 0, ig, t0, ib);
         tma_load_5d(sm + S_RB + 8192, &maps.B, &bar_a, kHalf, 0, ig, t0, ib);
-        if (rsu) bulk_load(sm + S_RS, rsu + t0, 512u, &bar_a);
+        if (rsu) bulk_load(sm + S_RS, rsu + static_cast<int64_t>(t0) * R, 512u, &bar_a);
         bulk_load(sm + S_PHI0, a.chunk_phi + (u * nch + c) * kHalf, 256u, &bar_a);
         s_lcnt[0] += 1;
     };
     auto issue_x = [&](int c) {
         mbar_arrive_expect_tx(&bar_x, 8192);
-        tma_load_5d(sm + S_XT, &maps.x, &bar_x, 0, 0, ih, c * kQ, ib);
+        tma_load_5d(sm + S_XT, &maps.x, &bar_x, 0, 0, ih, c * Q, ib);
         s_lcnt[1] += 1;
     };
     auto issue_h = [&](int c) {
@@ -225,8 +227,8 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         s_lcnt[2] += 1;
     };
     auto issue_b = [&](int c) {
-        const int t0 = c * kQ;
-        mbar_arrive_expect_tx(&bar_b, 8192 + 8192 + 16384);
+        const int t0 = c * Q;
+        mbar_arrive_expect_tx(&bar_b, Q * 128 + 8192 + 16384);
         tma_load_4d(sm + S_TH, &maps.theta, &bar_b, 0, ih, t0, ib);
         tma_load_5d(sm + S_DT, &maps.dy, &bar_b, 0, 0, ih, t0, ib);
         tma_load_5d(sm + S_CT, &maps.C, &bar_b, 0, 0, ig, t0, ib);
@@ -255,9 +257,9 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         }
     }
     if (warp == 0) tmem_alloc(&tslot, kTmemCols);
-    for (int i = tid; i < 2 * kN; i += kThreads) {
-        const float* bsrc = i < kN ? p.Bbias : p.Cbias;
-        s_bias[i] = bsrc ? bsrc[hh * kN + (i & (kN - 1))] : 0.f;
+    for (int i = tid; i < 2 * R * kN; i += kThreads) {
+        const float* bsrc = i < R * kN ? p.Bbias : p.Cbias;
+        s_bias[i] = bsrc ? bsrc[hh * R * kN + (i % (R * kN))] : 0.f;
     }
     if (tid < kHalf) s_car[tid] = a.dphi1 ? a.dphi1[u * kHalf + tid] : 0.f;
 
@@ -307,8 +309,8 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     const uint32_t tmem = tslot;
     const uint32_t lanebase = (32u * q4) << 16;
 
-    // per-thread bias sums over the rows this thread owns in every chunk (row t = 16 q4 +
-    // lane % 16; B and C columns col0 + k and col0 + 64 + k, k < 16)
+    // per-thread bias sums over the rows this thread owns in every chunk (row = 16 q4 +
+    // lane % 16, always of rank row % R; B and C columns col0 + k and col0 + 64 + k, k < 16)
     float accB[32], accC[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) accB[k] = accC[k] = 0.f;
@@ -327,16 +329,16 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         const int c = nch - 1 - it;
         const int cur = it & 1;
         const uint32_t par = static_cast<uint32_t>(it & 1);
-        const int t0 = c * kQ;
-        const int T = (L - t0) < kQ ? (L - t0) : kQ;
+        const int t0 = c * Q;
+        const int T = (L - t0) < Q ? (L - t0) : Q;   // tokens of this chunk
         if (!mbar_wait(&bar_a, par)) s_abort = 1;   // scalar boxes, raw B, scales, start angle
         if constexpr (kRaw) {
             // this head's column of the dt and lam boxes: softplus / sigmoid in place
             float* sSc = reinterpret_cast<float*>(sm + S_SC);
-            for (int i = tid; i < 2 * (kQ + 1); i += kThreads) {
-                const int t = i <= kQ ? i : i - (kQ + 1);
+            for (int i = tid; i < 2 * (Q + 1); i += kThreads) {
+                const int t = i <= Q ? i : i - (Q + 1);
                 if (t0 + t >= L) continue;
-                if (i <= kQ) {
+                if (i <= Q) {
                     float* d = sSc + t * 4 + hc;
                     *d = step_dt<true>(*d, dtb, p.flags);
                 } else {
@@ -370,7 +372,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             const float tot0 = __shfl_sync(0xffffffffu, s0, 31);
             const float s1 = warp_inclusive_scan(av[1]) + tot0;
             const float cum_end = __shfl_sync(0xffffffffu, s1, 31);   // padded tokens add 0
-            const float a_next = sSc[kQ * 4 + hc] * sSc[oA + kQ * 4 + hc];   // 0 past the end
+            const float a_next = sSc[Q * 4 + hc] * sSc[oA + Q * 4 + hc];   // 0 past the end
             const float cxT = cum_end + a_next;
             const float cum0 = __shfl_sync(0xffffffffu, s0, 0);
             // cum_{t+1} for every t (cx_T after the chunk's last real token)
@@ -395,10 +397,11 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 sf[F_DT + t] = dv[k];
                 sf[F_BETA + t] = bv[k];
             }
+            __syncwarp();
             if (lane == 0) {
-                sf[F_C2 + kQ] = cxT * kLog2e;
-                sf[F_BETA + kQ] = zoh ? 0.f
-                    : (1.f - sSc[oL + kQ * 4 + hc]) * sSc[kQ * 4 + hc] * __expf(a_next);
+                sf[F_C2 + Q] = cxT * kLog2e;
+                sf[F_BETA + Q] = zoh ? 0.f
+                    : (1.f - sSc[oL + Q * 4 + hc]) * sSc[Q * 4 + hc] * __expf(a_next);
                 sf[F_MISC + 0] = __expf(cxT - cum0);
                 sf[F_MISC + 1] = __expf(cum0);
                 const float d0 = sSc[hc], l0 = sSc[oL + hc];
@@ -412,7 +415,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         if (!mbar_wait(&bar_b, par)) s_abort = 1;   // theta, dY, raw C
         {
             const int jp = 2 * lane;
-            constexpr int TPS = kQ / 8;
+            constexpr int TPS = Q / 8;   // tokens per warp
             const float* phi0 = reinterpret_cast<const float*>(sm + S_PHI0);
             float inc[TPS][2];
             float sum0 = 0.f, sum1 = 0.f;
@@ -434,10 +437,6 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 const float2 v = s_seg[k * 32 + lane];
                 if (k < warp) { a0 += v.x; a1 += v.y; }
             }
-            const float2 bB0 = *reinterpret_cast<const float2*>(s_bias + jp);
-            const float2 bB1 = *reinterpret_cast<const float2*>(s_bias + jp + kHalf);
-            const float2 bC0 = *reinterpret_cast<const float2*>(s_bias + kN + jp);
-            const float2 bC1 = *reinterpret_cast<const float2*>(s_bias + kN + jp + kHalf);
 #pragma unroll
             for (int k = 0; k < TPS; ++k) {
                 const int t = warp * TPS + k;
@@ -447,10 +446,17 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 float2 cs, sn;
                 __sincosf(a0, &sn.x, &cs.x);
                 __sincosf(a1, &sn.y, &cs.y);
-                const float2 rs = (rsu && t < T) ? reinterpret_cast<const float2*>(sm + S_RS)[t]
-                                                 : make_float2(1.f, 1.f);
-                const uint32_t o = swz128(t, jp);
                 const float vn = sf[F_VN + t];
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                const int row = t * R + r;
+                const float2 bB0 = *reinterpret_cast<const float2*>(s_bias + r * kN + jp);
+                const float2 bB1 = *reinterpret_cast<const float2*>(s_bias + r * kN + jp + kHalf);
+                const float2 bC0 = *reinterpret_cast<const float2*>(s_bias + (R + r) * kN + jp);
+                const float2 bC1 = *reinterpret_cast<const float2*>(s_bias + (R + r) * kN + jp + kHalf);
+                const float2 rs = (rsu && t < T) ? reinterpret_cast<const float2*>(sm + S_RS)[row]
+                                                 : make_float2(1.f, 1.f);
+                const uint32_t o = swz128(row, jp);
                 {   // B: u = rs raw + bias, Bbar = (u0 c + u1 s, u1 c - u0 s); also vn Bbar
                     const float2 r0 = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + S_RB + o));
                     const float2 r1 = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + S_RB + 8192 + o));
@@ -473,6 +479,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                     *reinterpret_cast<uint32_t*>(sm + S_CT + 8192 + o) =
                         pack_bf16(fmaf(u1.x, cs.x, -u0.x * sn.x), fmaf(u1.y, cs.y, -u0.y * sn.y));
                 }
+                }
             }
         }
         // ---- Xs = diag(vn) X and Ds = diag(e^{cum - cum_0}) dY (rows keep their swizzle) ----
@@ -482,7 +489,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             const int e = tid + i * kThreads;
             const int row = e >> 3, ch = e & 7;
             const uint32_t o = static_cast<uint32_t>(row) * 128u + (static_cast<uint32_t>(ch) << 4);
-            const float fx = sf[F_VN + row], fd = sf[F_DS + row];
+            const float fx = sf[F_VN + row / R], fd = sf[F_DS + row / R];
             const uint4 vx = *reinterpret_cast<const uint4*>(sm + S_XT + o);
             const uint4 vd = *reinterpret_cast<const uint4*>(sm + S_DT + o);
             const uint32_t wx[4] = {vx.x, vx.y, vx.z, vx.w}, wd[4] = {vd.x, vd.y, vd.z, vd.w};
@@ -545,9 +552,10 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_S + 16u * wh, sv);
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_Z + 16u * wh, zv);
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_Q + 16u * wh, qv);
-            const int t = trow;
-            const float c2t = sf[F_C2 + t], c2t1 = sf[F_C2 + t + 1];
-            const float wt = sf[F_W + t], gt = sf[F_GAM + t];
+            const int t = trow;                 // operand row
+            const int tt = t / R;               // its token
+            const float c2t = sf[F_C2 + tt], c2t1 = sf[F_C2 + tt + 1];
+            const float wt = sf[F_W + tt], gt = sf[F_GAM + tt];
             float xv[16];
             load_row16(sm + S_XT, t, col0, xv);
             tmem_wait_ld();
@@ -559,11 +567,11 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 float pv[2], zz[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int s = col0 + j + e;
+                    const int s = (col0 + j + e) / R;   // the column's token
                     const float spv = sv[j + e], zvv = zv[j + e];
                     float m = 0.f;
                     cu[j + e] = 0.f;
-                    if (s > t) {
+                    if (s > tt) {
                         const float c2s = sf[F_C2 + s];
                         const float f = ex2_approx(c2s - c2t);
                         const float fb = ex2_approx(c2s - c2t1);
@@ -571,9 +579,9 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                         const float sz = spv * zvv;
                         kg = fmaf(f, sz, kg);
                         kb = fmaf(fb, sz, kb);
-                        cu[j + e] = m * sz;   // the pair (t, s) crosses every token in (t, s]
+                        cu[j + e] = m * sz;   // the pair crosses every token in (tt, s]
                         ru += cu[j + e];
-                    } else if (s == t) {
+                    } else if (s == tt) {   // the token's own R x R block
                         m = gt;
                         kg = fmaf(spv, zvv, kg);
                     }
@@ -709,16 +717,19 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             if (c > 0) issue_x(c - 1);   // X was last read by Z, Xs and the q sums
         }
         __syncwarp();
-        // per-token dg and the next token's db (threads 0..63, fixed summation order)
-        if (tid < kQ) {
+        // per-token dg and the next token's db (one thread per token, fixed summation order
+        // over the token's rows and the row partials)
+        if (tid < Q) {
             const int t = tid;
             float kg = 0.f, kb = 0.f, q = 0.f;
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                kg += red[(R_KG * 4 + s) * 64 + t];
-                kb += red[(R_KB * 4 + s) * 64 + t];
-                q += red[(R_Q * 4 + s) * 64 + t];
-            }
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    kg += red[(R_KG * 4 + s) * 64 + t * R + r];
+                    kb += red[(R_KB * 4 + s) * 64 + t * R + r];
+                    q += red[(R_Q * 4 + s) * 64 + t * R + r];
+                }
             const float dg = fmaf(sf[F_EE + t], q, kg), db1 = fmaf(sf[F_EB + t], q, kb);
             s_tok[t] = dg;
             s_tok[64 + t] = db1;
@@ -742,9 +753,10 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                         *reinterpret_cast<const uint4*>(sm + S_TH + 16 * e);
                 }
             }
-            const int t = trow;
-            const bool real = t < T;
-            const int64_t tok = static_cast<int64_t>(t0) + t;
+            const int t = trow;                 // operand row
+            const int tt = t / R, rk = t % R;   // its token and rank
+            const bool real = tt < T;
+            const int64_t tok = static_cast<int64_t>(t0) + tt;
             float vx[16], vb0[16], vb1[16], vc0[16], vc1[16];
             {
                 float yo[16], dyv[16];
@@ -768,11 +780,17 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             load_row16(sm + S_CT + 8192, t, col0, cbar1);
             tmem_wait_ld();
             float nb0[16], nb1[16], nc0[16], nc1[16];
-            float* ph = sphi + t * kPhiStride + col0;
+            // the token's angles; with R > 1 the token's R rows sit in consecutive lanes, which
+            // all read them before the sum of their angle adjoints replaces them
+            float* ph = sphi + tt * kPhiStride + col0;
+            float phv[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) phv[k] = ph[k];
+            if constexpr (R > 1) __syncwarp();
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 float sn, cs;
-                __sincosf(ph[k], &sn, &cs);
+                __sincosf(phv[k], &sn, &cs);
                 const float db0 = vb0[k], db1 = vb1[k], dc0 = vc0[k], dc1 = vc1[k];
                 nb0[k] = fmaf(db0, cs, -db1 * sn);
                 nb1[k] = fmaf(db0, sn, db1 * cs);
@@ -780,7 +798,9 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 nc1[k] = fmaf(dc0, sn, dc1 * cs);
                 float dl = fmaf(db0, bbar1[k], -db1 * bbar0[k]);
                 dl = fmaf(dc0, cbar1[k], fmaf(-dc1, cbar0[k], dl));
-                ph[k] = real ? dl : 0.f;
+#pragma unroll
+                for (int o = 1; o < R; o <<= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+                if (rk == 0) ph[k] = real ? dl : 0.f;
             }
             if (real) {
 #pragma unroll
@@ -788,15 +808,16 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                     accB[k] += nb0[k]; accB[16 + k] += nb1[k];
                     accC[k] += nc0[k]; accC[16 + k] += nc1[k];
                 }
-                float* dxr = a.dx + ((bb * L + tok) * H + hh) * kP + col0;
-                const float* px = (a.dprevx1 && tok == L - 1) ? a.dprevx1 + u * kP + col0 : nullptr;
+                float* dxr = a.dx + (((bb * L + tok) * H + hh) * R + rk) * kP + col0;
+                const float* px = (a.dprevx1 && tok == L - 1) ? a.dprevx1 + (u * R + rk) * kP + col0
+                                                              : nullptr;
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
                     float4 v = make_float4(vx[k], vx[k + 1], vx[k + 2], vx[k + 3]);
                     if (px) { v.x += px[k]; v.y += px[k + 1]; v.z += px[k + 2]; v.w += px[k + 3]; }
                     *reinterpret_cast<float4*>(dxr + k) = v;
                 }
-                const int64_t rowN = ((bb * L + tok) * H + hh) * kN;
+                const int64_t rowN = (((bb * L + tok) * H + hh) * R + rk) * kN;
                 float* db = a.wdB + rowN + col0;
                 float* dc = a.wdC + rowN + col0;
 #pragma unroll
@@ -815,18 +836,19 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         if (tid == 0 && c > 0) issue_b(c - 1);   // theta copied, dY and Cbar read
 
         // ---- the angle adjoint's suffix sum over the sequence: dPhi_t = carry + sum_{s>=t} dl_s;
-        // dtheta = dt dPhi; theta . dPhi per token (4 segments of 16 tokens per pair) ----
+        // dtheta = dt dPhi; theta . dPhi per token (4 segments of Q / 4 tokens per pair) ----
         {
+            constexpr int QS = Q / 4;
             const int i = tid & 63, sg = tid >> 6;
             float loc = 0.f;
-#pragma unroll 4
-            for (int k = 0; k < 16; ++k) loc += sphi[(16 * sg + k) * kPhiStride + i];
+#pragma unroll
+            for (int k = 0; k < QS; ++k) loc += sphi[(QS * sg + k) * kPhiStride + i];
             s_suf[sg * 64 + i] = loc;
             __syncthreads();
             float acc = s_car[i];
             for (int s2 = 3; s2 > sg; --s2) acc += s_suf[s2 * 64 + i];
-            for (int k = 15; k >= 0; --k) {
-                const int t = 16 * sg + k;
+            for (int k = QS - 1; k >= 0; --k) {
+                const int t = QS * sg + k;
                 acc += sphi[t * kPhiStride + i];
                 float thd = 0.f;
                 if (t < T) {
@@ -863,15 +885,21 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const int t = lane + 32 * k;
-                float ru = 0.f, q = 0.f, vv = 0.f;
-#pragma unroll
-                for (int s4 = 0; s4 < 4; ++s4) {
-                    ru += red[(R_RU * 4 + s4) * 64 + t];
-                    q += red[(R_Q * 4 + s4) * 64 + t];
-                    vv += red[(R_V * 4 + s4) * 64 + t];
-                }
-                const float cu = s_cu[t] + s_cu[64 + t] + s_cu[128 + t] + s_cu[192 + t];
+                float ru = 0.f, q = 0.f, vv = 0.f, cu = 0.f;
                 const bool real = t < T;
+                if (real) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const int row = t * R + r;
+#pragma unroll
+                        for (int s4 = 0; s4 < 4; ++s4) {
+                            ru += red[(R_RU * 4 + s4) * 64 + row];
+                            q += red[(R_Q * 4 + s4) * 64 + row];
+                            vv += red[(R_V * 4 + s4) * 64 + row];
+                            cu += s_cu[s4 * 64 + row];
+                        }
+                    }
+                }
                 g[k] = real ? ru - cu : 0.f;
                 p3[k] = real ? sf[F_VN + t] * q : 0.f;
                 v[k] = real ? sf[F_DS + t] * vv : 0.f;
@@ -903,7 +931,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                         const float dpn = k ? dp1_1 : (lane == 31 ? dp_32 : dp1_0);
                         dnx = dpn - sf[F_BETA + t + 1] * db1;
                     } else {
-                        dnx = dnext - sf[F_BETA + kQ] * db1;
+                        dnx = dnext - sf[F_BETA + Q] * db1;
                     }
                     // D'_t - D_{t+1} + gamma_t dg_t: the scalar kernel subtracts beta_t db_t and
                     // gamma_t dg_t again, leaving D_t - D_{t+1} (D_t = D'_t - beta_t db_t)
@@ -926,101 +954,127 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             for (int j = 0; j < 8; ++j)
                 dst[j] = make_float4(al0 * gr[4 * j], al0 * gr[4 * j + 1], al0 * gr[4 * j + 2], al0 * gr[4 * j + 3]);
         }
-        // Bbar_{-1} (the stored raw B, normalised, biased, rotated by phi0) and x_{-1}
-        float* pb = s_prev;            // [128] Bbar_{-1}
-        float* px = s_prev + 128;      // [64]  x_{-1}
-        float* pcs = s_prev + 192;     // [64]  cos, [64] sin
-        float* pgx = s_prev + 320;     // [2][128] (G_0 x_{-1}) halves
-        float* pdx = s_prev + 576;     // [4][64] dprevx partials
-        float* pred = s_prev + 832;    // [8] db_0 partials, [7] the RMS scale
-        float* pbias = s_prev + 848;   // [128] dBbar_{-1} rotated back, for the bias sum
-        if (warp == 0) {
+        // Bbar_{-1}[r] (the stored raw B, normalised, biased, rotated by phi0) and x_{-1}[r],
+        // in buffers the loop no longer uses (no copy is in flight after chunk 0)
+        float* w1 = reinterpret_cast<float*>(sm + S_CT);   // 8192 floats (raw C and raw B)
+        float* pb = w1;                // [R][128] Bbar_{-1}
+        float* px = w1 + 1024;         // [R][64]  x_{-1}
+        float* pcs = w1 + 1536;        // [64] cos, [64] sin of phi0
+        float* pred = w1 + 1664;       // [8] db_0 partials, [8 + r] the RMS scales
+        float* pgx = w1 + 1696;        // [2][R][128] (G_0 x_{-1}[r]) halves, then dBbar_{-1}
+        float* pdx = w1 + 3744;        // [4][R][64] dprevx partials
+        float* pbias = w1 + 5792;      // [R][128] dBbar_{-1} rotated back, for the bias sum
+        const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(p.prevB0);
+        if (warp < R) {
             float ss = 0.f;
-            const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(p.prevB0);
             for (int n = lane; n < kN; n += 32) {
-                const float v = pB ? __bfloat162float(pB[u * kN + n]) : 0.f;
+                const float v = pB ? __bfloat162float(pB[(u * R + warp) * kN + n]) : 0.f;
                 ss += v * v;
             }
             ss = warp_sum(ss);
-            if (lane == 0) pred[7] = p.bc_norm ? rsqrtf(ss / kN + p.eps) : 1.f;
+            if (lane == 0) pred[8 + warp] = p.bc_norm ? rsqrtf(ss / kN + p.eps) : 1.f;
         }
         __syncthreads();
-        if (tid < kHalf) {
-            const int i = tid;
-            const __nv_bfloat16* pB = static_cast<const __nv_bfloat16*>(p.prevB0);
-            const float rsp = pred[7];
-            const float u0 = (pB ? __bfloat162float(pB[u * kN + i]) : 0.f) * rsp + s_bias[i];
-            const float u1 = (pB ? __bfloat162float(pB[u * kN + i + kHalf]) : 0.f) * rsp + s_bias[i + kHalf];
+        for (int e = tid; e < R * kHalf; e += kThreads) {
+            const int r = e / kHalf, i = e % kHalf;
+            const float rsp = pred[8 + r];
+            const int64_t o = (u * R + r) * kN;
+            const float u0 = (pB ? __bfloat162float(pB[o + i]) : 0.f) * rsp + s_bias[r * kN + i];
+            const float u1 = (pB ? __bfloat162float(pB[o + i + kHalf]) : 0.f) * rsp + s_bias[r * kN + i + kHalf];
             float sn, cs;
             sincosf(p.phi0 ? p.phi0[u * kHalf + i] : 0.f, &sn, &cs);
-            pb[i] = u0 * cs + u1 * sn;
-            pb[i + kHalf] = u1 * cs - u0 * sn;
-            pcs[i] = cs;
-            pcs[kHalf + i] = sn;
-            px[i] = p.prevx0 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.prevx0)[u * kP + i]) : 0.f;
+            pb[r * kN + i] = u0 * cs + u1 * sn;
+            pb[r * kN + i + kHalf] = u1 * cs - u0 * sn;
+            if (r == 0) {
+                pcs[i] = cs;
+                pcs[kHalf + i] = sn;
+            }
+            px[e] = p.prevx0 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.prevx0)[u * R * kP + e]) : 0.f;
         }
         __syncthreads();
-        {
-            // (G_0 x_{-1})[n] partial over this thread's columns; dprevx0 partials over rows
+#pragma unroll 1
+        for (int r = 0; r < R; ++r) {
+            // (G_0 x_{-1}[r])[n] partial over this thread's columns; dprevx0 partials over rows
             float gx = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) gx = fmaf(gr[j], px[32 * wh + j], gx);
-            pgx[wh * 128 + nrow] = gx;
-            const float bn = pb[nrow];
+            for (int j = 0; j < 32; ++j) gx = fmaf(gr[j], px[r * kP + 32 * wh + j], gx);
+            pgx[(wh * R + r) * kN + nrow] = gx;
+            const float bn = pb[r * kN + nrow];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const float v = warp_sum(bn * gr[j]);
-                if (lane == j) pdx[q4 * 64 + 32 * wh + j] = v;
+                if (lane == j) pdx[(q4 * R + r) * kP + 32 * wh + j] = v;
             }
         }
         __syncthreads();
-        if (tid < kN) {
-            const int n = tid;
-            const float gx = pgx[n] + pgx[128 + n];
-            float v = pb[n] * gx;   // db_0 partial
+        {
+            float v = 0.f;   // db_0 partial
+            for (int e = tid; e < R * kN; e += kThreads) {
+                const int r = e / kN, n = e % kN;
+                const float gx = pgx[r * kN + n] + pgx[(R + r) * kN + n];
+                v = fmaf(pb[e], gx, v);
+                pgx[e] = be0 * gx;      // dBbar_{-1}[r][n]
+            }
             v = warp_sum(v);
             if (lane == 0) pred[warp] = v;
-            pgx[n] = be0 * gx;      // dBbar_{-1}
         }
         __syncthreads();
-        if (tid == 0) a.wsc[u * L * 4 + 0] = pred[0] + pred[1] + pred[2] + pred[3];
-        if (tid < kP && a.dprevx0)
-            a.dprevx0[u * kP + tid] = be0 * (pdx[tid] + pdx[64 + tid] + pdx[128 + tid] + pdx[192 + tid]);
+        if (tid == 0) {
+            float v = 0.f;
+            for (int w = 0; w < kThreads / 32; ++w) v += pred[w];
+            a.wsc[u * L * 4 + 0] = v;
+        }
+        if (a.dprevx0)
+            for (int e = tid; e < R * kP; e += kThreads) {
+                const int r = e / kP, pp = e % kP;
+                float v = 0.f;
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4) v += pdx[(w4 * R + r) * kP + pp];
+                a.dprevx0[u * R * kP + e] = be0 * v;
+            }
         if (tid < kHalf) {
             const int i = tid;
-            const float d0 = pgx[i], d1 = pgx[i + kHalf];
-            const float dl = d0 * pb[i + kHalf] - d1 * pb[i];
-            if (a.dphi0) a.dphi0[u * kHalf + i] = s_car[i] + dl;
             const float cs = pcs[i], sn = pcs[kHalf + i];
-            const float n0 = d0 * cs - d1 * sn, n1 = d0 * sn + d1 * cs;
-            a.wprev[u * kN + i] = n0;
-            a.wprev[u * kN + i + kHalf] = n1;
-            pbias[i] = n0;
-            pbias[kHalf + i] = n1;
+            float dl = 0.f;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const float d0 = pgx[r * kN + i], d1 = pgx[r * kN + i + kHalf];
+                dl += d0 * pb[r * kN + i + kHalf] - d1 * pb[r * kN + i];
+                const float n0 = d0 * cs - d1 * sn, n1 = d0 * sn + d1 * cs;
+                a.wprev[(u * R + r) * kN + i] = n0;
+                a.wprev[(u * R + r) * kN + i + kHalf] = n1;
+                pbias[r * kN + i] = n0;
+                pbias[r * kN + i + kHalf] = n1;
+            }
+            if (a.dphi0) a.dphi0[u * kHalf + i] = s_car[i] + dl;
         }
         __syncthreads();
-        // bias sums: over the 16 rows of each half-warp, then over the four row blocks
-        float* sb = reinterpret_cast<float*>(sm + S_PHI);   // [4][256]
+        // bias sums: over the rows of one rank within each half-warp (its lanes differ in the
+        // bits at and above R), then over the four row blocks, per rank
+        float* sb = reinterpret_cast<float*>(sm + S_BT);   // [4][2][R][128]
+        const int rk = trow % R;
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
             float vb = accB[k], vc = accC[k];
 #pragma unroll
-            for (int o = 1; o < 16; o <<= 1) {
+            for (int o = R; o < 16; o <<= 1) {
                 vb += __shfl_xor_sync(0xffffffffu, vb, o);
                 vc += __shfl_xor_sync(0xffffffffu, vc, o);
             }
-            if ((lane & 15) == 0) {
+            if ((lane & 15) < R) {
                 const int col = col0 + (k & 15) + (k >= 16 ? kHalf : 0);
-                sb[q4 * 256 + col] = vb;
-                sb[q4 * 256 + kN + col] = vc;
+                sb[((q4 * 2 + 0) * R + rk) * kN + col] = vb;
+                sb[((q4 * 2 + 1) * R + rk) * kN + col] = vc;
             }
         }
         __syncthreads();
-        {
-            const int n = tid;   // 0..127: B, 128..255: C
-            float v = sb[n] + sb[256 + n] + sb[512 + n] + sb[768 + n];
-            if (n < kN) v += pbias[n];
-            a.wbias[u * 2 * kN + n] = v;
+        for (int e = tid; e < 2 * R * kN; e += kThreads) {
+            const int isC = e / (R * kN), rem = e % (R * kN);
+            float v = 0.f;
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) v += sb[(w4 * 2 + isC) * R * kN + rem];
+            if (!isC) v += pbias[rem];
+            a.wbias[u * 2 * R * kN + e] = v;
         }
     }
 
@@ -1042,42 +1096,56 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
-// dB_bias[h] = sum over the batch of the units' sums (fixed order), and the same for C.
+// dB_bias[h] = sum over the batch of the units' sums (fixed order), and the same for C; RN is
+// R * N, the bias length per head.
 __global__ void __launch_bounds__(256) bwd_bias_sum_kernel(const float* __restrict__ wbias,
-                                                           int64_t b, int64_t H, float* dBbias,
-                                                           float* dCbias) {
+                                                           int64_t b, int64_t H, int RN,
+                                                           float* dBbias, float* dCbias) {
     const int64_t h = blockIdx.x;
-    const int n = threadIdx.x;   // 0..255
-    float v = 0.f;
-    for (int64_t i = 0; i < b; ++i) v += wbias[((i * H + h) * 2) * kN + n];
-    if (n < kN) {
-        if (dBbias) dBbias[h * kN + n] = v;
-    } else if (dCbias) {
-        dCbias[h * kN + n - kN] = v;
+    for (int n = threadIdx.x; n < 2 * RN; n += blockDim.x) {
+        float v = 0.f;
+        for (int64_t i = 0; i < b; ++i) v += wbias[(i * H + h) * 2 * RN + n];
+        if (n < RN) {
+            if (dBbias) dBbias[h * RN + n] = v;
+        } else if (dCbias) {
+            dCbias[h * RN + n - RN] = v;
+        }
     }
+}
+
+template <int R>
+cudaError_t launch_bwd_tc_r(const BwdTcArgs& a, const BwdMaps& maps, int64_t units, bool raw,
+                            cudaStream_t s) {
+    auto kern = raw ? bwd_tc_kernel<R, true> : bwd_tc_kernel<R, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(units), kThreads, kSmemBytes, s>>>(a, maps);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 bool bwd_tc_supported(const ScanParams& p, bool bf16) {
+    if (p.R != 1 && p.R != 2 && p.R != 4 && p.R != 8) return false;
     ScanParams q = p;
-    q.Q = kQ;
-    return bf16 && p.R == 1 && tc_scan_supported(q, true);
+    q.Q = kQ / p.R;
+    return bf16 && tc_scan_supported(q, true);
 }
 
 size_t bwd_tc_workspace_bytes(const ScanParams& p) {
-    const int64_t nch = (p.L + kQ - 1) / kQ, units = p.b * p.H;
+    const int64_t Q = kQ / p.R, nch = (p.L + Q - 1) / Q, units = p.b * p.H;
     auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
     return r256(static_cast<size_t>(units) * nch * 16384) +
            r256(static_cast<size_t>(units) * nch * kHalf * 4) +
            r256(static_cast<size_t>(units) * kN * kP * 4) +
            r256(static_cast<size_t>(units) * (kHalf + 1) * 4) +
-           r256(static_cast<size_t>(units) * 2 * kN * 4) +
-           r256(static_cast<size_t>(p.b) * nch * kQ * p.G * sizeof(float2));
+           r256(static_cast<size_t>(units) * 2 * p.R * kN * 4) +
+           r256(static_cast<size_t>(p.b) * nch * Q * p.G * p.R * sizeof(float2));
 }
 
 cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cudaStream_t s) {
-    const int64_t nch = (p.L + kQ - 1) / kQ, units = p.b * p.H;
+    const int64_t R = p.R, Q = kQ / R, nch = (p.L + Q - 1) / Q, units = p.b * p.H;
     auto r256 = [](size_t v) { return (v + 255) / 256 * 256; };
     uint8_t* w = static_cast<uint8_t*>(ws);
     BwdTcArgs a{};
@@ -1089,7 +1157,7 @@ cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cuda
     float* phifin = reinterpret_cast<float*>(w);
     float* lamfin = phifin + units * kHalf;
     w += r256(static_cast<size_t>(units) * (kHalf + 1) * 4);
-    float* wbias = reinterpret_cast<float*>(w); w += r256(static_cast<size_t>(units) * 2 * kN * 4);
+    float* wbias = reinterpret_cast<float*>(w); w += r256(static_cast<size_t>(units) * 2 * R * kN * 4);
     float2* rs = p.bc_norm ? reinterpret_cast<float2*>(w) : nullptr;
 
     // the forward state pass: e^{cum_0} H0' and the angle before every chunk, the final state
@@ -1097,34 +1165,35 @@ cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cuda
     if (e != cudaSuccess) return e;
 
     BwdMaps maps;
-    const uint64_t H = p.H, Lq = p.L, b = p.b, G = p.G;
-    {
-        const uint64_t dims[5] = {kP, 1, H, Lq, b};
-        const uint64_t str[4] = {kP * 2, kP * 2, H * kP * 2, Lq * H * kP * 2};
-        const uint32_t box[5] = {kP, 1, 1, kQ, 1};
+    const uint64_t H = p.H, Lq = p.L, b = p.b, G = p.G, Ru = static_cast<uint64_t>(R);
+    const uint32_t Qb = static_cast<uint32_t>(Q), Rb = static_cast<uint32_t>(R);
+    {   // x, dy [b][L][H][R][P], box (P, R, 1, Q, 1)
+        const uint64_t dims[5] = {kP, Ru, H, Lq, b};
+        const uint64_t str[4] = {kP * 2, Ru * kP * 2, H * Ru * kP * 2, Lq * H * Ru * kP * 2};
+        const uint32_t box[5] = {kP, Rb, 1, Qb, 1};
         if (!encode_tmap(&maps.x, true, 5, p.x, dims, str, box, true) ||
             !encode_tmap(&maps.dy, true, 5, o.dy, dims, str, box, true))
             return cudaErrorInvalidValue;
     }
-    {
+    {   // theta [b][L][H][N/2], box (64, 1, Q, 1)
         const uint64_t dims[4] = {kHalf, H, Lq, b};
         const uint64_t str[3] = {kHalf * 2, H * kHalf * 2, Lq * H * kHalf * 2};
-        const uint32_t box[4] = {kHalf, 1, kQ, 1};
+        const uint32_t box[4] = {kHalf, 1, Qb, 1};
         if (!encode_tmap(&maps.theta, true, 4, p.theta, dims, str, box, true))
             return cudaErrorInvalidValue;
     }
-    {
-        const uint64_t dims[5] = {kN, 1, G, Lq, b};
-        const uint64_t str[4] = {kN * 2, kN * 2, G * kN * 2, Lq * G * kN * 2};
-        const uint32_t box[5] = {kHalf, 1, 1, kQ, 1};
+    {   // B, C [b][L][G][R][N], box (64 columns, R, 1, Q, 1)
+        const uint64_t dims[5] = {kN, Ru, G, Lq, b};
+        const uint64_t str[4] = {kN * 2, Ru * kN * 2, G * Ru * kN * 2, Lq * G * Ru * kN * 2};
+        const uint32_t box[5] = {kHalf, Rb, 1, Qb, 1};
         if (!encode_tmap(&maps.B, true, 5, p.B, dims, str, box, true) ||
             !encode_tmap(&maps.C, true, 5, p.C, dims, str, box, true))
             return cudaErrorInvalidValue;
     }
-    {
+    {   // dt, A, lam [b][L][H] fp32, box (4 heads, Q + 1 tokens, 1)
         const uint64_t dims[3] = {H, Lq, b};
         const uint64_t str[2] = {H * 4, Lq * H * 4};
-        const uint32_t box[3] = {4, kQ + 1, 1};
+        const uint32_t box[3] = {4, Qb + 1, 1};
         if (!encode_tmap(&maps.dt, false, 3, p.dt, dims, str, box, false) ||
             !encode_tmap(&maps.A, false, 3, p.A, dims, str, box, false) ||
             !encode_tmap(&maps.lam, false, 3, p.lam, dims, str, box, false))
@@ -1149,15 +1218,18 @@ cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cuda
     a.dphi0 = o.dphi0;
     a.dprevx0 = o.dprevx0;
     a.status = o.status;
-    auto kern = p.flags ? bwd_tc_kernel<true> : bwd_tc_kernel<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes));
+    const bool raw = p.flags != 0;
+    switch (R) {
+        case 1: e = launch_bwd_tc_r<1>(a, maps, units, raw, s); break;
+        case 2: e = launch_bwd_tc_r<2>(a, maps, units, raw, s); break;
+        case 4: e = launch_bwd_tc_r<4>(a, maps, units, raw, s); break;
+        case 8: e = launch_bwd_tc_r<8>(a, maps, units, raw, s); break;
+        default: return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(units), kThreads, kSmemBytes, s>>>(a, maps);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (o.dBbias || o.dCbias) {
-        bwd_bias_sum_kernel<<<static_cast<unsigned>(p.H), 256, 0, s>>>(wbias, p.b, p.H, o.dBbias,
-                                                                      o.dCbias);
+        bwd_bias_sum_kernel<<<static_cast<unsigned>(p.H), 256, 0, s>>>(
+            wbias, p.b, p.H, static_cast<int>(R * kN), o.dBbias, o.dCbias);
         e = cudaGetLastError();
     }
     return e;

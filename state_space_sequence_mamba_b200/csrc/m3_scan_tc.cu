@@ -1232,11 +1232,11 @@ bool encode_tmap(void* map, bool bf16, int rank, const void* base, const uint64_
 cudaError_t launch_bwd_states_tc(const ScanParams& p_in, float2* rs, uint8_t* chunk_h,
                                  float* chunk_phi, float* hfin, float* phifin, float* lamfin,
                                  cudaStream_t s) {
-    if (p_in.b * p_in.H == 0 || p_in.R != 1) return cudaErrorInvalidValue;
+    if (p_in.b * p_in.H == 0) return cudaErrorInvalidValue;
     ScanParams p = p_in;
-    p.Q = 64;
+    p.Q = 64 / p.R;
     SegArgs sa;
-    sa.seg_chunks = static_cast<int>((p.L + 63) / 64);
+    sa.seg_chunks = static_cast<int>((p.L + p.Q - 1) / p.Q);
     sa.nseg = 1;
     sa.out_h = hfin;
     sa.out_phi = phifin;
@@ -1244,7 +1244,14 @@ cudaError_t launch_bwd_states_tc(const ScanParams& p_in, float2* rs, uint8_t* ch
     sa.save_init = false;
     sa.chunk_h = chunk_h;
     sa.chunk_phi = chunk_phi;
-    return p.flags ? launch_tc_t<1, true>(p, rs, sa, s, true) : launch_tc_t<1, false>(p, rs, sa, s, true);
+    const bool raw = p.flags != 0;
+    switch (p.R) {
+        case 1: return raw ? launch_tc_t<1, true>(p, rs, sa, s, true) : launch_tc_t<1, false>(p, rs, sa, s, true);
+        case 2: return raw ? launch_tc_t<2, true>(p, rs, sa, s, true) : launch_tc_t<2, false>(p, rs, sa, s, true);
+        case 4: return raw ? launch_tc_t<4, true>(p, rs, sa, s, true) : launch_tc_t<4, false>(p, rs, sa, s, true);
+        case 8: return raw ? launch_tc_t<8, true>(p, rs, sa, s, true) : launch_tc_t<8, false>(p, rs, sa, s, true);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_scan_state_tc(const ScanParams& p, void* ws_body, size_t body_bytes,
