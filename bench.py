@@ -31,8 +31,8 @@ METRIC = "SSM prefill tokens/s + decode µs/step at 1.5B shapes; % of HBM/TC roo
 # source file when it was captured: reported while that file is unchanged, else null.
 SCAN_TRAFFIC = {"kernel": "scan_tc_kernel",
                 "source": "state_space_sequence_mamba_b200/csrc/m3_scan_tc.cu",
-                "sha256": "aefbe39b9b54335d624cdc2897f0b27fdf066f2be18b7fc6cc9fab2c9fc49890",
-                "bytes": 186.45e6}
+                "sha256": "0987a86f8a47ce05cb03c949cc42428ab50417a13d9b95527b7e1b7b1338848d",
+                "bytes": 186.534144e6}
 # kernels one scan launches: the per-token RMS-scale pre-pass of B and C, then the scan
 KERNELS_PER_SCAN = 2
 WORKLOAD = "SISO prefill b4 H64 P64 N128 L2048 chunk64 bf16/fp32-state BCNorm+bias"

@@ -559,6 +559,9 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             float xv[16];
             load_row16(sm + S_XT, t, col0, xv);
             tmem_wait_ld();
+            // e^{cum_s - cum_t} = e^{cum_s - cum_{t+1}} alpha_{t+1}: one exponential per element,
+            // both factors <= 1; the selects keep the warp on one path
+            const float alpha1 = ex2_approx(fminf(c2t1 - c2t, 0.f));
             float kg = 0.f, kb = 0.f, qq = 0.f, ru = 0.f;
             float cu[16];
             uint32_t ps[8], pz[8];
@@ -569,22 +572,15 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 for (int e = 0; e < 2; ++e) {
                     const int s = (col0 + j + e) / R;   // the column's token
                     const float spv = sv[j + e], zvv = zv[j + e];
-                    float m = 0.f;
-                    cu[j + e] = 0.f;
-                    if (s > tt) {
-                        const float c2s = sf[F_C2 + s];
-                        const float f = ex2_approx(c2s - c2t);
-                        const float fb = ex2_approx(c2s - c2t1);
-                        m = f * wt;
-                        const float sz = spv * zvv;
-                        kg = fmaf(f, sz, kg);
-                        kb = fmaf(fb, sz, kb);
-                        cu[j + e] = m * sz;   // the pair crosses every token in (tt, s]
-                        ru += cu[j + e];
-                    } else if (s == tt) {   // the token's own R x R block
-                        m = gt;
-                        kg = fmaf(spv, zvv, kg);
-                    }
+                    const bool after = s > tt, same = s == tt;   // same: the token's R x R block
+                    const float fb = ex2_approx(fminf(sf[F_C2 + s] - c2t1, 0.f));
+                    const float f = after ? fb * alpha1 : (same ? 1.f : 0.f);
+                    const float m = after ? f * wt : (same ? gt : 0.f);
+                    const float sz = spv * zvv;
+                    kg = fmaf(f, sz, kg);
+                    kb = fmaf(after ? fb : 0.f, sz, kb);
+                    cu[j + e] = after ? m * sz : 0.f;   // the pair crosses every token in (tt, s]
+                    ru += cu[j + e];
                     pv[e] = m * spv;
                     zz[e] = m * zvv;
                 }
