@@ -127,6 +127,19 @@ __device__ __forceinline__ void load_row16(const uint8_t* tile, int row, int c, 
     }
 }
 
+// A [64 rows][64 fp32] staging tile: 16-byte chunk ch of row r at r * 256 + (ch ^ (r & 15)) * 16,
+// so that 16 rows written at the same columns, or one row read whole, hit distinct banks.
+__device__ __forceinline__ uint32_t staged_off(int row, int ch) {
+    return static_cast<uint32_t>(row) * 256u + (static_cast<uint32_t>(ch ^ (row & 15)) << 4);
+}
+// 16 consecutive fp32 of row `row` starting at column c (a multiple of 4) into a staging tile
+__device__ __forceinline__ void stage_row(uint8_t* tile, int row, int c, const float (&v)[16]) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<float4*>(tile + staged_off(row, c / 4 + m)) =
+            make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+}
+
 }  // namespace
 
 struct BwdTcArgs {
@@ -804,25 +817,39 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                     accB[k] += nb0[k]; accB[16 + k] += nb1[k];
                     accC[k] += nc0[k]; accC[16 + k] += nc1[k];
                 }
-                float* dxr = a.dx + (((bb * L + tok) * H + hh) * R + rk) * kP + col0;
-                const float* px = (a.dprevx1 && tok == L - 1) ? a.dprevx1 + (u * R + rk) * kP + col0
-                                                              : nullptr;
+                if (a.dprevx1 && tok == L - 1) {
+                    const float* px = a.dprevx1 + (u * R + rk) * kP + col0;
 #pragma unroll
-                for (int k = 0; k < 16; k += 4) {
-                    float4 v = make_float4(vx[k], vx[k + 1], vx[k + 2], vx[k + 3]);
-                    if (px) { v.x += px[k]; v.y += px[k + 1]; v.z += px[k + 2]; v.w += px[k + 3]; }
-                    *reinterpret_cast<float4*>(dxr + k) = v;
+                    for (int k = 0; k < 16; ++k) vx[k] += px[k];
                 }
-                const int64_t rowN = (((bb * L + tok) * H + hh) * R + rk) * kN;
-                float* db = a.wdB + rowN + col0;
-                float* dc = a.wdC + rowN + col0;
-#pragma unroll
-                for (int k = 0; k < 16; k += 4) {
-                    *reinterpret_cast<float4*>(db + k) = make_float4(nb0[k], nb0[k + 1], nb0[k + 2], nb0[k + 3]);
-                    *reinterpret_cast<float4*>(db + kHalf + k) = make_float4(nb1[k], nb1[k + 1], nb1[k + 2], nb1[k + 3]);
-                    *reinterpret_cast<float4*>(dc + k) = make_float4(nc0[k], nc0[k + 1], nc0[k + 2], nc0[k + 3]);
-                    *reinterpret_cast<float4*>(dc + kHalf + k) = make_float4(nc1[k], nc1[k + 1], nc1[k + 2], nc1[k + 3]);
-                }
+            }
+            // The rows go out through shared memory so that each half-warp stores one whole
+            // 256-byte row (a thread holds 64 bytes of one row, 16 rows per half-warp):
+            // dx and dBbar now (the buffers of Xs/Ds, Bs and this chunk's G_n operand, whose
+            // readers have finished), dCbar after them.
+            stage_row(sm + S_XS, t, col0, vx);
+            stage_row(sm + S_BS, t, col0, nb0);
+            stage_row(sm + S_GN + cur * 16384, t, col0, nb1);
+            __syncthreads();
+            for (int e = tid; e < 3 * 64 * 16; e += kThreads) {
+                const int tile = e >> 10, row = (e >> 4) & 63, ch = e & 15;
+                if (row / R >= T) continue;
+                const int64_t grow = ((bb * L + t0 + row / R) * H + hh) * R + row % R;
+                const uint8_t* src = tile == 0 ? sm + S_XS : tile == 1 ? sm + S_BS : sm + S_GN + cur * 16384;
+                float* dst = tile == 0 ? a.dx + grow * kP : a.wdB + grow * kN + (tile == 2 ? kHalf : 0);
+                *reinterpret_cast<float4*>(dst + 4 * ch) = *reinterpret_cast<const float4*>(src + staged_off(row, ch));
+            }
+            __syncthreads();
+            stage_row(sm + S_BS, t, col0, nc0);
+            stage_row(sm + S_GN + cur * 16384, t, col0, nc1);
+            __syncthreads();
+            for (int e = tid; e < 2 * 64 * 16; e += kThreads) {
+                const int tile = e >> 10, row = (e >> 4) & 63, ch = e & 15;
+                if (row / R >= T) continue;
+                const int64_t grow = ((bb * L + t0 + row / R) * H + hh) * R + row % R;
+                const uint8_t* src = tile == 0 ? sm + S_BS : sm + S_GN + cur * 16384;
+                float* dst = a.wdC + grow * kN + (tile == 1 ? kHalf : 0);
+                *reinterpret_cast<float4*>(dst + 4 * ch) = *reinterpret_cast<const float4*>(src + staged_off(row, ch));
             }
         }
         fence_before_sync();
