@@ -10,7 +10,7 @@
 // chunk, with alpha_n = 1), each chunk of Q = 64 tokens needs:
 //     S' = Bbar Cbar^T,  Z = X dY^T,  Q1 = Bbar G_n                 (tensor cores, M64)
 //     Ps = M^T o S',  Pz = M^T o Z                                   (CUDA cores)
-//     dx    = Ps dY + diag(w e^{cx_T - cum}) Bbar G_n                (tensor cores)
+//     dx    = Ps dY + diag(w e^{cx_T - cum}) Q1                      (tensor cores, then Q1 scaled)
 //     dBbar = Pz Cbar + diag(w e^{cx_T - cum}) X G_n^T               (tensor cores, N128)
 //     dCbar = Pz^T Bbar + diag(e^{cum - cum_0}) dY (e^{cum_0} H0')^T (tensor cores, N128)
 //     G_0   = Cbar^T diag(e^{cum - cum_0}) dY + e^{cx_T - cum_0} G_n (tensor cores, M128)
@@ -56,7 +56,7 @@ constexpr uint32_t S_DS = 24576;      // diag(e^{cum - cum_0}) dY
 constexpr uint32_t S_PS = 32768;      // Ps = M^T o S'
 constexpr uint32_t S_PZ = 40960;      // Pz = M^T o Z
 constexpr uint32_t S_BT = 49152;      // Bbar [t][n]
-constexpr uint32_t S_BS = 65536;      // diag(vn) Bbar
+constexpr uint32_t S_BS = 65536;      // staging of the epilogue's rows (16 KB)
 constexpr uint32_t S_CT = 81920;      // raw C (TMA), rotated in place to Cbar
 constexpr uint32_t S_RB = 98304;      // raw B (TMA)
 constexpr uint32_t S_GN = 114688;     // G_n bf16 [n][p], two buffers of 16384
@@ -334,7 +334,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
     const uint32_t aXT = smem_u32(sm + S_XT), aDT = smem_u32(sm + S_DT);
     const uint32_t aXS = smem_u32(sm + S_XS), aDS = smem_u32(sm + S_DS);
     const uint32_t aPS = smem_u32(sm + S_PS), aPZ = smem_u32(sm + S_PZ);
-    const uint32_t aBT = smem_u32(sm + S_BT), aBS = smem_u32(sm + S_BS);
+    const uint32_t aBT = smem_u32(sm + S_BT);
     const uint32_t aCT = smem_u32(sm + S_CT), aHS = smem_u32(sm + S_HS);
     const uint32_t aGN = smem_u32(sm + S_GN);
 
@@ -459,7 +459,6 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 float2 cs, sn;
                 __sincosf(a0, &sn.x, &cs.x);
                 __sincosf(a1, &sn.y, &cs.y);
-                const float vn = sf[F_VN + t];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                 const int row = t * R + r;
@@ -470,7 +469,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 const float2 rs = (rsu && t < T) ? reinterpret_cast<const float2*>(sm + S_RS)[row]
                                                  : make_float2(1.f, 1.f);
                 const uint32_t o = swz128(row, jp);
-                {   // B: u = rs raw + bias, Bbar = (u0 c + u1 s, u1 c - u0 s); also vn Bbar
+                {   // B: u = rs raw + bias, Bbar = (u0 c + u1 s, u1 c - u0 s)
                     const float2 r0 = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + S_RB + o));
                     const float2 r1 = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + S_RB + 8192 + o));
                     const float2 u0 = make_float2(fmaf(r0.x, rs.x, bB0.x), fmaf(r0.y, rs.x, bB0.y));
@@ -479,8 +478,6 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                     const float2 v1 = make_float2(fmaf(u1.x, cs.x, -u0.x * sn.x), fmaf(u1.y, cs.y, -u0.y * sn.y));
                     *reinterpret_cast<uint32_t*>(sm + S_BT + o) = pack_bf16(v0.x, v0.y);
                     *reinterpret_cast<uint32_t*>(sm + S_BT + 8192 + o) = pack_bf16(v1.x, v1.y);
-                    *reinterpret_cast<uint32_t*>(sm + S_BS + o) = pack_bf16(vn * v0.x, vn * v0.y);
-                    *reinterpret_cast<uint32_t*>(sm + S_BS + 8192 + o) = pack_bf16(vn * v1.x, vn * v1.y);
                 }
                 {   // C, in place
                     const float2 r0 = bf2_to_f2(*reinterpret_cast<const uint32_t*>(sm + S_CT + o));
@@ -682,21 +679,16 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
             const uint32_t loPS = desc_lo(aPS, 16), loPZ = desc_lo(aPZ, 16);
             const uint32_t loPZt = desc_lo(aPZ, 8192);
             const uint32_t loDTm = desc_lo(aDT, 8192);
-            const uint32_t loBS = desc_lo(aBS, 16), loXS = desc_lo(aXS, 16), loDS = desc_lo(aDS, 16);
-            const uint32_t loGn = desc_lo(aGN + cur * 16384, 16384);
+            const uint32_t loXS = desc_lo(aXS, 16), loDS = desc_lo(aDS, 16);
             const uint32_t loGk = desc_lo(aGN + cur * 16384, 16);
             const uint32_t loHk = desc_lo(aHS, 16);
             const uint32_t loCt = desc_lo(aCT, 8192), loBt = desc_lo(aBT, 8192);
             const uint32_t loC2 = desc_lo(aCT, 16);
-            // dx = Ps dY + Bs G_n
+            // dx = Ps dY (+ diag(vn) Bbar G_n from the Q1 accumulator in the epilogue)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 mma_bf16(tmem + T_S, desc_pack(loPS + (kmajor_off(k, 8192) >> 4), hi),
                          desc_pack(loDTm + (mnmajor_off(k) >> 4), hi), id64, k > 0);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16(tmem + T_S, desc_pack(loBS + (kmajor_off(k, 8192) >> 4), hi),
-                         desc_pack(loGn + (mnmajor_off(k) >> 4), hi), id64, 1);
             // dBbar = Pz Cbar + Xs G_n^T
 #pragma unroll
             for (int k = 0; k < 4; ++k)
@@ -777,7 +769,15 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 for (int k = 0; k < 16; ++k) v = fmaf(yo[k], dyv[k], v);
                 red[(R_V * 4 + slot) * 64 + t] = v;
             }
-            tmem_ld_16x32bx2_x16(tmem + lanebase + T_S + 16u * wh, vx);
+            {   // dx = Ps dY + vn (Bbar G_n): the boundary term is Q1, still in TMEM, scaled
+                float q1[16];
+                tmem_ld_16x32bx2_x16(tmem + lanebase + T_S + 16u * wh, vx);
+                tmem_ld_16x32bx2_x16(tmem + lanebase + T_Q + 16u * wh, q1);
+                tmem_wait_ld();
+                const float vn = sf[F_VN + tt];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) vx[k] = fmaf(vn, q1[k], vx[k]);
+            }
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_DB + 16u * wh, vb0);
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_DB + 64u + 16u * wh, vb1);
             tmem_ld_16x32bx2_x16(tmem + lanebase + T_DC + 16u * wh, vc0);
