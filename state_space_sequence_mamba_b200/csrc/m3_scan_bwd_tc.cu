@@ -863,20 +863,27 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         {
             constexpr int QS = Q / 4;
             const int i = tid & 63, sg = tid >> 6;
+            // the segment's angle adjoints in registers first, so that the loads do not wait on
+            // one another
+            float dlv[QS];
             float loc = 0.f;
 #pragma unroll
-            for (int k = 0; k < QS; ++k) loc += sphi[(QS * sg + k) * kPhiStride + i];
+            for (int k = 0; k < QS; ++k) {
+                dlv[k] = sphi[(QS * sg + k) * kPhiStride + i];
+                loc += dlv[k];
+            }
             s_suf[sg * 64 + i] = loc;
             __syncthreads();
             float acc = s_car[i];
             for (int s2 = 3; s2 > sg; --s2) acc += s_suf[s2 * 64 + i];
+            float* dth = a.dtheta + ((bb * L + t0) * H + hh) * kHalf + i;
+#pragma unroll
             for (int k = QS - 1; k >= 0; --k) {
                 const int t = QS * sg + k;
-                acc += sphi[t * kPhiStride + i];
+                acc += dlv[k];
                 float thd = 0.f;
                 if (t < T) {
-                    const int64_t tok = static_cast<int64_t>(t0) + t;
-                    a.dtheta[((bb * L + tok) * H + hh) * kHalf + i] = sf[F_DT + t] * acc;
+                    dth[static_cast<int64_t>(t) * H * kHalf] = sf[F_DT + t] * acc;
                     const uint16_t thb = *reinterpret_cast<const uint16_t*>(sm + S_PS + swz128(t, i));
                     thd = __uint_as_float(static_cast<uint32_t>(thb) << 16) * acc;
                 }
