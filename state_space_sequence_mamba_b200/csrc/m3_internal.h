@@ -174,8 +174,8 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
 bool bwd_tc_supported(const ScanParams& p, bool bf16);
 size_t bwd_tc_workspace_bytes(const ScanParams& p);
 // Where the chunked backward writes: the sequential backward's intermediate buffers (wdB,
-// wdC [b,L,H,N], wsc [units][L][4], wprev [units][N], wF [units]) and the gradients it
-// produces itself.
+// wdC [b,L,H,R,N], here as bf16; wsc [units][L][4], wprev [units][R][N], wF [units]) and the
+// gradients it produces itself.
 struct BwdTcOut {
     const void* dy;
     const float* dh1;
@@ -183,8 +183,8 @@ struct BwdTcOut {
     const float* dprevx1;
     float* dx;
     float* dtheta;
-    float* wdB;
-    float* wdC;
+    void* wdB;
+    void* wdC;
     float* wsc;
     float* wprev;
     float* wF;

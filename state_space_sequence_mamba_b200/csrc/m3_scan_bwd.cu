@@ -138,6 +138,7 @@ struct BwdArgs {
     float* dprevx0;
     float* wdC;    // [b,L,H,R,N] dCbar (forward sweep), then dC after the rotation (reverse)
     float* wdB;    // [b,L,H,R,N] dB after the rotation
+    int wd_bf16;   // the chunked form wrote wdB and wdC as bf16 (the norm kernel reads them so)
     float* wphi;   // [units][nchunks][N/2] angle before each chunk
     float* wF;     // [units] <dL/dh_final, h_final>
     float* wsc;    // [units][L][4] db, dg, dy.y, theta.dPhi per token
@@ -1049,8 +1050,9 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
     int64_t src_off;
     float* dst;
     const float* extra = nullptr;   // final state's prev_B gradient, summed over the group
-    int64_t h_first = 0, nh = 0, dn_stride = 0;
+    int64_t h_first = 0, nh = 0, dn_stride = 0, dn_off = 0;
     const float* dn_base;
+    bool dn_h = false;   // the per-head rows are bf16
     if (item < ntok) {
         const int isC = static_cast<int>(item & 1);
         const int64_t rest = item >> 1;
@@ -1061,7 +1063,9 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
         dst = (isC ? a.dC : a.dB) + src_off;
         h_first = g * hpg;
         nh = hpg;
-        dn_base = (isC ? a.wdC : a.wdB) + ((tok * H + h_first) * R + r) * N;
+        dn_off = ((tok * H + h_first) * R + r) * N;
+        dn_base = isC ? a.wdC : a.wdB;
+        dn_h = a.wd_bf16 != 0;
         dn_stride = R * N;
         if (!isC && t == L - 1 && a.dprevB1) extra = a.dprevB1 + ((bb * H + h_first) * R + r) * N;
     } else {
@@ -1071,7 +1075,8 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
         src_off = j * N;
         dst = a.dprevB0 + j * N;
         nh = 1;
-        dn_base = a.wprev + j * N;
+        dn_base = a.wprev;
+        dn_off = j * N;
         dn_stride = 0;
     }
     // N <= 256: at most eight elements per lane, kept in registers
@@ -1083,7 +1088,12 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
         dnv[j] = 0.f;
         vv[j] = 0.f;
         if (n < N) {
-            for (int64_t h = 0; h < nh; ++h) dnv[j] += dn_base[h * dn_stride + n];
+            if (dn_h) {
+                const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(dn_base) + dn_off;
+                for (int64_t h = 0; h < nh; ++h) dnv[j] += __bfloat162float(hb[h * dn_stride + n]);
+            } else {
+                for (int64_t h = 0; h < nh; ++h) dnv[j] += dn_base[dn_off + h * dn_stride + n];
+            }
             vv[j] = src ? raw(src, src_off + n) : 0.f;
             ss = fmaf(vv[j], vv[j], ss);
             dot = fmaf(vv[j], dnv[j], dot);
@@ -1183,6 +1193,7 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
         o.dh1 = g.dh1; o.dphi1 = g.dphi1; o.dprevx1 = g.dprevx1;
         o.dx = g.dx; o.dtheta = g.dtheta;
         o.wdB = a.wdB; o.wdC = a.wdC; o.wsc = a.wsc; o.wprev = a.wprev; o.wF = a.wF;
+        a.wd_bf16 = 1;
         o.dh0 = g.dh0; o.dphi0 = g.dphi0; o.dprevx0 = g.dprevx0;
         o.dBbias = g.dBbias; o.dCbias = g.dCbias;
         o.status = status;

@@ -139,6 +139,20 @@ __device__ __forceinline__ void stage_row(uint8_t* tile, int row, int c, const f
         *reinterpret_cast<float4*>(tile + staged_off(row, c / 4 + m)) =
             make_float4(v[4 * m], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
 }
+// The same tile read as [64 rows][128 bf16]: columns c .. c + 15 from lo and 64 + c .. 79 + c
+// from hi (c a multiple of 8), each rounded to bf16
+__device__ __forceinline__ void stage_row_bf16(uint8_t* tile, int row, int c, const float (&lo)[16],
+                                               const float (&hi)[16]) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        *reinterpret_cast<uint4*>(tile + staged_off(row, c / 8 + m)) =
+            make_uint4(pack_bf16(lo[8 * m], lo[8 * m + 1]), pack_bf16(lo[8 * m + 2], lo[8 * m + 3]),
+                       pack_bf16(lo[8 * m + 4], lo[8 * m + 5]), pack_bf16(lo[8 * m + 6], lo[8 * m + 7]));
+        *reinterpret_cast<uint4*>(tile + staged_off(row, 8 + c / 8 + m)) =
+            make_uint4(pack_bf16(hi[8 * m], hi[8 * m + 1]), pack_bf16(hi[8 * m + 2], hi[8 * m + 3]),
+                       pack_bf16(hi[8 * m + 4], hi[8 * m + 5]), pack_bf16(hi[8 * m + 6], hi[8 * m + 7]));
+    }
+}
 
 }  // namespace
 
@@ -153,8 +167,8 @@ struct BwdTcArgs {
     const float* dprevx1;
     float* dx;                 // [b, L, H, R, P]
     float* dtheta;             // [b, L, H, N/2]
-    float* wdB;                // [b, L, H, R, N]: dBbar rotated back (per head)
-    float* wdC;
+    __nv_bfloat16* wdB;        // [b, L, H, R, N]: dBbar rotated back (per head), bf16
+    __nv_bfloat16* wdC;
     float* wsc;                // [units][L][4]: db, dg, decay term, theta.dPhi per token
     float* wprev;              // [units][R][N]: the same for the initial state's previous B
     float* wF;                 // [units]: <dL/dh_final, h_final>
@@ -824,32 +838,22 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 }
             }
             // The rows go out through shared memory so that each half-warp stores one whole
-            // 256-byte row (a thread holds 64 bytes of one row, 16 rows per half-warp):
-            // dx and dBbar now (the buffers of Xs/Ds, Bs and this chunk's G_n operand, whose
-            // readers have finished), dCbar after them.
+            // 256-byte row (a thread holds 64 bytes of one row, 16 rows per half-warp), in the
+            // buffers of Xs/Ds, Bs and this chunk's G_n operand, whose readers have finished:
+            // dx in fp32, and the per-head dBbar and dCbar rows in bf16 (only their sums over
+            // the group's heads are used, by the norm kernel).
             stage_row(sm + S_XS, t, col0, vx);
-            stage_row(sm + S_BS, t, col0, nb0);
-            stage_row(sm + S_GN + cur * 16384, t, col0, nb1);
+            stage_row_bf16(sm + S_BS, t, col0, nb0, nb1);
+            stage_row_bf16(sm + S_GN + cur * 16384, t, col0, nc0, nc1);
             __syncthreads();
             for (int e = tid; e < 3 * 64 * 16; e += kThreads) {
                 const int tile = e >> 10, row = (e >> 4) & 63, ch = e & 15;
                 if (row / R >= T) continue;
                 const int64_t grow = ((bb * L + t0 + row / R) * H + hh) * R + row % R;
                 const uint8_t* src = tile == 0 ? sm + S_XS : tile == 1 ? sm + S_BS : sm + S_GN + cur * 16384;
-                float* dst = tile == 0 ? a.dx + grow * kP : a.wdB + grow * kN + (tile == 2 ? kHalf : 0);
-                *reinterpret_cast<float4*>(dst + 4 * ch) = *reinterpret_cast<const float4*>(src + staged_off(row, ch));
-            }
-            __syncthreads();
-            stage_row(sm + S_BS, t, col0, nc0);
-            stage_row(sm + S_GN + cur * 16384, t, col0, nc1);
-            __syncthreads();
-            for (int e = tid; e < 2 * 64 * 16; e += kThreads) {
-                const int tile = e >> 10, row = (e >> 4) & 63, ch = e & 15;
-                if (row / R >= T) continue;
-                const int64_t grow = ((bb * L + t0 + row / R) * H + hh) * R + row % R;
-                const uint8_t* src = tile == 0 ? sm + S_BS : sm + S_GN + cur * 16384;
-                float* dst = a.wdC + grow * kN + (tile == 1 ? kHalf : 0);
-                *reinterpret_cast<float4*>(dst + 4 * ch) = *reinterpret_cast<const float4*>(src + staged_off(row, ch));
+                const uint4 v = *reinterpret_cast<const uint4*>(src + staged_off(row, ch));
+                if (tile == 0) *reinterpret_cast<uint4*>(a.dx + grow * kP + 4 * ch) = v;
+                else *reinterpret_cast<uint4*>((tile == 1 ? a.wdB : a.wdC) + grow * kN + 8 * ch) = v;
             }
         }
         fence_before_sync();
@@ -1238,8 +1242,8 @@ cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cuda
     a.dprevx1 = o.dprevx1;
     a.dx = o.dx;
     a.dtheta = o.dtheta;
-    a.wdB = o.wdB;
-    a.wdC = o.wdC;
+    a.wdB = static_cast<__nv_bfloat16*>(o.wdB);
+    a.wdC = static_cast<__nv_bfloat16*>(o.wdC);
     a.wsc = o.wsc;
     a.wprev = o.wprev;
     a.wF = o.wF;
