@@ -249,11 +249,11 @@ M3_API size_t m3_scan_bwd_workspace_bytes(const m3_dims* dims);
  * at least m3_scan_bwd_workspace_bytes. Any supported N, P, R, dtype and flags; asynchronous
  * on `stream`.
  * Two forms compute the same gradients:
- *  - bf16 inputs with R = 1, N = 128, P = 64 and H a multiple of 4 run the chunked form on the
- *    tensor cores (64-token chunks, bf16 operands with fp32 accumulators, fp32 state
- *    adjoint), bitwise reproducible run to run except the dt_bias gradient (an atomic sum
- *    over units). Its bounded waits report a timeout through the workspace's status word,
- *    which m3_scan_check reads after the stream has synchronised.
+ *  - bf16 inputs with R in {1, 2, 4, 8}, N = 128, P = 64 and H a multiple of 4 run the
+ *    chunked form on the tensor cores (chunks of 64 (token, rank) rows, bf16 operands with
+ *    fp32 accumulators, fp32 state adjoint), bitwise reproducible run to run. Its bounded
+ *    waits report a timeout through the workspace's status word, which m3_scan_check reads
+ *    after the stream has synchronised.
  *  - every other shape, and any shape with M3_BWD_FP32 in dims->flags, runs two sequential
  *    sweeps in fp32 on the CUDA cores; not bitwise reproducible run to run (some sums use
  *    atomic adds, whose order varies in the last bits). */

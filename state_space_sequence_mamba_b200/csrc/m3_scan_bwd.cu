@@ -30,10 +30,11 @@
 // so the loop has no barrier; the next chunk's global loads (cp.async) fly during the loop.
 // bwd_rms_kernel computes the RMS scales of all B and C rows once, before the sweeps.
 //
-// Summation order: the cross-warp sums of dx and of the per-token scalar partials are
-// shared-memory atomic adds, and the bias and dt_bias sums over units are global atomic
-// adds, so the gradients are not bitwise reproducible run to run (they differ in the last
-// bits; the forward scan and the decode step are reproducible).
+// Summation order: in the sweeps, the cross-warp sums of dx and of the per-token scalar
+// partials are shared-memory atomic adds and the B and C bias sums over units are global
+// atomic adds, so the sweeps' gradients are not bitwise reproducible run to run (they differ
+// in the last bits). The dt_bias sum over units has a fixed order (per-unit shares, then a
+// sum over the batch), as every sum of the chunked tensor-core form does.
 #include <cuda_bf16.h>
 
 #include "m3_common.cuh"
@@ -1026,9 +1027,20 @@ __global__ void __launch_bounds__(kScalThreads) bwd_scalar_kernel(const BwdArgs 
         if (tid == 0) {
             float s = 0.f;
             for (int w = 0; w < kScalThreads / 32; ++w) s += red[w];
-            atomicAdd(a.ddtbias + hh, s);
+            a.wphi[u] = s;   // this unit's share; bwd_dtbias_kernel sums the batch in order
         }
     }
+}
+
+// dt_bias[h] = sum over the batch of the units' shares, in a fixed order (the per-chunk angle
+// buffer, no longer needed, holds the shares).
+__global__ void __launch_bounds__(256) bwd_dtbias_kernel(const float* __restrict__ share,
+                                                         int64_t b, int64_t H, float* ddtbias) {
+    const int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (h >= H) return;
+    float v = 0.f;
+    for (int64_t i = 0; i < b; ++i) v += share[i * H + h];
+    ddtbias[h] = v;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1219,6 +1231,11 @@ cudaError_t launch_scan_bwd(const ScanParams& f, const BwdGrads& g, bool bf16, f
     }
     bwd_scalar_kernel<<<static_cast<unsigned>(units), kScalThreads, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.ddtbias && (f.flags & M3_DT_SOFTPLUS)) {
+        bwd_dtbias_kernel<<<static_cast<unsigned>((f.H + 255) / 256), 256, 0, s>>>(a.wphi, f.b, f.H,
+                                                                                  a.ddtbias);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     const int64_t items = f.b * f.L * f.G * f.R * 2 + units * f.R;
     const int64_t blocks = (items * 32 + 255) / 256;
     bwd_norm_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(a, bf16 ? 1 : 0);

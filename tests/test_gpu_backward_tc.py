@@ -87,10 +87,12 @@ def test_tc_backward_without_final_gradient(cuda_dev):
     compare_tc(got, oracle_grads(pr, dy, None), pr)
 
 
-def test_tc_backward_is_reproducible(cuda_dev):
-    """Fixed summation order: two runs give the same bits in every gradient."""
-    pr = make_problem(2, 300, 8, 1, 64, 128, rank=1, chunk=64, dtype=torch.bfloat16,
-                      bc_norm=True, bias_std=0.1, seed=42, with_state=True)
+@pytest.mark.parametrize("R", [1, 4])
+def test_tc_backward_is_reproducible(cuda_dev, R):
+    """Fixed summation order: two runs give the same bits in every gradient, the bias and
+    dt_bias sums over units included (raw scalars, so dt_bias has a gradient)."""
+    pr = make_problem(2, 300, 8, 1, 64, 128, rank=R, chunk=64 // R, dtype=torch.bfloat16,
+                      bc_norm=True, bias_std=0.1, seed=42, with_state=True, raw_scalars=True)
     dy, dfin = draw_grads(pr, seed=6)
     a = gpu_grads(pr, dy, dfin, cuda_dev, exact=False)
     b = gpu_grads(pr, dy, dfin, cuda_dev, exact=False)
