@@ -135,6 +135,18 @@ def test_backward_workspace_and_argument_checks(lib):
                                                              flags=bd.M3_BWD_FP32))) == base
     assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(batch=2, seqlen=100, nheads=4,
                                                              in_dtype=bd.M3_F32))) == base
+    # MIMO R4: chunks of 16 tokens (64 rows), the bias sums and scales per rank
+    d4 = dims(batch=2, seqlen=100, nheads=4, dstate=128, rank=4, chunk=16)
+    nch4 = (100 + 3) // 4   # the sweeps stage 16 / R = 4 tokens at a time
+    simt4 = 4 * (2 * r64(2 * 100 * 4 * 4 * 128) + r64(units * nch4 * 64) + r64(units)
+                 + r64(units * 100 * 4) + r64(units * 4 * 128) + r64(2 * 2 * 100 * 4 * 4)
+                 + r64(units * 4))
+    n16 = (100 + 15) // 16
+    tc4 = (r256(units * n16 * 16384) + r256(units * n16 * 64 * 4) + r256(units * 128 * 64 * 4)
+           + r256(units * 65 * 4) + r256(units * 2 * 4 * 128 * 4) + r256(2 * n16 * 16 * 1 * 4 * 8))
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d4)) == 256 + r256(simt4) + tc4
+    d4f = dims(batch=2, seqlen=100, nheads=4, dstate=128, rank=4, chunk=16, flags=bd.M3_BWD_FP32)
+    assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(d4f)) == 256 + r256(simt4)
     assert lib.m3_scan_bwd_workspace_bytes(ctypes.byref(dims(rank=3))) == 0
     assert ctypes.sizeof(bd.Grads) == 10 * 8
     ins = fake_inputs()
