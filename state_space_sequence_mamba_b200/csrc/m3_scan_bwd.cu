@@ -1101,7 +1101,9 @@ __global__ void __launch_bounds__(256) bwd_norm_kernel(const BwdArgs a, int bf16
         vv[j] = 0.f;
         if (n < N) {
             if (dn_h) {
+                // the group's heads in order, eight loads in flight
                 const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(dn_base) + dn_off;
+#pragma unroll 8
                 for (int64_t h = 0; h < nh; ++h) dnv[j] += __bfloat162float(hb[h * dn_stride + n]);
             } else {
                 for (int64_t h = 0; h < nh; ++h) dnv[j] += dn_base[dn_off + h * dn_stride + n];
