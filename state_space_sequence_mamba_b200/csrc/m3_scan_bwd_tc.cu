@@ -1,5 +1,7 @@
 // Chunked backward of the prefill scan on the sm_100a tensor cores (bf16 operands, fp32
-// accumulators in TMEM, fp32 state adjoint), for SISO bf16 inputs with N = 128, P = 64.
+// accumulators in TMEM, fp32 state adjoint), for bf16 inputs with N = 128, P = 64 and rank
+// R in {1, 2, 4, 8}: a chunk is 64 operand rows, Q = 64 / R tokens of R (token, rank) rows,
+// as in the forward scan, and the token mask acts on full R x R blocks.
 //
 // Method ("Mamba-3: Improved Sequence Modeling using State Space Principles", Sec. 3.1.3
 // eq. 7 for the chunk mask M = L1 . L2, Sec. 3.3 for the chunked algorithm, and the chain
@@ -7,7 +9,7 @@
 // dt A, w_t = gamma_t + (1 - lam_{t+1}) dt_{t+1}, M[t,s] = e^{cum_t - cum_s} w_s for s < t,
 // gamma_t on the diagonal, H0' the primed state before the chunk) and G_n the state adjoint
 // dL/dh at the first token of the next chunk (the final state's gradient after the last
-// chunk, with alpha_n = 1), each chunk of Q = 64 tokens needs:
+// chunk, with alpha_n = 1), each chunk needs:
 //     S' = Bbar Cbar^T,  Z = X dY^T,  Q1 = Bbar G_n                 (tensor cores, M64)
 //     Ps = M^T o S',  Pz = M^T o Z                                   (CUDA cores)
 //     dx    = Ps dY + diag(w e^{cx_T - cum}) Q1                      (tensor cores, then Q1 scaled)
@@ -15,16 +17,17 @@
 //     dCbar = Pz^T Bbar + diag(e^{cum - cum_0}) dY (e^{cum_0} H0')^T (tensor cores, N128)
 //     G_0   = Cbar^T diag(e^{cum - cum_0}) dY + e^{cx_T - cum_0} G_n (tensor cores, M128)
 // where cx_T = cum_end + dt_n A_n (alpha_n = e^{dt_n A_n} of the next chunk's first token).
-// The per-token scalars the decay, step and trapezoid gradients need are row sums of the
-// element-wise products of the two Q x Q matrices:
+// The per-token scalars the step and trapezoid gradients need are row sums of the element-
+// wise products of the two 64 x 64 matrices, summed over the token's rows:
 //     dg_t = <G_t, u_t>     = sum_{s>=t} e^{cum_s - cum_t} S'[t,s] Z[t,s] + e^{cx_T - cum_t} q_t
 //     db_{t+1} = <G_{t+1}, u_t> = sum_{s>t} e^{cum_s - cum_{t+1}} S'[t,s] Z[t,s]
 //                                 + e^{cx_T - cum_{t+1}} q_t,     q_t = (Bbar_t G_n) . x_t
-// dy . y_t = <Cbar_t, dCbar_t>, and the angle adjoint dPhi_t (the cross products of dBbar and
-// dCbar with Bbar and Cbar, summed from the end of the sequence) gives dtheta = dt dPhi.
-// dBbar and dCbar are rotated back to the normalised, biased frame; the RMS-norm backward,
-// the sum over the heads of a group and the step-scalar chain rule run in the kernels the
-// sequential backward also uses.
+// The decay gradient D_t = <G_t, alpha_t h_{t-1}> is formed per chunk from sums that do not
+// cancel (see the per-token term below), the angle adjoint dPhi_t (the cross products of
+// dBbar and dCbar with Bbar and Cbar, summed from the end of the sequence) gives
+// dtheta = dt dPhi. dBbar and dCbar are rotated back to the normalised, biased frame; the
+// RMS-norm backward, the sum over the heads of a group and the step-scalar chain rule run in
+// the kernels the sequential backward also uses.
 //
 // One CTA per (batch, head) unit walks its chunks from the last to the first, carrying G_n
 // (fp32 in registers, bf16 as an operand) and the angle adjoint. The primed chunk-start
