@@ -13,10 +13,12 @@ primed state before the chunk and G_n the state adjoint at the next chunk's firs
     T2 = sum_{s >= t} e^{cum_s} dy_s . (H0'^T Cbar_s),
     T3 = sum_{s' < t} w_s' e^{cx_T - cum_s'} <G_n, Bbar_s' x_s'^T>,
     T4 = e^{cx_T} <G_n, H0'>.
+For MIMO (rank R) the rows are (token, rank) pairs: S' and Z run over rows, the crossing
+pairs are rows of different tokens s' < t <= s, and u_t = sum_r Bbar_t[r] x_t[r]^T.
 This file checks that form against D_t computed token by token from the plain recurrence and
-its adjoint, for several chunk sizes, ragged ends and both discretisations, and that the
-per-token values the kernel hands to the scalar step (D'_t - D_{t+1} + gamma_t dg_t) give
-back D_t through that step's suffix sum.
+its adjoint, for several chunk sizes, ranks 1, 2 and 4, ragged ends and both
+discretisations, and that the per-token values the kernel hands to the scalar step
+(D'_t - D_{t+1} + gamma_t dg_t) give back D_t through that step's suffix sum.
 """
 import math
 
@@ -26,7 +28,7 @@ import pytest
 from test_backward_algorithm import rot_T
 
 
-def problem(rng, L, N, P, zoh):
+def problem(rng, L, N, P, zoh, R=1):
     d = np.log1p(np.exp(rng.standard_normal(L) - 1.0))
     a_rate = -np.exp(rng.uniform(-1, 1, L))
     lam = rng.uniform(0.05, 0.95, L)
@@ -43,14 +45,14 @@ def problem(rng, L, N, P, zoh):
     theta = rng.uniform(-math.pi, math.pi, (L, N // 2))
     phi0 = rng.uniform(-math.pi, math.pi, N // 2)
     Phi = phi0 + np.cumsum(d[:, None] * theta, 0)
-    Bn = rng.standard_normal((L, N))
-    Cn = rng.standard_normal((L, N))
-    Bbar = rot_T(Bn, Phi)
-    Cbar = rot_T(Cn, Phi)
-    Bm1 = rot_T(rng.standard_normal(N), phi0)
-    x = rng.standard_normal((L, P))
-    xm1 = rng.standard_normal(P)
-    dy = rng.standard_normal((L, P))
+    Bn = rng.standard_normal((L, R, N))
+    Cn = rng.standard_normal((L, R, N))
+    Bbar = rot_T(Bn, Phi[:, None])
+    Cbar = rot_T(Cn, Phi[:, None])
+    Bm1 = rot_T(rng.standard_normal((R, N)), phi0)
+    x = rng.standard_normal((L, R, P))
+    xm1 = rng.standard_normal((R, P))
+    dy = rng.standard_normal((L, R, P))
     h0 = rng.standard_normal((N, P))
     dh1 = rng.standard_normal((N, P))
     return dict(d=d, a=d * a_rate, al=al, be=be, ga=ga, c=c, w=ga + c[1:], Bbar=Bbar,
@@ -60,8 +62,8 @@ def problem(rng, L, N, P, zoh):
 def sequential(q):
     """h_t, G_t, D_t = alpha_t <G_t, h_{t-1}>, db_t, dg_t and <dh1, h_final>, token by token."""
     L = len(q["d"])
-    u = [np.outer(q["Bbar"][t], q["x"][t]) for t in range(L)]
-    um1 = np.outer(q["Bm1"], q["xm1"])
+    u = [np.einsum("rn,rp->np", q["Bbar"][t], q["x"][t]) for t in range(L)]
+    um1 = np.einsum("rn,rp->np", q["Bm1"], q["xm1"])
     h, prev, uprev = [], q["h0"], um1
     for t in range(L):
         cur = q["al"][t] * prev + q["be"][t] * uprev + q["ga"][t] * u[t]
@@ -70,7 +72,7 @@ def sequential(q):
     G = [None] * L
     nxt = q["dh1"]
     for t in range(L - 1, -1, -1):
-        G[t] = np.outer(q["Cbar"][t], q["dy"][t]) + nxt
+        G[t] = np.einsum("rn,rp->np", q["Cbar"][t], q["dy"][t]) + nxt
         nxt = q["al"][t] * G[t]
     hm = [q["h0"]] + h[:-1]
     um = [um1] + u[:-1]
@@ -93,31 +95,37 @@ def chunked_D(q, Q, h, G):
         else:
             cxT, Gn = cum[-1], q["dh1"]
         hprev = h[t0 - 1] if t0 > 0 else q["h0"]
-        uprev = np.outer(q["Bbar"][t0 - 1], q["x"][t0 - 1]) if t0 > 0 else np.outer(q["Bm1"], q["xm1"])
+        uprev = (np.einsum("rn,rp->np", q["Bbar"][t0 - 1], q["x"][t0 - 1]) if t0 > 0
+                 else np.einsum("rn,rp->np", q["Bm1"], q["xm1"]))
         H0 = hprev + q["c"][t0] * uprev                       # primed state before the chunk
-        B, C, X, dY, w = (q[k][t0:t1] for k in ("Bbar", "Cbar", "x", "dy", "w"))
-        S = B @ C.T                                           # S'[s', s] = Bbar_s' . Cbar_s
-        Z = X @ dY.T                                          # Z[s', s] = x_s' . dy_s
-        idx = np.arange(T)
-        Acr = np.where(idx[:, None] < idx[None, :],
-                       np.exp(cum[None, :] - cum[:, None]) * w[:, None] * S * Z, 0.0)
-        v = np.exp(cum) * np.einsum("sp,np,sn->s", dY, H0, C)
-        qv = np.einsum("sn,np,sp->s", B, Gn, X)
+        R = q["x"].shape[1]
+        rows = lambda k: q[k][t0:t1].reshape(T * R, -1)      # row = token * R + rank
+        B, C, X, dY = rows("Bbar"), rows("Cbar"), rows("x"), rows("dy")
+        w = q["w"][t0:t1]
+        tok = np.arange(T * R) // R
+        S = B @ C.T                                           # S'[i, j] = Bbar_i . Cbar_j
+        Z = X @ dY.T                                          # Z[i, j] = x_i . dy_j
+        Acr = np.where(tok[:, None] < tok[None, :],
+                       np.exp(cum[tok][None, :] - cum[tok][:, None]) * w[tok][:, None] * S * Z, 0.0)
+        v = np.exp(cum[tok]) * np.einsum("jp,np,jn->j", dY, H0, C)
+        qv = np.einsum("in,np,ip->i", B, Gn, X)
         T4 = math.exp(cxT) * (Gn * H0).sum()
         for t in range(T):
-            T1 = Acr[:t, t:].sum()
-            T2 = v[t:].sum()
-            T3 = (w[:t] * np.exp(cxT - cum[:t]) * qv[:t]).sum()
+            before, after = tok < t, tok >= t
+            T1 = Acr[np.ix_(before, after)].sum()
+            T2 = v[after].sum()
+            T3 = (w[tok] * np.exp(cxT - cum[tok]) * qv)[before].sum()
             Dp[t0 + t] = T1 + T2 + T3 + T4
     return Dp
 
 
+@pytest.mark.parametrize("R", [1, 2, 4])
 @pytest.mark.parametrize("zoh", [False, True])
 @pytest.mark.parametrize("Q", [1, 4, 5, 16])
-def test_direct_chunk_form_of_the_decay_gradient(Q, zoh):
-    rng = np.random.default_rng(90 + Q + 7 * zoh)
+def test_direct_chunk_form_of_the_decay_gradient(Q, zoh, R):
+    rng = np.random.default_rng(90 + Q + 7 * zoh + 31 * R)
     L, N, P = 13, 8, 3
-    q = problem(rng, L, N, P, zoh)
+    q = problem(rng, L, N, P, zoh, R)
     h, G, D, db, dg, F = sequential(q)
     Dp = chunked_D(q, Q, h, G)
     np.testing.assert_allclose(Dp - q["be"] * db, D, rtol=1e-10, atol=1e-10)
