@@ -34,6 +34,8 @@
 // states come from a forward state pass (the tensor-core scan's state-only form), which
 // stores e^{cum_0} H0' per chunk in the swizzled bf16 operand layout and the angle before each
 // chunk. Every sum has a fixed order: the gradients are reproducible run to run.
+#include <cstdlib>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -257,6 +259,9 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
         s_lcnt[2] += 1;
     };
     auto issue_b = [&](int c) {
+        // test hook: CTA 0 skips this group for the chunk it reaches at step test_skip_theta,
+        // so that its bounded wait runs out (a load that nothing issues)
+        if (blockIdx.x == 0 && p.test_skip_theta > 0 && c == nch - 1 - p.test_skip_theta) return;
         const int t0 = c * Q;
         mbar_arrive_expect_tx(&bar_b, Q * 128 + 8192 + 16384);
         tma_load_4d(sm + S_TH, &maps.theta, &bar_b, 0, ih, t0, ib);
@@ -1255,6 +1260,9 @@ cudaError_t launch_bwd_tc(const ScanParams& p, const BwdTcOut& o, void* ws, cuda
     a.dphi0 = o.dphi0;
     a.dprevx0 = o.dprevx0;
     a.status = o.status;
+    // test hook of the timeout path (as for the forward scans): > 0 makes CTA 0 skip the
+    // theta / dY / raw C load of that step, so that its bounded wait gives up
+    if (const char* env = std::getenv("M3_TEST_SKIP_THETA_LOAD")) a.p.test_skip_theta = std::atoi(env);
     const bool raw = p.flags != 0;
     switch (R) {
         case 1: e = launch_bwd_tc_r<1>(a, maps, units, raw, s); break;

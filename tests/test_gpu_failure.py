@@ -50,6 +50,44 @@ def test_timeout_is_reported_and_the_workspace_reusable(cuda_dev, R, chunk):
     compare(pr, y, fin, yo, so)
 
 
+@pytest.mark.parametrize("R", [1, 4])
+def test_backward_timeout_is_reported_and_the_workspace_reusable(cuda_dev, R):
+    """The chunked tensor-core backward: CTA 0 skips one load group (theta, dY, raw C) of its
+    second step, so its bounded wait gives up; m3_scan_check reports the timeout on the
+    backward's workspace and the next call on the same workspace matches the oracle (the
+    drain of the CTA's copies and MMAs and the TMEM release worked)."""
+    from test_gpu_backward import draw_grads, oracle_grads
+    from test_gpu_backward_tc import compare_tc
+    pr = make_problem(1, 200, 4, 1, 64, 128, rank=R, chunk=64 // R, dtype=torch.bfloat16,
+                      bc_norm=True, bias_std=0.1, seed=171 + R, with_state=True)
+    dy, dfin = draw_grads(pr, seed=5)
+    g = pr.to(cuda_dev)
+    t = g.tensors()
+    dims = m3.make_dims(t["x"], t["B"], 1, True, 1e-6)
+    ws = torch.zeros(m3.scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=cuda_dev)
+    init = m3.State.from_dict(g.state)
+    df = {k: v.to(cuda_dev) for k, v in dfin.items()}
+
+    def call():
+        return m3.scan_bwd(**t, dy=dy.to(cuda_dev), init=init, dfinal=df, bc_norm=True,
+                           workspace=ws)
+
+    os.environ["M3_TEST_SKIP_THETA_LOAD"] = "1"
+    try:
+        call()
+        torch.cuda.synchronize()
+    finally:
+        del os.environ["M3_TEST_SKIP_THETA_LOAD"]
+    with pytest.raises(m3.M3Error) as ei:
+        m3.scan_check(ws)
+    assert ei.value.status == m3.M3_ERR_TIMEOUT
+    assert int(ws[:256].count_nonzero()) == 0          # the header is zero again
+    got = call()
+    torch.cuda.synchronize()
+    m3.scan_check(ws)
+    compare_tc(got, oracle_grads(pr, dy, dfin), pr)
+
+
 PAT = 0x5A   # the guard bytes
 BAND = 4096  # bytes before and after each output
 
