@@ -49,7 +49,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 256;
-constexpr int kN = 128, kP = 64, kHalf = 64, kQ = 64;
+constexpr int kN = 128, kP = 64, kHalf = 64, kQ = 64;   // kQ: operand rows per chunk
 constexpr int kPhiStride = 68;   // floats per row of the angle tile (padded against conflicts)
 
 // Shared memory (bytes from a 1024-byte aligned base). Operand tiles are 64 rows of 128 bytes
@@ -946,7 +946,7 @@ bwd_tc_kernel(const BwdTcArgs a, const __grid_constant__ BwdMaps maps) {
                 p3[k] = real ? sf[F_VN + t] * q : 0.f;
                 v[k] = real ? sf[F_DS + t] * vv : 0.f;
             }
-            // exclusive prefixes of g and p3, inclusive suffix of v, over the 64 tokens
+            // exclusive prefixes of g and p3, inclusive suffix of v, over the chunk's tokens (<= 64)
             const float gi0 = warp_inclusive_scan(g[0]), gi1 = warp_inclusive_scan(g[1]);
             const float pi0 = warp_inclusive_scan(p3[0]), pi1 = warp_inclusive_scan(p3[1]);
             const float vi0 = warp_inclusive_scan(v[0]), vi1 = warp_inclusive_scan(v[1]);
