@@ -510,6 +510,15 @@ def bwd_bytes(pr) -> int:
     return reads + writes
 
 
+def bwd_chunked(m3, dims) -> bool:
+    """Whether m3_scan_bwd runs the chunked tensor-core form for these dims, as the library
+    decides it: only that form needs workspace beyond the fp32 sweeps' (its chunk states)."""
+    import copy
+    fp32 = copy.copy(dims)
+    fp32.flags = dims.flags | m3.BWD_FP32
+    return m3.scan_bwd_workspace_bytes(dims) > m3.scan_bwd_workspace_bytes(fp32)
+
+
 def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cpu=False,
                    exact=False):
     """m3_scan_bwd on a prefill workload with a carried initial state and dy ~ N(0,1); with
@@ -527,8 +536,7 @@ def bench_backward(m3, dev, cfg, hbm, world, dist, seed, reps=5, seqlen=None, cp
         sa["flags"] = sa["flags"] | m3.BWD_FP32
     dims = m3.make_dims(pr.x, pr.B, 1, d.bc_norm, d.norm_eps, sa["flags"])
     ws = torch.empty(m3.scan_bwd_workspace_bytes(dims), dtype=torch.uint8, device=dev)
-    tc = (not exact and d.dtype == torch.bfloat16 and d.rank in (1, 2, 4, 8)
-          and d.dstate == 128 and d.headdim == 64 and d.nheads % 4 == 0)
+    tc = bwd_chunked(m3, dims)
     stream = torch.cuda.current_stream()
 
     def step():   # the config's own BC norm, eps and scalar form, as the CPU baseline reads them

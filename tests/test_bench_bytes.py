@@ -60,3 +60,24 @@ def test_quoted_workload_bytes():
     pr = make_problem(4, 2048, 64, 1, 64, 128, rank=1, dtype=torch.bfloat16, bc_norm=True,
                       bias_std=0.1, seed=1)
     assert bench.scan_bytes(pr) == 220430336
+
+
+def test_backward_form_follows_the_library():
+    """The form the backward bench line reports is the one the library picks: the chunked
+    tensor-core form for the bf16 prefill workloads (SISO and MIMO R4), the fp32 sweeps with
+    M3_BWD_FP32, for fp32 inputs and for a head size the chunked form does not take."""
+    from state_space_sequence_mamba_b200 import binding as m3
+    from state_space_sequence_mamba_b200.inputs import make_config
+    b = _bench()
+    for cfg in (1, 2):
+        pr = make_config(cfg, with_state=True, batch=1, nheads=4, seqlen=64)
+        dims = m3.make_dims(pr.x, pr.B, 1, True, 1e-6, 0)
+        assert b.bwd_chunked(m3, dims), cfg
+        dims.flags = m3.BWD_FP32
+        assert not b.bwd_chunked(m3, dims), cfg
+    for kw in (dict(dtype=torch.float32), dict(P=32)):
+        P = kw.get("P", 64)
+        pr = make_problem(1, 64, 4, 1, P, 128, rank=1, chunk=64,
+                          dtype=kw.get("dtype", torch.bfloat16), bc_norm=True, seed=3)
+        dims = m3.make_dims(pr.x, pr.B, 1, True, 1e-6, 0)
+        assert not b.bwd_chunked(m3, dims), kw
